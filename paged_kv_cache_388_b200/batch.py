@@ -1,0 +1,84 @@
+"""Turn a workload description into the host arrays the kernels consume.
+
+Runs the block allocator step by step the way a serving engine would for one
+iteration: sequences that already hold their earlier context, the new tokens
+of this step appended one by one (taking blocks on demand and copying shared
+blocks before they are written), then one attention call over everything.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from .allocator import BlockAllocator
+
+
+@dataclass
+class Batch:
+    block_tables: np.ndarray       # int32 [S, max_blocks]
+    context_lens: np.ndarray       # int32 [S], includes this step's tokens
+    query_start_loc: np.ndarray | None  # int32 [S+1], None = one query token per sequence
+    slot_mapping: np.ndarray       # int64 [T_new] slots of this step's new tokens
+    cow_pairs: np.ndarray          # int64 [P, 2] (src, dst) block copies before the writes
+    max_query_len: int
+    allocator: BlockAllocator
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max()) if self.num_seqs else 0
+
+
+def build_batch(wl) -> Batch:
+    """``wl`` is a ``workloads.Workload``."""
+    alloc = BlockAllocator(wl.num_blocks, wl.block_size, wl.free_order)
+    slots: list[int] = []
+    cows: list[tuple[int, int]] = []
+    sids: list[int] = []
+
+    def append(sid):
+        s, cow = alloc.append_slot(sid)
+        slots.append(s)
+        if cow is not None:
+            cows.append(cow)
+
+    if wl.kind in ("decode", "mixed"):
+        for L, Q in zip(wl.context_lens, wl.query_lens):
+            sid = alloc.new_sequence(L - Q)
+            for _ in range(Q):
+                append(sid)
+            sids.append(sid)
+        qlens = list(wl.query_lens)
+    elif wl.kind == "shared_prefix":
+        for p in range(wl.num_prompts):
+            root = alloc.new_sequence(wl.prompt_len)
+            group = [root] + [alloc.fork(root) for _ in range(wl.samples - 1)]
+            sids.extend(group)
+        for sid, tail in zip(sids, wl.tails):
+            for _ in range(tail):
+                append(sid)
+        qlens = [1] * len(sids)
+    else:
+        raise ValueError(wl.kind)
+
+    qsl = None
+    if any(q != 1 for q in qlens):
+        qsl = np.zeros(len(qlens) + 1, dtype=np.int32)
+        qsl[1:] = np.cumsum(qlens)
+    return Batch(
+        block_tables=alloc.block_tables_array(sids),
+        context_lens=alloc.context_lens_array(sids),
+        query_start_loc=qsl,
+        slot_mapping=np.asarray(slots, dtype=np.int64),
+        cow_pairs=np.asarray(cows, dtype=np.int64).reshape(-1, 2),
+        max_query_len=max(qlens) if qlens else 0,
+        allocator=alloc,
+    )

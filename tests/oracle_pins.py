@@ -1,0 +1,425 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each pin takes the oracle shared library handle, so the same pins run on the
+real oracle (tests/test_oracle.py) and on deliberately broken copies of it
+(tests/test_oracle_mutants.py, which shows every planted mistake fails one).
+
+The pins: the pages' worked examples (tests/golden/), NumPy brute force on
+contiguous, never-paged K/V, closed forms of softmax attention, and the
+invariants of paging (placement, sharing, causal truncation, GQA grouping).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle
+from oracle import alloc_model
+from oracle.brute import attention_contiguous
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------
+# helpers: build paged inputs from contiguous per-sequence K/V (test side)
+# ----------------------------------------------------------------------------
+def _bits(x, dtype):
+    """float64 array -> storage array of the cache dtype."""
+    if dtype == "f32":
+        return x.astype(np.float32)
+    if dtype == "f16":
+        return x.astype(np.float16)
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _as_f64(a, dtype):
+    if dtype == "bf16":
+        import torch
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    return a.astype(np.float64)
+
+
+def page_sequences(ks, vs, bs, nb, rng, perm=None):
+    """Place contiguous K/V ([L_i, Hk, D] each) into a pool [nb, Hk, bs, D]:
+    logical block j of sequence i goes to the next block of a random
+    permutation of the pool.  Returns (k_pool, v_pool, tables)."""
+    hk, d = ks[0].shape[1], ks[0].shape[2]
+    k_pool = rng.standard_normal((nb, hk, bs, d))  # junk in unused slots
+    v_pool = rng.standard_normal((nb, hk, bs, d))
+    order = list(rng.permutation(nb)) if perm is None else list(perm)
+    tables = []
+    for k, v in zip(ks, vs):
+        L = k.shape[0]
+        nblk = -(-L // bs)
+        t = [int(order.pop(0)) for _ in range(nblk)]
+        for j, pb in enumerate(t):
+            lo, hi = j * bs, min(L, (j + 1) * bs)
+            # pool[pb, head, offset, :] holds token j*bs + offset
+            k_pool[pb, :, : hi - lo, :] = np.transpose(k[lo:hi], (1, 0, 2))
+            v_pool[pb, :, : hi - lo, :] = np.transpose(v[lo:hi], (1, 0, 2))
+        tables.append(t)
+    width = max(len(t) for t in tables)
+    bt = np.zeros((len(tables), width), dtype=np.int32)
+    for i, t in enumerate(tables):
+        bt[i, : len(t)] = t
+    return k_pool, v_pool, bt
+
+
+def random_case(rng, lens, qlens, H, Hk, D, bs, dtype, nb_extra=3):
+    """Contiguous K/V and queries, rounded to the dtype, plus their paged form."""
+    ks = [_as_f64(_bits(rng.standard_normal((L, Hk, D)), dtype), dtype) for L in lens]
+    vs = [_as_f64(_bits(rng.standard_normal((L, Hk, D)), dtype), dtype) for L in lens]
+    nb = sum(-(-L // bs) for L in lens) + nb_extra
+    k_pool, v_pool, bt = page_sequences(ks, vs, bs, nb, rng)
+    tq = sum(qlens)
+    q = _as_f64(_bits(rng.standard_normal((tq, H, D)), dtype), dtype)
+    qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    return dict(ks=ks, vs=vs, q=q, k_pool=_bits(k_pool, dtype), v_pool=_bits(v_pool, dtype),
+                bt=bt, cl=np.asarray(lens, np.int32), qsl=qsl, H=H, Hk=Hk, D=D, bs=bs,
+                dtype=dtype)
+
+
+def run_oracle(lib, c, scale, use_qsl=True, rows=None):
+    return oracle.decode(_bits(c["q"], c["dtype"]), c["k_pool"], c["v_pool"], c["bt"], c["cl"],
+                         scale, c["dtype"], query_start_loc=c["qsl"] if use_qsl else None,
+                         rows=rows, lib=lib)
+
+
+def run_brute(c, scale):
+    outs = []
+    for i, (k, v) in enumerate(zip(c["ks"], c["vs"])):
+        q = c["q"][c["qsl"][i]: c["qsl"][i + 1]]
+        outs.append(attention_contiguous(q, k, v, scale, c["H"] // c["Hk"]))
+    return np.concatenate(outs, axis=0)
+
+
+# ----------------------------------------------------------------------------
+# pins
+# ----------------------------------------------------------------------------
+def pin_brute_force(lib):
+    """Paged oracle == NumPy attention on contiguous K/V, many shapes."""
+    rng = np.random.default_rng(7)
+    shapes = [  # (lens, qlens, H, Hk, D, bs, dtype)
+        ([17, 33, 64, 100], [1, 1, 1, 1], 4, 4, 64, 16, "f32"),
+        ([1, 16, 31, 50], [1, 1, 1, 1], 8, 2, 64, 16, "f16"),
+        ([40, 70], [1, 1], 16, 2, 128, 32, "bf16"),
+        ([37, 65, 20], [5, 1, 20], 8, 2, 64, 16, "bf16"),
+        ([48], [16], 4, 1, 64, 32, "f32"),
+    ]
+    for lens, qlens, H, Hk, D, bs, dt in shapes:
+        c = random_case(rng, lens, qlens, H, Hk, D, bs, dt)
+        scale = 1.0 / math.sqrt(D)
+        got = run_oracle(lib, c, scale)
+        want = run_brute(c, scale)
+        assert np.allclose(got, want, rtol=1e-12, atol=1e-12), (lens, H, Hk, D, bs, dt)
+
+
+def pin_decode_without_qsl(lib):
+    """query_start_loc=None means one query token per sequence."""
+    rng = np.random.default_rng(8)
+    c = random_case(rng, [5, 19, 33], [1, 1, 1], 4, 2, 64, 16, "f32")
+    a = run_oracle(lib, c, 0.125, use_qsl=True)
+    b = run_oracle(lib, c, 0.125, use_qsl=False)
+    assert np.array_equal(a, b)
+
+
+def pin_identical_keys_mean(lib):
+    """All keys equal -> every weight equal -> output = mean of visible V."""
+    rng = np.random.default_rng(9)
+    L, H, Hk, D, bs = 37, 4, 2, 64, 16
+    krow = rng.standard_normal((Hk, D))
+    ks = [np.broadcast_to(krow, (L, Hk, D)).copy()]
+    vs = [_as_f64(_bits(rng.standard_normal((L, Hk, D)), "f32"), "f32")]
+    kp, vp, bt = page_sequences(ks, vs, bs, 6, rng)
+    q = rng.standard_normal((1, H, D))
+    out = oracle.decode(_bits(q, "f32"), _bits(kp, "f32"), _bits(vp, "f32"), bt,
+                        np.asarray([L], np.int32), 0.7, "f32", lib=lib)
+    for h in range(H):
+        want = vs[0][:, h // (H // Hk), :].mean(axis=0)
+        assert np.allclose(out[0, h], want, rtol=1e-12, atol=1e-13)
+
+
+def pin_single_key(lib):
+    """One visible key -> output equals that V row exactly."""
+    rng = np.random.default_rng(10)
+    for dt in ("f32", "f16", "bf16"):
+        c = random_case(rng, [1, 1], [1, 1], 4, 2, 64, 16, dt)
+        out = run_oracle(lib, c, 0.125)
+        for i in range(2):
+            for h in range(4):
+                assert np.array_equal(out[i, h], c["vs"][i][0, h // 2, :])
+
+
+def pin_dominant_logit(lib):
+    """q parallel to K[j] and large -> softmax is one-hot on j -> output V[j]."""
+    rng = np.random.default_rng(11)
+    L, D, bs = 40, 64, 16
+    k = rng.standard_normal((L, 1, D))
+    k /= np.linalg.norm(k, axis=2, keepdims=True)
+    v = rng.standard_normal((L, 1, D))
+    kp, vp, bt = page_sequences([k], [v], bs, 5, rng)
+    for j in (0, 17, 39):
+        q = (60.0 * k[j, 0, :]).reshape(1, 1, D) * 8.0  # scale 1/8 undone
+        out = oracle.decode(_bits(q, "f32"), _bits(kp, "f32"), _bits(vp, "f32"), bt,
+                            np.asarray([L], np.int32), 0.125, "f32", lib=lib)
+        vj = _as_f64(_bits(v[j, 0, :], "f32"), "f32")
+        assert np.allclose(out[0, 0], vj, atol=1e-6), j
+    # logits large enough to overflow exp() unless the maximum is subtracted
+    q = (2000.0 * k[5, 0, :]).reshape(1, 1, D)
+    out = oracle.decode(_bits(q, "f32"), _bits(kp, "f32"), _bits(vp, "f32"), bt,
+                        np.asarray([L], np.int32), 1.0, "f32", lib=lib)
+    assert np.all(np.isfinite(out))
+
+
+def pin_v_linearity(lib):
+    """Doubling V doubles the output exactly (power-of-two scaling is exact)."""
+    rng = np.random.default_rng(12)
+    c = random_case(rng, [29, 50], [1, 3], 8, 4, 64, 16, "f32")
+    a = run_oracle(lib, c, 0.125)
+    c2 = dict(c)
+    c2["v_pool"] = (c["v_pool"] * 2).astype(np.float32)
+    b = run_oracle(lib, c2, 0.125)
+    assert np.array_equal(b, 2 * a)
+
+
+def pin_scale_zero_mean(lib):
+    """scale = 0 -> uniform weights -> mean of visible V (per causal row)."""
+    rng = np.random.default_rng(13)
+    c = random_case(rng, [23], [4], 4, 2, 64, 16, "f32")
+    out = run_oracle(lib, c, 0.0)
+    for t in range(4):
+        n = 23 - 4 + t + 1
+        for h in range(4):
+            want = c["vs"][0][:n, h // 2, :].mean(axis=0)
+            assert np.allclose(out[t, h], want, rtol=1e-12, atol=1e-13)
+
+
+def pin_hand_example(lib):
+    """A two-key example worked by hand: D=2, scale 1, q=(1,0),
+    K=((0,0),(ln 3, 0)) -> weights (1/4, 3/4); V=((4,0),(8,2)) -> (7, 1.5)."""
+    kp = np.zeros((1, 1, 16, 2))
+    vp = np.zeros((1, 1, 16, 2))
+    kp[0, 0, 1] = (math.log(3.0), 0.0)
+    vp[0, 0, 0] = (4.0, 0.0)
+    vp[0, 0, 1] = (8.0, 2.0)
+    q = np.array([[[1.0, 0.0]]])
+    out = oracle.decode(_bits(q, "f32"), _bits(kp, "f32"), _bits(vp, "f32"),
+                        np.zeros((1, 1), np.int32), np.asarray([2], np.int32), 1.0, "f32", lib=lib)
+    # ln 3 is rounded to fp32; the weight of key 1 is exp(fl(ln3))/(1+exp(fl(ln3)))
+    assert np.allclose(out[0, 0], [7.0, 1.5], atol=1e-6)
+
+
+def pin_gqa_equals_replicated_mha(lib):
+    """GQA over Hk heads == MHA after replicating every KV head g times."""
+    rng = np.random.default_rng(14)
+    H, Hk, D, bs = 8, 2, 64, 16
+    g = H // Hk
+    c = random_case(rng, [21, 45], [1, 2], H, Hk, D, bs, "f32")
+    a = run_oracle(lib, c, 0.125)
+    rep = lambda p: np.repeat(p, g, axis=1)  # noqa: E731  kv head j -> heads j*g..j*g+g-1
+    b = oracle.decode(_bits(c["q"], "f32"), rep(c["k_pool"]), rep(c["v_pool"]), c["bt"], c["cl"],
+                      0.125, "f32", query_start_loc=c["qsl"], lib=lib)
+    assert np.array_equal(a, b)
+
+
+def pin_placement_invariance(lib):
+    """Relabelling physical blocks (moving the data, rewriting the tables)
+    leaves every output bit-identical."""
+    rng = np.random.default_rng(15)
+    c = random_case(rng, [30, 64, 7], [1, 4, 1], 8, 2, 64, 16, "bf16")
+    a = run_oracle(lib, c, 0.125)
+    nb = c["k_pool"].shape[0]
+    pi = rng.permutation(nb)             # old block b -> new block pi[b]
+    kp = np.empty_like(c["k_pool"])
+    vp = np.empty_like(c["v_pool"])
+    kp[pi] = c["k_pool"]
+    vp[pi] = c["v_pool"]
+    c2 = dict(c, k_pool=kp, v_pool=vp, bt=pi[c["bt"]].astype(np.int32))
+    # unused table entries are never read; keep them in range
+    b = run_oracle(lib, c2, 0.125)
+    assert np.array_equal(a, b)
+
+
+def pin_shared_equals_duplicated(lib):
+    """Sequences pointing at the same physical blocks give the same outputs as
+    sequences holding private copies of those blocks."""
+    rng = np.random.default_rng(16)
+    H, Hk, D, bs, P = 8, 2, 64, 16, 48
+    prompt_k = rng.standard_normal((P, Hk, D))
+    prompt_v = rng.standard_normal((P, Hk, D))
+    tails = [5, 17, 1]
+    ks = [np.concatenate([prompt_k, rng.standard_normal((t, Hk, D))]) for t in tails]
+    vs = [np.concatenate([prompt_v, rng.standard_normal((t, Hk, D))]) for t in tails]
+    kp, vp, bt = page_sequences(ks, vs, bs, 20, rng)           # private copies
+    shared_bt = bt.copy()
+    shared_bt[:, : P // bs] = bt[0, : P // bs]                  # all point at seq 0's prompt
+    q = _bits(rng.standard_normal((3, H, D)), "f32")
+    lens = np.asarray([P + t for t in tails], np.int32)
+    a = oracle.decode(q, _bits(kp, "f32"), _bits(vp, "f32"), bt, lens, 0.125, "f32", lib=lib)
+    b = oracle.decode(q, _bits(kp, "f32"), _bits(vp, "f32"), shared_bt, lens, 0.125, "f32", lib=lib)
+    assert np.array_equal(a, b)
+
+
+def pin_causal_truncation(lib):
+    """Row t of a Q-token chunk == a decode of the same sequence truncated to
+    L - Q + t + 1 tokens."""
+    rng = np.random.default_rng(17)
+    L, Q = 70, 12
+    c = random_case(rng, [L], [Q], 8, 2, 64, 16, "f32")
+    full = run_oracle(lib, c, 0.125)
+    for t in (0, 5, 11):
+        n = L - Q + t + 1
+        one = oracle.decode(_bits(c["q"][t: t + 1], "f32"), c["k_pool"], c["v_pool"], c["bt"],
+                            np.asarray([n], np.int32), 0.125, "f32", lib=lib)
+        assert np.array_equal(full[t], one[0]), t
+
+
+def pin_empty_context(lib):
+    """Context length 0 gives a zero output (defined edge case)."""
+    rng = np.random.default_rng(18)
+    c = random_case(rng, [9], [1], 4, 4, 64, 16, "f32")
+    out = oracle.decode(_bits(c["q"], "f32"), c["k_pool"], c["v_pool"], c["bt"],
+                        np.asarray([0], np.int32), 0.125, "f32", lib=lib)
+    assert np.array_equal(out, np.zeros_like(out))
+
+
+def pin_dtype_decoding(lib):
+    """Exact fp16 / bf16 -> double decoding, checked on every 16-bit pattern
+    against the library conversions (L = 1 returns V unchanged)."""
+    import torch
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    for dt in ("f16", "bf16"):
+        D = 64
+        n = pats.size // D
+        vp = pats.reshape(n, 1, 1, D)
+        vp = np.concatenate([vp, np.zeros((n, 1, 15, D), np.uint16)], axis=2)
+        kp = np.zeros_like(vp)
+        if dt == "f16":
+            want = pats.view(np.float16).astype(np.float64)
+            v_arr, k_arr, q = vp.view(np.float16), kp.view(np.float16), np.zeros((n, 1, D), np.float16)
+        else:
+            want = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+            v_arr, k_arr, q = vp, kp, np.zeros((n, 1, D), np.uint16)
+        bt = np.arange(n, dtype=np.int32).reshape(n, 1)
+        out = oracle.decode(q, k_arr, v_arr, bt, np.ones(n, np.int32), 1.0, dt, lib=lib)
+        got = out.reshape(-1)
+        fin = np.isfinite(want)
+        assert np.array_equal(got[fin], want[fin]), dt
+        assert np.array_equal(np.isnan(got), np.isnan(want)), dt
+
+
+def pin_worked_block_table(lib):
+    """The pages' table [5, 2, 8, 1]: tokens 0-63 of one sequence sit where
+    the page says; checked through the oracle's gather (single-key reads)."""
+    g = golden("block_table_worked_example.json")
+    bs = g["block_size"]
+    table = g["block_table"]
+    for lo, hi, pb in g["logical_ranges"]:
+        for p in (lo, hi):
+            assert table[p // bs] == pb
+    for tok, slot in g["slots_derived_by_hand"].items():
+        assert alloc_model.slot_of(table, int(tok), bs) == slot
+    # Through the oracle: mark every (block, offset) of the pool with its own
+    # slot number in V; a query whose only visible key is logical token p
+    # (causal row of a 64-token chunk, first row sees token 0 ...) returns the
+    # slot number that the gather visited.
+    nb, D = 9, 64
+    vp = np.zeros((nb, 1, bs, D), np.float32)
+    for b in range(nb):
+        for o in range(bs):
+            vp[b, 0, o, :] = b * bs + o
+    kp = np.zeros_like(vp)
+    q = np.zeros((64, 1, D), np.float32)
+    bt = np.asarray([table], np.int32)
+    # scale 0 -> row t returns the mean of the slot numbers of tokens 0..t
+    out = oracle.decode(q, kp, vp, bt, np.asarray([64], np.int32), 0.0, "f32",
+                        query_start_loc=np.asarray([0, 64], np.int32), lib=lib)
+    means = out[:, 0, 0]
+    slots = [means[0]] + [(t + 1) * means[t] - t * means[t - 1] for t in range(1, 64)]
+    for tok, slot in g["slots_derived_by_hand"].items():
+        assert abs(slots[int(tok)] - slot) < 1e-9, tok
+
+
+def pin_block_counts(lib):
+    g = golden("block_count_worked_example.json")
+    bs, n = g["block_size"], g["tokens"]
+    assert alloc_model.blocks_needed(n, bs) == g["blocks"]
+    assert n - (g["blocks"] - 1) * bs == g["tokens_in_last_block"]
+    m = alloc_model.PoolModel(range(20), bs)
+    m.new_sequence("a", n)
+    assert len(m.tables["a"]) == g["blocks"]
+    g = golden("on_demand_growth.json")
+    m = alloc_model.PoolModel(g["free_order_head"] + list(range(10, 20)), g["block_size"])
+    m.new_sequence("a", 0)
+    for n in range(1, 65):
+        m.append("a")
+        if str(n) in g["table_after_tokens"]:
+            assert m.tables["a"] == g["table_after_tokens"][str(n)], n
+
+
+def pin_reshape_then_gather(lib):
+    """Writing every token of a sequence with reshape_and_cache (slots from the
+    worked table rule) and reading them back through the oracle's gather
+    reproduces NumPy attention over the contiguous K/V."""
+    rng = np.random.default_rng(19)
+    H, Hk, D, bs, L = 8, 2, 64, 16, 45
+    k = rng.standard_normal((L, Hk, D)).astype(np.float32)
+    v = rng.standard_normal((L, Hk, D)).astype(np.float32)
+    nb = 8
+    kp = rng.standard_normal((nb, Hk, bs, D)).astype(np.float32)
+    vp = rng.standard_normal((nb, Hk, bs, D)).astype(np.float32)
+    before_k, before_v = kp.copy(), vp.copy()
+    table = [6, 1, 3]
+    slots = np.asarray([alloc_model.slot_of(table, p, bs) for p in range(L)], np.int64)
+    slots_pad = np.concatenate([slots[:20], [-1], slots[20:]])       # a padding token
+    kk = np.concatenate([k[:20], np.full((1, Hk, D), 99, np.float32), k[20:]])
+    vv = np.concatenate([v[:20], np.full((1, Hk, D), 99, np.float32), v[20:]])
+    oracle.reshape_and_cache(kp, vp, kk, vv, slots_pad, "f32", lib=lib)
+    # untouched blocks and the tail of the last block keep their bytes
+    for b in range(nb):
+        if b not in table:
+            assert np.array_equal(kp[b], before_k[b]) and np.array_equal(vp[b], before_v[b])
+    assert np.array_equal(kp[3, :, L - 32:], before_k[3, :, L - 32:])
+    q = rng.standard_normal((3, H, D)).astype(np.float32)
+    bt = np.asarray([table], np.int32)
+    out = oracle.decode(q, kp, vp, bt, np.asarray([L], np.int32), 0.125, "f32",
+                        query_start_loc=np.asarray([0, 3], np.int32), lib=lib)
+    want = attention_contiguous(q.astype(np.float64), k, v, 0.125, H // Hk)
+    assert np.allclose(out, want, rtol=1e-12, atol=1e-12)
+
+
+def pin_copy_blocks(lib):
+    """Copy-on-write copies: dst gets src's bytes, every other block keeps its
+    own; with a chain (a->b, b->c) c receives b's bytes from before the call."""
+    rng = np.random.default_rng(20)
+    nb, Hk, bs, D = 10, 2, 16, 64
+    for dt in ("f32", "bf16"):
+        kp = _bits(rng.standard_normal((nb, Hk, bs, D)), dt)
+        vp = _bits(rng.standard_normal((nb, Hk, bs, D)), dt)
+        k0, v0 = kp.copy(), vp.copy()
+        pairs = [(1, 7), (4, 2), (7, 9)]          # 7 is read (for 9) and written (from 1)
+        oracle.copy_blocks(kp, vp, pairs, dt, lib=lib)
+        assert np.array_equal(kp[7], k0[1]) and np.array_equal(vp[7], v0[1])
+        assert np.array_equal(kp[2], k0[4]) and np.array_equal(vp[2], v0[4])
+        assert np.array_equal(kp[9], k0[7]) and np.array_equal(vp[9], v0[7])
+        for b in set(range(nb)) - {7, 2, 9}:
+            assert np.array_equal(kp[b], k0[b]) and np.array_equal(vp[b], v0[b])
+
+
+ALL_PINS = [
+    pin_brute_force, pin_decode_without_qsl, pin_identical_keys_mean, pin_single_key,
+    pin_dominant_logit, pin_v_linearity, pin_scale_zero_mean, pin_hand_example,
+    pin_gqa_equals_replicated_mha, pin_placement_invariance, pin_shared_equals_duplicated,
+    pin_causal_truncation, pin_empty_context, pin_dtype_decoding, pin_worked_block_table,
+    pin_block_counts, pin_reshape_then_gather, pin_copy_blocks,
+]
