@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark: one decode step of paged attention on the Llama-3-8B-shaped GQA batch.
+
+A step is the whole hot path over one batch: copy-on-write block copies (none
+in this batch), reshape_and_cache of the step's 256 new tokens, then paged
+decode attention of the 256 query tokens over their block-table KV cache
+(32 query heads / 8 KV heads, head_dim 128, block size 16, bf16, context
+lengths lognormal with median 800 capped at 4096, shuffled pool).
+
+Printed (rank 0, one JSON line): achieved HBM GB/s of the step (algorithmic
+bytes / device time), decode tokens/s, the dominant kernel's roofline, an
+end-to-end figure through the public API with host buffers, and the CPU oracle
+timed on a bounded sample as a baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torchrun: every rank runs its own batch (weak scaling,
+no collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+from paged_kv_cache_388_b200.batch import build_batch  # noqa: E402
+
+METRIC = "paged decode attention: achieved HBM GB/s (% of peak) and decode tokens/s"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def elem_bytes(dtype):
+    return {"f32": 4, "f16": 2, "bf16": 2}[dtype]
+
+
+def seq_bytes(wl, batch, seqs):
+    """Algorithmic bytes of the step restricted to sequences `seqs`: every
+    byte the method has to move, once (shared physical blocks once)."""
+    e = elem_bytes(wl.dtype)
+    H, Hk, D, bs = wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
+    seen = set()
+    kv_tokens = 0
+    nblk_total = 0
+    qrows = 0
+    for i in seqs:
+        L = int(batch.context_lens[i])
+        nblk = -(-L // bs)
+        nblk_total += nblk
+        for j in range(nblk):
+            pb = int(batch.block_tables[i, j])
+            if pb not in seen:
+                seen.add(pb)
+                kv_tokens += min(bs, L - j * bs)
+        qsl = batch.query_start_loc
+        qrows += 1 if qsl is None else int(qsl[i + 1] - qsl[i])
+    decode = kv_tokens * 2 * Hk * D * e + 2 * qrows * H * D * e + nblk_total * 4 + len(seqs) * 4
+    return decode, kv_tokens, qrows
+
+
+def step_bytes(wl, batch):
+    e = elem_bytes(wl.dtype)
+    Hk, D, bs = wl.num_kv_heads, wl.head_dim, wl.block_size
+    decode, kv_tokens, qrows = seq_bytes(wl, batch, range(batch.num_seqs))
+    t_new = wl.num_new_tokens
+    reshape = 2 * (2 * t_new * Hk * D * e) + t_new * 8
+    copy = int(batch.cow_pairs.shape[0]) * 2 * (2 * Hk * bs * D * e)
+    return {"decode": decode, "reshape": reshape, "copy_blocks": copy,
+            "step": decode + reshape + copy, "kv_tokens": kv_tokens, "q_rows": qrows}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.fh = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        self.fh = os.fdopen(fd, "w")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.fh.close()
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        try:
+            with open(self.path) as f:
+                lines = f.readlines()
+            os.unlink(self.path)
+        except OSError:
+            lines = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(self.NAMES, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle legs (cpu_baseline and --impl reference)
+# --------------------------------------------------------------------------
+def oracle_runner(wl, vals, batch):
+    """Returns run(n_seqs) -> (seconds, bytes, n_seqs): the oracle doing the
+    step for the first n_seqs sequences (their new tokens' writes into a copy
+    of the pool, then their decode rows over all heads)."""
+    import oracle
+    kp0 = workloads.to_numpy_raw(vals["k_pool"])
+    vp0 = workloads.to_numpy_raw(vals["v_pool"])
+    key = workloads.to_numpy_raw(vals["new_key"])
+    value = workloads.to_numpy_raw(vals["new_value"])
+    q = workloads.to_numpy_raw(vals["q"])
+    assert batch.query_start_loc is None and batch.cow_pairs.shape[0] == 0
+    e = elem_bytes(wl.dtype)
+
+    def run(n):
+        kp, vp = kp0.copy(), vp0.copy()
+        t0 = time.perf_counter()
+        oracle.reshape_and_cache(kp, vp, key[:n], value[:n], batch.slot_mapping[:n], wl.dtype)
+        oracle.decode(q, kp, vp, batch.block_tables, batch.context_lens, wl.scale, wl.dtype,
+                      rows=range(n))
+        dt = time.perf_counter() - t0
+        dec, _, _ = seq_bytes(wl, batch, range(n))
+        nbytes = dec + 2 * (2 * n * wl.num_kv_heads * wl.head_dim * e) + n * 8
+        return dt, nbytes, n
+
+    return run, oracle.max_threads()
+
+
+def size_sample(run, total, target_s):
+    """Pick the number of sequences whose oracle step takes about target_s."""
+    n = min(8, total)
+    dt, _, _ = run(n)
+    while dt < 0.2 * target_s and n < total:
+        n = min(total, n * 4)
+        dt, _, _ = run(n)
+    n = int(min(total, max(1, n * target_s / max(dt, 1e-6))))
+    return n
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle, as it stands, on the host cores."""
+    wl = workloads.make(args.config)
+    batch = build_batch(wl)
+    vals = workloads.values(wl)
+    run, cores = oracle_runner(wl, vals, batch)
+    n = size_sample(run, batch.num_seqs, target_s=4.0)
+    for _ in range(args.warmup):
+        run(n)
+    times, nbytes = [], 0
+    for _ in range(args.steps):
+        dt, nbytes, _ = run(n)
+        times.append(dt)
+    total = sum(times)
+    value = nbytes * args.steps / total / 1e9
+    sample = (f"first {n} of {batch.num_seqs} sequences per step (their reshape_and_cache writes "
+              f"and decode rows, all {wl.num_heads} heads)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------------
+# GPU leg
+# --------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+
+    from paged_kv_cache_388_b200 import _lib
+    from paged_kv_cache_388_b200.session import PagedKVCache
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    wl = workloads.make(args.config)
+    batch = build_batch(wl)
+    vals = workloads.values(wl)
+    nbytes = step_bytes(wl, batch)
+
+    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                         k_cache=vals["k_pool"].to(dev), v_cache=vals["v_pool"].to(dev))
+    q = vals["q"].to(dev)
+    key = vals["new_key"].to(dev)
+    value = vals["new_value"].to(dev)
+    slot = torch.from_numpy(batch.slot_mapping).to(dev)
+    bt = torch.from_numpy(batch.block_tables).to(dev)
+    cl = torch.from_numpy(batch.context_lens).to(dev)
+    qsl = None if batch.query_start_loc is None else torch.from_numpy(batch.query_start_loc).to(dev)
+    cow = torch.from_numpy(np.ascontiguousarray(batch.cow_pairs)).to(dev)
+    out = torch.empty_like(q)
+    mcl = batch.max_context_len
+    ws_bytes = _lib.pa_decode_workspace_size(batch.num_seqs, wl.num_heads, wl.num_kv_heads,
+                                             wl.head_dim, wl.block_size, mcl, 0)
+    cache.workspace(batch.num_seqs, wl.num_heads, mcl)
+    stream = torch.cuda.current_stream(dev)
+
+    K = args.steps
+    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(K + args.warmup)]
+          for k in ("d0", "d1", "r0", "r1")}
+
+    def step(i):
+        if cow.shape[0]:
+            cache.copy_blocks(cow)
+        ev["r0"][i].record(stream)
+        cache.write(key, value, slot)
+        ev["r1"][i].record(stream)
+        ev["d0"][i].record(stream)
+        cache.attend(q, bt, cl, wl.scale, out=out, query_start_loc=qsl,
+                     max_query_len=batch.max_query_len, max_context_len=mcl)
+        ev["d1"][i].record(stream)
+
+    for i in range(args.warmup):
+        step(K + i)
+    torch.cuda.synchronize(dev)
+    assert _lib.pa_get_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        t_start.record(stream)
+        for i in range(K):
+            step(i)
+        t_end.record(stream)
+        barrier()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = [ev["d0"][i].elapsed_time(ev["d1"][i]) for i in range(K)]
+    res_ms = [ev["r0"][i].elapsed_time(ev["r1"][i]) for i in range(K)]
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert _lib.pa_get_device_error() == 0
+    clk = clocks.summary()
+
+    # ---- end to end through the public API, host (pinned) buffers ----------
+    hq = vals["q"].pin_memory()
+    hkey = vals["new_key"].pin_memory()
+    hval = vals["new_value"].pin_memory()
+    hslot = torch.from_numpy(batch.slot_mapping).pin_memory()
+    hbt = torch.from_numpy(batch.block_tables).pin_memory()
+    hcl = torch.from_numpy(batch.context_lens).pin_memory()
+    hout = torch.empty_like(hq).pin_memory()
+    h2d = PagedKVCache.host_bytes(hq, hkey, hval, hslot, hbt, hcl)
+    d2h = PagedKVCache.host_bytes(hout)
+    e2e_ok = batch.query_start_loc is None and cow.shape[0] == 0
+    e2e = None
+    if e2e_ok:
+        for _ in range(args.warmup):
+            cache.step_from_host(hq, hkey, hval, hslot, hbt, hcl, hout, wl.scale, max_context_len=mcl)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            cache.step_from_host(hq, hkey, hval, hslot, hbt, hcl, hout, wl.scale, max_context_len=mcl)
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": nbytes["step"] * world * K / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / K}
+
+    # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1) -----------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and batch.query_start_loc is None:
+        run, cores = oracle_runner(wl, vals, batch)
+        n = size_sample(run, batch.num_seqs, target_s=12.0)
+        dt, ob, _ = run(n)
+        cpu = {"value": ob / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"first {n} of {batch.num_seqs} sequences (reshape_and_cache of their "
+                         f"new tokens + decode rows over all {wl.num_heads} heads), "
+                         f"one run of {dt:.1f} s"}
+
+    splits = ws_bytes > 0
+    launches_per_step = 1 + 1 + (1 if splits else 0) + (1 if cow.shape[0] else 0) + \
+        (1 if batch.max_query_len > 1 else 0)
+    peak, peak_kind = hbm_peak()
+    dec_avg = statistics.mean(dec_ms)
+    achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
+    value = nbytes["step"] * world * K / (ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic",
+        "config": {
+            "workload": wl.name,
+            "global_batch": batch.num_seqs * world,
+            "heads": f"{wl.num_heads}q/{wl.num_kv_heads}kv",
+            "head_dim": wl.head_dim,
+            "block_size": wl.block_size,
+            "kv_tokens": nbytes["kv_tokens"],
+            "step_bytes": nbytes["step"],
+            "l2": f"inputs larger than L2 ({nbytes['decode'] / 1e9:.2f} GB of KV per step vs "
+                  f"{L2_BYTES / 2**20:.0f} MiB L2); no flush",
+            "parallelism": f"dp{world} (independent batches)",
+        },
+        "decode_tokens_per_s": batch.num_seqs * world * K / (ms * 1e-3),
+        "pct_of_nominal_8TBps": 100.0 * value / NOMINAL_HBM_GBS,
+        "roofline": {
+            "kernel": "pa_decode (paged_decode_kernel + reduce_kernel)",
+            "bound": "hbm",
+            "achieved": achieved,
+            "peak": peak,
+            "peak_kind": f"{peak_kind} copy bandwidth",
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
+            "traffic": None,
+            "algorithmic_bytes": nbytes["decode"],
+            "avg_ms": dec_avg,
+        },
+        "kernels_ms": {"pa_decode": dec_avg, "pa_reshape_and_cache": statistics.mean(res_ms)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged KV-cache attention on NVIDIA B200 (sm_100a).
+ *
+ * The KV cache of every sequence is stored in fixed-size blocks (16 or 32
+ * tokens) that sit anywhere in one global pool; a per-sequence block table
+ * maps logical block i to a physical block id, and several sequences may point
+ * at the same physical block to share a prefix ("核心概念" (vLLM concepts
+ * page), sections 核心概念：块（Block）, 逻辑视图与物理视图分离 and 内存共享;
+ * "理解 vLLM PagedAttention", sections 三 and 六).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are caller-owned DEVICE pointers to contiguous
+ *    row-major arrays; the library never allocates, frees or keeps them.
+ *  - Element types: PA_F32 (float), PA_F16 (IEEE half), PA_BF16 (bfloat16).
+ *    q, out and both caches share one dtype; accumulation is fp32.
+ *  - Layouts (fixed by this library; the pages prescribe none):
+ *        k_cache, v_cache   [num_blocks][num_kv_heads][block_size][head_dim]
+ *        key, value         [num_tokens][num_kv_heads][head_dim]
+ *        q, out             [num_q_tokens][num_heads][head_dim]
+ *        block_tables       int32 [num_seqs][max_blocks_per_seq]
+ *    Every (block, kv-head) tile is one contiguous block_size*head_dim run.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and return once the work is enqueued.
+ *  - Supported: head_dim in {64, 128}; block_size in {16, 32};
+ *    num_heads % num_kv_heads == 0 with group = num_heads / num_kv_heads a
+ *    multiple of one of {4, 2, 1} and group / {4|2|1} <= 8.  Pointers to
+ *    caches, q, out, key and value must be 16-byte aligned.
+ *  - Errors: a negative pa_status is returned and NOTHING is launched when
+ *    an argument is invalid or unsupported (checked on the host).  Values
+ *    only the device sees (block ids, slots, context lengths) are checked by
+ *    the kernels: a bad item is skipped, its outputs are written as zeros and
+ *    a bit is OR-ed into a per-device error word (PA_DEVERR_*), which
+ *    pa_get_device_error() reads and clears.  Kernels never trap and every
+ *    wait inside them is bounded in time.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer, ... */
+  PA_ERR_UNSUPPORTED = -2, /* head_dim / block_size / group outside the list above */
+  PA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
+  PA_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Bits of the device error word. */
+#define PA_DEVERR_BLOCK_ID 0x1u    /* block id outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 0x2u        /* slot outside [0, num_blocks*block_size) */
+#define PA_DEVERR_CONTEXT_LEN 0x4u /* context_len < 0 or > max_blocks_per_seq*block_size */
+#define PA_DEVERR_QUERY_LEN 0x8u   /* query rows of a sequence exceed its context */
+#define PA_DEVERR_TIMEOUT 0x10u    /* a bounded wait inside a kernel expired */
+
+/*
+ * pa_reshape_and_cache -- write this step's new K/V into their cache slots.
+ *
+ * Defined by: each step computes only the current token's K and V and stores
+ * them for later steps ("核心概念", section 为什么需要 KV Cache); a token at
+ * position pos of a sequence with block table T goes to slot
+ * T[pos / block_size] * block_size + pos % block_size, i.e. block
+ * slot / block_size, offset slot % block_size (section 逻辑视图与物理视图分离).
+ *
+ *   key, value      [num_tokens][num_kv_heads][head_dim], dtype
+ *   k_cache,v_cache [num_blocks][num_kv_heads][block_size][head_dim], written
+ *   slot_mapping    int64 [num_tokens]; a negative slot skips the token
+ *                   (padding).  Two tokens must not share a slot.
+ * Byte-exact copy; no arithmetic on the values.
+ */
+int pa_reshape_and_cache(const void *key, const void *value, void *k_cache,
+                         void *v_cache, const int64_t *slot_mapping,
+                         int num_tokens, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, int dtype,
+                         struct CUstream_st *stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copy.
+ *
+ * Defined by: sequences share physical blocks until they diverge; the shared
+ * block is then copied so that each writer owns its block ("理解 vLLM
+ * PagedAttention", section 六; "PagedAttention 实战", section PagedAttention
+ * 的核心, item 3).
+ *
+ *   block_mapping  int64 [num_pairs][2] = {src, dst}; copies K and V of all
+ *                  KV heads of block src onto block dst.  A dst must not
+ *                  appear twice nor also be a src in the same call (the
+ *                  result would depend on ordering).
+ * Byte-exact copy.
+ */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping,
+                   int num_pairs, int num_kv_heads, int head_dim,
+                   int block_size, int num_blocks, int dtype,
+                   struct CUstream_st *stream);
+
+/*
+ * pa_decode_workspace_size -- bytes of device scratch pa_decode needs for
+ * split-KV partial results (0 when no sequence is split).  Arguments as for
+ * pa_decode; depends on the current device's SM count.
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                int head_dim, int block_size,
+                                int max_context_len, int kv_split_tokens);
+
+/*
+ * pa_decode -- attention of each sequence's query token(s) over its paged KV.
+ *
+ * Defined by: at each step the new token attends to all earlier tokens of its
+ * sequence, whose K/V are read from the cache ("核心概念", section 为什么需要
+ * KV Cache); decode reads the whole KV history and is bound by memory
+ * traffic ("PagedAttention 实战", section 先理解 KV Cache, Decode).  For query
+ * head h (KV head h / group), context length L and query rows t = 0..Q-1 of
+ * a sequence (Q = 1 for decode, Q > 1 for a chunked-prefill chunk, section
+ * Chunked Prefill), row t sees keys 0 .. L-Q+t and
+ *     out = softmax(scale * q . K^T) V        (fp32 accumulation).
+ * Long contexts are split across CTAs (split-KV) and merged by a second
+ * kernel, following the decode-scheduling idea of organising work by page,
+ * KV-head group and sequence split ("PagedAttention 实战", section 2026 年的
+ * 新变化).
+ *
+ *   out, q            [num_q_tokens][num_heads][head_dim]; out must not alias q
+ *   block_tables      int32 [num_seqs][max_blocks_per_seq]; only the first
+ *                     ceil(context_len / block_size) entries of a row are read
+ *   context_lens      int32 [num_seqs]: tokens in the cache for the sequence,
+ *                     this step's tokens included (they must already have been
+ *                     written with pa_reshape_and_cache)
+ *   query_start_loc   int32 [num_seqs + 1] prefix offsets of each sequence's
+ *                     query rows in q, or NULL for one row per sequence
+ *                     (num_q_tokens == num_seqs)
+ *   max_query_len     host-side upper bound of the rows of any sequence (1 for
+ *                     pure decode); rows of sequences with Q > 1 go to the
+ *                     chunked-query kernel
+ *   scale             softmax scale (typically 1/sqrt(head_dim))
+ *   max_context_len   host-side upper bound of context_lens (0: use
+ *                     max_blocks_per_seq * block_size)
+ *   kv_split_tokens   0: library policy; > 0: split every sequence's KV into
+ *                     pieces of this many tokens (rounded down to blocks)
+ *   workspace         device scratch of >= pa_decode_workspace_size(...) bytes
+ *                     (may be NULL when that size is 0); contents need no
+ *                     initialisation and are not meaningful after the call.
+ * Context length 0 gives zero output.
+ */
+int pa_decode(void *out, const void *q, const void *k_cache,
+              const void *v_cache, const int32_t *block_tables,
+              int max_blocks_per_seq, const int32_t *context_lens,
+              const int32_t *query_start_loc, int num_seqs, int num_q_tokens,
+              int max_query_len, int num_heads, int num_kv_heads, int head_dim,
+              int block_size, int num_blocks, float scale, int max_context_len,
+              int kv_split_tokens, int dtype, void *workspace,
+              size_t workspace_bytes, struct CUstream_st *stream);
+
+/*
+ * pa_get_device_error -- synchronise `stream`, then read and clear the
+ * current device's error word (PA_DEVERR_* bits, 0 = none) into *code_out.
+ */
+int pa_get_device_error(unsigned int *code_out, struct CUstream_st *stream);
+
+/* Human-readable name of a pa_status value (static string). */
+const char *pa_status_string(int status);
+
+/* ABI version of this header: (major << 16) | minor. */
+int pa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

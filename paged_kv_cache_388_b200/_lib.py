@@ -1,0 +1,163 @@
+"""Thin ctypes binding of libpa.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+computation of its own: it reads shapes off the tensors, checks that they are
+contiguous CUDA tensors of the right dtype, and passes raw device pointers and
+the current CUDA stream to the library.  There is no fallback: if the CUDA
+library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_388_b200.build` "
+        "(nvcc, sm_100a).  There is no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+F = ctypes.c_float
+SZ = ctypes.c_size_t
+
+_lib.pa_reshape_and_cache.restype = I
+_lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
+_lib.pa_copy_blocks.restype = I
+_lib.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P]
+_lib.pa_decode_workspace_size.restype = SZ
+_lib.pa_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
+_lib.pa_decode.restype = I
+_lib.pa_decode.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, I, I, P, SZ, P]
+_lib.pa_get_device_error.restype = I
+_lib.pa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
+_lib.pa_status_string.restype = ctypes.c_char_p
+_lib.pa_status_string.argtypes = [I]
+_lib.pa_abi_version.restype = I
+_lib.pa_abi_version.argtypes = []
+
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+
+PA_DEVERR_BLOCK_ID = 0x1
+PA_DEVERR_SLOT = 0x2
+PA_DEVERR_CONTEXT_LEN = 0x4
+PA_DEVERR_QUERY_LEN = 0x8
+PA_DEVERR_TIMEOUT = 0x10
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.pa_status_string(status).decode()} ({status})")
+
+
+def library():
+    """The loaded ctypes library (for tests that call entry points directly)."""
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, name, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise PAError(rc, what)
+
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
+    """key/value [T, Hk, D]; caches [NB, Hk, bs, D]; slot_mapping int64 [T]."""
+    _dev(key, "key")
+    _dev(value, "value", key.dtype)
+    _dev(k_cache, "k_cache", key.dtype)
+    _dev(v_cache, "v_cache", key.dtype)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    nb, hk, bs, d = k_cache.shape
+    rc = _lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(slot_mapping), key.shape[0], hk, d, bs, nb,
+                                   _DT[key.dtype], _stream(stream))
+    _check(rc, "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
+    """block_mapping int64 [P, 2] of (src, dst) physical block ids."""
+    _dev(k_cache, "k_cache")
+    _dev(v_cache, "v_cache", k_cache.dtype)
+    _dev(block_mapping, "block_mapping", torch.int64)
+    nb, hk, bs, d = k_cache.shape
+    rc = _lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping),
+                             block_mapping.shape[0], hk, d, bs, nb, _DT[k_cache.dtype],
+                             _stream(stream))
+    _check(rc, "pa_copy_blocks")
+
+
+def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                             max_context_len, kv_split_tokens=0) -> int:
+    return int(_lib.pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                             block_size, max_context_len, kv_split_tokens))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+              query_start_loc=None, max_query_len=1, max_context_len=0, kv_split_tokens=0,
+              workspace=None, stream=None):
+    """out/q [Tq, H, D]; caches [NB, Hk, bs, D]; block_tables int32 [S, mbps];
+    context_lens int32 [S]; query_start_loc int32 [S+1] or None; workspace: a
+    uint8 CUDA tensor of >= pa_decode_workspace_size(...) bytes (or None when
+    that size is 0)."""
+    _dev(q, "q")
+    _dev(out, "out", q.dtype)
+    _dev(k_cache, "k_cache", q.dtype)
+    _dev(v_cache, "v_cache", q.dtype)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    if query_start_loc is not None:
+        _dev(query_start_loc, "query_start_loc", torch.int32)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+    tq, h, d = q.shape
+    nb, hk, bs, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    s, mbps = block_tables.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                        mbps, _ptr(context_lens), _ptr(query_start_loc), s, tq,
+                        int(max_query_len), h, hk, d, bs, nb, float(scale), int(max_context_len),
+                        int(kv_split_tokens), _DT[q.dtype], _ptr(workspace), ws_bytes,
+                        _stream(stream))
+    _check(rc, "pa_decode")
+
+
+def pa_get_device_error(stream=None) -> int:
+    """Synchronise the stream, return and clear the device error word."""
+    code = ctypes.c_uint(0)
+    rc = _lib.pa_get_device_error(ctypes.byref(code), _stream(stream))
+    _check(rc, "pa_get_device_error")
+    return int(code.value)
+
+
+def pa_abi_version() -> int:
+    return int(_lib.pa_abi_version())

@@ -1,0 +1,688 @@
+// decode.cu -- paged decode attention (one query token per sequence) for B200.
+//
+// Work decomposition
+//   A work item is (sequence, KV head, split): the GROUP query heads that read
+//   one KV head share every K/V byte loaded for that item (GQA), and long
+//   contexts are cut into splits of `split_blocks` KV blocks so that the 148
+//   SMs stay busy and the tail is short (sequence split / KV-head group /
+//   work queue, "PagedAttention 实战", section 2026 年的新变化).  The kernel is
+//   persistent: each CTA scans context_lens once, builds the prefix sum of
+//   per-sequence split counts in shared memory and then walks items
+//   blockIdx.x, blockIdx.x + gridDim.x, ... (dense enumeration, so CTAs get
+//   item counts within one of each other).
+//
+// Data movement (the whole cost of decode: "PagedAttention 实战", section
+// 先理解 KV Cache, Decode is memory-bound)
+//   One producer warp walks the block table of each item and, for every KV
+//   block, issues two bulk asynchronous copies (TMA, non-tensor form) of the
+//   contiguous (block, kv-head) K and V tiles -- block_size*head_dim elements
+//   each -- into a ring of shared-memory stages guarded by full/empty
+//   mbarriers.  The block table is read 32 entries at a time with one
+//   coalesced load.
+//
+// Math (fp32 on the CUDA cores; decode is not a dense contraction)
+//   Consumer warps take whole KV blocks round-robin; warps that share a block
+//   (group > 4) split the query heads between them.  Within a warp a lane
+//   owns one 16-byte slice of a K/V row: q.K partial dot products are formed
+//   with packed fp32x2 FMAs, combined with a butterfly reduce-scatter across
+//   the lanes of a row, and fed to an online softmax in base 2 (scale*log2 e
+//   folded into q).  P.V accumulates into per-lane fp32 registers.  At the end
+//   of an item the warps' (m, l, acc) states are merged through shared memory
+//   and either written to `out` (single split) or to the split workspace,
+//   which reduce_kernel combines.
+#include <float.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kMaxSeqsPerLaunch = 2048;
+constexpr int kRingBytes = 64 * 1024;
+constexpr int kMaxConsumerWarps = 8;
+
+template <typename T, int D, int BS, int GW>
+struct DecodeCfg {
+  static constexpr int kElem = sizeof(T);
+  static constexpr int ELEMS = 16 / kElem;      // elements per 16-byte vector
+  static constexpr int PAIRS = ELEMS / 2;
+  static constexpr int LPR = D / ELEMS;         // lanes per K/V row
+  static constexpr int RPP = 32 / LPR;          // rows per pass (row groups per warp)
+  static constexpr int CHUNK = 16;              // rows per softmax step
+  static constexpr int PASSES = CHUNK / RPP;
+  static constexpr int NV = PASSES * GW;        // partial scores per lane per chunk
+  static constexpr int VPL = NV >= LPR ? NV / LPR : 1;  // reduced scores kept per lane
+  static constexpr int DUP = NV >= LPR ? 1 : LPR / NV;  // lanes holding the same score
+  static constexpr int LPH = LPR / GW;          // lanes of one head in a row group
+  static constexpr int TILE = BS * D * kElem;   // bytes of one (block, kv-head) tile
+  static constexpr int STAGE = 2 * TILE;        // K tile + V tile
+  static constexpr int STAGES = kRingBytes / STAGE < 2 ? 2 : kRingBytes / STAGE;
+  static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row must map onto whole lanes");
+  static_assert(PASSES >= 1 && CHUNK % RPP == 0, "chunk must hold whole passes");
+  static_assert(GW <= LPR, "a lane's reduced scores must belong to one head");
+  static_assert(BS % CHUNK == 0, "block size must be a multiple of 16");
+};
+
+// Shared-memory layout (dynamic).  Offsets are 128-byte aligned.
+template <typename C>
+struct Smem {
+  static constexpr int kRing = 0;
+  static constexpr int kFull = kRing + C::STAGES * C::STAGE;           // uint64 [STAGES]
+  static constexpr int kEmpty = kFull + 8 * C::STAGES;                 // uint64 [STAGES]
+  static constexpr int kBad = kEmpty + 8 * C::STAGES;                  // int [STAGES]
+  static constexpr int kMisc = (kBad + 4 * C::STAGES + 127) / 128 * 128;  // int [4]
+  static constexpr int kPrefix = kMisc + 128;                          // int [kMaxSeqs+1]
+  static constexpr int kScan = kPrefix + 4 * (kMaxSeqsPerLaunch + 8);  // int [32]
+  static constexpr int kP = (kScan + 128 + 127) / 128 * 128;           // float [NCW][16][GW]
+  static constexpr int kMerge = kP + kMaxConsumerWarps * 16 * 4 * 4;   // float [NCW][GW][D+4]
+  static constexpr int kBytes = kMerge + kMaxConsumerWarps * 4 * (128 + 4) * 4;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Work items contributed by sequence s: its splits for a decode sequence
+// (one query row); for a chunk of Q > 1 rows, Q single-row items in row mode
+// and none otherwise (the chunk kernel takes them).
+__device__ __forceinline__ bool seq_len_ok(const AttnArgs &a, int L) {
+  return L >= 0 && L <= a.max_context_len;
+}
+
+// Query rows [q0, q0 + qlen) of sequence gs; false if they do not fit in q.
+__device__ __forceinline__ bool seq_rows(const AttnArgs &a, int gs, int *q0, int *qlen) {
+  if (!a.query_start_loc) {
+    *q0 = gs;
+    *qlen = 1;
+    return true;
+  }
+  *q0 = a.query_start_loc[gs];
+  *qlen = a.query_start_loc[gs + 1] - *q0;
+  return *q0 >= 0 && *qlen >= 0 && *q0 + *qlen <= a.num_q_tokens;
+}
+
+__device__ __forceinline__ int seq_items(const AttnArgs &a, int s) {
+  const int gs = a.seq_begin + s;
+  int q0, qlen;
+  if (!seq_rows(a, gs, &q0, &qlen)) {
+    raise_error(a.err, PA_DEVERR_QUERY_LEN);
+    return 0;
+  }
+  if (qlen <= 0) return 0;
+  if (qlen > 1) return a.rows_mode ? qlen : 0;
+  const int L = a.context_lens[gs];
+  if (L <= 0 || !seq_len_ok(a, L)) return 1;  // zero-output item
+  return ceil_div(ceil_div(L, a.block_size), a.split_blocks);
+}
+
+struct Item {
+  int seq;     // global sequence index
+  int qrow;    // query row (token index into q / out)
+  int split;
+  int nsplit;
+  int kvh;
+  int b0, b1;  // KV blocks [b0, b1) of the sequence
+  int L;       // keys visible to the row (valid only if ok)
+  unsigned int bad_bits;  // PA_DEVERR_* of an invalid sequence (0: ok)
+};
+
+__device__ __forceinline__ Item decode_item(const AttnArgs &a, const int *prefix, int n, int w) {
+  Item it;
+  const int f = w / a.num_kv_heads;
+  it.kvh = w - f * a.num_kv_heads;
+  int lo = 0, hi = n;  // find s with prefix[s] <= f < prefix[s+1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= f) lo = mid; else hi = mid;
+  }
+  it.seq = a.seq_begin + lo;
+  const int L = a.context_lens[it.seq];
+  int q0, qlen;
+  seq_rows(a, it.seq, &q0, &qlen);  // valid: sequences with bad rows contribute no items
+  it.bad_bits = 0;
+  if (!seq_len_ok(a, L)) it.bad_bits = PA_DEVERR_CONTEXT_LEN;
+  else if (qlen > L && L > 0) it.bad_bits = PA_DEVERR_QUERY_LEN;
+  if (qlen > 1) {  // row mode: one item per query row, never split
+    const int t = f - prefix[lo];
+    it.qrow = q0 + t;
+    it.split = 0;
+    it.nsplit = 1;
+    it.L = L - qlen + t + 1;
+  } else {
+    it.qrow = q0;
+    it.split = f - prefix[lo];
+    it.nsplit = prefix[lo + 1] - prefix[lo];
+    it.L = L;
+  }
+  if (it.bad_bits || it.L <= 0) {
+    it.b0 = it.b1 = 0;
+  } else {
+    const int nblk = ceil_div(it.L, a.block_size);
+    it.b0 = qlen > 1 ? 0 : it.split * a.split_blocks;
+    it.b1 = qlen > 1 ? nblk : min(nblk, it.b0 + a.split_blocks);
+  }
+  return it;
+}
+
+template <int NV, int LPR>
+__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
+  int cnt = NV;
+#pragma unroll
+  for (int m = LPR / 2; m >= 1; m >>= 1) {
+    if (cnt > 1) {
+      const int half = cnt / 2;
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < NV / 2; ++i) {
+        if (i < half) {
+          const float send = up ? v[i] : v[i + half];
+          const float keep = up ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      cnt = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+    }
+  }
+}
+
+template <typename T, int D, int BS, int GW>
+__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
+    paged_decode_kernel(const AttnArgs a, int ncw, int hsplit) {
+  using C = DecodeCfg<T, D, BS, GW>;
+  using S = Smem<C>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::kFull);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + S::kEmpty);
+  int *bad = reinterpret_cast<int *>(smem + S::kBad);
+  volatile int *abort_flag = reinterpret_cast<int *>(smem + S::kMisc);
+  int *prefix = reinterpret_cast<int *>(smem + S::kPrefix);
+  int *scan = reinterpret_cast<int *>(smem + S::kScan);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int nthreads = blockDim.x;
+  const int n = a.num_seqs;
+
+  // ---- prologue: barriers + prefix sum of items per sequence ---------------
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], hsplit);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  {
+    const int per = ceil_div(n, nthreads);
+    const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; ++s) local += seq_items(a, s);
+    // block exclusive scan of `local`
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) scan[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = nthreads >> 5;
+      int w = lane < nw ? scan[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < nw) scan[lane] = w;  // inclusive warp totals
+    }
+    __syncthreads();
+    int run = (warp ? scan[warp - 1] : 0) + x - local;
+    for (int s = s0; s < s1; ++s) {
+      prefix[s] = run;
+      run += seq_items(a, s);
+    }
+    if (tid == nthreads - 1) prefix[n] = run;
+  }
+  __syncthreads();
+  const int total_items = prefix[n] * a.num_kv_heads;
+
+  unsigned char *ring = smem + S::kRing;
+
+  if (warp == ncw) {
+    // ======================= producer warp ===================================
+    uint32_t it = 0;
+    for (int w = blockIdx.x; w < total_items; w += gridDim.x) {
+      const Item item = decode_item(a, prefix, n, w);
+      const int32_t *table = a.block_tables + (int64_t)item.seq * a.max_blocks_per_seq;
+      for (int b = item.b0; b < item.b1; b += 32) {
+        const int cnt = min(32, item.b1 - b);
+        const int my_id = lane < cnt ? table[b + lane] : 0;
+        for (int k = 0; k < cnt; ++k) {
+          const int pb = __shfl_sync(0xffffffffu, my_id, k);
+          const uint32_t slot = it % C::STAGES;
+          const uint32_t par = ((it / C::STAGES) & 1u) ^ 1u;
+          ++it;
+          bool ok = !*abort_flag;
+          if (ok) ok = mbar_wait(&empty[slot], par);
+          if (lane == 0) {
+            if (!ok) {
+              if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+              *abort_flag = 1;
+              bad[slot] = 1;
+              mbar_arrive(&full[slot]);
+            } else if (pb < 0 || pb >= a.num_blocks) {
+              raise_error(a.err, PA_DEVERR_BLOCK_ID);
+              bad[slot] = 1;
+              mbar_arrive(&full[slot]);
+            } else {
+              bad[slot] = 0;
+              const int64_t tile = ((int64_t)pb * a.num_kv_heads + item.kvh) * (BS * D);
+              unsigned char *dst = ring + slot * C::STAGE;
+              fence_proxy_async_smem();
+              mbar_arrive_expect_tx(&full[slot], C::STAGE);
+              bulk_load(dst, static_cast<const T *>(a.k_cache) + tile, C::TILE, &full[slot]);
+              bulk_load(dst + C::TILE, static_cast<const T *>(a.v_cache) + tile, C::TILE,
+                        &full[slot]);
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+    return;
+  }
+
+  // ======================= consumer warps ==================================
+  const int hs = warp % hsplit;   // which GW-head subset of the group
+  const int bl = warp / hsplit;   // block lane: blocks bl, bl+nbl, ...
+  const int nbl = ncw / hsplit;
+  const int rg = lane / C::LPR;   // row group
+  const int li = lane % C::LPR;   // lane within row
+  // reduced-score ownership of this lane (see reduce_scatter)
+  const int v0 = C::NV >= C::LPR ? li * C::VPL : li / C::DUP;
+  const int my_head = v0 / C::PASSES;
+  const bool owner = (li % C::DUP) == 0;
+
+  float *p_s = reinterpret_cast<float *>(smem + S::kP) + warp * 16 * GW;
+  float *merge = reinterpret_cast<float *>(smem + S::kMerge);
+  const int mstride = GW * (D + 4);  // floats per warp in the merge area
+
+  uint32_t it_base = 0;
+  for (int w = blockIdx.x; w < total_items; w += gridDim.x) {
+    const Item item = decode_item(a, prefix, n, w);
+    const int nblocks = item.b1 - item.b0;
+    const int qrow = item.qrow;
+    const int head0 = item.kvh * a.group + hs * GW;
+
+    // q slice of this lane, pre-scaled by scale*log2(e)
+    float2 q2[GW][C::PAIRS];
+#pragma unroll
+    for (int h = 0; h < GW; ++h) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(
+          static_cast<const T *>(a.q) + ((int64_t)qrow * a.num_heads + head0 + h) * D +
+          li * C::ELEMS);
+      Elem<T>::to_f2(raw, q2[h]);
+#pragma unroll
+      for (int e = 0; e < C::PAIRS; ++e) {
+        q2[h][e].x *= a.scale_log2;
+        q2[h][e].y *= a.scale_log2;
+      }
+    }
+
+    float m[GW];
+    float2 acc[GW][C::PAIRS];
+#pragma unroll
+    for (int h = 0; h < GW; ++h) {
+      m[h] = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < C::PAIRS; ++e) acc[h][e] = make_float2(0.f, 0.f);
+    }
+    float l_lane = 0.f;
+    bool item_bad = item.bad_bits != 0;
+    if (item.bad_bits && tid == 0 && item.kvh == 0) raise_error(a.err, item.bad_bits);
+
+    for (int j = bl; j < nblocks; j += nbl) {
+      const uint32_t itn = it_base + j;
+      const uint32_t slot = itn % C::STAGES;
+      const uint32_t par = (itn / C::STAGES) & 1u;
+      bool ok = !*abort_flag;
+      if (ok) {
+        ok = mbar_wait(&full[slot], par);
+        if (!ok && lane == 0) {
+          if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+      }
+      if (ok && bad[slot]) ok = false;
+      if (!ok) {
+        item_bad = true;
+      } else {
+        const int b = item.b0 + j;
+        const int nvalid = min(BS, item.L - b * BS);
+        const unsigned char *ks = ring + slot * C::STAGE;
+        const unsigned char *vs = ks + C::TILE;
+#pragma unroll
+        for (int r0 = 0; r0 < BS; r0 += C::CHUNK) {
+          if (r0 < nvalid) {
+            // ---- scores: partial dot products over this lane's slice ----
+            float sc[C::NV];
+#pragma unroll
+            for (int p = 0; p < C::PASSES; ++p) {
+              const int row = r0 + p * C::RPP + rg;
+              const uint4 raw =
+                  *reinterpret_cast<const uint4 *>(ks + (row * D + li * C::ELEMS) * C::kElem);
+              float2 k2[C::PAIRS];
+              Elem<T>::to_f2(raw, k2);
+#pragma unroll
+              for (int h = 0; h < GW; ++h) {
+                float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int e = 0; e < C::PAIRS; ++e) d2 = ffma2(q2[h][e], k2[e], d2);
+                sc[h * C::PASSES + p] = d2.x + d2.y;
+              }
+            }
+            reduce_scatter<C::NV, C::LPR>(sc, lane);
+
+            // ---- online softmax (base 2) ----
+            float cmax = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < C::VPL; ++i) {
+              const int v = v0 + i;
+              const int row = r0 + (v % C::PASSES) * C::RPP + rg;
+              if (row >= nvalid) sc[i] = -INFINITY;
+              cmax = fmaxf(cmax, sc[i]);
+            }
+#pragma unroll
+            for (int o = 1; o < C::LPH; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+#pragma unroll
+            for (int o = C::LPR; o < 32; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+            float alpha[GW];
+            float m_mine = 0.f;
+#pragma unroll
+            for (int h = 0; h < GW; ++h) {
+              const float cm = __shfl_sync(0xffffffffu, cmax, h * C::LPH);
+              const float mn = fmaxf(m[h], cm);
+              alpha[h] = fast_exp2(m[h] - mn);
+              m[h] = mn;
+              if (h == my_head) m_mine = mn;
+            }
+            float psum = 0.f;
+#pragma unroll
+            for (int i = 0; i < C::VPL; ++i) {
+              const float pv = fast_exp2(sc[i] - m_mine);
+              psum += pv;
+              const int v = v0 + i;
+              const int crow = (v % C::PASSES) * C::RPP + rg;  // row within chunk
+              if (owner) p_s[crow * GW + my_head] = pv;
+            }
+            float a_mine = 1.f;
+#pragma unroll
+            for (int h = 0; h < GW; ++h)
+              if (h == my_head) a_mine = alpha[h];
+            l_lane = l_lane * a_mine + (owner ? psum : 0.f);
+            __syncwarp();
+
+            // ---- rescale and accumulate P.V ----
+#pragma unroll
+            for (int h = 0; h < GW; ++h) {
+              const float2 a2 = make_float2(alpha[h], alpha[h]);
+#pragma unroll
+              for (int e = 0; e < C::PAIRS; ++e) acc[h][e] = __fmul2_rn(acc[h][e], a2);
+            }
+#pragma unroll
+            for (int p = 0; p < C::PASSES; ++p) {
+              const int crow = p * C::RPP + rg;
+              const int row = r0 + crow;
+              const uint4 raw =
+                  *reinterpret_cast<const uint4 *>(vs + (row * D + li * C::ELEMS) * C::kElem);
+              float2 v2[C::PAIRS];
+              Elem<T>::to_f2(raw, v2);
+              if (row >= nvalid) {
+#pragma unroll
+                for (int e = 0; e < C::PAIRS; ++e) v2[e] = make_float2(0.f, 0.f);
+              }
+              float pr[GW];
+              if constexpr (GW == 4) {
+                const float4 t = *reinterpret_cast<const float4 *>(p_s + crow * 4);
+                pr[0] = t.x; pr[1] = t.y; pr[2] = t.z; pr[3] = t.w;
+              } else if constexpr (GW == 2) {
+                const float2 t = *reinterpret_cast<const float2 *>(p_s + crow * 2);
+                pr[0] = t.x; pr[1] = t.y;
+              } else {
+                pr[0] = p_s[crow];
+              }
+#pragma unroll
+              for (int h = 0; h < GW; ++h) {
+                const float2 pp = make_float2(pr[h], pr[h]);
+#pragma unroll
+                for (int e = 0; e < C::PAIRS; ++e) acc[h][e] = ffma2(pp, v2[e], acc[h][e]);
+              }
+            }
+            __syncwarp();
+          }
+        }
+      }
+      // release the stage
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    it_base += nblocks;
+
+    // ---- per-warp totals: sum acc over row groups, l over the head's lanes ----
+#pragma unroll
+    for (int o = C::LPR; o < 32; o <<= 1) {
+#pragma unroll
+      for (int h = 0; h < GW; ++h)
+#pragma unroll
+        for (int e = 0; e < C::PAIRS; ++e) {
+          acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
+          acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
+        }
+    }
+#pragma unroll
+    for (int o = 1; o < C::LPH; o <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
+#pragma unroll
+    for (int o = C::LPR; o < 32; o <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, o);
+
+    float *mw = merge + warp * mstride;
+    if (rg == 0) {
+#pragma unroll
+      for (int h = 0; h < GW; ++h) {
+        float *dst = mw + h * (D + 4) + li * C::ELEMS;
+#pragma unroll
+        for (int e = 0; e < C::PAIRS; ++e) {
+          dst[2 * e] = acc[h][e].x;
+          dst[2 * e + 1] = acc[h][e].y;
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < GW; ++h) {
+      const float lh = __shfl_sync(0xffffffffu, l_lane, h * C::LPH);
+      if (lane == 0) {
+        mw[h * (D + 4) + D] = m[h];
+        mw[h * (D + 4) + D + 1] = lh;
+        mw[h * (D + 4) + D + 2] = item_bad ? 1.f : 0.f;
+      }
+    }
+    named_sync(1, ncw * 32);
+
+    // ---- merge the warps that worked on the same heads; write out ----------
+    {
+      const int D4 = D / 4;
+      const int total4 = a.group * D4;
+      const bool direct = item.nsplit == 1;
+      for (int idx = tid; idx < total4; idx += ncw * 32) {
+        const int hg = idx / D4;           // head within the group
+        const int d4 = idx - hg * D4;
+        const int hsub = hg / GW, h = hg - hsub * GW;
+        float M = -INFINITY;
+        bool anybad = false;
+        for (int b2 = 0; b2 < nbl; ++b2) {
+          const float *src = merge + (b2 * hsplit + hsub) * mstride + h * (D + 4);
+          M = fmaxf(M, src[D]);
+          anybad |= src[D + 2] != 0.f;
+        }
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum = 0.f;
+        for (int b2 = 0; b2 < nbl; ++b2) {
+          const float *src = merge + (b2 * hsplit + hsub) * mstride + h * (D + 4);
+          const float mb = src[D];
+          const float wgt = mb == -INFINITY ? 0.f : fast_exp2(mb - M);
+          Lsum += wgt * src[D + 1];
+          const float4 x = *reinterpret_cast<const float4 *>(src + d4 * 4);
+          o.x += wgt * x.x;
+          o.y += wgt * x.y;
+          o.z += wgt * x.z;
+          o.w += wgt * x.w;
+        }
+        const int head = item.kvh * a.group + hg;
+        if (direct) {
+          float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
+          T *dst = static_cast<T *>(a.out) + ((int64_t)qrow * a.num_heads + head) * D + d4 * 4;
+          dst[0] = Elem<T>::from_f(o.x * inv);
+          dst[1] = Elem<T>::from_f(o.y * inv);
+          dst[2] = Elem<T>::from_f(o.z * inv);
+          dst[3] = Elem<T>::from_f(o.w * inv);
+        } else {
+          const int64_t pidx = ((int64_t)item.seq * a.num_heads + head) * a.max_splits + item.split;
+          *reinterpret_cast<float4 *>(a.part_o + pidx * D + d4 * 4) = o;
+          if (d4 == 0) {
+            a.part_ml[2 * pidx] = M;
+            a.part_ml[2 * pidx + 1] = anybad ? __int_as_float(0x7fc00000) : Lsum;
+          }
+        }
+      }
+    }
+    named_sync(1, ncw * 32);
+  }
+}
+
+// Combine split partials: one warp per (sequence, head).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) reduce_kernel(const AttnArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= a.num_seqs * a.num_heads) return;
+  const int s = gw / a.num_heads;
+  const int head = gw - s * a.num_heads;
+  const int gs = a.seq_begin + s;
+  int qrow, qlen;
+  if (!seq_rows(a, gs, &qrow, &qlen) || qlen != 1) return;
+  const int L = a.context_lens[gs];
+  if (L <= 0 || !seq_len_ok(a, L)) return;  // written by the main kernel
+  const int nsplit = ceil_div(ceil_div(L, a.block_size), a.split_blocks);
+  if (nsplit <= 1 || nsplit > a.max_splits) return;
+  const int64_t base = ((int64_t)gs * a.num_heads + head) * a.max_splits;
+
+  float M = -INFINITY;
+  bool poisoned = false;
+  for (int sp = lane; sp < nsplit; sp += 32) {
+    M = fmaxf(M, a.part_ml[2 * (base + sp)]);
+    poisoned |= isnan(a.part_ml[2 * (base + sp) + 1]);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  poisoned = __any_sync(0xffffffffu, poisoned);
+
+  constexpr int PER = D / 32;  // elements per lane
+  float o[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) o[e] = 0.f;
+  float Lsum = 0.f;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const float ms = a.part_ml[2 * (base + sp)];
+    const float wgt = ms == -INFINITY ? 0.f : fast_exp2(ms - M);
+    Lsum += wgt * a.part_ml[2 * (base + sp) + 1];
+    const float *src = a.part_o + (base + sp) * D + lane * PER;
+    if constexpr (PER == 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(src);
+      o[0] += wgt * x.x; o[1] += wgt * x.y; o[2] += wgt * x.z; o[3] += wgt * x.w;
+    } else {
+      const float2 x = *reinterpret_cast<const float2 *>(src);
+      o[0] += wgt * x.x; o[1] += wgt * x.y;
+    }
+  }
+  const float inv = (Lsum > 0.f && !poisoned) ? 1.f / Lsum : 0.f;
+  T *dst = static_cast<T *>(a.out) + ((int64_t)qrow * a.num_heads + head) * D + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) dst[e] = Elem<T>::from_f(o[e] * inv);
+}
+
+template <typename T, int D, int BS, int GW>
+cudaError_t launch_decode_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
+  using C = DecodeCfg<T, D, BS, GW>;
+  using S = Smem<C>;
+  auto kern = paged_decode_kernel<T, D, BS, GW>;
+  static int occ = -1;  // resident CTAs per SM (per instantiation; same on every B200)
+  if (occ < 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::kBytes);
+    if (e != cudaSuccess) return e;
+    int o = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, 32 * (kMaxConsumerWarps + 1),
+                                                      S::kBytes);
+    if (e != cudaSuccess) return e;
+    occ = o > 0 ? o : 1;
+  }
+  const int hsplit = a.group / GW;
+  const int nbl = hsplit >= 4 ? 1 : 4 / hsplit;
+  const int ncw = hsplit * nbl;
+  // upper bound of items in this launch
+  const int64_t max_items = (int64_t)a.num_seqs * a.num_kv_heads * a.max_splits;
+  int64_t grid = (int64_t)sm_count * occ;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, 32 * (ncw + 1), S::kBytes, stream>>>(a, ncw, hsplit);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int BS>
+cudaError_t dispatch_gw(const AttnArgs &a, int sm_count, cudaStream_t s) {
+  if (a.group % 4 == 0) return launch_decode_t<T, D, BS, 4>(a, sm_count, s);
+  if (a.group % 2 == 0) return launch_decode_t<T, D, BS, 2>(a, sm_count, s);
+  return launch_decode_t<T, D, BS, 1>(a, sm_count, s);
+}
+
+template <typename T, int D>
+cudaError_t dispatch_bs(const AttnArgs &a, int sm_count, cudaStream_t s) {
+  return a.block_size == 16 ? dispatch_gw<T, D, 16>(a, sm_count, s)
+                            : dispatch_gw<T, D, 32>(a, sm_count, s);
+}
+
+template <typename T>
+cudaError_t dispatch_d(const AttnArgs &a, int sm_count, cudaStream_t s) {
+  return a.head_dim == 64 ? dispatch_bs<T, 64>(a, sm_count, s) : dispatch_bs<T, 128>(a, sm_count, s);
+}
+
+template <typename T>
+cudaError_t launch_reduce_t(const AttnArgs &a, cudaStream_t stream) {
+  const int64_t warps = (int64_t)a.num_seqs * a.num_heads;
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  if (a.head_dim == 64)
+    reduce_kernel<T, 64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  else
+    reduce_kernel<T, 128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_max_seqs_per_launch() { return kMaxSeqsPerLaunch; }
+
+cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream) {
+  if (dtype == PA_F32) return dispatch_d<float>(a, sm_count, stream);
+  if (dtype == PA_F16) return dispatch_d<__half>(a, sm_count, stream);
+  return dispatch_d<__nv_bfloat16>(a, sm_count, stream);
+}
+
+cudaError_t launch_reduce(const AttnArgs &a, int dtype, cudaStream_t stream) {
+  if (dtype == PA_F32) return launch_reduce_t<float>(a, stream);
+  if (dtype == PA_F16) return launch_reduce_t<__half>(a, stream);
+  return launch_reduce_t<__nv_bfloat16>(a, stream);
+}
+
+}  // namespace pa

@@ -1,0 +1,254 @@
+// pa_api.cu -- the C ABI of libpa.so: argument checks, split policy, launches.
+//
+// Nothing here allocates device memory.  The only device state the library
+// owns is one error word per device (a file-scope __device__ variable), whose
+// address is looked up once per device.
+#include <mutex>
+
+#include "../../include/pa.h"
+#include "pa_internal.h"
+
+namespace pa {
+
+__device__ unsigned int g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DevInfo g_dev[kMaxDevices];
+bool g_dev_ok[kMaxDevices];
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+bool dtype_ok(int dtype) { return dtype == PA_F32 || dtype == PA_F16 || dtype == PA_BF16; }
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Heads handled by one warp (4, 2 or 1) and how many warps share a KV block.
+bool group_supported(int group) {
+  if (group <= 0) return false;
+  const int gw = group % 4 == 0 ? 4 : (group % 2 == 0 ? 2 : 1);
+  return group / gw <= 8;
+}
+
+}  // namespace
+
+cudaError_t device_info(DevInfo *info) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_dev_ok[dev]) {
+    DevInfo d;
+    e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_error_word);
+    if (e != cudaSuccess) return e;
+    d.err = static_cast<unsigned int *>(p);
+    g_dev[dev] = d;
+    g_dev_ok[dev] = true;
+  }
+  *info = g_dev[dev];
+  return cudaSuccess;
+}
+
+void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
+                  int kv_split_tokens, int sm_count, int *split_blocks, int *max_splits) {
+  const int nblk_max = max_context_len > 0 ? ceil_div(max_context_len, block_size) : 1;
+  int sb;
+  if (kv_split_tokens > 0) {
+    sb = kv_split_tokens / block_size;
+    if (sb < 1) sb = 1;
+  } else {
+    // Pieces of 512 tokens (256 KiB of K+V per KV head at head_dim 128, 16-bit)
+    // keep the merge cost near 1% while giving each CTA many items; very long
+    // contexts use at most 64 pieces; small batches split finer (>= 128 tokens)
+    // until there are about four items per resident CTA slot.
+    int tok = 512;
+    if (max_context_len > 64 * 512) tok = ceil_div(ceil_div(max_context_len, 64), block_size) * block_size;
+    while (tok > 128 && (int64_t)num_seqs * num_kv_heads * ceil_div(max_context_len, tok) <
+                            (int64_t)4 * sm_count)
+      tok /= 2;
+    sb = tok / block_size;
+    if (sb < 1) sb = 1;
+  }
+  *split_blocks = sb;
+  *max_splits = ceil_div(nblk_max, sb);
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+int pa_abi_version(void) { return (1 << 16) | 0; }
+
+const char *pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    default: return "PA_UNKNOWN_STATUS";
+  }
+}
+
+int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, int dtype,
+                         struct CUstream_st *stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !dtype_ok(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  cudaError_t e = launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, num_tokens,
+                                           num_kv_heads, head_dim, block_size, num_blocks,
+                                           elem_bytes(dtype), dev.err, (cudaStream_t)stream);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
+                   int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                   struct CUstream_st *stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !dtype_ok(dtype))
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  cudaError_t e = launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, num_kv_heads,
+                                     head_dim, block_size, num_blocks, elem_bytes(dtype), dev.err,
+                                     (cudaStream_t)stream);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                int block_size, int max_context_len, int kv_split_tokens) {
+  if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_context_len <= 0)
+    return 0;
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return 0;
+  int sb = 0, ms = 0;
+  split_policy(num_seqs, num_kv_heads, block_size, max_context_len, kv_split_tokens,
+               dev.sm_count, &sb, &ms);
+  if (ms <= 1) return 0;
+  return (size_t)num_seqs * num_heads * ms * (head_dim + 2) * sizeof(float) + 256;
+}
+
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+              const int32_t *query_start_loc, int num_seqs, int num_q_tokens, int max_query_len,
+              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+              float scale, int max_context_len, int kv_split_tokens, int dtype, void *workspace,
+              size_t workspace_bytes, struct CUstream_st *stream) {
+  if (num_seqs < 0 || num_q_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+      num_blocks <= 0 || max_blocks_per_seq <= 0 || !dtype_ok(dtype) || kv_split_tokens < 0)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_heads / num_kv_heads;
+  if (!group_supported(group)) return PA_ERR_UNSUPPORTED;
+  if (!query_start_loc) {
+    if (num_q_tokens != num_seqs) return PA_ERR_INVALID_ARG;
+    max_query_len = 1;
+  } else if (max_query_len < 1) {
+    return PA_ERR_INVALID_ARG;
+  }
+  if (num_seqs == 0 || num_q_tokens == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (out == q) return PA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30) return PA_ERR_UNSUPPORTED;
+  const int cap = max_blocks_per_seq * block_size;
+  if (max_context_len <= 0 || max_context_len > cap) max_context_len = cap;
+  if (max_query_len > 1 && group > 64) return PA_ERR_UNSUPPORTED;
+
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  int split_blocks = 0, max_splits = 0;
+  split_policy(num_seqs, num_kv_heads, block_size, max_context_len, kv_split_tokens, dev.sm_count,
+               &split_blocks, &max_splits);
+
+  AttnArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start_loc = query_start_loc;
+  a.err = dev.err;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.split_blocks = split_blocks;
+  a.max_splits = max_splits;
+  a.max_query_len = max_query_len;
+  a.max_context_len = max_context_len;
+  a.num_q_tokens = num_q_tokens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  // fp32 chunk rows have no tensor-core kernel: the decode kernel takes them
+  // one query row per work item.
+  a.rows_mode = (max_query_len > 1 && dtype == PA_F32) ? 1 : 0;
+
+  if (max_splits > 1) {
+    const size_t need = (size_t)num_seqs * num_heads * max_splits * (head_dim + 2) * sizeof(float);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+    a.part_o = static_cast<float *>(workspace);
+    a.part_ml = a.part_o + (size_t)num_seqs * num_heads * max_splits * head_dim;
+  }
+
+  cudaStream_t s = (cudaStream_t)stream;
+  const int step = decode_max_seqs_per_launch();
+  for (int s0 = 0; s0 < num_seqs; s0 += step) {
+    a.seq_begin = s0;
+    a.num_seqs = num_seqs - s0 < step ? num_seqs - s0 : step;
+    cudaError_t e = launch_decode(a, dtype, dev.sm_count, s);
+    if (e == cudaSuccess && max_splits > 1) e = launch_reduce(a, dtype, s);
+    if (e == cudaSuccess && max_query_len > 1 && !a.rows_mode)
+      e = launch_chunk(a, dtype, num_q_tokens, s);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+int pa_get_device_error(unsigned int *code_out, struct CUstream_st *stream) {
+  if (!code_out) return PA_ERR_INVALID_ARG;
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned int host = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyAsync(&host, dev.err, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemsetAsync(dev.err, 0, sizeof host, s) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  *code_out = host;
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+"""User-facing wrapper: one layer's paged KV cache resident in device memory.
+
+``PagedKVCache`` owns the K and V block pools and the split-KV workspace and
+exposes the three operations of the hot path (``write`` = reshape_and_cache,
+``copy_blocks``, ``attend`` = decode), each a single C-ABI call on the current
+CUDA stream.  ``step_from_host`` runs one whole decode step from host (pinned)
+buffers: copy the step's inputs in, write the new K/V, attend, copy the output
+back -- the end-to-end path a serving loop takes every iteration.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks, num_kv_heads, head_dim, block_size, dtype=torch.bfloat16,
+                 device="cuda", k_cache=None, v_cache=None):
+        shape = (num_blocks, num_kv_heads, block_size, head_dim)
+        self.k_cache = k_cache if k_cache is not None else torch.empty(shape, dtype=dtype, device=device)
+        self.v_cache = v_cache if v_cache is not None else torch.empty(shape, dtype=dtype, device=device)
+        assert tuple(self.k_cache.shape) == shape and tuple(self.v_cache.shape) == shape
+        self.num_blocks, self.num_kv_heads, self.head_dim, self.block_size = shape[0], shape[1], shape[3], shape[2]
+        self.dtype = self.k_cache.dtype
+        self.device = self.k_cache.device
+        self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self._staging = {}
+
+    # ---- the three device operations --------------------------------------
+    def write(self, key, value, slot_mapping):
+        _lib.pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slot_mapping)
+
+    def copy_blocks(self, block_mapping):
+        if block_mapping.shape[0]:
+            _lib.pa_copy_blocks(self.k_cache, self.v_cache, block_mapping)
+
+    def workspace(self, num_seqs, num_heads, max_context_len, kv_split_tokens=0):
+        need = _lib.pa_decode_workspace_size(num_seqs, num_heads, self.num_kv_heads, self.head_dim,
+                                             self.block_size, max_context_len, kv_split_tokens)
+        if self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._ws if need else None
+
+    def attend(self, q, block_tables, context_lens, scale, out=None, query_start_loc=None,
+               max_query_len=1, max_context_len=0, kv_split_tokens=0):
+        if out is None:
+            out = torch.empty_like(q)
+        mcl = max_context_len or block_tables.shape[1] * self.block_size
+        ws = self.workspace(block_tables.shape[0], q.shape[1], mcl, kv_split_tokens)
+        _lib.pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
+                       query_start_loc=query_start_loc, max_query_len=max_query_len,
+                       max_context_len=mcl, kv_split_tokens=kv_split_tokens, workspace=ws)
+        return out
+
+    # ---- one step from host memory ------------------------------------------
+    def _dev_like(self, name, t):
+        buf = self._staging.get(name)
+        if buf is None or buf.shape != t.shape or buf.dtype != t.dtype:
+            buf = torch.empty(t.shape, dtype=t.dtype, device=self.device)
+            self._staging[name] = buf
+        return buf
+
+    def step_from_host(self, q, key, value, slot_mapping, block_tables, context_lens, out, scale,
+                       max_context_len=0, kv_split_tokens=0):
+        """All arguments are host tensors (pinned for asynchronous copies);
+        ``out`` receives the attention output.  Returns after enqueueing."""
+        d = {}
+        for name, t in (("q", q), ("key", key), ("value", value), ("slot_mapping", slot_mapping),
+                        ("block_tables", block_tables), ("context_lens", context_lens)):
+            d[name] = self._dev_like(name, t)
+            d[name].copy_(t, non_blocking=True)
+        self.write(d["key"], d["value"], d["slot_mapping"])
+        o = self._dev_like("out", out)
+        self.attend(d["q"], d["block_tables"], d["context_lens"], scale, out=o,
+                    max_context_len=max_context_len, kv_split_tokens=kv_split_tokens)
+        out.copy_(o, non_blocking=True)
+        return out
+
+    @staticmethod
+    def host_bytes(*tensors) -> int:
+        return int(sum(t.numel() * t.element_size() for t in tensors))
