@@ -52,9 +52,13 @@ def build_batch(wl) -> Batch:
 
     if wl.kind in ("decode", "mixed"):
         for L, Q in zip(wl.context_lens, wl.query_lens):
-            sid = alloc.new_sequence(L - Q)
-            for _ in range(Q):
-                append(sid)
+            if L < Q:  # empty context: the query token has no K/V to write (padding slot)
+                sid = alloc.new_sequence(L)
+                slots.extend([-1] * Q)
+            else:
+                sid = alloc.new_sequence(L - Q)
+                for _ in range(Q):
+                    append(sid)
             sids.append(sid)
         qlens = list(wl.query_lens)
     elif wl.kind == "shared_prefix":

@@ -15,12 +15,12 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
-BUILD = os.path.join(PKG, "_build")
-LIB = os.path.join(PKG, "libpa.so")
+BUILD = os.environ.get("PA_BUILD_DIR", os.path.join(PKG, "_build"))
+LIB = os.environ.get("PA_LIB_OUT", os.path.join(PKG, "libpa.so"))
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
-         "-Xptxas", "-warn-spills", "-I", INCLUDE]
+         "-Xptxas", "-warn-spills", "-I", INCLUDE] + os.environ.get("PA_NVCC_DEFINES", "").split()
 
 
 def _headers():

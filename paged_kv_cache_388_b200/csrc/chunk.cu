@@ -26,8 +26,13 @@ constexpr int kPad = 8;    // elements of padding per smem row
 template <typename T>
 struct Mma;
 
+// P (softmax weights in [0, 1]) is fed to the P.V product in the cache's
+// 16-bit type.  bf16 keeps 8 significant bits, which on rows with few keys
+// leaves errors near 2^-9 of |V|; such rows split P into hi + lo bf16 parts
+// (two products, P exact to ~2^-17).  fp16 keeps 11 bits and needs no split.
 template <>
 struct Mma<__nv_bfloat16> {
+  static constexpr bool kSplitP = true;
   __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
     asm volatile(
@@ -40,10 +45,17 @@ struct Mma<__nv_bfloat16> {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
   }
+  // residual of pack(): (lo - bf16(lo), hi - bf16(hi)) in bf16
+  __device__ __forceinline__ static uint32_t pack_residual(float lo, float hi) {
+    const float rl = lo - __bfloat162float(__float2bfloat16_rn(lo));
+    const float rh = hi - __bfloat162float(__float2bfloat16_rn(hi));
+    return pack(rl, rh);
+  }
 };
 
 template <>
 struct Mma<__half> {
+  static constexpr bool kSplitP = false;
   __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
     asm volatile(
@@ -56,6 +68,7 @@ struct Mma<__half> {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
   }
+  __device__ __forceinline__ static uint32_t pack_residual(float, float) { return 0u; }
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
@@ -249,6 +262,7 @@ __global__ void __launch_bounds__(128) chunk_kernel(const AttnArgs a, int tiles_
     m_b = mn_b;
     float rs_a = 0.f, rs_b = 0.f;
     uint32_t pa[kKT / 16][4];
+    uint32_t pr[Mma<T>::kSplitP ? kKT / 16 : 1][4];
 #pragma unroll
     for (int i = 0; i < kKT / 8; ++i) {
       const float p0 = fast_exp2(s[i][0] - mn_a), p1 = fast_exp2(s[i][1] - mn_a);
@@ -257,6 +271,10 @@ __global__ void __launch_bounds__(128) chunk_kernel(const AttnArgs a, int tiles_
       rs_b += p2 + p3;
       pa[i / 2][(i & 1) * 2 + 0] = Mma<T>::pack(p0, p1);
       pa[i / 2][(i & 1) * 2 + 1] = Mma<T>::pack(p2, p3);
+      if constexpr (Mma<T>::kSplitP) {
+        pr[i / 2][(i & 1) * 2 + 0] = Mma<T>::pack_residual(p0, p1);
+        pr[i / 2][(i & 1) * 2 + 1] = Mma<T>::pack_residual(p2, p3);
+      }
     }
     l_a = l_a * al_a + rs_a;
     l_b = l_b * al_b + rs_b;
@@ -279,6 +297,10 @@ __global__ void __launch_bounds__(128) chunk_kernel(const AttnArgs a, int tiles_
         ldsm_x4_t(b, tV + key * LD + c);
         Mma<T>::run(o[2 * dp], pa[kk], b[0], b[1]);
         Mma<T>::run(o[2 * dp + 1], pa[kk], b[2], b[3]);
+        if constexpr (Mma<T>::kSplitP) {
+          Mma<T>::run(o[2 * dp], pr[kk], b[0], b[1]);
+          Mma<T>::run(o[2 * dp + 1], pr[kk], b[2], b[3]);
+        }
       }
     }
     __syncthreads();

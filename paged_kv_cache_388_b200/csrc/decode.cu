@@ -38,9 +38,17 @@
 namespace pa {
 namespace {
 
+// Tunables (compile-time): ring of K/V stages per CTA and the CTAs per SM the
+// 4-consumer-warp variant is register-limited to.
+#ifndef PA_DECODE_RING_KB
+#define PA_DECODE_RING_KB 48
+#endif
+#ifndef PA_DECODE_MIN_CTAS
+#define PA_DECODE_MIN_CTAS 3
+#endif
+
 constexpr int kMaxSeqsPerLaunch = 2048;
-constexpr int kRingBytes = 64 * 1024;
-constexpr int kMaxConsumerWarps = 8;
+constexpr int kRingBytes = PA_DECODE_RING_KB * 1024;
 
 template <typename T, int D, int BS, int GW>
 struct DecodeCfg {
@@ -51,9 +59,13 @@ struct DecodeCfg {
   static constexpr int RPP = 32 / LPR;          // rows per pass (row groups per warp)
   static constexpr int CHUNK = 16;              // rows per softmax step
   static constexpr int PASSES = CHUNK / RPP;
-  static constexpr int NV = PASSES * GW;        // partial scores per lane per chunk
-  static constexpr int VPL = NV >= LPR ? NV / LPR : 1;  // reduced scores kept per lane
-  static constexpr int DUP = NV >= LPR ? 1 : LPR / NV;  // lanes holding the same score
+  // Scores are reduced in sub-chunks of PPS passes so that a sub-chunk holds at
+  // most LPR partial sums per lane (registers) and leaves one reduced score per
+  // lane (DUP lanes share it when a sub-chunk has fewer scores than lanes).
+  static constexpr int PPS = PASSES * GW >= LPR ? LPR / GW : PASSES;  // passes per sub-chunk
+  static constexpr int NSUB = PASSES / PPS;     // sub-chunks per chunk = scores kept per lane
+  static constexpr int NVS = PPS * GW;          // partial scores per lane per sub-chunk
+  static constexpr int DUP = LPR / NVS;         // lanes holding the same reduced score
   static constexpr int LPH = LPR / GW;          // lanes of one head in a row group
   static constexpr int TILE = BS * D * kElem;   // bytes of one (block, kv-head) tile
   static constexpr int STAGE = 2 * TILE;        // K tile + V tile
@@ -61,56 +73,50 @@ struct DecodeCfg {
   static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row must map onto whole lanes");
   static_assert(PASSES >= 1 && CHUNK % RPP == 0, "chunk must hold whole passes");
   static_assert(GW <= LPR, "a lane's reduced scores must belong to one head");
+  static_assert(NVS <= LPR && LPR % NVS == 0 && PASSES % PPS == 0, "sub-chunk shape");
   static_assert(BS % CHUNK == 0, "block size must be a multiple of 16");
 };
 
-// Shared-memory layout (dynamic).  Offsets are 128-byte aligned.
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// Dynamic shared-memory layout; depends on the launch (sequences in this
+// launch, consumer warps, group size), computed identically on host and device.
 template <typename C>
-struct Smem {
-  static constexpr int kRing = 0;
-  static constexpr int kFull = kRing + C::STAGES * C::STAGE;           // uint64 [STAGES]
-  static constexpr int kEmpty = kFull + 8 * C::STAGES;                 // uint64 [STAGES]
-  static constexpr int kBad = kEmpty + 8 * C::STAGES;                  // int [STAGES]
-  static constexpr int kMisc = (kBad + 4 * C::STAGES + 127) / 128 * 128;  // int [4]
-  static constexpr int kPrefix = kMisc + 128;                          // int [kMaxSeqs+1]
-  static constexpr int kScan = kPrefix + 4 * (kMaxSeqsPerLaunch + 8);  // int [32]
-  static constexpr int kP = (kScan + 128 + 127) / 128 * 128;           // float [NCW][16][GW]
-  static constexpr int kMerge = kP + kMaxConsumerWarps * 16 * 4 * 4;   // float [NCW][GW][D+4]
-  static constexpr int kBytes = kMerge + kMaxConsumerWarps * 4 * (128 + 4) * 4;
+struct Layout {
+  int ring, qbuf, full, empty, qfull, qempty, bad, misc, len, q0, ql, prefix, scan, p, merge, bytes;
+  int qbytes;  // bytes of one item's query rows (GROUP heads)
+  __host__ __device__ Layout(int n, int ncw, int group) {
+    constexpr int D = C::LPR * C::ELEMS;
+    qbytes = group * D * C::kElem;
+    ring = 0;
+    qbuf = ring + C::STAGES * C::STAGE;
+    full = align_up(qbuf + 2 * qbytes, 128);
+    empty = full + 8 * C::STAGES;
+    qfull = empty + 8 * C::STAGES;
+    qempty = qfull + 16;
+    bad = qempty + 16;
+    misc = align_up(bad + 4 * C::STAGES, 16);
+    len = misc + 16;
+    q0 = len + 4 * n;
+    ql = q0 + 4 * n;
+    prefix = ql + 4 * n;
+    scan = align_up(prefix + 4 * (n + 1), 16);
+    p = align_up(scan + 4 * 32, 128);
+    merge = align_up(p + ncw * 16 * 4 * 4, 128);
+    bytes = merge + ncw * 4 * (D + 4) * 4;
+  }
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Work items contributed by sequence s: its splits for a decode sequence
-// (one query row); for a chunk of Q > 1 rows, Q single-row items in row mode
-// and none otherwise (the chunk kernel takes them).
-__device__ __forceinline__ bool seq_len_ok(const AttnArgs &a, int L) {
-  return L >= 0 && L <= a.max_context_len;
-}
-
-// Query rows [q0, q0 + qlen) of sequence gs; false if they do not fit in q.
-__device__ __forceinline__ bool seq_rows(const AttnArgs &a, int gs, int *q0, int *qlen) {
-  if (!a.query_start_loc) {
-    *q0 = gs;
-    *qlen = 1;
-    return true;
-  }
-  *q0 = a.query_start_loc[gs];
-  *qlen = a.query_start_loc[gs + 1] - *q0;
-  return *q0 >= 0 && *qlen >= 0 && *q0 + *qlen <= a.num_q_tokens;
-}
-
-__device__ __forceinline__ int seq_items(const AttnArgs &a, int s) {
-  const int gs = a.seq_begin + s;
-  int q0, qlen;
-  if (!seq_rows(a, gs, &q0, &qlen)) {
-    raise_error(a.err, PA_DEVERR_QUERY_LEN);
-    return 0;
-  }
+// Work items contributed by a sequence: its splits for a decode sequence (one
+// query row); for a chunk of Q > 1 rows, Q single-row items in row mode and
+// none otherwise (the chunk kernel takes them).  len/q0/qlen come from the
+// shared-memory copies made in the prologue.
+__device__ __forceinline__ int seq_items(const AttnArgs &a, int L, int qlen) {
   if (qlen <= 0) return 0;
   if (qlen > 1) return a.rows_mode ? qlen : 0;
-  const int L = a.context_lens[gs];
-  if (L <= 0 || !seq_len_ok(a, L)) return 1;  // zero-output item
+  if (L <= 0 || L > a.max_context_len) return 1;  // zero-output item
   return ceil_div(ceil_div(L, a.block_size), a.split_blocks);
 }
 
@@ -121,11 +127,13 @@ struct Item {
   int nsplit;
   int kvh;
   int b0, b1;  // KV blocks [b0, b1) of the sequence
-  int L;       // keys visible to the row (valid only if ok)
+  int L;       // keys visible to the row
   unsigned int bad_bits;  // PA_DEVERR_* of an invalid sequence (0: ok)
 };
 
-__device__ __forceinline__ Item decode_item(const AttnArgs &a, const int *prefix, int n, int w) {
+__device__ __forceinline__ Item decode_item(const AttnArgs &a, const int *prefix,
+                                            const int *s_len, const int *s_q0, const int *s_ql,
+                                            int n, int w) {
   Item it;
   const int f = w / a.num_kv_heads;
   it.kvh = w - f * a.num_kv_heads;
@@ -135,11 +143,11 @@ __device__ __forceinline__ Item decode_item(const AttnArgs &a, const int *prefix
     if (prefix[mid] <= f) lo = mid; else hi = mid;
   }
   it.seq = a.seq_begin + lo;
-  const int L = a.context_lens[it.seq];
-  int q0, qlen;
-  seq_rows(a, it.seq, &q0, &qlen);  // valid: sequences with bad rows contribute no items
+  const int L = s_len[lo];
+  const int q0 = s_q0[lo];
+  const int qlen = s_ql[lo];
   it.bad_bits = 0;
-  if (!seq_len_ok(a, L)) it.bad_bits = PA_DEVERR_CONTEXT_LEN;
+  if (L < 0 || L > a.max_context_len) it.bad_bits = PA_DEVERR_CONTEXT_LEN;
   else if (qlen > L && L > 0) it.bad_bits = PA_DEVERR_QUERY_LEN;
   if (qlen > 1) {  // row mode: one item per query row, never split
     const int t = f - prefix[lo];
@@ -186,30 +194,66 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
   }
 }
 
-template <typename T, int D, int BS, int GW>
-__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
+template <typename T>
+__device__ __forceinline__ void store4(T *dst, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float *dst, float4 v) {
+  *reinterpret_cast<float4 *>(dst) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *dst, float4 v) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t *>(&lo);
+  u.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = u;
+}
+template <>
+__device__ __forceinline__ void store4<__half>(__half *dst, float4 v) {
+  __half2 lo = __floats2half2_rn(v.x, v.y), hi = __floats2half2_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t *>(&lo);
+  u.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(dst) = u;
+}
+
+// MAXW = most consumer warps a launch of this variant uses (4: three CTAs per
+// SM fit; 8: the wide variant for large head groups).
+template <typename T, int D, int BS, int GW, int MAXW>
+__global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTAS : 1)
     paged_decode_kernel(const AttnArgs a, int ncw, int hsplit) {
   using C = DecodeCfg<T, D, BS, GW>;
-  using S = Smem<C>;
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::kFull);
-  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + S::kEmpty);
-  int *bad = reinterpret_cast<int *>(smem + S::kBad);
-  volatile int *abort_flag = reinterpret_cast<int *>(smem + S::kMisc);
-  int *prefix = reinterpret_cast<int *>(smem + S::kPrefix);
-  int *scan = reinterpret_cast<int *>(smem + S::kScan);
+  const int n = a.num_seqs;
+  const Layout<C> lay(n, ncw, a.group);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.full);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + lay.empty);
+  uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + lay.qfull);
+  uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + lay.qempty);
+  int *bad = reinterpret_cast<int *>(smem + lay.bad);
+  volatile int *abort_flag = reinterpret_cast<int *>(smem + lay.misc);
+  int *s_len = reinterpret_cast<int *>(smem + lay.len);
+  int *s_q0 = reinterpret_cast<int *>(smem + lay.q0);
+  int *s_ql = reinterpret_cast<int *>(smem + lay.ql);
+  int *prefix = reinterpret_cast<int *>(smem + lay.prefix);
+  int *scan = reinterpret_cast<int *>(smem + lay.scan);
+  unsigned char *ring = smem + lay.ring;
+  unsigned char *qbuf = smem + lay.qbuf;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int nthreads = blockDim.x;
-  const int n = a.num_seqs;
 
-  // ---- prologue: barriers + prefix sum of items per sequence ---------------
+  // ---- prologue: barriers, per-sequence lengths and rows, item prefix sum --
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], hsplit);
+      mbar_init(&empty[s], ncw);  // every consumer warp releases every stage
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], ncw);
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -218,7 +262,23 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
     const int per = ceil_div(n, nthreads);
     const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
     int local = 0;
-    for (int s = s0; s < s1; ++s) local += seq_items(a, s);
+    for (int s = s0; s < s1; ++s) {
+      const int gs = a.seq_begin + s;
+      int q0 = gs, q1 = gs + 1;
+      if (a.query_start_loc) {
+        q0 = a.query_start_loc[gs];
+        q1 = a.query_start_loc[gs + 1];
+        if (q0 < 0 || q1 < q0 || q1 > a.num_q_tokens) {  // rows outside q: no items
+          raise_error(a.err, PA_DEVERR_QUERY_LEN);
+          q1 = q0 = 0;
+        }
+      }
+      const int L = a.context_lens[gs];
+      s_len[s] = L;
+      s_q0[s] = q0;
+      s_ql[s] = q1 - q0;
+      local += seq_items(a, L, q1 - q0);
+    }
     // block exclusive scan of `local`
     int x = local;
 #pragma unroll
@@ -242,26 +302,44 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
     int run = (warp ? scan[warp - 1] : 0) + x - local;
     for (int s = s0; s < s1; ++s) {
       prefix[s] = run;
-      run += seq_items(a, s);
+      run += seq_items(a, s_len[s], s_ql[s]);
     }
     if (tid == nthreads - 1) prefix[n] = run;
   }
   __syncthreads();
   const int total_items = prefix[n] * a.num_kv_heads;
 
-  unsigned char *ring = smem + S::kRing;
-
   if (warp == ncw) {
     // ======================= producer warp ===================================
-    uint32_t it = 0;
-    for (int w = blockIdx.x; w < total_items; w += gridDim.x) {
-      const Item item = decode_item(a, prefix, n, w);
+    uint32_t it = 0, k = 0;
+    for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
+      const Item item = decode_item(a, prefix, s_len, s_q0, s_ql, n, w);
+      // this item's query rows -> qbuf[k & 1]
+      {
+        const uint32_t qs = k & 1u;
+        bool ok = !*abort_flag;
+        if (ok) ok = mbar_wait(&qempty[qs], ((k >> 1) & 1u) ^ 1u);
+        if (lane == 0) {
+          if (!ok) {
+            if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            mbar_arrive(&qfull[qs]);
+          } else {
+            mbar_arrive_expect_tx(&qfull[qs], lay.qbytes);
+            bulk_load(qbuf + qs * lay.qbytes,
+                      static_cast<const T *>(a.q) +
+                          ((int64_t)item.qrow * a.num_heads + item.kvh * a.group) * D,
+                      lay.qbytes, &qfull[qs]);
+          }
+        }
+        __syncwarp();
+      }
       const int32_t *table = a.block_tables + (int64_t)item.seq * a.max_blocks_per_seq;
       for (int b = item.b0; b < item.b1; b += 32) {
         const int cnt = min(32, item.b1 - b);
         const int my_id = lane < cnt ? table[b + lane] : 0;
-        for (int k = 0; k < cnt; ++k) {
-          const int pb = __shfl_sync(0xffffffffu, my_id, k);
+        for (int j = 0; j < cnt; ++j) {
+          const int pb = __shfl_sync(0xffffffffu, my_id, j);
           const uint32_t slot = it % C::STAGES;
           const uint32_t par = ((it / C::STAGES) & 1u) ^ 1u;
           ++it;
@@ -281,7 +359,6 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
               bad[slot] = 0;
               const int64_t tile = ((int64_t)pb * a.num_kv_heads + item.kvh) * (BS * D);
               unsigned char *dst = ring + slot * C::STAGE;
-              fence_proxy_async_smem();
               mbar_arrive_expect_tx(&full[slot], C::STAGE);
               bulk_load(dst, static_cast<const T *>(a.k_cache) + tile, C::TILE, &full[slot]);
               bulk_load(dst + C::TILE, static_cast<const T *>(a.v_cache) + tile, C::TILE,
@@ -301,35 +378,48 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
   const int nbl = ncw / hsplit;
   const int rg = lane / C::LPR;   // row group
   const int li = lane % C::LPR;   // lane within row
-  // reduced-score ownership of this lane (see reduce_scatter)
-  const int v0 = C::NV >= C::LPR ? li * C::VPL : li / C::DUP;
-  const int my_head = v0 / C::PASSES;
+  // reduced-score ownership of this lane (see reduce_scatter): in every
+  // sub-chunk the lane keeps score v = li / DUP, i.e. head v / PPS of pass
+  // v % PPS of that sub-chunk.
+  const int vsub = li / C::DUP;
+  const int my_head = vsub / C::PPS;
+  const int my_pass = vsub % C::PPS;
   const bool owner = (li % C::DUP) == 0;
 
-  float *p_s = reinterpret_cast<float *>(smem + S::kP) + warp * 16 * GW;
-  float *merge = reinterpret_cast<float *>(smem + S::kMerge);
+  float *p_s = reinterpret_cast<float *>(smem + lay.p) + warp * 16 * GW;
+  float *merge = reinterpret_cast<float *>(smem + lay.merge);
   const int mstride = GW * (D + 4);  // floats per warp in the merge area
 
-  uint32_t it_base = 0;
-  for (int w = blockIdx.x; w < total_items; w += gridDim.x) {
-    const Item item = decode_item(a, prefix, n, w);
+  uint32_t it_base = 0, k = 0;
+  for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
+    const Item item = decode_item(a, prefix, s_len, s_q0, s_ql, n, w);
     const int nblocks = item.b1 - item.b0;
-    const int qrow = item.qrow;
-    const int head0 = item.kvh * a.group + hs * GW;
 
-    // q slice of this lane, pre-scaled by scale*log2(e)
+    // q slice of this lane from the prefetched rows, pre-scaled by scale*log2(e)
     float2 q2[GW][C::PAIRS];
-#pragma unroll
-    for (int h = 0; h < GW; ++h) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(
-          static_cast<const T *>(a.q) + ((int64_t)qrow * a.num_heads + head0 + h) * D +
-          li * C::ELEMS);
-      Elem<T>::to_f2(raw, q2[h]);
-#pragma unroll
-      for (int e = 0; e < C::PAIRS; ++e) {
-        q2[h][e].x *= a.scale_log2;
-        q2[h][e].y *= a.scale_log2;
+    {
+      const uint32_t qs = k & 1u;
+      bool ok = !*abort_flag;
+      if (ok) {
+        ok = mbar_wait(&qfull[qs], (k >> 1) & 1u);
+        if (!ok && lane == 0) {
+          if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
       }
+      const T *qrow = reinterpret_cast<const T *>(qbuf + qs * lay.qbytes) + hs * GW * D;
+#pragma unroll
+      for (int h = 0; h < GW; ++h) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(qrow + h * D + li * C::ELEMS);
+        Elem<T>::to_f2(raw, q2[h]);
+#pragma unroll
+        for (int e = 0; e < C::PAIRS; ++e) {
+          q2[h][e].x *= a.scale_log2;
+          q2[h][e].y *= a.scale_log2;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qempty[qs]);
     }
 
     float m[GW];
@@ -344,19 +434,35 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
     bool item_bad = item.bad_bits != 0;
     if (item.bad_bits && tid == 0 && item.kvh == 0) raise_error(a.err, item.bad_bits);
 
-    for (int j = bl; j < nblocks; j += nbl) {
-      const uint32_t itn = it_base + j;
+    // Every consumer warp waits for and releases every stage in ring order
+    // (so no parity wait is ever more than one phase ahead of its barrier),
+    // but computes only the blocks j = bl, bl + nbl, ... of this item.
+    auto wait_stage = [&](uint32_t itn) -> bool {
       const uint32_t slot = itn % C::STAGES;
-      const uint32_t par = (itn / C::STAGES) & 1u;
       bool ok = !*abort_flag;
       if (ok) {
-        ok = mbar_wait(&full[slot], par);
+        ok = mbar_wait(&full[slot], (itn / C::STAGES) & 1u);
         if (!ok && lane == 0) {
           if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
           *abort_flag = 1;
         }
       }
-      if (ok && bad[slot]) ok = false;
+      return ok && !bad[slot];
+    };
+    auto release_stage = [&](uint32_t itn) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[itn % C::STAGES]);
+    };
+    int next = 0;  // first block of the item not yet waited for by this warp
+    for (int j = bl; j < nblocks; j += nbl) {
+      for (; next < j; ++next) {
+        wait_stage(it_base + next);
+        release_stage(it_base + next);
+      }
+      next = j + 1;
+      const uint32_t itn = it_base + j;
+      const uint32_t slot = itn % C::STAGES;
+      const bool ok = wait_stage(itn);
       if (!ok) {
         item_bad = true;
       } else {
@@ -367,61 +473,64 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
 #pragma unroll
         for (int r0 = 0; r0 < BS; r0 += C::CHUNK) {
           if (r0 < nvalid) {
-            // ---- scores: partial dot products over this lane's slice ----
-            float sc[C::NV];
+            // ---- scores: partial dot products over this lane's slice, reduced
+            //      across the row's lanes one sub-chunk at a time ----
+            float sc[C::NSUB];
 #pragma unroll
-            for (int p = 0; p < C::PASSES; ++p) {
-              const int row = r0 + p * C::RPP + rg;
-              const uint4 raw =
-                  *reinterpret_cast<const uint4 *>(ks + (row * D + li * C::ELEMS) * C::kElem);
-              float2 k2[C::PAIRS];
-              Elem<T>::to_f2(raw, k2);
+            for (int u = 0; u < C::NSUB; ++u) {
+              float part[C::NVS];
 #pragma unroll
-              for (int h = 0; h < GW; ++h) {
-                float2 d2 = make_float2(0.f, 0.f);
+              for (int pp = 0; pp < C::PPS; ++pp) {
+                const int row = r0 + (u * C::PPS + pp) * C::RPP + rg;
+                const uint4 raw =
+                    *reinterpret_cast<const uint4 *>(ks + (row * D + li * C::ELEMS) * C::kElem);
+                float2 k2[C::PAIRS];
+                Elem<T>::to_f2(raw, k2);
 #pragma unroll
-                for (int e = 0; e < C::PAIRS; ++e) d2 = ffma2(q2[h][e], k2[e], d2);
-                sc[h * C::PASSES + p] = d2.x + d2.y;
+                for (int h = 0; h < GW; ++h) {
+                  float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+                  for (int e = 0; e < C::PAIRS; ++e) d2 = ffma2(q2[h][e], k2[e], d2);
+                  part[h * C::PPS + pp] = d2.x + d2.y;
+                }
               }
+              reduce_scatter<C::NVS, C::LPR>(part, lane);
+              sc[u] = part[0];
             }
-            reduce_scatter<C::NV, C::LPR>(sc, lane);
 
             // ---- online softmax (base 2) ----
             float cmax = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < C::VPL; ++i) {
-              const int v = v0 + i;
-              const int row = r0 + (v % C::PASSES) * C::RPP + rg;
-              if (row >= nvalid) sc[i] = -INFINITY;
-              cmax = fmaxf(cmax, sc[i]);
+            for (int u = 0; u < C::NSUB; ++u) {
+              const int row = r0 + (u * C::PPS + my_pass) * C::RPP + rg;
+              if (row >= nvalid) sc[u] = -INFINITY;
+              cmax = fmaxf(cmax, sc[u]);
             }
 #pragma unroll
-            for (int o = 1; o < C::LPH; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+            for (int o = C::DUP; o < C::LPH; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
 #pragma unroll
             for (int o = C::LPR; o < 32; o <<= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
             float alpha[GW];
-            float m_mine = 0.f;
+            float m_mine = 0.f, a_mine = 1.f;
 #pragma unroll
             for (int h = 0; h < GW; ++h) {
               const float cm = __shfl_sync(0xffffffffu, cmax, h * C::LPH);
               const float mn = fmaxf(m[h], cm);
               alpha[h] = fast_exp2(m[h] - mn);
               m[h] = mn;
-              if (h == my_head) m_mine = mn;
+              if (h == my_head) {
+                m_mine = mn;
+                a_mine = alpha[h];
+              }
             }
             float psum = 0.f;
 #pragma unroll
-            for (int i = 0; i < C::VPL; ++i) {
-              const float pv = fast_exp2(sc[i] - m_mine);
+            for (int u = 0; u < C::NSUB; ++u) {
+              const float pv = fast_exp2(sc[u] - m_mine);
               psum += pv;
-              const int v = v0 + i;
-              const int crow = (v % C::PASSES) * C::RPP + rg;  // row within chunk
+              const int crow = (u * C::PPS + my_pass) * C::RPP + rg;  // row within chunk
               if (owner) p_s[crow * GW + my_head] = pv;
             }
-            float a_mine = 1.f;
-#pragma unroll
-            for (int h = 0; h < GW; ++h)
-              if (h == my_head) a_mine = alpha[h];
             l_lane = l_lane * a_mine + (owner ? psum : 0.f);
             __syncwarp();
 
@@ -465,9 +574,11 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
           }
         }
       }
-      // release the stage
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      release_stage(itn);
+    }
+    for (; next < nblocks; ++next) {
+      wait_stage(it_base + next);
+      release_stage(it_base + next);
     }
     it_base += nblocks;
 
@@ -491,12 +602,10 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
     if (rg == 0) {
 #pragma unroll
       for (int h = 0; h < GW; ++h) {
-        float *dst = mw + h * (D + 4) + li * C::ELEMS;
+        float4 *dst = reinterpret_cast<float4 *>(mw + h * (D + 4) + li * C::ELEMS);
 #pragma unroll
-        for (int e = 0; e < C::PAIRS; ++e) {
-          dst[2 * e] = acc[h][e].x;
-          dst[2 * e + 1] = acc[h][e].y;
-        }
+        for (int e = 0; e < C::PAIRS; e += 2)
+          dst[e / 2] = make_float4(acc[h][e].x, acc[h][e].y, acc[h][e + 1].x, acc[h][e + 1].y);
       }
     }
 #pragma unroll
@@ -541,12 +650,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 1))
         }
         const int head = item.kvh * a.group + hg;
         if (direct) {
-          float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
-          T *dst = static_cast<T *>(a.out) + ((int64_t)qrow * a.num_heads + head) * D + d4 * 4;
-          dst[0] = Elem<T>::from_f(o.x * inv);
-          dst[1] = Elem<T>::from_f(o.y * inv);
-          dst[2] = Elem<T>::from_f(o.z * inv);
-          dst[3] = Elem<T>::from_f(o.w * inv);
+          const float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
+          T *dst = static_cast<T *>(a.out) + ((int64_t)item.qrow * a.num_heads + head) * D + d4 * 4;
+          store4<T>(dst, make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv));
         } else {
           const int64_t pidx = ((int64_t)item.seq * a.num_heads + head) * a.max_splits + item.split;
           *reinterpret_cast<float4 *>(a.part_o + pidx * D + d4 * 4) = o;
@@ -570,10 +676,14 @@ __global__ void __launch_bounds__(256) reduce_kernel(const AttnArgs a) {
   const int s = gw / a.num_heads;
   const int head = gw - s * a.num_heads;
   const int gs = a.seq_begin + s;
-  int qrow, qlen;
-  if (!seq_rows(a, gs, &qrow, &qlen) || qlen != 1) return;
+  int qrow = gs, qlen = 1;
+  if (a.query_start_loc) {
+    qrow = a.query_start_loc[gs];
+    qlen = a.query_start_loc[gs + 1] - qrow;
+    if (qrow < 0 || qlen != 1 || qrow + 1 > a.num_q_tokens) return;
+  }
   const int L = a.context_lens[gs];
-  if (L <= 0 || !seq_len_ok(a, L)) return;  // written by the main kernel
+  if (L <= 0 || L > a.max_context_len) return;  // written by the main kernel
   const int nsplit = ceil_div(ceil_div(L, a.block_size), a.split_blocks);
   if (nsplit <= 1 || nsplit > a.max_splits) return;
   const int64_t base = ((int64_t)gs * a.num_heads + head) * a.max_splits;
@@ -612,32 +722,45 @@ __global__ void __launch_bounds__(256) reduce_kernel(const AttnArgs a) {
   for (int e = 0; e < PER; ++e) dst[e] = Elem<T>::from_f(o[e] * inv);
 }
 
-template <typename T, int D, int BS, int GW>
-cudaError_t launch_decode_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
+template <typename T, int D, int BS, int GW, int MAXW>
+cudaError_t launch_variant(const AttnArgs &a, int sm_count, int ncw, int hsplit,
+                           cudaStream_t stream) {
   using C = DecodeCfg<T, D, BS, GW>;
-  using S = Smem<C>;
-  auto kern = paged_decode_kernel<T, D, BS, GW>;
-  static int occ = -1;  // resident CTAs per SM (per instantiation; same on every B200)
-  if (occ < 0) {
+  auto kern = paged_decode_kernel<T, D, BS, GW, MAXW>;
+  const Layout<C> lay(a.num_seqs, ncw, a.group);
+  // Opt in to the largest layout once; resident CTAs per SM for this launch.
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    const Layout<C> big(kMaxSeqsPerLaunch, MAXW, 32);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         S::kBytes);
+                                         big.bytes);
     if (e != cudaSuccess) return e;
-    int o = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, 32 * (kMaxConsumerWarps + 1),
-                                                      S::kBytes);
-    if (e != cudaSuccess) return e;
-    occ = o > 0 ? o : 1;
+    attr_set[dev] = true;
   }
-  const int hsplit = a.group / GW;
-  const int nbl = hsplit >= 4 ? 1 : 4 / hsplit;
-  const int ncw = hsplit * nbl;
-  // upper bound of items in this launch
-  const int64_t max_items = (int64_t)a.num_seqs * a.num_kv_heads * a.max_splits;
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (ncw + 1),
+                                                                lay.bytes);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  const int64_t max_items = (int64_t)a.num_seqs * a.num_kv_heads *
+                            (a.rows_mode ? (a.max_splits > a.max_query_len ? a.max_splits : a.max_query_len)
+                                         : a.max_splits);
   int64_t grid = (int64_t)sm_count * occ;
   if (grid > max_items) grid = max_items;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, 32 * (ncw + 1), S::kBytes, stream>>>(a, ncw, hsplit);
+  kern<<<(unsigned)grid, 32 * (ncw + 1), lay.bytes, stream>>>(a, ncw, hsplit);
   return cudaGetLastError();
+}
+
+template <typename T, int D, int BS, int GW>
+cudaError_t launch_decode_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
+  const int hsplit = a.group / GW;
+  const int nbl = hsplit >= 4 ? 1 : 4 / hsplit;
+  const int ncw = hsplit * nbl;
+  if (ncw <= 4) return launch_variant<T, D, BS, GW, 4>(a, sm_count, ncw, hsplit, stream);
+  return launch_variant<T, D, BS, GW, 8>(a, sm_count, ncw, hsplit, stream);
 }
 
 template <typename T, int D, int BS>

@@ -10,9 +10,13 @@ def model_batch(wl):
     slots, sids = [], []
     if wl.kind in ("decode", "mixed"):
         for i, (L, Q) in enumerate(zip(wl.context_lens, wl.query_lens)):
-            m.new_sequence(i, L - Q)
-            for _ in range(Q):
-                slots.append(m.append(i))
+            if L < Q:
+                m.new_sequence(i, L)
+                slots.extend([-1] * Q)
+            else:
+                m.new_sequence(i, L - Q)
+                for _ in range(Q):
+                    slots.append(m.append(i))
             sids.append(i)
         qlens = list(wl.query_lens)
     else:

@@ -53,7 +53,8 @@ def test_batch_matches_oracle_rules(cfg):
     else:
         assert np.array_equal(b.query_start_loc, m["query_start_loc"])
     # slots unique (several writers to one slot would make the result ambiguous)
-    assert len(set(b.slot_mapping.tolist())) == b.slot_mapping.size
+    real = b.slot_mapping[b.slot_mapping >= 0]
+    assert len(set(real.tolist())) == real.size
     # refcounts: each block in use is referenced by exactly refcount tables
     refs = np.zeros(wl.num_blocks, np.int64)
     for i, L in enumerate(b.context_lens):
@@ -63,6 +64,15 @@ def test_batch_matches_oracle_rules(cfg):
     for pb in range(wl.num_blocks):
         assert refs[pb] == b.allocator.refcount(pb)
     assert b.allocator.num_free + np.count_nonzero(refs) == wl.num_blocks
+
+
+def test_empty_context_gets_padding_slot():
+    wl = workloads.decode_workload("edge", 1, [0, 1, 16, 17], 8, 2, 64, 16, "f32")
+    b = build_batch(wl)
+    m = model_batch(wl)
+    assert b.slot_mapping[0] == -1 and np.array_equal(b.slot_mapping, m["slot_mapping"])
+    assert b.context_lens.tolist() == [0, 1, 16, 17]
+    assert np.array_equal(b.block_tables, m["block_tables"])
 
 
 def test_shared_prefix_cow_counts():
