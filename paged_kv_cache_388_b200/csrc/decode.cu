@@ -31,12 +31,15 @@
 //   and either written to `out` (single split) or to the split workspace,
 //   which reduce_kernel combines.
 #include <float.h>
+#include <stdlib.h>
+#include <string.h>
 
-#include "pa_device.cuh"
-#include "pa_internal.h"
+#include "decode_common.cuh"
 
 namespace pa {
 namespace {
+
+using namespace dec;
 
 // Tunables (compile-time): ring of K/V stages per CTA and the CTAs per SM the
 // 4-consumer-warp variant is register-limited to.
@@ -77,13 +80,11 @@ struct DecodeCfg {
   static_assert(BS % CHUNK == 0, "block size must be a multiple of 16");
 };
 
-__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
-
 // Dynamic shared-memory layout; depends on the launch (sequences in this
 // launch, consumer warps, group size), computed identically on host and device.
 template <typename C>
 struct Layout {
-  int ring, qbuf, full, empty, qfull, qempty, bad, misc, len, q0, ql, prefix, scan, p, merge, bytes;
+  int ring, qbuf, full, empty, qfull, qempty, bad, misc, batch, p, merge, bytes;
   int qbytes;  // bytes of one item's query rows (GROUP heads)
   __host__ __device__ Layout(int n, int ncw, int group) {
     constexpr int D = C::LPR * C::ELEMS;
@@ -96,80 +97,12 @@ struct Layout {
     qempty = qfull + 16;
     bad = qempty + 16;
     misc = align_up(bad + 4 * C::STAGES, 16);
-    len = misc + 16;
-    q0 = len + 4 * n;
-    ql = q0 + 4 * n;
-    prefix = ql + 4 * n;
-    scan = align_up(prefix + 4 * (n + 1), 16);
-    p = align_up(scan + 4 * 32, 128);
+    batch = misc + 16;
+    p = align_up(batch + BatchSmem::bytes(n), 128);
     merge = align_up(p + ncw * 16 * 4 * 4, 128);
     bytes = merge + ncw * 4 * (D + 4) * 4;
   }
 };
-
-__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
-
-// Work items contributed by a sequence: its splits for a decode sequence (one
-// query row); for a chunk of Q > 1 rows, Q single-row items in row mode and
-// none otherwise (the chunk kernel takes them).  len/q0/qlen come from the
-// shared-memory copies made in the prologue.
-__device__ __forceinline__ int seq_items(const AttnArgs &a, int L, int qlen) {
-  if (qlen <= 0) return 0;
-  if (qlen > 1) return a.rows_mode ? qlen : 0;
-  if (L <= 0 || L > a.max_context_len) return 1;  // zero-output item
-  return ceil_div(ceil_div(L, a.block_size), a.split_blocks);
-}
-
-struct Item {
-  int seq;     // global sequence index
-  int qrow;    // query row (token index into q / out)
-  int split;
-  int nsplit;
-  int kvh;
-  int b0, b1;  // KV blocks [b0, b1) of the sequence
-  int L;       // keys visible to the row
-  unsigned int bad_bits;  // PA_DEVERR_* of an invalid sequence (0: ok)
-};
-
-__device__ __forceinline__ Item decode_item(const AttnArgs &a, const int *prefix,
-                                            const int *s_len, const int *s_q0, const int *s_ql,
-                                            int n, int w) {
-  Item it;
-  const int f = w / a.num_kv_heads;
-  it.kvh = w - f * a.num_kv_heads;
-  int lo = 0, hi = n;  // find s with prefix[s] <= f < prefix[s+1]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (prefix[mid] <= f) lo = mid; else hi = mid;
-  }
-  it.seq = a.seq_begin + lo;
-  const int L = s_len[lo];
-  const int q0 = s_q0[lo];
-  const int qlen = s_ql[lo];
-  it.bad_bits = 0;
-  if (L < 0 || L > a.max_context_len) it.bad_bits = PA_DEVERR_CONTEXT_LEN;
-  else if (qlen > L && L > 0) it.bad_bits = PA_DEVERR_QUERY_LEN;
-  if (qlen > 1) {  // row mode: one item per query row, never split
-    const int t = f - prefix[lo];
-    it.qrow = q0 + t;
-    it.split = 0;
-    it.nsplit = 1;
-    it.L = L - qlen + t + 1;
-  } else {
-    it.qrow = q0;
-    it.split = f - prefix[lo];
-    it.nsplit = prefix[lo + 1] - prefix[lo];
-    it.L = L;
-  }
-  if (it.bad_bits || it.L <= 0) {
-    it.b0 = it.b1 = 0;
-  } else {
-    const int nblk = ceil_div(it.L, a.block_size);
-    it.b0 = qlen > 1 ? 0 : it.split * a.split_blocks;
-    it.b1 = qlen > 1 ? nblk : min(nblk, it.b0 + a.split_blocks);
-  }
-  return it;
-}
 
 template <int NV, int LPR>
 __device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
@@ -194,29 +127,6 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
   }
 }
 
-template <typename T>
-__device__ __forceinline__ void store4(T *dst, float4 v);
-template <>
-__device__ __forceinline__ void store4<float>(float *dst, float4 v) {
-  *reinterpret_cast<float4 *>(dst) = v;
-}
-template <>
-__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *dst, float4 v) {
-  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-  uint2 u;
-  u.x = *reinterpret_cast<uint32_t *>(&lo);
-  u.y = *reinterpret_cast<uint32_t *>(&hi);
-  *reinterpret_cast<uint2 *>(dst) = u;
-}
-template <>
-__device__ __forceinline__ void store4<__half>(__half *dst, float4 v) {
-  __half2 lo = __floats2half2_rn(v.x, v.y), hi = __floats2half2_rn(v.z, v.w);
-  uint2 u;
-  u.x = *reinterpret_cast<uint32_t *>(&lo);
-  u.y = *reinterpret_cast<uint32_t *>(&hi);
-  *reinterpret_cast<uint2 *>(dst) = u;
-}
-
 // MAXW = most consumer warps a launch of this variant uses (4: three CTAs per
 // SM fit; 8: the wide variant for large head groups).
 template <typename T, int D, int BS, int GW, int MAXW>
@@ -232,11 +142,8 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
   uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + lay.qempty);
   int *bad = reinterpret_cast<int *>(smem + lay.bad);
   volatile int *abort_flag = reinterpret_cast<int *>(smem + lay.misc);
-  int *s_len = reinterpret_cast<int *>(smem + lay.len);
-  int *s_q0 = reinterpret_cast<int *>(smem + lay.q0);
-  int *s_ql = reinterpret_cast<int *>(smem + lay.ql);
-  int *prefix = reinterpret_cast<int *>(smem + lay.prefix);
-  int *scan = reinterpret_cast<int *>(smem + lay.scan);
+  BatchSmem bsm;
+  bsm.carve(smem + lay.batch, n);
   unsigned char *ring = smem + lay.ring;
   unsigned char *qbuf = smem + lay.qbuf;
 
@@ -258,62 +165,14 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
     *abort_flag = 0;
     mbar_init_fence();
   }
-  {
-    const int per = ceil_div(n, nthreads);
-    const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
-    int local = 0;
-    for (int s = s0; s < s1; ++s) {
-      const int gs = a.seq_begin + s;
-      int q0 = gs, q1 = gs + 1;
-      if (a.query_start_loc) {
-        q0 = a.query_start_loc[gs];
-        q1 = a.query_start_loc[gs + 1];
-        if (q0 < 0 || q1 < q0 || q1 > a.num_q_tokens) {  // rows outside q: no items
-          raise_error(a.err, PA_DEVERR_QUERY_LEN);
-          q1 = q0 = 0;
-        }
-      }
-      const int L = a.context_lens[gs];
-      s_len[s] = L;
-      s_q0[s] = q0;
-      s_ql[s] = q1 - q0;
-      local += seq_items(a, L, q1 - q0);
-    }
-    // block exclusive scan of `local`
-    int x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) scan[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      const int nw = nthreads >> 5;
-      int w = lane < nw ? scan[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      if (lane < nw) scan[lane] = w;  // inclusive warp totals
-    }
-    __syncthreads();
-    int run = (warp ? scan[warp - 1] : 0) + x - local;
-    for (int s = s0; s < s1; ++s) {
-      prefix[s] = run;
-      run += seq_items(a, s_len[s], s_ql[s]);
-    }
-    if (tid == nthreads - 1) prefix[n] = run;
-  }
-  __syncthreads();
-  const int total_items = prefix[n] * a.num_kv_heads;
+  scan_batch(a, bsm, n);
+  const int total_items = bsm.prefix[n] * a.num_kv_heads;
 
   if (warp == ncw) {
     // ======================= producer warp ===================================
     uint32_t it = 0, k = 0;
     for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
-      const Item item = decode_item(a, prefix, s_len, s_q0, s_ql, n, w);
+      const Item item = decode_item(a, bsm, n, w);
       // this item's query rows -> qbuf[k & 1]
       {
         const uint32_t qs = k & 1u;
@@ -392,7 +251,7 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
 
   uint32_t it_base = 0, k = 0;
   for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
-    const Item item = decode_item(a, prefix, s_len, s_q0, s_ql, n, w);
+    const Item item = decode_item(a, bsm, n, w);
     const int nblocks = item.b1 - item.b0;
 
     // q slice of this lane from the prefetched rows, pre-scaled by scale*log2(e)
@@ -620,49 +479,7 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
     named_sync(1, ncw * 32);
 
     // ---- merge the warps that worked on the same heads; write out ----------
-    {
-      const int D4 = D / 4;
-      const int total4 = a.group * D4;
-      const bool direct = item.nsplit == 1;
-      for (int idx = tid; idx < total4; idx += ncw * 32) {
-        const int hg = idx / D4;           // head within the group
-        const int d4 = idx - hg * D4;
-        const int hsub = hg / GW, h = hg - hsub * GW;
-        float M = -INFINITY;
-        bool anybad = false;
-        for (int b2 = 0; b2 < nbl; ++b2) {
-          const float *src = merge + (b2 * hsplit + hsub) * mstride + h * (D + 4);
-          M = fmaxf(M, src[D]);
-          anybad |= src[D + 2] != 0.f;
-        }
-        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-        float Lsum = 0.f;
-        for (int b2 = 0; b2 < nbl; ++b2) {
-          const float *src = merge + (b2 * hsplit + hsub) * mstride + h * (D + 4);
-          const float mb = src[D];
-          const float wgt = mb == -INFINITY ? 0.f : fast_exp2(mb - M);
-          Lsum += wgt * src[D + 1];
-          const float4 x = *reinterpret_cast<const float4 *>(src + d4 * 4);
-          o.x += wgt * x.x;
-          o.y += wgt * x.y;
-          o.z += wgt * x.z;
-          o.w += wgt * x.w;
-        }
-        const int head = item.kvh * a.group + hg;
-        if (direct) {
-          const float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
-          T *dst = static_cast<T *>(a.out) + ((int64_t)item.qrow * a.num_heads + head) * D + d4 * 4;
-          store4<T>(dst, make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv));
-        } else {
-          const int64_t pidx = ((int64_t)item.seq * a.num_heads + head) * a.max_splits + item.split;
-          *reinterpret_cast<float4 *>(a.part_o + pidx * D + d4 * 4) = o;
-          if (d4 == 0) {
-            a.part_ml[2 * pidx] = M;
-            a.part_ml[2 * pidx + 1] = anybad ? __int_as_float(0x7fc00000) : Lsum;
-          }
-        }
-      }
-    }
+    merge_store<T, D>(a, item, merge, mstride, GW, hsplit, nbl, ncw, tid);
     named_sync(1, ncw * 32);
   }
 }
@@ -797,6 +614,11 @@ cudaError_t launch_reduce_t(const AttnArgs &a, cudaStream_t stream) {
 int decode_max_seqs_per_launch() { return kMaxSeqsPerLaunch; }
 
 cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream) {
+  // 16-bit caches: tensor-core kernel unless PA_DECODE_KERNEL=simt asks for
+  // the CUDA-core one (kept for fp32, odd head groups and comparison).
+  const char *sel = getenv("PA_DECODE_KERNEL");
+  const bool want_simt = sel && strcmp(sel, "simt") == 0;
+  if (!want_simt && decode_mma_supported(a, dtype)) return launch_decode_mma(a, dtype, sm_count, stream);
   if (dtype == PA_F32) return dispatch_d<float>(a, sm_count, stream);
   if (dtype == PA_F16) return dispatch_d<__half>(a, sm_count, stream);
   return dispatch_d<__nv_bfloat16>(a, sm_count, stream);

@@ -1,0 +1,567 @@
+// decode_mma.cu -- paged decode attention on the tensor cores (16-bit caches).
+//
+// Why tensor cores here: with GQA, the GROUP query heads that share a KV head
+// all read every K/V element of the item, so the per-block products
+//     S^T[keys x heads] = K[keys x D] . Q^T[D x heads]
+//     O^T[D x heads]   += V^T[D x keys] . P^T[keys x heads]
+// are dense contractions of the loaded tile with a GROUP-wide operand.  Done
+// on the CUDA cores they cost ~1000 instructions per 16-key block (fp32 FMAs,
+// bf16 widening, cross-lane reductions) and the kernel is issue-bound well
+// below HBM speed; as mma.sync m16n8k16 (keys / head dims on M, the group's
+// heads on N) they take 24 MMAs and 16 ldmatrix per block and leave the
+// kernel bound by HBM, which is what decode is ("PagedAttention 实战",
+// section 先理解 KV Cache, Decode).  The operands are consumed straight from the
+// staged cache tiles; nothing is rearranged in memory to form them.
+//
+// Data movement: one producer warp per CTA walks each item's block table and,
+// per KV block, issues tensor-map TMA loads of the (block, kv-head) K and V
+// tiles (two 64-column boxes each at head_dim 128) with the 128-byte swizzle,
+// so that ldmatrix reads of 8 rows at one column are bank-conflict free.
+// Stages live in a shared-memory ring guarded by full/empty mbarriers.
+//
+// Softmax: online, base 2 (scale*log2 e applied to S in fp32).  P is rounded
+// to the cache type for the P.V product; for bf16 (8 significant bits) P is
+// split into hi + lo bf16 parts, two products, so P enters exact to ~2^-17.
+//
+// Work items, the batch scan and the final merge are shared with the
+// CUDA-core kernel (decode_common.cuh).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "decode_common.cuh"
+
+namespace pa {
+namespace {
+
+using namespace dec;
+
+#ifndef PA_MMA_RING_KB
+#define PA_MMA_RING_KB 48
+#endif
+#ifndef PA_MMA_MIN_CTAS
+#define PA_MMA_MIN_CTAS 3
+#endif
+#ifndef PA_MMA_WARPS
+#define PA_MMA_WARPS 4
+#endif
+
+constexpr int kMaxSeqsPerLaunch = 2048;
+
+template <typename T>
+struct MmaT;
+
+template <>
+struct MmaT<__nv_bfloat16> {
+  static constexpr bool kSplitP = true;
+  static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  __device__ __forceinline__ static uint16_t bits(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
+  }
+  __device__ __forceinline__ static float back(uint16_t u) {
+    return __uint_as_float(static_cast<uint32_t>(u) << 16);
+  }
+};
+
+template <>
+struct MmaT<__half> {
+  static constexpr bool kSplitP = false;
+  static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  __device__ __forceinline__ static void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  __device__ __forceinline__ static uint16_t bits(float x) {
+    __half h = __float2half_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
+  }
+  __device__ __forceinline__ static float back(uint16_t u) {
+    return __half2float(*reinterpret_cast<__half *>(&u));
+  }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// A staged tile is BS rows x D columns of 16-bit values held as D/64 boxes of
+// BS rows x 128 bytes, each written by TMA with the 128-byte swizzle: the
+// 16-byte chunk c of row r sits at chunk position c ^ (r % 8).  Box bases are
+// 1024-byte aligned.  Byte address of the 8-element group (r, c8*8):
+template <int BS>
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int r, int c8) {
+  const int box = c8 >> 3, chunk = c8 & 7;
+  return tile + box * (BS * 128) + r * 128 + ((chunk ^ (r & 7)) << 4);
+}
+
+template <int D, int BS, int NT, int NCW>
+struct MmaLayout {
+  static constexpr int kTile = BS * D * 2;   // bytes of one (block, kv-head) K or V tile
+  static constexpr int kStage = 2 * kTile;
+  static constexpr int kStages = (PA_MMA_RING_KB * 1024) / kStage < 2 ? 2 : (PA_MMA_RING_KB * 1024) / kStage;
+  static constexpr int kHeads = 8 * NT;      // heads per warp (padded group)
+  static constexpr int kPbuf = NT * 2 * 8 * 16 * 2;  // per warp: P^T hi+lo [nt][8 heads][16 keys]
+  int ring, qbuf, full, empty, qfull, qempty, bad, misc, batch, pbuf, merge, bytes, qbytes;
+  // merge area: [warp][group heads][D + 4] floats
+  __host__ __device__ MmaLayout(int n, int group) {
+    qbytes = group * D * 2;
+    ring = 0;  // relative to a 1024-byte aligned base
+    qbuf = ring + kStages * kStage;
+    full = align_up(qbuf + 2 * qbytes, 128);
+    empty = full + 8 * kStages;
+    qfull = empty + 8 * kStages;
+    qempty = qfull + 16;
+    bad = qempty + 16;
+    misc = align_up(bad + 4 * kStages, 16);
+    batch = misc + 16;
+    pbuf = align_up(batch + BatchSmem::bytes(n), 128);
+    merge = align_up(pbuf + NCW * kPbuf, 128);
+    bytes = merge + NCW * group * (D + 4) * 4 + 1024;  // + alignment slack
+  }
+};
+
+template <typename T, int D, int BS, int NT, int NCW>
+__global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
+    paged_decode_mma_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv) {
+  using L = MmaLayout<D, BS, NT, NCW>;
+  constexpr int KS = D / 16;    // k-steps of the QK product (head dim)
+  constexpr int MT = D / 16;    // m-tiles of the PV product (head dim)
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int n = a.num_seqs;
+  const L lay(n, a.group);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.full);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + lay.empty);
+  uint64_t *qfull = reinterpret_cast<uint64_t *>(smem + lay.qfull);
+  uint64_t *qempty = reinterpret_cast<uint64_t *>(smem + lay.qempty);
+  int *bad = reinterpret_cast<int *>(smem + lay.bad);
+  volatile int *abort_flag = reinterpret_cast<int *>(smem + lay.misc);
+  BatchSmem bsm;
+  bsm.carve(smem + lay.batch, n);
+  const uint32_t ring = smem_addr(smem + lay.ring);
+  unsigned char *qbuf = smem + lay.qbuf;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qempty[s], NCW);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  scan_batch(a, bsm, n);
+  const int total_items = bsm.prefix[n] * a.num_kv_heads;
+
+  if (warp == NCW) {
+    // ======================= producer warp ===================================
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+    }
+    uint32_t it = 0, k = 0;
+    for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
+      const Item item = decode_item(a, bsm, n, w);
+      {  // the item's GROUP query rows -> qbuf[k & 1]
+        const uint32_t qs = k & 1u;
+        bool ok = !*abort_flag;
+        if (ok) ok = mbar_wait(&qempty[qs], ((k >> 1) & 1u) ^ 1u);
+        if (lane == 0) {
+          if (!ok) {
+            if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            mbar_arrive(&qfull[qs]);
+          } else {
+            mbar_arrive_expect_tx(&qfull[qs], lay.qbytes);
+            bulk_load(qbuf + qs * lay.qbytes,
+                      static_cast<const T *>(a.q) +
+                          ((int64_t)item.qrow * a.num_heads + item.kvh * a.group) * D,
+                      lay.qbytes, &qfull[qs]);
+          }
+        }
+        __syncwarp();
+      }
+      const int32_t *table = a.block_tables + (int64_t)item.seq * a.max_blocks_per_seq;
+      for (int b = item.b0; b < item.b1; b += 32) {
+        const int cnt = min(32, item.b1 - b);
+        const int my_id = lane < cnt ? table[b + lane] : 0;
+        for (int j = 0; j < cnt; ++j) {
+          const int pb = __shfl_sync(0xffffffffu, my_id, j);
+          const uint32_t slot = it % L::kStages;
+          const uint32_t par = ((it / L::kStages) & 1u) ^ 1u;
+          ++it;
+          bool ok = !*abort_flag;
+          if (ok) ok = mbar_wait(&empty[slot], par);
+          if (lane == 0) {
+            if (!ok) {
+              if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+              *abort_flag = 1;
+              bad[slot] = 1;
+              mbar_arrive(&full[slot]);
+            } else if (pb < 0 || pb >= a.num_blocks) {
+              raise_error(a.err, PA_DEVERR_BLOCK_ID);
+              bad[slot] = 1;
+              mbar_arrive(&full[slot]);
+            } else {
+              bad[slot] = 0;
+              const int row = (pb * a.num_kv_heads + item.kvh) * BS;
+              const uint32_t dst = ring + slot * L::kStage;
+              mbar_arrive_expect_tx(&full[slot], L::kStage);
+#pragma unroll
+              for (int bx = 0; bx < D / 64; ++bx) {
+                tma_load_2d(dst + bx * (BS * 128), &tmk, bx * 64, row, &full[slot]);
+                tma_load_2d(dst + L::kTile + bx * (BS * 128), &tmv, bx * 64, row, &full[slot]);
+              }
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+    return;
+  }
+
+  // ======================= consumer warps ==================================
+  const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
+  unsigned char *pbuf = smem + lay.pbuf + warp * L::kPbuf;  // [nt][hi|lo][8 heads][16 keys] 16-bit
+  float *merge = reinterpret_cast<float *>(smem + lay.merge);
+  const int mstride = a.group * (D + 4);
+  const float sl2 = a.scale_log2;
+
+  uint32_t it_base = 0, k = 0;
+  for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
+    const Item item = decode_item(a, bsm, n, w);
+    const int nblocks = item.b1 - item.b0;
+
+    // q as the B operand of S^T = K Q^T: b0 = Q[head][16ks+2t..], b1 = +8
+    uint32_t qb[NT][KS][2];
+    {
+      const uint32_t qs = k & 1u;
+      bool ok = !*abort_flag;
+      if (ok) {
+        ok = mbar_wait(&qfull[qs], (k >> 1) & 1u);
+        if (!ok && lane == 0) {
+          if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+      }
+      const uint16_t *qr = reinterpret_cast<const uint16_t *>(qbuf + qs * lay.qbytes);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int head = nt * 8 + g;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          if (head < a.group) {
+            qb[nt][ks][0] = *reinterpret_cast<const uint32_t *>(qr + head * D + ks * 16 + 2 * t);
+            qb[nt][ks][1] = *reinterpret_cast<const uint32_t *>(qr + head * D + ks * 16 + 8 + 2 * t);
+          } else {
+            qb[nt][ks][0] = qb[nt][ks][1] = 0u;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qempty[qs]);
+    }
+
+    float o[NT][MT][4];
+    float m[NT][2], l[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+    }
+    bool item_bad = item.bad_bits != 0;
+    if (item.bad_bits && tid == 0 && item.kvh == 0) raise_error(a.err, item.bad_bits);
+
+    // Every consumer warp waits for and releases every stage in ring order
+    // (no parity wait is ever more than one phase ahead of its barrier) but
+    // computes only the blocks j = warp, warp + NCW, ... of the item.
+    auto wait_stage = [&](uint32_t itn) -> bool {
+      const uint32_t slot = itn % L::kStages;
+      bool ok = !*abort_flag;
+      if (ok) {
+        ok = mbar_wait(&full[slot], (itn / L::kStages) & 1u);
+        if (!ok && lane == 0) {
+          if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
+        }
+      }
+      return ok && !bad[slot];
+    };
+    auto release_stage = [&](uint32_t itn) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[itn % L::kStages]);
+    };
+    int next = 0;
+    for (int j = warp; j < nblocks; j += NCW) {
+      for (; next < j; ++next) {
+        wait_stage(it_base + next);
+        release_stage(it_base + next);
+      }
+      next = j + 1;
+      const uint32_t itn = it_base + j;
+      if (!wait_stage(itn)) {
+        item_bad = true;
+      } else {
+        const int nvalid = min(BS, item.L - (item.b0 + j) * BS);
+        const uint32_t ktile = ring + (itn % L::kStages) * L::kStage;
+        const uint32_t vtile = ktile + L::kTile;
+#pragma unroll
+        for (int r0 = 0; r0 < BS; r0 += 16) {
+          if (r0 < nvalid) {
+            // ---- S^T = K Q^T over this 16-key sub-tile ----
+            float s[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+            {
+              const int mi = lane >> 3;
+              const int kr = r0 + (lane & 7) + (mi & 1) * 8;
+#pragma unroll
+              for (int ks = 0; ks < KS; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(af, swz<BS>(ktile, kr, ks * 2 + (mi >> 1)));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) MmaT<T>::mma(s[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+              }
+            }
+            // ---- online softmax: thread holds keys r0+g, r0+g+8 of heads 2t, 2t+1 ----
+            const bool v0 = r0 + g < nvalid, v1 = r0 + g + 8 < nvalid;
+            uint32_t pb_hi[NT][2], pb_lo[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              float p[4];
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const float x0 = v0 ? s[nt][hh] * sl2 : -INFINITY;
+                const float x1 = v1 ? s[nt][2 + hh] * sl2 : -INFINITY;
+                float mx = fmaxf(x0, x1);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mn = fmaxf(m[nt][hh], mx);
+                const float alpha = fast_exp2(m[nt][hh] - mn);
+                m[nt][hh] = mn;
+                p[hh] = fast_exp2(x0 - mn);
+                p[2 + hh] = fast_exp2(x1 - mn);
+                l[nt][hh] = l[nt][hh] * alpha + p[hh] + p[2 + hh];
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                  o[nt][mt][hh] *= alpha;
+                  o[nt][mt][2 + hh] *= alpha;
+                }
+              }
+              // P^T via shared memory: P[head][key] 16-bit, rows of 16 keys
+              uint16_t *ph = reinterpret_cast<uint16_t *>(pbuf) + nt * 2 * 128;
+              uint16_t *pl = ph + 128;
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int head = 2 * t + (c & 1), key = g + (c >> 1) * 8;
+                const uint16_t hi = MmaT<T>::bits(p[c]);
+                ph[head * 16 + key] = hi;
+                if constexpr (MmaT<T>::kSplitP) pl[head * 16 + key] = MmaT<T>::bits(p[c] - MmaT<T>::back(hi));
+              }
+              __syncwarp();
+              pb_hi[nt][0] = *reinterpret_cast<const uint32_t *>(ph + g * 16 + 2 * t);
+              pb_hi[nt][1] = *reinterpret_cast<const uint32_t *>(ph + g * 16 + 8 + 2 * t);
+              if constexpr (MmaT<T>::kSplitP) {
+                pb_lo[nt][0] = *reinterpret_cast<const uint32_t *>(pl + g * 16 + 2 * t);
+                pb_lo[nt][1] = *reinterpret_cast<const uint32_t *>(pl + g * 16 + 8 + 2 * t);
+              }
+              __syncwarp();
+            }
+            // ---- rows past the context end may hold anything (even NaN):
+            //      zero them in the staged V tile, as P is 0 there ----
+            if (r0 + 16 > nvalid) {
+              const int z0 = nvalid;
+              const int nz = (r0 + 16 - z0) * (D / 8);
+              for (int c = lane; c < nz; c += 32) {
+                const int r = z0 + c / (D / 8), ch = c % (D / 8);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(swz<BS>(vtile, r, ch)),
+                             "r"(0u)
+                             : "memory");
+              }
+              fence_proxy_async_smem();  // before the next TMA write of this stage
+              __syncwarp();
+            }
+            // ---- O^T += V^T P^T ----
+            {
+              const int mi = lane >> 3;
+              const int vr = r0 + (lane & 7) + (mi >> 1) * 8;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                uint32_t af[4];
+                ldsm_x4_t(af, swz<BS>(vtile, vr, mt * 2 + (mi & 1)));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  MmaT<T>::mma(o[nt][mt], af, pb_hi[nt][0], pb_hi[nt][1]);
+                  if constexpr (MmaT<T>::kSplitP) MmaT<T>::mma(o[nt][mt], af, pb_lo[nt][0], pb_lo[nt][1]);
+                }
+              }
+            }
+          }
+        }
+      }
+      release_stage(itn);
+    }
+    for (; next < nblocks; ++next) {
+      wait_stage(it_base + next);
+      release_stage(it_base + next);
+    }
+    it_base += nblocks;
+
+    // ---- warp totals -> merge area [warp][head][D + 4] ----
+    float *mw = merge + warp * mstride;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float lt = l[nt][hh];
+        lt += __shfl_xor_sync(0xffffffffu, lt, 4);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+        const int head = nt * 8 + 2 * t + hh;
+        if (head < a.group) {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            mw[head * (D + 4) + mt * 16 + g] = o[nt][mt][hh];
+            mw[head * (D + 4) + mt * 16 + g + 8] = o[nt][mt][2 + hh];
+          }
+          if (g == 0) {
+            mw[head * (D + 4) + D] = m[nt][hh];
+            mw[head * (D + 4) + D + 1] = lt;
+            mw[head * (D + 4) + D + 2] = item_bad ? 1.f : 0.f;
+          }
+        }
+      }
+    }
+    named_sync(1, NCW * 32);
+    merge_store<T, D>(a, item, merge, mstride, a.group, 1, NCW, NCW, tid);
+    named_sync(1, NCW * 32);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D view of a cache: rows = num_blocks * num_kv_heads * block_size, columns
+// = head_dim; boxes of 64 columns x block_size rows, 128-byte swizzle.
+template <typename T, int D, int BS>
+bool make_map(CUtensorMap *map, const void *base, int num_blocks, int num_kv_heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)num_blocks * num_kv_heads * BS};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)BS};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, MmaT<T>::kTmaType, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int BS, int NT>
+cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
+  constexpr int NCW = PA_MMA_WARPS;
+  using L = MmaLayout<D, BS, NT, NCW>;
+  auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW>;
+  CUtensorMap tmk, tmv;
+  if (!make_map<T, D, BS>(&tmk, a.k_cache, a.num_blocks, a.num_kv_heads) ||
+      !make_map<T, D, BS>(&tmv, a.v_cache, a.num_blocks, a.num_kv_heads))
+    return cudaErrorInvalidValue;
+  const L lay(a.num_seqs, a.group);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    const L big(kMaxSeqsPerLaunch, 8 * NT);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, big.bytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1), lay.bytes);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  const int64_t max_items = (int64_t)a.num_seqs * a.num_kv_heads *
+                            (a.rows_mode ? (a.max_splits > a.max_query_len ? a.max_splits : a.max_query_len)
+                                         : a.max_splits);
+  int64_t grid = (int64_t)sm_count * occ;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, 32 * (NCW + 1), lay.bytes, stream>>>(a, tmk, tmv);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int BS>
+cudaError_t mma_nt(const AttnArgs &a, int sm_count, cudaStream_t s) {
+  return a.group <= 8 ? launch_mma_t<T, D, BS, 1>(a, sm_count, s)
+                      : launch_mma_t<T, D, BS, 2>(a, sm_count, s);
+}
+
+template <typename T, int D>
+cudaError_t mma_bs(const AttnArgs &a, int sm_count, cudaStream_t s) {
+  return a.block_size == 16 ? mma_nt<T, D, 16>(a, sm_count, s) : mma_nt<T, D, 32>(a, sm_count, s);
+}
+
+template <typename T>
+cudaError_t mma_d(const AttnArgs &a, int sm_count, cudaStream_t s) {
+  return a.head_dim == 64 ? mma_bs<T, 64>(a, sm_count, s) : mma_bs<T, 128>(a, sm_count, s);
+}
+
+}  // namespace
+
+bool decode_mma_supported(const AttnArgs &a, int dtype) {
+  return (dtype == PA_F16 || dtype == PA_BF16) && a.group >= 1 && a.group <= 16 &&
+         encode_fn() != nullptr;
+}
+
+cudaError_t launch_decode_mma(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream) {
+  if (dtype == PA_F16) return mma_d<__half>(a, sm_count, stream);
+  return mma_d<__nv_bfloat16>(a, sm_count, stream);
+}
+
+}  // namespace pa

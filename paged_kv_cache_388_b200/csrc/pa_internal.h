@@ -50,6 +50,10 @@ cudaError_t device_info(DevInfo *info);
 void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
                   int kv_split_tokens, int sm_count, int *split_blocks, int *max_splits);
 
+// Implemented in decode_mma.cu (tensor-core decode for 16-bit caches)
+bool decode_mma_supported(const AttnArgs &a, int dtype);
+cudaError_t launch_decode_mma(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream);
+
 // Implemented in decode.cu
 cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnArgs &a, int dtype, cudaStream_t stream);

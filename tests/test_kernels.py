@@ -36,9 +36,20 @@ def _check_workload(lib, wl, kv_split_tokens=0, rows=None):
     return out, ref, err
 
 
+@pytest.fixture(params=["auto", "simt"])
+def decode_kernel(request, monkeypatch):
+    """Run with the library's default decode kernel (tensor cores for 16-bit
+    caches) and with the CUDA-core kernel forced."""
+    if request.param == "simt":
+        monkeypatch.setenv("PA_DECODE_KERNEL", "simt")
+    else:
+        monkeypatch.delenv("PA_DECODE_KERNEL", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("split", [0, 32, 1 << 20], ids=["policy", "split32", "nosplit"])
 @pytest.mark.parametrize("cfg", workloads.SMALL_CONFIGS)
-def test_small_config_parity(lib, cfg, split):
+def test_small_config_parity(lib, cfg, split, decode_kernel):
     _check_workload(lib, workloads.make(cfg), kv_split_tokens=split)
 
 
@@ -65,7 +76,7 @@ def test_full_config_sampled(lib, cfg):
     _check_workload(lib, wl, rows=rows)
 
 
-def test_split_agrees_with_nosplit(lib):
+def test_split_agrees_with_nosplit(lib, decode_kernel):
     wl = workloads.make("3s")
     vals = workloads.values(wl)
     batch = build_batch(wl)
@@ -83,7 +94,7 @@ def test_split_agrees_with_nosplit(lib):
 @pytest.mark.parametrize("H,Hk,D,dtype", [(32, 8, 128, "bf16"), (8, 4, 64, "f16"),
                                           (32, 2, 128, "bf16"), (4, 4, 64, "f32"),
                                           (16, 2, 64, "f32")])
-def test_edge_lengths(lib, H, Hk, D, dtype, bs):
+def test_edge_lengths(lib, H, Hk, D, dtype, bs, decode_kernel):
     lens = [0, 1, 15, 16, 17, 31, 32, 33, 513, 4096]
     wl = workloads.decode_workload(f"edge_{H}_{Hk}_{D}_{dtype}_{bs}", 3100, lens, H, Hk, D, bs, dtype)
     out, ref, _ = _check_workload(lib, wl, kv_split_tokens=64)
@@ -93,7 +104,7 @@ def test_edge_lengths(lib, H, Hk, D, dtype, bs):
 
 @pytest.mark.parametrize("dtype,D,bs", [("bf16", 128, 16), ("f16", 64, 32), ("f32", 64, 16),
                                         ("bf16", 64, 32)])
-def test_chunked_rows(lib, dtype, D, bs):
+def test_chunked_rows(lib, dtype, D, bs, decode_kernel):
     wl = workloads.mixed_workload(f"chunk_{dtype}_{D}_{bs}", 3200, 2, 100, 900, 3, 150, 37,
                                   16, 4, D, bs, dtype)
     _check_workload(lib, wl)
@@ -122,7 +133,7 @@ def _tiny_decode(lib, lens=(20, 40), dtype=torch.bfloat16, bs=16):
     return kc, vc, q, bt, cl
 
 
-def test_bad_block_id_sets_error_and_zeroes_row(lib):
+def test_bad_block_id_sets_error_and_zeroes_row(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib)
     bt[1, 1] = 10_000
     out = torch.full_like(q, 7.0)
@@ -134,7 +145,7 @@ def test_bad_block_id_sets_error_and_zeroes_row(lib):
     assert lib.pa_get_device_error() == 0  # cleared
 
 
-def test_bad_block_id_split_path(lib):
+def test_bad_block_id_split_path(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib, lens=(20, 60))
     bt[1, 3] = -5
     ws = torch.empty(lib.pa_decode_workspace_size(2, 8, 2, 128, 16, 64, 16), dtype=torch.uint8,
@@ -145,7 +156,7 @@ def test_bad_block_id_split_path(lib):
     assert torch.count_nonzero(out[1]) == 0
 
 
-def test_bad_context_len(lib):
+def test_bad_context_len(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib)
     cl[0] = 4 * 16 + 1  # beyond max_blocks_per_seq * block_size
     out = torch.full_like(q, 7.0)
@@ -224,3 +235,20 @@ def test_empty_calls_are_noops(lib):
     lib.pa_copy_blocks(kc, vc, torch.empty(0, 2, dtype=torch.int64, device="cuda"))
     assert torch.equal(kc, k0)
     assert lib.pa_get_device_error() == 0
+
+
+def test_nan_in_unused_slots_does_not_leak(lib, decode_kernel):
+    """Slots past a sequence's length may hold anything; NaN there must not
+    reach the output."""
+    kc, vc, q, bt, cl = _tiny_decode(lib, lens=(20, 37))
+    nan = torch.tensor(float("nan"), dtype=kc.dtype, device="cuda")
+    ref_out = torch.empty_like(q)
+    lib.pa_decode(ref_out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20)
+    kc[bt[0, 1], :, 4:] = nan  # seq 0: tokens 20.. of block 1 are unused
+    vc[bt[0, 1], :, 4:] = nan
+    kc[bt[1, 2], :, 5:] = nan  # seq 1: tokens 37.. of block 2
+    vc[bt[1, 2], :, 5:] = nan
+    out = torch.empty_like(q)
+    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20)
+    assert lib.pa_get_device_error() == 0
+    assert torch.equal(out, ref_out)
