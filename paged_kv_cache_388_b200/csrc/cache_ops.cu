@@ -16,6 +16,11 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4 *__restrict__ key, const uint4 *__restrict__ value, uint4 *__restrict__ k_cache,
     uint4 *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping, int num_tokens,
     int num_kv_heads, int vpr, int block_size, int64_t num_slots, unsigned int *err) {
+  // Launched as a programmatic dependent of the previous kernel: wait for its
+  // writes before touching memory; then let the next grid (the decode kernel)
+  // be scheduled -- it waits for this grid's writes before reading the cache.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t per_token = (int64_t)num_kv_heads * vpr;
   const int64_t total = (int64_t)num_tokens * per_token;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
@@ -47,6 +52,7 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ k_
                                                           const int64_t *__restrict__ mapping,
                                                           int64_t blk_vecs, int num_blocks,
                                                           unsigned int *err) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int pair = blockIdx.x;
   uint4 *base = blockIdx.y ? v_cache : k_cache;
   const int64_t src = mapping[2 * (int64_t)pair];
@@ -83,11 +89,19 @@ cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  reshape_and_cache_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-      static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
-      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), slot_mapping, num_tokens,
-      num_kv_heads, vpr, block_size, (int64_t)num_blocks * block_size, err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, reshape_and_cache_kernel, static_cast<const uint4 *>(key),
+                            static_cast<const uint4 *>(value), static_cast<uint4 *>(k_cache),
+                            static_cast<uint4 *>(v_cache), slot_mapping, num_tokens, num_kv_heads,
+                            vpr, block_size, (int64_t)num_blocks * block_size, err);
 }
 
 cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping,

@@ -479,7 +479,13 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
     named_sync(1, ncw * 32);
 
     // ---- merge the warps that worked on the same heads; write out ----------
-    merge_store<T, D>(a, item, merge, mstride, GW, hsplit, nbl, ncw, tid);
+    {
+      Seg seg;
+      seg.it = item;
+      seg.out = item.nsplit == 1 ? kOutDirect : kOutSplit;
+      seg.index = item.split;
+      merge_store<T, D>(a, seg, merge, mstride, GW, hsplit, nbl, ncw, tid);
+    }
     named_sync(1, ncw * 32);
   }
 }
@@ -614,11 +620,6 @@ cudaError_t launch_reduce_t(const AttnArgs &a, cudaStream_t stream) {
 int decode_max_seqs_per_launch() { return kMaxSeqsPerLaunch; }
 
 cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream) {
-  // 16-bit caches: tensor-core kernel unless PA_DECODE_KERNEL=simt asks for
-  // the CUDA-core one (kept for fp32, odd head groups and comparison).
-  const char *sel = getenv("PA_DECODE_KERNEL");
-  const bool want_simt = sel && strcmp(sel, "simt") == 0;
-  if (!want_simt && decode_mma_supported(a, dtype)) return launch_decode_mma(a, dtype, sm_count, stream);
   if (dtype == PA_F32) return dispatch_d<float>(a, sm_count, stream);
   if (dtype == PA_F16) return dispatch_d<__half>(a, sm_count, stream);
   return dispatch_d<__nv_bfloat16>(a, sm_count, stream);

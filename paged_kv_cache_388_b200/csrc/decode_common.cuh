@@ -60,7 +60,17 @@ struct BatchSmem {
   }
 };
 
-// Called by every thread of the CTA; ends with __syncthreads().
+// KV blocks of a decode sequence (one query row, valid length), else 0: the
+// unit of the balanced partition.
+__device__ __forceinline__ int unit_blocks(const AttnArgs &a, int L, int qlen) {
+  if (qlen != 1 || L <= 0 || L > a.max_context_len) return 0;
+  return ceil_div(L, a.block_size);
+}
+
+// Called by every thread of the CTA; ends with __syncthreads().  prefix[s]
+// counts items (BAL = false) or KV blocks per KV head (BAL = true) of the
+// sequences before s.
+template <bool BAL = false>
 __device__ __forceinline__ void scan_batch(const AttnArgs &a, const BatchSmem &b, int n) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
   const int per = ceil_div(n, nthreads);
@@ -81,7 +91,7 @@ __device__ __forceinline__ void scan_batch(const AttnArgs &a, const BatchSmem &b
     b.len[s] = L;
     b.q0[s] = q0;
     b.ql[s] = q1 - q0;
-    local += seq_items(a, L, q1 - q0);
+    local += BAL ? unit_blocks(a, L, q1 - q0) : seq_items(a, L, q1 - q0);
   }
   int x = local;  // block exclusive scan of `local`
 #pragma unroll
@@ -105,7 +115,7 @@ __device__ __forceinline__ void scan_batch(const AttnArgs &a, const BatchSmem &b
   int run = (warp ? b.scan[warp - 1] : 0) + x - local;
   for (int s = s0; s < s1; ++s) {
     b.prefix[s] = run;
-    run += seq_items(a, b.len[s], b.ql[s]);
+    run += BAL ? unit_blocks(a, b.len[s], b.ql[s]) : seq_items(a, b.len[s], b.ql[s]);
   }
   if (tid == nthreads - 1) b.prefix[n] = run;
   __syncthreads();
@@ -149,6 +159,96 @@ __device__ __forceinline__ Item decode_item(const AttnArgs &a, const BatchSmem &
   return it;
 }
 
+// ---------------------------------------------------------------------------
+// Balanced partition.  The work of the launch is the concatenation, over
+// decode sequences s and then KV heads, of each (s, kvh) pair's KV blocks:
+// W = sum_s blocks(s) * Hk blocks.  CTA i of G takes the flat range
+// [i*W/G, (i+1)*W/G), so every CTA moves the same number of bytes (+-1 block)
+// whatever the length mix.  A pair wholly inside one CTA's range is finished
+// there (written to `out`); a pair cut by range boundaries leaves one partial
+// (m, l, acc) record per covering CTA -- a CTA cuts at most its first and its
+// last segment -- and balanced_reduce_kernel merges them.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t bal_start(int i, int64_t W, int G) {
+  return (int64_t)i * W / G;
+}
+
+// Largest i with bal_start(i) <= pos (pos < W).
+__device__ __forceinline__ int bal_owner(int64_t pos, int64_t W, int G) {
+  int i = (int)(pos * G / W);
+  if (i >= G) i = G - 1;
+  while (i + 1 < G && bal_start(i + 1, W, G) <= pos) ++i;
+  while (i > 0 && bal_start(i, W, G) > pos) --i;
+  return i;
+}
+
+// Output of a segment: direct to `out`, a fixed-split partial (index = split)
+// or a balanced-partition record (index = 0 first / 1 last segment of the CTA).
+enum SegOut { kOutDirect = 0, kOutSplit = 1, kOutRecord = 2 };
+
+struct Seg {
+  Item it;      // seq, qrow, kvh, b0, b1, L, bad_bits (+ split for kOutSplit)
+  int out;      // SegOut
+  int index;
+};
+
+// Iterates the segments of this CTA in either scheme; producer and consumer
+// warps call it in lock step and see the same sequence.
+struct SegIter {
+  int w;             // fixed scheme: next item
+  int64_t pos, end;  // balanced scheme: flat block range still to do
+  bool first;
+  __device__ void init(const AttnArgs &a, const BatchSmem &b, int n) {
+    w = blockIdx.x;
+    if (a.balanced) {
+      const int64_t W = (int64_t)b.prefix[n] * a.num_kv_heads;
+      pos = bal_start(blockIdx.x, W, gridDim.x);
+      end = bal_start(blockIdx.x + 1, W, gridDim.x);
+      first = true;
+    }
+  }
+  __device__ bool next(const AttnArgs &a, const BatchSmem &b, int n, Seg *seg) {
+    if (!a.balanced) {
+      if (w >= b.prefix[n] * a.num_kv_heads) return false;
+      seg->it = decode_item(a, b, n, w);
+      seg->out = seg->it.nsplit == 1 ? kOutDirect : kOutSplit;
+      seg->index = seg->it.split;
+      w += gridDim.x;
+      return true;
+    }
+    if (pos >= end) return false;
+    // sequence s holding flat position pos: prefix[s]*Hk <= pos < prefix[s+1]*Hk
+    const int Hk = a.num_kv_heads;
+    int lo = 0, hi = n;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((int64_t)b.prefix[mid] * Hk <= pos) lo = mid; else hi = mid;
+    }
+    const int nb = b.prefix[lo + 1] - b.prefix[lo];  // > 0: empty sequences own no range
+    const int64_t off = pos - (int64_t)b.prefix[lo] * Hk;
+    const int kvh = (int)(off / nb);
+    const int b0 = (int)(off - (int64_t)kvh * nb);
+    const int64_t left = end - pos;
+    const int b1 = left < nb - b0 ? b0 + (int)left : nb;
+    Item &it = seg->it;
+    it.seq = a.seq_begin + lo;
+    it.qrow = b.q0[lo];
+    it.split = 0;
+    it.nsplit = 1;
+    it.kvh = kvh;
+    it.b0 = b0;
+    it.b1 = b1;
+    it.L = b.len[lo];
+    it.bad_bits = 0;
+    const bool complete = b0 == 0 && b1 == nb;
+    seg->out = complete ? kOutDirect : kOutRecord;
+    seg->index = first ? 0 : 1;
+    first = false;
+    pos += b1 - b0;
+    return true;
+  }
+};
+
 template <typename T>
 __device__ __forceinline__ void store4(T *dst, float4 v);
 template <>
@@ -180,12 +280,12 @@ __device__ __forceinline__ void store4<__half>(__half *dst, float4 v) {
 // the blocks j = bl (mod nbl).  All consumer threads (ncw*32) call this;
 // direct items go to `out`, split items to the workspace.
 template <typename T, int D>
-__device__ __forceinline__ void merge_store(const AttnArgs &a, const Item &item,
+__device__ __forceinline__ void merge_store(const AttnArgs &a, const Seg &seg,
                                             const float *merge, int mstride, int gw,
                                             int hsplit, int nbl, int ncw, int tid) {
+  const Item &item = seg.it;
   constexpr int D4 = D / 4;
   const int total4 = a.group * D4;
-  const bool direct = item.nsplit == 1;
   for (int idx = tid; idx < total4; idx += ncw * 32) {
     const int hg = idx / D4;  // head within the group
     const int d4 = idx - hg * D4;
@@ -211,16 +311,25 @@ __device__ __forceinline__ void merge_store(const AttnArgs &a, const Item &item,
       o.w += wgt * x.w;
     }
     const int head = item.kvh * a.group + hg;
-    if (direct) {
+    if (seg.out == kOutDirect) {
       const float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
       T *dst = static_cast<T *>(a.out) + ((int64_t)item.qrow * a.num_heads + head) * D + d4 * 4;
       store4<T>(dst, make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv));
     } else {
-      const int64_t pidx = ((int64_t)item.seq * a.num_heads + head) * a.max_splits + item.split;
-      *reinterpret_cast<float4 *>(a.part_o + pidx * D + d4 * 4) = o;
+      float *po, *pml;
+      if (seg.out == kOutSplit) {
+        const int64_t pidx = ((int64_t)item.seq * a.num_heads + head) * a.max_splits + seg.index;
+        po = a.part_o + pidx * D;
+        pml = a.part_ml + 2 * pidx;
+      } else {  // record of this CTA: [cta][slot][group head][D + 4] (16-byte rows)
+        const int64_t ridx = ((int64_t)blockIdx.x * 2 + seg.index) * a.group + hg;
+        po = a.part_o + ridx * (D + 4);
+        pml = po + D;
+      }
+      *reinterpret_cast<float4 *>(po + d4 * 4) = o;
       if (d4 == 0) {
-        a.part_ml[2 * pidx] = M;
-        a.part_ml[2 * pidx + 1] = anybad ? __int_as_float(0x7fc00000) : Lsum;
+        pml[0] = M;
+        pml[1] = anybad ? __int_as_float(0x7fc00000) : Lsum;
       }
     }
   }

@@ -127,7 +127,6 @@ struct MmaLayout {
   static constexpr int kTile = BS * D * 2;   // bytes of one (block, kv-head) K or V tile
   static constexpr int kStage = 2 * kTile;
   static constexpr int kStages = (PA_MMA_RING_KB * 1024) / kStage < 2 ? 2 : (PA_MMA_RING_KB * 1024) / kStage;
-  static constexpr int kHeads = 8 * NT;      // heads per warp (padded group)
   static constexpr int kPbuf = NT * 2 * 8 * 16 * 2;  // per warp: P^T hi+lo [nt][8 heads][16 keys]
   int ring, qbuf, full, empty, qfull, qempty, bad, misc, batch, pbuf, merge, bytes, qbytes;
   // merge area: [warp][group heads][D + 4] floats
@@ -184,8 +183,31 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
     *abort_flag = 0;
     mbar_init_fence();
   }
-  scan_batch(a, bsm, n);
-  const int total_items = bsm.prefix[n] * a.num_kv_heads;
+  // Launched as a programmatic dependent of the previous kernel: nothing is
+  // read from global memory before that kernel's writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // ... and let the merge kernel that follows get scheduled while this runs.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (a.balanced && tid == 0) a.bal_desc[4 * blockIdx.x] = -1;  // no cut pair starts here (yet)
+  if (a.balanced) {
+    scan_batch<true>(a, bsm, n);
+    if (blockIdx.x == 0)  // block prefix for the merge kernel
+      for (int s = tid; s <= n; s += blockDim.x) a.bal_prefix[s] = bsm.prefix[s];
+    // Decode sequences with no KV blocks (empty or invalid context) own no
+    // part of the partition: their rows are written as zeros here.
+    if (warp < NCW) {
+      for (int s = blockIdx.x; s < n; s += gridDim.x) {
+        if (bsm.ql[s] != 1 || bsm.prefix[s + 1] != bsm.prefix[s]) continue;
+        const int L = bsm.len[s];
+        if (L != 0 && tid == 0) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
+        T *row = static_cast<T *>(a.out) + (int64_t)bsm.q0[s] * a.num_heads * D;
+        for (int i = tid; i < a.num_heads * D / 4; i += NCW * 32)
+          store4<T>(row + 4 * i, make_float4(0.f, 0.f, 0.f, 0.f));
+      }
+    }
+  } else {
+    scan_batch<false>(a, bsm, n);
+  }
 
   if (warp == NCW) {
     // ======================= producer warp ===================================
@@ -194,9 +216,12 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
     }
     uint32_t it = 0, k = 0;
-    for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
-      const Item item = decode_item(a, bsm, n, w);
-      {  // the item's GROUP query rows -> qbuf[k & 1]
+    SegIter iter;
+    iter.init(a, bsm, n);
+    Seg seg;
+    for (; iter.next(a, bsm, n, &seg); ++k) {
+      const Item &item = seg.it;
+      {  // the segment's GROUP query rows -> qbuf[k & 1]
         const uint32_t qs = k & 1u;
         bool ok = !*abort_flag;
         if (ok) ok = mbar_wait(&qempty[qs], ((k >> 1) & 1u) ^ 1u);
@@ -263,8 +288,11 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
   const float sl2 = a.scale_log2;
 
   uint32_t it_base = 0, k = 0;
-  for (int w = blockIdx.x; w < total_items; w += gridDim.x, ++k) {
-    const Item item = decode_item(a, bsm, n, w);
+  SegIter iter;
+  iter.init(a, bsm, n);
+  Seg seg;
+  for (; iter.next(a, bsm, n, &seg); ++k) {
+    const Item &item = seg.it;
     const int nblocks = item.b1 - item.b0;
 
     // q as the B operand of S^T = K Q^T: b0 = Q[head][16ks+2t..], b1 = +8
@@ -471,9 +499,72 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
       }
     }
     named_sync(1, NCW * 32);
-    merge_store<T, D>(a, item, merge, mstride, a.group, 1, NCW, NCW, tid);
+    merge_store<T, D>(a, seg, merge, mstride, a.group, 1, NCW, NCW, tid);
+    if (seg.out == kOutRecord && item.b0 == 0 && tid == 0) {
+      // This CTA holds the first piece of a pair cut at its range end: leave
+      // the merge kernel a descriptor {record slot, kv head, last covering
+      // CTA, query row}.
+      const int nb = ceil_div(item.L, a.block_size);
+      const int64_t W = (int64_t)bsm.prefix[n] * a.num_kv_heads;
+      const int64_t ps = (int64_t)bsm.prefix[item.seq - a.seq_begin] * a.num_kv_heads +
+                         (int64_t)item.kvh * nb;
+      int *d = a.bal_desc + 4 * blockIdx.x;
+      d[1] = item.kvh;
+      d[2] = bal_owner(ps + nb - 1, W, gridDim.x);
+      d[3] = item.qrow;
+      d[0] = seg.index;  // record slot of this piece in this CTA
+    }
     named_sync(1, NCW * 32);
   }
+}
+
+// Merge the partial records of the (sequence, KV head) pairs that the
+// balanced partition cut.  The decode kernel leaves, for every CTA holding
+// the first piece of a cut pair, a descriptor {sequence, kv head, last
+// covering CTA, query row}; one warp per (CTA, group head) merges that
+// pair's head from the records of CTAs first .. last.  Launched as a programmatic
+// dependent of the decode grid: griddepcontrol.wait returns once that grid
+// has finished and its writes are visible.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) balanced_merge_kernel(const AttnArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int w = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);  // (CTA, group head)
+  const int lane = threadIdx.x & 31;
+  const int G = a.grid, grp = a.group;
+  const int first = w / grp, hg = w - first * grp;
+  if (first >= G) return;
+  const int4 d = *reinterpret_cast<const int4 *>(a.bal_desc + 4 * first);
+  const int64_t W = (int64_t)a.bal_prefix[a.num_seqs] * a.num_kv_heads;
+  if (d.x < 0) return;  // no cut pair starts in this CTA
+  const int slot0 = d.x, kvh = d.y, last = d.z, qrow = d.w;
+  constexpr int PER = D / 32;
+  float M = -INFINITY, Lsum = 0.f;
+  bool poisoned = false;
+  float o[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) o[e] = 0.f;
+  for (int c = first; c <= last; ++c) {
+    if (c > first && bal_start(c + 1, W, G) == bal_start(c, W, G)) continue;  // empty range
+    // the pair's piece is record slot0 of CTA `first` and the first segment
+    // (slot 0) of every later CTA
+    const float *r = a.part_o + (((int64_t)c * 2 + (c == first ? slot0 : 0)) * grp + hg) * (D + 4);
+    float x[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) x[e] = r[lane * PER + e];
+    const float m = r[D], l = r[D + 1];
+    poisoned |= isnan(l);
+    const float Mn = fmaxf(M, m);
+    const float sa = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+    const float sb = m == -INFINITY ? 0.f : fast_exp2(m - Mn);
+    Lsum = Lsum * sa + l * sb;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] = o[e] * sa + x[e] * sb;
+    M = Mn;
+  }
+  const float inv = (Lsum > 0.f && !poisoned) ? 1.f / Lsum : 0.f;
+  T *dst = static_cast<T *>(a.out) + ((int64_t)qrow * a.num_heads + kvh * grp + hg) * D + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) dst[e] = Elem<T>::from_f(o[e] * inv);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -526,14 +617,76 @@ cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1), lay.bytes);
   if (e != cudaSuccess) return e;
   if (occ < 1) occ = 1;
-  const int64_t max_items = (int64_t)a.num_seqs * a.num_kv_heads *
-                            (a.rows_mode ? (a.max_splits > a.max_query_len ? a.max_splits : a.max_query_len)
-                                         : a.max_splits);
   int64_t grid = (int64_t)sm_count * occ;
-  if (grid > max_items) grid = max_items;
+  if (a.balanced) {
+    grid = a.grid;  // fixed by the host (records are per CTA)
+  } else {
+    const int64_t max_items = (int64_t)a.num_seqs * a.num_kv_heads * a.max_splits;
+    if (grid > max_items) grid = max_items;
+  }
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, 32 * (NCW + 1), lay.bytes, stream>>>(a, tmk, tmv);
-  return cudaGetLastError();
+  // programmatic dependent launch: the grid may be scheduled while the
+  // previous kernel in the stream finishes; it waits (griddepcontrol.wait)
+  // before touching global memory.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(32 * (NCW + 1));
+  cfg.dynamicSmemBytes = lay.bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, tmk, tmv);
+}
+
+template <typename T, int D, int BS, int NT>
+int grid_mma_t(const AttnArgs &a, int sm_count) {
+  constexpr int NCW = PA_MMA_WARPS;
+  using L = MmaLayout<D, BS, NT, NCW>;
+  auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    const L big(kMaxSeqsPerLaunch, 8 * NT);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, big.bytes) != cudaSuccess)
+      return 0;
+    attr_set[dev] = true;
+  }
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1),
+                                                    L(a.num_seqs, a.group).bytes) != cudaSuccess)
+    return 0;
+  return sm_count * (occ < 1 ? 1 : occ);
+}
+
+template <typename T>
+int grid_mma_d(const AttnArgs &a, int sm_count) {
+  if (a.head_dim == 64)
+    return a.block_size == 16 ? (a.group <= 8 ? grid_mma_t<T, 64, 16, 1>(a, sm_count) : grid_mma_t<T, 64, 16, 2>(a, sm_count))
+                              : (a.group <= 8 ? grid_mma_t<T, 64, 32, 1>(a, sm_count) : grid_mma_t<T, 64, 32, 2>(a, sm_count));
+  return a.block_size == 16 ? (a.group <= 8 ? grid_mma_t<T, 128, 16, 1>(a, sm_count) : grid_mma_t<T, 128, 16, 2>(a, sm_count))
+                            : (a.group <= 8 ? grid_mma_t<T, 128, 32, 1>(a, sm_count) : grid_mma_t<T, 128, 32, 2>(a, sm_count));
+}
+
+template <typename T>
+cudaError_t launch_bal_reduce_t(const AttnArgs &a, cudaStream_t stream) {
+  const int warps = a.grid * a.group;  // one per (CTA descriptor, group head)
+  if (warps <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((warps * 32 + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.head_dim == 64) return cudaLaunchKernelEx(&cfg, balanced_merge_kernel<T, 64>, a);
+  return cudaLaunchKernelEx(&cfg, balanced_merge_kernel<T, 128>, a);
 }
 
 template <typename T, int D, int BS>
@@ -553,6 +706,15 @@ cudaError_t mma_d(const AttnArgs &a, int sm_count, cudaStream_t s) {
 }
 
 }  // namespace
+
+int decode_mma_grid(const AttnArgs &a, int dtype, int sm_count) {
+  return dtype == PA_F16 ? grid_mma_d<__half>(a, sm_count) : grid_mma_d<__nv_bfloat16>(a, sm_count);
+}
+
+cudaError_t launch_balanced_reduce(const AttnArgs &a, int dtype, cudaStream_t stream) {
+  return dtype == PA_F16 ? launch_bal_reduce_t<__half>(a, stream)
+                         : launch_bal_reduce_t<__nv_bfloat16>(a, stream);
+}
 
 bool decode_mma_supported(const AttnArgs &a, int dtype) {
   return (dtype == PA_F16 || dtype == PA_BF16) && a.group >= 1 && a.group <= 16 &&

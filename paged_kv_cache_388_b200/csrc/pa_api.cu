@@ -3,6 +3,9 @@
 // Nothing here allocates device memory.  The only device state the library
 // owns is one error word per device (a file-scope __device__ variable), whose
 // address is looked up once per device.
+#include <stdlib.h>
+#include <string.h>
+
 #include <mutex>
 
 #include "../../include/pa.h"
@@ -148,8 +151,14 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
   int sb = 0, ms = 0;
   split_policy(num_seqs, num_kv_heads, block_size, max_context_len, kv_split_tokens,
                dev.sm_count, &sb, &ms);
-  if (ms <= 1) return 0;
-  return (size_t)num_seqs * num_heads * ms * (head_dim + 2) * sizeof(float) + 256;
+  size_t fixed = ms <= 1 ? 0 : (size_t)num_seqs * num_heads * ms * (head_dim + 2) * sizeof(float) + 256;
+  if (kv_split_tokens > 0 || num_heads % num_kv_heads != 0) return fixed;
+  // balanced partition (tensor-core kernel): per-CTA records for at most 8
+  // resident CTAs per SM, plus the block prefix of one launch
+  const int n = num_seqs < decode_max_seqs_per_launch() ? num_seqs : decode_max_seqs_per_launch();
+  const size_t bal = balanced_record_bytes(dev.sm_count * 8, num_heads / num_kv_heads, head_dim) +
+                     balanced_desc_bytes(dev.sm_count * 8) + (size_t)(n + 1) * sizeof(int) + 256;
+  return fixed > bal ? fixed : bal;
 }
 
 int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -215,7 +224,27 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
   // one query row per work item.
   a.rows_mode = (max_query_len > 1 && dtype == PA_F32) ? 1 : 0;
 
-  if (max_splits > 1) {
+  // Kernel: tensor cores for 16-bit caches (PA_DECODE_KERNEL=simt forces the
+  // CUDA-core kernel, kept for fp32, unusual head groups and comparison).
+  const char *sel = getenv("PA_DECODE_KERNEL");
+  const bool want_simt = sel && strcmp(sel, "simt") == 0;
+  const bool use_mma = !want_simt && !a.rows_mode && decode_mma_supported(a, dtype);
+  // Balanced partition unless the caller fixed the split size.
+  a.balanced = (use_mma && kv_split_tokens == 0) ? 1 : 0;
+  const int step = decode_max_seqs_per_launch();
+  if (a.balanced) {
+    AttnArgs probe = a;
+    probe.num_seqs = num_seqs < step ? num_seqs : step;
+    a.grid = decode_mma_grid(probe, dtype, dev.sm_count);
+    if (a.grid <= 0) return PA_ERR_CUDA;
+    const size_t rec = balanced_record_bytes(a.grid, group, head_dim);
+    const size_t desc = balanced_desc_bytes(a.grid);
+    const size_t need = rec + desc + (size_t)(probe.num_seqs + 1) * sizeof(int);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+    a.part_o = static_cast<float *>(workspace);
+    a.bal_desc = reinterpret_cast<int *>(static_cast<char *>(workspace) + rec);
+    a.bal_prefix = reinterpret_cast<int *>(static_cast<char *>(workspace) + rec + desc);
+  } else if (max_splits > 1) {
     const size_t need = (size_t)num_seqs * num_heads * max_splits * (head_dim + 2) * sizeof(float);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
     a.part_o = static_cast<float *>(workspace);
@@ -223,12 +252,13 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
   }
 
   cudaStream_t s = (cudaStream_t)stream;
-  const int step = decode_max_seqs_per_launch();
   for (int s0 = 0; s0 < num_seqs; s0 += step) {
     a.seq_begin = s0;
     a.num_seqs = num_seqs - s0 < step ? num_seqs - s0 : step;
-    cudaError_t e = launch_decode(a, dtype, dev.sm_count, s);
-    if (e == cudaSuccess && max_splits > 1) e = launch_reduce(a, dtype, s);
+    cudaError_t e = use_mma ? launch_decode_mma(a, dtype, dev.sm_count, s)
+                            : launch_decode(a, dtype, dev.sm_count, s);
+    if (e == cudaSuccess && a.balanced) e = launch_balanced_reduce(a, dtype, s);
+    else if (e == cudaSuccess && max_splits > 1) e = launch_reduce(a, dtype, s);
     if (e == cudaSuccess && max_query_len > 1 && !a.rows_mode)
       e = launch_chunk(a, dtype, num_q_tokens, s);
     if (e != cudaSuccess) return PA_ERR_CUDA;

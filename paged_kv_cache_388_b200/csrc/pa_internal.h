@@ -35,6 +35,10 @@ struct AttnArgs {
   int max_context_len;  // host bound; longer sequences are rejected on the device
   int num_q_tokens;
   int rows_mode;      // 1: the decode kernel also takes rows of Q>1 sequences (one item per row)
+  int balanced;       // 1: balanced flat partition (records in part_o), 0: fixed splits
+  int grid;           // CTAs of the balanced launch (records are per CTA)
+  int *bal_prefix;    // balanced: [num_seqs + 1] block prefix written by CTA 0
+  int *bal_desc;      // balanced: [grid][4] cut-pair descriptors written by the decode kernel
   float scale_log2;   // scale * log2(e)
 };
 
@@ -53,8 +57,16 @@ void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_contex
 // Implemented in decode_mma.cu (tensor-core decode for 16-bit caches)
 bool decode_mma_supported(const AttnArgs &a, int dtype);
 cudaError_t launch_decode_mma(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream);
+int decode_mma_grid(const AttnArgs &a, int dtype, int sm_count);  // CTAs of a balanced launch
+cudaError_t launch_balanced_reduce(const AttnArgs &a, int dtype, cudaStream_t stream);
+// Workspace of the balanced scheme: per-CTA partial records, the per-CTA
+// cut-pair descriptors, then the block prefix.
+inline size_t balanced_record_bytes(int grid, int group, int head_dim) {
+  return ((size_t)grid * 2 * group * (head_dim + 4) * sizeof(float) + 255) / 256 * 256;
+}
+inline size_t balanced_desc_bytes(int grid) { return ((size_t)grid * 4 * sizeof(int) + 255) / 256 * 256; }
 
-// Implemented in decode.cu
+// Implemented in decode.cu (CUDA-core kernel, fixed-split scheme)
 cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnArgs &a, int dtype, cudaStream_t stream);
 int decode_max_seqs_per_launch();

@@ -77,6 +77,22 @@ class PagedKVCache:
         out.copy_(o, non_blocking=True)
         return out
 
+    def capture_step_from_host(self, q, key, value, slot_mapping, block_tables, context_lens, out,
+                               scale, max_context_len=0, warmup=2):
+        """Capture ``step_from_host`` on these (pinned) host buffers into a CUDA
+        graph and return a callable that replays it: each call copies the
+        buffers' current contents in, runs the step and copies ``out`` back.
+        The caller refills the host buffers between calls."""
+        for _ in range(warmup):  # one-time library setup happens outside capture
+            self.step_from_host(q, key, value, slot_mapping, block_tables, context_lens, out,
+                                scale, max_context_len=max_context_len)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step_from_host(q, key, value, slot_mapping, block_tables, context_lens, out,
+                                scale, max_context_len=max_context_len)
+        return g.replay
+
     @staticmethod
     def host_bytes(*tensors) -> int:
         return int(sum(t.numel() * t.element_size() for t in tensors))

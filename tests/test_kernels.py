@@ -121,6 +121,11 @@ def test_chunk_whole_prompt(lib):
     _check_workload(lib, wl)
 
 
+def _ws(lib, n, split=0, H=8, Hk=2, D=128, bs=16, max_ctx=64):
+    size = lib.pa_decode_workspace_size(n, H, Hk, D, bs, max_ctx, split)
+    return torch.empty(max(size, 16), dtype=torch.uint8, device="cuda")
+
+
 def _tiny_decode(lib, lens=(20, 40), dtype=torch.bfloat16, bs=16):
     torch.manual_seed(0)
     H, Hk, D = 8, 2, 128
@@ -137,7 +142,7 @@ def test_bad_block_id_sets_error_and_zeroes_row(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib)
     bt[1, 1] = 10_000
     out = torch.full_like(q, 7.0)
-    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20)
+    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20, workspace=_ws(lib, 2))
     code = lib.pa_get_device_error()
     assert code & lib.PA_DEVERR_BLOCK_ID
     assert torch.count_nonzero(out[1]) == 0
@@ -160,7 +165,7 @@ def test_bad_context_len(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib)
     cl[0] = 4 * 16 + 1  # beyond max_blocks_per_seq * block_size
     out = torch.full_like(q, 7.0)
-    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1)
+    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, workspace=_ws(lib, 2))
     assert lib.pa_get_device_error() & lib.PA_DEVERR_CONTEXT_LEN
     assert torch.count_nonzero(out[0]) == 0
 
@@ -243,12 +248,16 @@ def test_nan_in_unused_slots_does_not_leak(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib, lens=(20, 37))
     nan = torch.tensor(float("nan"), dtype=kc.dtype, device="cuda")
     ref_out = torch.empty_like(q)
-    lib.pa_decode(ref_out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20)
+    ws = _ws(lib, 2)
+    lib.pa_decode(ref_out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20, workspace=ws)
     kc[bt[0, 1], :, 4:] = nan  # seq 0: tokens 20.. of block 1 are unused
     vc[bt[0, 1], :, 4:] = nan
     kc[bt[1, 2], :, 5:] = nan  # seq 1: tokens 37.. of block 2
     vc[bt[1, 2], :, 5:] = nan
     out = torch.empty_like(q)
-    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20)
+    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20, workspace=ws)
+    assert lib.pa_get_device_error() == 0
+    assert torch.equal(out, ref_out)
+    lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, workspace=ws)  # balanced partition
     assert lib.pa_get_device_error() == 0
     assert torch.equal(out, ref_out)
