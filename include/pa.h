@@ -160,6 +160,45 @@ int pa_decode(void *out, const void *q, const void *k_cache,
               size_t workspace_bytes, struct CUstream_st *stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode without a caller-supplied workspace.
+ *
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory -- a plugin whose host framework owns
+ * all device memory, a runtime whose memory budget is fixed at start-up, or a
+ * serving loop that must not call cudaMalloc on its hot path (an allocation
+ * can synchronise the device and is not allowed in every stream-capture
+ * mode).  The scratch that pa_decode would take from `workspace` comes
+ * instead from a static device array of PA_NOALLOC_SCRATCH_BYTES bytes built
+ * into the library; every GPU that loads the library holds it until the
+ * process exits.  This function allocates nothing and calls no allocating
+ * routine.
+ *
+ * Arguments and results are those of pa_decode (without workspace).
+ * PA_ERR_WORKSPACE (nothing launched) if the batch needs more scratch than
+ * the array holds; pa_decode_workspace_size() tells how much a batch may
+ * need (16-bit caches with kv_split_tokens = 0 need about
+ * 8 * SMs * 2 * group * (head_dim + 4) * 4 bytes, well inside the array).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents:
+ * nothing in it has to start at zero, but calls whose kernels overlap on the
+ * GPU (other streams, other host threads) race on it -- serialise them.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+int pa_decode_noalloc(void *out, const void *q, const void *k_cache,
+                      const void *v_cache, const int32_t *block_tables,
+                      int max_blocks_per_seq, const int32_t *context_lens,
+                      const int32_t *query_start_loc, int num_seqs,
+                      int num_q_tokens, int max_query_len, int num_heads,
+                      int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, float scale, int max_context_len,
+                      int kv_split_tokens, int dtype, struct CUstream_st *stream);
+
+/* Size of the static scratch array pa_decode_noalloc uses, in bytes. */
+size_t pa_noalloc_scratch_bytes(void);
+
+/*
  * pa_get_device_error -- synchronise `stream`, then read and clear the
  * current device's error word (PA_DEVERR_* bits, 0 = none) into *code_out.
  */

@@ -36,6 +36,10 @@ _lib.pa_decode_workspace_size.restype = SZ
 _lib.pa_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
 _lib.pa_decode.restype = I
 _lib.pa_decode.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, I, I, P, SZ, P]
+_lib.pa_decode_noalloc.restype = I
+_lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, I, I, P]
+_lib.pa_noalloc_scratch_bytes.restype = SZ
+_lib.pa_noalloc_scratch_bytes.argtypes = []
 _lib.pa_get_device_error.restype = I
 _lib.pa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), P]
 _lib.pa_status_string.restype = ctypes.c_char_p
@@ -149,6 +153,38 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                         int(kv_split_tokens), _DT[q.dtype], _ptr(workspace), ws_bytes,
                         _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                      query_start_loc=None, max_query_len=1, max_context_len=0, kv_split_tokens=0,
+                      stream=None):
+    """pa_decode with the library's static scratch instead of a workspace, for
+    callers that cannot allocate device memory.  Calls must not overlap on
+    the GPU (they share the scratch); make the first call on a device before
+    any stream capture."""
+    _dev(q, "q")
+    _dev(out, "out", q.dtype)
+    _dev(k_cache, "k_cache", q.dtype)
+    _dev(v_cache, "v_cache", q.dtype)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    if query_start_loc is not None:
+        _dev(query_start_loc, "query_start_loc", torch.int32)
+    tq, h, d = q.shape
+    nb, hk, bs, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    s, mbps = block_tables.shape
+    rc = _lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), mbps, _ptr(context_lens), _ptr(query_start_loc),
+                                s, tq, int(max_query_len), h, hk, d, bs, nb, float(scale),
+                                int(max_context_len), int(kv_split_tokens), _DT[q.dtype],
+                                _stream(stream))
+    _check(rc, "pa_decode_noalloc")
+
+
+def pa_noalloc_scratch_bytes() -> int:
+    return int(_lib.pa_noalloc_scratch_bytes())
 
 
 def pa_get_device_error(stream=None) -> int:
