@@ -54,6 +54,34 @@ def hbm_peak():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = ("paged_kv_cache_388_b200/csrc/decode_mma.cu",
+                  "paged_kv_cache_388_b200/csrc/decode_common.cuh",
+                  "paged_kv_cache_388_b200/csrc/pa_device.cuh",
+                  "paged_kv_cache_388_b200/csrc/pa_internal.h")
+PROFILE = os.path.join(ROOT, "profiles", "paged_decode_mma_kernel_cfg3.md")
+
+
+def profiled_traffic(config):
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, or None if that summary is for other sources or another workload."""
+    import hashlib
+    if config != "3" or not os.path.exists(PROFILE):
+        return None
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    fields = {}
+    with open(PROFILE, encoding="utf-8") as fh:
+        for line in fh:
+            if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch", "source_sha256"):
+                k, val = line.split(":", 1)
+                fields[k.strip()] = val.strip()
+    if fields.get("source_sha256") != h.hexdigest():
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def elem_bytes(dtype):
     return {"f32": 4, "f16": 2, "bf16": 2}[dtype]
 
@@ -158,6 +186,19 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle legs (cpu_baseline and --impl reference)
 # --------------------------------------------------------------------------
+def aggregate(local_bytes, local_ms, device):
+    """Whole-job totals over ranks: bytes summed, time = the slowest rank's.
+    No-op without an initialised process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(local_bytes), float(local_ms)
+    b = torch.tensor([float(local_bytes)], dtype=torch.float64, device=device)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(b.item()), float(t.item())
+
+
 def oracle_runner(wl, vals, batch):
     """Returns run(n_seqs) -> (seconds, bytes, n_seqs): the oracle doing the
     step for the first n_seqs sequences (their new tokens' writes into a copy
@@ -240,7 +281,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
 
-    wl = workloads.make(args.config)
+    # weak scaling: every rank runs its own batch of the workload's shape
+    wl = workloads.make(args.config, replica=rank)
     batch = build_batch(wl)
     vals = workloads.values(wl)
     nbytes = step_bytes(wl, batch)
@@ -308,11 +350,8 @@ def run_ours(args, rank, world, local_rank):
         g_steps.replay()
         t_end.record(stream)
         barrier()
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms_local = t_start.elapsed_time(t_end)
+    job_bytes, ms = aggregate(nbytes["step"] * K, ms_local, dev)
     assert _lib.pa_get_device_error() == 0
     clk = clocks.summary()
     del g_steps, g_warm
@@ -365,12 +404,8 @@ def run_ours(args, rank, world, local_rank):
             replay()
         e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": nbytes["step"] * world * K / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+        e2e_bytes, e2e_ms = aggregate(nbytes["step"] * K, e0.elapsed_time(e1), dev)
+        e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / K, "path": "PagedKVCache.capture_step_from_host (CUDA graph)"}
 
@@ -390,7 +425,7 @@ def run_ours(args, rank, world, local_rank):
         (1 if batch.max_query_len > 1 else 0)
     peak, peak_kind = hbm_peak()
     achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
-    value = nbytes["step"] * world * K / (ms * 1e-3) / 1e9
+    value = job_bytes / (ms * 1e-3) / 1e9
     res = {
         "metric": METRIC,
         "value": value,
@@ -427,7 +462,9 @@ def run_ours(args, rank, world, local_rank):
             "unit": "GB/s",
             "frac": achieved / peak,
             "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
-            "traffic": None,
+            "traffic": profiled_traffic(args.config),
+            "traffic_source": "profiles/paged_decode_mma_kernel_cfg3.md (ncu dram__bytes_read+write "
+                              "of the decode kernel; null when the kernel sources changed since)",
             "algorithmic_bytes": nbytes["decode"],
             "avg_ms": dec_avg,
         },

@@ -135,65 +135,86 @@ def mixed_workload(name, seed, n_decode, dec_lo, dec_hi, n_chunk, prefix, chunk,
                     query_lens=[qls[i] for i in order])
 
 
+def _reseed(config, seed):
+    """The named workload drawn again from another seed (same shapes/recipe)."""
+    global _SEED_OVERRIDE
+    _SEED_OVERRIDE = seed
+    try:
+        return make(config)
+    finally:
+        _SEED_OVERRIDE = None
+
+
+_SEED_OVERRIDE = None
+
+
+def _seed(default):
+    return default if _SEED_OVERRIDE is None else _SEED_OVERRIDE
+
+
 def lognormal_lengths(rng, n, median, sigma, cap):
     z = rng.standard_normal(n)
     return np.clip(np.rint(np.exp(np.log(median) + sigma * z)), 1, cap).astype(np.int64).tolist()
 
 
-def make(config: str) -> Workload:
+def make(config: str, replica: int = 0) -> Workload:
     """Named workloads: the five full-size configurations and small variants
-    ('s' suffix) of the same shapes that the oracle finishes in seconds."""
+    ('s' suffix) of the same shapes that the oracle finishes in seconds.
+    ``replica`` > 0 gives an independent batch of the same shape (seeds offset
+    by 100000 * replica) -- one per rank when N GPUs each run their own batch."""
+    if replica:
+        return _reseed(config, make(config).seed + 100000 * replica)
     c = config
     if c == "1":
-        return decode_workload("cfg1_tiny_fp32", 1001, [17, 33, 64, 100], 4, 4, 64, 16,
+        return decode_workload("cfg1_tiny_fp32", _seed(1001), [17, 33, 64, 100], 4, 4, 64, 16,
                                "f32", num_blocks=64)
     if c == "2":
-        rng = np.random.default_rng(1002)
+        rng = np.random.default_rng(_seed(1002))
         lens = rng.integers(128, 2048 + 1, size=64).tolist()
-        return decode_workload("cfg2_llama2_7b_mha_fp16", 1002, lens, 32, 32, 128, 16, "f16",
+        return decode_workload("cfg2_llama2_7b_mha_fp16", _seed(1002), lens, 32, 32, 128, 16, "f16",
                                rng=rng)
     if c == "3":
-        rng = np.random.default_rng(1003)
+        rng = np.random.default_rng(_seed(1003))
         lens = lognormal_lengths(rng, 256, 800, 0.8, 4096)
-        return decode_workload("cfg3_llama3_8b_gqa_bf16", 1003, lens, 32, 8, 128, 16, "bf16",
+        return decode_workload("cfg3_llama3_8b_gqa_bf16", _seed(1003), lens, 32, 8, 128, 16, "bf16",
                                rng=rng)
     if c == "4":
-        return shared_prefix_workload("cfg4_shared_prefix_70b_bf16", 1004, 32, 8, 1024, 512,
+        return shared_prefix_workload("cfg4_shared_prefix_70b_bf16", _seed(1004), 32, 8, 1024, 512,
                                       64, 8, 128, 16, "bf16")
     if c == "4cow":
-        return shared_prefix_workload("cfg4cow_shared_prefix_1016_bf16", 1014, 32, 8, 1016, 512,
+        return shared_prefix_workload("cfg4cow_shared_prefix_1016_bf16", _seed(1014), 32, 8, 1016, 512,
                                       64, 8, 128, 16, "bf16")
     if c == "5":
-        return mixed_workload("cfg5_long_mixed_bf16_bs16", 1005, 8, 32768, 131072, 4, 16384,
+        return mixed_workload("cfg5_long_mixed_bf16_bs16", _seed(1005), 8, 32768, 131072, 4, 16384,
                               512, 32, 8, 128, 16, "bf16")
     if c == "5bs32":
-        return mixed_workload("cfg5_long_mixed_bf16_bs32", 1005, 8, 32768, 131072, 4, 16384,
+        return mixed_workload("cfg5_long_mixed_bf16_bs32", _seed(1005), 8, 32768, 131072, 4, 16384,
                               512, 32, 8, 128, 32, "bf16")
     # ---- small variants: same head shapes, dtypes and structure ----
     if c == "2s":
-        rng = np.random.default_rng(2002)
+        rng = np.random.default_rng(_seed(2002))
         lens = rng.integers(1, 700 + 1, size=12).tolist()
-        return decode_workload("cfg2s_mha_fp16_small", 2002, lens, 32, 32, 128, 16, "f16", rng=rng)
+        return decode_workload("cfg2s_mha_fp16_small", _seed(2002), lens, 32, 32, 128, 16, "f16", rng=rng)
     if c == "3s":
-        rng = np.random.default_rng(2003)
+        rng = np.random.default_rng(_seed(2003))
         lens = lognormal_lengths(rng, 40, 200, 0.8, 1100)
-        return decode_workload("cfg3s_gqa_bf16_small", 2003, lens, 32, 8, 128, 16, "bf16", rng=rng)
+        return decode_workload("cfg3s_gqa_bf16_small", _seed(2003), lens, 32, 8, 128, 16, "bf16", rng=rng)
     if c == "3s32":
-        rng = np.random.default_rng(2013)
+        rng = np.random.default_rng(_seed(2013))
         lens = lognormal_lengths(rng, 24, 200, 0.8, 1100)
-        return decode_workload("cfg3s_gqa_bf16_bs32_small", 2013, lens, 32, 8, 128, 32, "bf16",
+        return decode_workload("cfg3s_gqa_bf16_bs32_small", _seed(2013), lens, 32, 8, 128, 32, "bf16",
                                rng=rng)
     if c == "4s":
-        return shared_prefix_workload("cfg4s_shared_prefix_small", 2004, 2, 8, 128, 70,
+        return shared_prefix_workload("cfg4s_shared_prefix_small", _seed(2004), 2, 8, 128, 70,
                                       64, 8, 128, 16, "bf16")
     if c == "4cows":
-        return shared_prefix_workload("cfg4cows_shared_prefix_cow_small", 2014, 2, 8, 120, 70,
+        return shared_prefix_workload("cfg4cows_shared_prefix_cow_small", _seed(2014), 2, 8, 120, 70,
                                       64, 8, 128, 16, "bf16")
     if c == "5s":
-        return mixed_workload("cfg5s_mixed_bf16_bs16_small", 2005, 3, 1500, 5000, 2, 700, 96,
+        return mixed_workload("cfg5s_mixed_bf16_bs16_small", _seed(2005), 3, 1500, 5000, 2, 700, 96,
                               32, 8, 128, 16, "bf16")
     if c == "5s32":
-        return mixed_workload("cfg5s_mixed_bf16_bs32_small", 2005, 3, 1500, 5000, 2, 700, 96,
+        return mixed_workload("cfg5s_mixed_bf16_bs32_small", _seed(2005), 3, 1500, 5000, 2, 700, 96,
                               32, 8, 128, 32, "bf16")
     raise KeyError(config)
 
