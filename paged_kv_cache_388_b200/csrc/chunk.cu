@@ -13,6 +13,9 @@
 // (row stride D+8 elements: conflict-free ldmatrix), double-buffered.
 // S = Q K^T and O += P V use mma.sync m16n8k16 (bf16/f16 in, fp32 out); the
 // softmax is the online (running max / running sum) form in base 2.
+#include <stdlib.h>
+#include <string.h>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -363,6 +366,11 @@ cudaError_t chunk_d(const AttnArgs &a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int /*num_q_tokens*/, cudaStream_t stream) {
+  // head_dim 128: tcgen05 kernel (chunk_tc.cu) unless PA_CHUNK_KERNEL=mma asks
+  // for this mma.sync kernel, which also serves head_dim 64.
+  const char *sel = getenv("PA_CHUNK_KERNEL");
+  const bool want_mma = sel && strcmp(sel, "mma") == 0;
+  if (!want_mma && chunk_tc_supported(a, dtype)) return launch_chunk_tc(a, dtype, stream);
   if (dtype == PA_F16) return chunk_d<__half>(a, stream);
   if (dtype == PA_BF16) return chunk_d<__nv_bfloat16>(a, stream);
   return cudaErrorNotSupported;  // fp32 chunks run through the decode kernel's row mode

@@ -1,0 +1,566 @@
+// chunk_tc.cu -- chunked-prefill attention on the 5th-generation tensor cores.
+//
+// A chunk of Q > 1 query tokens of one sequence attends causally over the
+// sequence's paged KV (row t sees keys 0 .. L-Q+t; "PagedAttention 实战",
+// section Chunked Prefill).  Per (sequence, KV head) the GROUP query heads of
+// every token read the same K/V, so a 128-row tile (128/GROUP tokens x GROUP
+// heads) against 64-key tiles is a dense contraction: S = Q K^T
+// (128x64x128) and O += P V (128x128x64) run as tcgen05.mma with fp32
+// accumulators in tensor memory.
+//
+// CTA = (sequence, KV head, 128 query rows); 6 warps:
+//   warps 0-3  softmax: thread r owns row r (TMEM lane r).  Reads S from TMEM,
+//              masks, keeps a running max that is only moved (and O rescaled
+//              in TMEM) when the tile max exceeds it by more than 2^8, writes
+//              P = 2^(s - m) as bf16 hi + lo (or fp16) into swizzled shared
+//              memory, and at the end writes O / l.
+//   warp 4     producer: TMA loads of Q (once) and of each 64-key K/V tile,
+//              block by block through the block table (128-byte swizzle).
+//   warp 5     MMA issue (one elected thread) and TMEM allocation.
+// TMEM: S double buffer (2 x 64 columns) and O (128 columns).
+// Shared memory: Q 32 KB, kStagesTC K/V stages of 32 KB, 2 P buffers of 32 KB.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kRowsTC = 128;   // query rows per CTA (MMA M)
+constexpr int kKeysTC = 64;    // keys per tile (MMA N of S, K of P.V)
+constexpr int kHeadDim = 128;
+#ifndef PA_CHUNK_TC_STAGES
+#define PA_CHUNK_TC_STAGES 3
+#endif
+constexpr int kStagesTC = PA_CHUNK_TC_STAGES;  // K/V tiles in flight
+constexpr int kThreadsTC = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between rescales
+
+template <typename T>
+struct TcType;
+template <>
+struct TcType<__nv_bfloat16> {
+  static constexpr uint32_t kFmt = 1;  // instruction-descriptor a/b format: BF16
+  static constexpr bool kSplitP = true;
+  static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  __device__ __forceinline__ static uint32_t pack(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+  __device__ __forceinline__ static float2 unpack(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+  __device__ __forceinline__ static uint16_t bits(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
+  }
+};
+template <>
+struct TcType<__half> {
+  static constexpr uint32_t kFmt = 0;  // F16
+  static constexpr bool kSplitP = false;
+  static constexpr CUtensorMapDataType kTma = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  __device__ __forceinline__ static uint32_t pack(float a, float b) {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+  __device__ __forceinline__ static float2 unpack(uint32_t u) {
+    return __half22float2(*reinterpret_cast<__half2 *>(&u));
+  }
+  __device__ __forceinline__ static uint16_t bits(float x) {
+    __half h = __float2half_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
+  }
+};
+
+// ---- shared-memory layout (offsets from a 1024-byte aligned base) ---------
+struct TcLayout {
+  static constexpr int kQ = 0;                                   // 2 halves x [128 rows x 128 B]
+  static constexpr int kKV = kQ + kRowsTC * kHeadDim * 2;        // stages: K (2x8 KB) + V (2x8 KB)
+  static constexpr int kStageBytes = 2 * kKeysTC * kHeadDim * 2;
+  static constexpr int kP = kKV + kStagesTC * kStageBytes;       // 2 buffers x (hi, lo) x [128 x 128 B]
+  static constexpr int kPBuf = 2 * kRowsTC * kKeysTC * 2;
+  static constexpr int kBar = kP + 2 * kPBuf;
+  static constexpr int kBytes = kBar + 256 + 1024;               // barriers etc. + alignment slack
+};
+
+// barrier indices within the barrier block
+enum {
+  kQFull = 0,
+  kKvFull = 1,                       // [kStagesTC]
+  kKvEmpty = kKvFull + kStagesTC,    // [kStagesTC]
+  kSFull = kKvEmpty + kStagesTC,     // [2]
+  kSFree = kSFull + 2,               // [2]
+  kPFull = kSFree + 2,               // [2]
+  kPvDone = kPFull + 2,              // [2]
+  kDone = kPvDone + 2,
+  kNumBars = kDone + 1
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            int z, int w, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// UMMA shared-memory descriptor, 128-byte swizzle (Blackwell format, version 1).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // version
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor for kind::f16 with fp32 accumulation.
+__host__ __device__ constexpr uint32_t umma_idesc(uint32_t fmt, uint32_t a_mn_major,
+                                                  uint32_t b_mn_major, int M, int N) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                   "r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+template <typename T, int BS>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    chunk_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmq,
+                    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                    int tiles_per_seq) {
+  using TT = TcType<T>;
+  constexpr int D = kHeadDim;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TcLayout::kBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TcLayout::kBar + 8 * kNumBars);
+  volatile int *flags = reinterpret_cast<volatile int *>(tmem_slot + 1);  // [0] abort, [1] bad block
+  const uint32_t sbase = smem_addr(smem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int tile = blockIdx.x % tiles_per_seq;
+  const int rest = blockIdx.x / tiles_per_seq;
+  const int kvh = rest % a.num_kv_heads;
+  const int seq = a.seq_begin + rest / a.num_kv_heads;
+  const int q0 = a.query_start_loc[seq];
+  const int Q = a.query_start_loc[seq + 1] - q0;
+  if (Q <= 1 || q0 < 0 || q0 + Q > a.num_q_tokens) return;  // CTA-uniform exits, before any barrier
+  if (Q > a.max_query_len) {
+    if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
+    return;
+  }
+  const int G = a.group;
+  const int TPT = kRowsTC / G;
+  const int t0 = tile * TPT;
+  if (t0 >= Q) return;
+  const int ntok = min(TPT, Q - t0);
+  const int L = a.context_lens[seq];
+  if (L < Q || L > a.max_context_len) {
+    if (tid == 0 && tile == 0 && kvh == 0)
+      raise_error(a.err, (L < 0 || L > a.max_context_len) ? PA_DEVERR_CONTEXT_LEN : PA_DEVERR_QUERY_LEN);
+    for (int idx = tid; idx < ntok * G * D; idx += blockDim.x) {
+      const int r = idx / D, dd = idx - r * D;
+      static_cast<T *>(a.out)[((int64_t)(q0 + t0 + r / G) * a.num_heads + kvh * G + r % G) * D + dd] =
+          Elem<T>::from_f(0.f);
+    }
+    return;
+  }
+  const int kend = L - Q + t0 + ntok;              // keys [0, kend) visible to some row
+  const int ntiles = (kend + kKeysTC - 1) / kKeysTC;
+  const int nblk = (L + BS - 1) / BS;              // blocks that hold the sequence
+
+  // ---- set-up: barriers, TMEM ------------------------------------------------
+  if (tid == 0) {
+    mbar_init(&bars[kQFull], 1);
+    for (int s = 0; s < kStagesTC; ++s) {
+      mbar_init(&bars[kKvFull + s], 1);
+      mbar_init(&bars[kKvEmpty + s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[kSFull + b], 1);
+      mbar_init(&bars[kSFree + b], 4);
+      mbar_init(&bars[kPFull + b], 4);
+      mbar_init(&bars[kPvDone + b], 1);
+    }
+    mbar_init(&bars[kDone], 1);
+    flags[0] = 0;
+    flags[1] = 0;
+    mbar_init_fence();
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s0 = tmem, tmem_o = tmem + 128;
+
+  auto fail = [&](void) {
+    if (!flags[0]) raise_error(a.err, PA_DEVERR_TIMEOUT);
+    flags[0] = 1;
+  };
+
+  if (warp == 4) {
+    // ======================= producer =======================================
+    if (lane == 0) {
+      const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
+      // Q: 128 rows (token, head) of this CTA, two 64-column boxes
+      mbar_arrive_expect_tx(&bars[kQFull], kRowsTC * D * 2);
+      for (int h = 0; h < 2; ++h)
+        tma_load_4d(sbase + TcLayout::kQ + h * kRowsTC * 128, &tmq, h * 64, 0, kvh, q0 + t0,
+                    &bars[kQFull]);
+      for (int j = 0; j < ntiles && !flags[0]; ++j) {
+        const int st = j % kStagesTC;
+        if (!mbar_wait(&bars[kKvEmpty + st], ((j / kStagesTC) & 1) ^ 1)) { fail(); break; }
+        const int b0 = j * (kKeysTC / BS);
+        const int nb = min(kKeysTC / BS, nblk - b0);  // blocks of this tile inside the sequence
+        mbar_arrive_expect_tx(&bars[kKvFull + st], nb * 2 * BS * D * 2);
+        const uint32_t kdst = sbase + TcLayout::kKV + st * TcLayout::kStageBytes;
+        const uint32_t vdst = kdst + TcLayout::kStageBytes / 2;
+        for (int b = 0; b < nb; ++b) {
+          int pb = table[b0 + b];
+          if (pb < 0 || pb >= a.num_blocks) {
+            raise_error(a.err, PA_DEVERR_BLOCK_ID);
+            flags[1] = 1;
+            pb = 0;  // load a valid block; the tile's rows are written as zeros
+          }
+          const int row = (pb * a.num_kv_heads + kvh) * BS;
+          for (int h = 0; h < 2; ++h) {
+            tma_load_2d(kdst + h * kKeysTC * 128 + b * BS * 128, &tmk, h * 64, row, &bars[kKvFull + st]);
+            tma_load_2d(vdst + h * kKeysTC * 128 + b * BS * 128, &tmv, h * 64, row, &bars[kKvFull + st]);
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ======================= MMA issue ======================================
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc(TT::kFmt, 0, 0, kRowsTC, kKeysTC);
+      constexpr uint32_t idesc_pv = umma_idesc(TT::kFmt, 0, 1, kRowsTC, D);
+      bool ok = mbar_wait(&bars[kQFull], 0);
+      if (!ok) fail();
+      auto issue_pv = [&](int jj) {
+        const int pbuf = jj & 1;
+        if (!mbar_wait(&bars[kPFull + pbuf], (jj >> 1) & 1)) { fail(); return false; }
+        tc_fence_after();
+        const uint32_t vst = sbase + TcLayout::kKV + (jj % kStagesTC) * TcLayout::kStageBytes +
+                             TcLayout::kStageBytes / 2;
+        const uint32_t pbase = sbase + TcLayout::kP + pbuf * TcLayout::kPBuf;
+        const int nparts = TT::kSplitP ? 2 : 1;
+        for (int part = 0; part < nparts; ++part) {
+          for (int ks = 0; ks < kKeysTC / 16; ++ks) {
+            const uint64_t da = umma_desc(pbase + part * (kRowsTC * 128) + ks * 32, 16, 1024);
+            const uint64_t db = umma_desc(vst + ks * 16 * 128, kKeysTC * 128, 1024);
+            umma(tmem_o, da, db, idesc_pv, (jj > 0 || part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&bars[kPvDone + pbuf]);
+        umma_commit(&bars[kKvEmpty + (jj % kStagesTC)]);
+        return true;
+      };
+      for (int j = 0; ok && j < ntiles && !flags[0]; ++j) {
+        const int st = j % kStagesTC, sb = j & 1;
+        if (!mbar_wait(&bars[kKvFull + st], (j / kStagesTC) & 1)) { fail(); break; }
+        if (!mbar_wait(&bars[kSFree + sb], ((j >> 1) & 1) ^ 1)) { fail(); break; }
+        tc_fence_after();
+        const uint32_t kst = sbase + TcLayout::kKV + st * TcLayout::kStageBytes;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int h = ks >> 2, kk = ks & 3;
+          const uint64_t da = umma_desc(sbase + TcLayout::kQ + h * kRowsTC * 128 + kk * 32, 16, 1024);
+          const uint64_t db = umma_desc(kst + h * kKeysTC * 128 + kk * 32, 16, 1024);
+          umma(tmem_s0 + sb * kKeysTC, da, db, idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars[kSFull + sb]);
+        if (j > 0 && !issue_pv(j - 1)) break;
+      }
+      if (ok && !flags[0] && ntiles > 0) issue_pv(ntiles - 1);
+      umma_commit(&bars[kDone]);  // completes when every MMA above has finished
+      if (!mbar_wait(&bars[kDone], 0)) fail();
+    }
+  } else {
+    // ======================= softmax warps (row r = tid) ======================
+    const int r = tid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int tok = r / G;
+    const int limit = L - Q + t0 + tok;  // last key this row may see
+    const float sl2 = a.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < ntiles; ++j) {
+      const int sb = j & 1;
+      bool ok = !flags[0] && mbar_wait(&bars[kSFull + sb], (j >> 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) { fail(); break; }  // warp-uniform: tcgen05.ld is collective
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(tmem_s0 + lane_off + sb * kKeysTC, sr[0]);
+      tmem_ld32(tmem_s0 + lane_off + sb * kKeysTC + 32, sr[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kSFree + sb]);
+      // scale and causal mask in place (as float bits), tile max
+      float mx = -INFINITY;
+      const int k0 = j * kKeysTC;
+#pragma unroll
+      for (int c = 0; c < kKeysTC; ++c) {
+        const float v = (k0 + c <= limit) ? __uint_as_float(sr[c >> 5][c & 31]) * sl2 : -INFINITY;
+        sr[c >> 5][c & 31] = __float_as_uint(v);
+        mx = fmaxf(mx, v);
+      }
+      // lazy rescale: move the reference max only when the tile max exceeds it
+      // by more than 2^8 (first tile: always)
+      const bool need = mx > m_used + kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = m_used == -INFINITY ? 0.f : fast_exp2(m_used - mx);
+        m_used = mx;
+        l *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O (in TMEM) is complete up to tile j-1 once that tile's P.V is done
+        const bool done = mbar_wait(&bars[kPvDone + ((j - 1) & 1)], ((j - 1) >> 1) & 1);
+        if (!__all_sync(0xffffffffu, done)) { fail(); break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int cblk = 0; cblk < D / 32; ++cblk) {
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_off + cblk * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem_o + lane_off + cblk * 32, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+      }
+      // the P buffer of tile j was last read by tile j-2's P.V
+      if (j >= 2 && !mbar_wait(&bars[kPvDone + sb], ((j - 2) >> 1) & 1)) { fail(); break; }
+      // P = 2^(x - m_used) -> shared memory (K-major, 128-byte swizzle), hi and lo
+      const uint32_t prow = sbase + TcLayout::kP + sb * TcLayout::kPBuf + r * 128;
+      float psum = 0.f;
+#pragma unroll
+      for (int c8 = 0; c8 < kKeysTC / 8; ++c8) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = c8 * 8 + 2 * i;
+          const float p0 = fast_exp2(__uint_as_float(sr[c >> 5][c & 31]) - m_used);
+          const float p1 = fast_exp2(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]) - m_used);
+          psum += p0 + p1;
+          hi[i] = TT::pack(p0, p1);
+          if constexpr (TT::kSplitP) {
+            const float2 h = TT::unpack(hi[i]);
+            lo[i] = TT::pack(p0 - h.x, p1 - h.y);
+          }
+        }
+        const uint32_t addr = prow + ((c8 ^ (r & 7)) << 4);
+        st_shared_v4(addr, hi[0], hi[1], hi[2], hi[3]);
+        if constexpr (TT::kSplitP) st_shared_v4(addr + kRowsTC * 128, lo[0], lo[1], lo[2], lo[3]);
+      }
+      l += psum;
+      // keys past the context end in the last tile: zero their V rows (P is 0
+      // there, but the slots may hold anything and 0 * NaN is NaN)
+      if (j == ntiles - 1 && (j + 1) * kKeysTC > L) {
+        const uint32_t vst = sbase + TcLayout::kKV + (j % kStagesTC) * TcLayout::kStageBytes +
+                             TcLayout::kStageBytes / 2;
+        const int z0 = L - j * kKeysTC;  // first stale row of the tile
+        const int nz = (kKeysTC - z0) * 16;  // 16-byte chunks over both halves
+        // all of the tile's K/V bytes must have landed before they are overwritten
+        if (mbar_wait(&bars[kKvFull + (j % kStagesTC)], (j / kStagesTC) & 1)) {
+          for (int c = r; c < nz; c += kRowsTC) {
+            const int row = z0 + c / 16, ch = c % 16;
+            const int h = ch >> 3, cc = ch & 7;
+            st_shared_v4(vst + h * kKeysTC * 128 + row * 128 + ((cc ^ (row & 7)) << 4), 0, 0, 0, 0);
+          }
+        } else {
+          fail();
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kPFull + sb]);
+    }
+    // ---- epilogue: O / l -> out ----
+    bool ok = !flags[0] && ntiles > 0 &&
+              mbar_wait(&bars[kPvDone + ((ntiles - 1) & 1)], ((ntiles - 1) >> 1) & 1);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && ntiles > 0) fail();
+    tc_fence_after();
+    const bool write = tok < ntok && r < TPT * G;
+    const float inv = (ok && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
+    T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * D;
+#pragma unroll 1
+    for (int cblk = 0; cblk < D / 32; ++cblk) {
+      uint32_t o[32];
+      tmem_ld32(tmem_o + lane_off + cblk * 32, o);
+      tmem_wait_ld();
+      if (write) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 v;
+          v.x = TT::pack(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+          v.y = TT::pack(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+          v.z = TT::pack(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+          v.w = TT::pack(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+          *reinterpret_cast<uint4 *>(dst + cblk * 32 + i) = v;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_tc() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+template <typename T, int BS>
+cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
+  auto fn = encode_fn_tc();
+  if (!fn) return cudaErrorNotSupported;
+  constexpr int D = kHeadDim;
+  const int G = a.group;
+  const int TPT = kRowsTC / G;
+  CUtensorMap tmq, tmk, tmv;
+  {  // q viewed as [tokens][Hk][G][D]; box = TPT tokens x G heads x 64 columns
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)G, (cuuint64_t)a.num_kv_heads,
+                          (cuuint64_t)a.num_q_tokens};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)G * D * 2, (cuuint64_t)a.num_heads * D * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)TPT};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (fn(&tmq, TcType<T>::kTma, 4, const_cast<void *>(a.q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  for (int i = 0; i < 2; ++i) {
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)a.num_blocks * a.num_kv_heads * BS};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)BS};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(i ? &tmv : &tmk, TcType<T>::kTma, 2, const_cast<void *>(i ? a.v_cache : a.k_cache), dims,
+           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto kern = chunk_tc_kernel<T, BS>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcLayout::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int tiles = (a.max_query_len + TPT - 1) / TPT;
+  const int64_t grid = (int64_t)a.num_seqs * a.num_kv_heads * tiles;
+  if (grid == 0) return cudaSuccess;
+  kern<<<(unsigned)grid, kThreadsTC, TcLayout::kBytes, stream>>>(a, tmq, tmk, tmv, tiles);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_tc_supported(const AttnArgs &a, int dtype) {
+  return (dtype == PA_BF16 || dtype == PA_F16) && a.head_dim == kHeadDim && a.group >= 1 &&
+         a.group <= kRowsTC && kRowsTC % a.group == 0 && encode_fn_tc() != nullptr;
+}
+
+cudaError_t launch_chunk_tc(const AttnArgs &a, int dtype, cudaStream_t stream) {
+  if (dtype == PA_BF16)
+    return a.block_size == 16 ? launch_tc_t<__nv_bfloat16, 16>(a, stream)
+                              : launch_tc_t<__nv_bfloat16, 32>(a, stream);
+  return a.block_size == 16 ? launch_tc_t<__half, 16>(a, stream) : launch_tc_t<__half, 32>(a, stream);
+}
+
+}  // namespace pa

@@ -71,6 +71,10 @@ cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream
 cudaError_t launch_reduce(const AttnArgs &a, int dtype, cudaStream_t stream);
 int decode_max_seqs_per_launch();
 
+// Implemented in chunk_tc.cu (tcgen05 chunked-query kernel, head_dim 128)
+bool chunk_tc_supported(const AttnArgs &a, int dtype);
+cudaError_t launch_chunk_tc(const AttnArgs &a, int dtype, cudaStream_t stream);
+
 // Implemented in chunk.cu
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int num_q_tokens, cudaStream_t stream);
 

@@ -47,6 +47,17 @@ def decode_kernel(request, monkeypatch):
     return request.param
 
 
+@pytest.fixture(params=["auto", "mma"])
+def chunk_kernel(request, monkeypatch):
+    """Chunked-query rows through the default kernel (tcgen05 at head_dim 128)
+    and through the mma.sync kernel forced."""
+    if request.param == "mma":
+        monkeypatch.setenv("PA_CHUNK_KERNEL", "mma")
+    else:
+        monkeypatch.delenv("PA_CHUNK_KERNEL", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("split", [0, 32, 1 << 20], ids=["policy", "split32", "nosplit"])
 @pytest.mark.parametrize("cfg", workloads.SMALL_CONFIGS)
 def test_small_config_parity(lib, cfg, split, decode_kernel):
@@ -104,20 +115,30 @@ def test_edge_lengths(lib, H, Hk, D, dtype, bs, decode_kernel):
 
 @pytest.mark.parametrize("dtype,D,bs", [("bf16", 128, 16), ("f16", 64, 32), ("f32", 64, 16),
                                         ("bf16", 64, 32)])
-def test_chunked_rows(lib, dtype, D, bs, decode_kernel):
+def test_chunked_rows(lib, dtype, D, bs, decode_kernel, chunk_kernel):
     wl = workloads.mixed_workload(f"chunk_{dtype}_{D}_{bs}", 3200, 2, 100, 900, 3, 150, 37,
                                   16, 4, D, bs, dtype)
     _check_workload(lib, wl)
 
 
-def test_chunk_group_eight(lib):
+def test_chunk_group_eight(lib, chunk_kernel):
     wl = workloads.mixed_workload("chunk_g8", 3300, 1, 300, 400, 2, 64, 20, 64, 8, 128, 16, "bf16")
     _check_workload(lib, wl)
 
 
-def test_chunk_whole_prompt(lib):
+def test_chunk_whole_prompt(lib, chunk_kernel):
     # a chunk that is the whole context (L == Q): row t sees keys 0..t
     wl = workloads.mixed_workload("chunk_full", 3400, 1, 5, 9, 2, 0, 77, 32, 8, 128, 16, "bf16")
+    _check_workload(lib, wl)
+
+
+@pytest.mark.parametrize("G,bs,dtype", [(1, 16, "bf16"), (2, 32, "f16"), (8, 32, "bf16"),
+                                        (16, 16, "bf16"), (4, 16, "f16")])
+def test_chunk_shapes(lib, G, bs, dtype, chunk_kernel):
+    # groups 1..16, both block sizes, chunk lengths that leave ragged tiles
+    Hk = 2
+    wl = workloads.mixed_workload(f"chunk_shapes_{G}_{bs}_{dtype}", 3500 + G, 2, 50, 400, 3, 131, 45,
+                                  G * Hk, Hk, 128, bs, dtype)
     _check_workload(lib, wl)
 
 
