@@ -488,8 +488,19 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--memory-report", action="store_true",
+                    help="host only: KV slots held by paged blocks vs max-length reservation")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.memory_report:
+        from paged_kv_cache_388_b200.memory import pool_usage, waste_report
+        for cfg, max_len in (("1", 100), ("2", 2048), ("3", 4096), ("4", 1536), ("4cow", 1528),
+                             ("5", 131072), ("5bs32", 131072)):
+            wl = workloads.make(cfg)
+            rep = waste_report(wl.seq_context_lens(), wl.block_size, max_len)
+            rep["pool"] = pool_usage(build_batch(wl).allocator)
+            print(json.dumps({"config": wl.name, "reservation_len": max_len, **rep}), flush=True)
+        return
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
