@@ -82,6 +82,44 @@ def profiled_traffic(config):
     return int(fields["traffic_bytes_per_launch"])
 
 
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def chunk_flops(batch):
+    """Multiply-add FLOPs of the chunked-query rows (QK^T and PV over the keys
+    each row may see): sum over rows of visible keys * H * D * 4."""
+    qsl = batch.query_start_loc
+    if qsl is None:
+        return 0
+    total = 0
+    for i, L in enumerate(batch.context_lens.tolist()):
+        Q = int(qsl[i + 1] - qsl[i])
+        if Q <= 1:
+            continue
+        total += sum(L - Q + t + 1 for t in range(Q))
+    return total
+
+
+def sub_batch(batch, keep):
+    """Rows of the batch for the sequences `keep` (decode-only or chunk-only)."""
+    keep = list(keep)
+    bt = batch.block_tables[keep]
+    cl = batch.context_lens[keep]
+    qsl = batch.query_start_loc
+    if qsl is None:
+        return bt, cl, None, np.asarray(keep, dtype=np.int64)
+    rows, starts = [], [0]
+    for i in keep:
+        rows.extend(range(int(qsl[i]), int(qsl[i + 1])))
+        starts.append(len(rows))
+    return bt, cl, np.asarray(starts, dtype=np.int32), np.asarray(rows, dtype=np.int64)
+
+
 def elem_bytes(dtype):
     return {"f32": 4, "f16": 2, "bf16": 2}[dtype]
 
@@ -378,6 +416,35 @@ def run_ours(args, rank, world, local_rank):
                                               max_context_len=mcl))
     res_avg = time_graph(lambda: cache.write(key, value, slot))
 
+    # Mixed batches: the decode rows and the chunked-query rows, each timed alone
+    parts = {}
+    if batch.query_start_loc is not None:
+        qsl_np = batch.query_start_loc
+        dec_ids = [i for i in range(batch.num_seqs) if qsl_np[i + 1] - qsl_np[i] == 1]
+        chk_ids = [i for i in range(batch.num_seqs) if qsl_np[i + 1] - qsl_np[i] > 1]
+        for name, ids in (("decode_rows", dec_ids), ("chunk_rows", chk_ids)):
+            if not ids:
+                continue
+            sbt, scl, sqsl, srows = sub_batch(batch, ids)
+            sq = q[torch.from_numpy(srows).to(dev)].contiguous()
+            sout = torch.empty_like(sq)
+            t_bt = torch.from_numpy(np.ascontiguousarray(sbt)).to(dev)
+            t_cl = torch.from_numpy(np.ascontiguousarray(scl)).to(dev)
+            t_qsl = None if sqsl is None else torch.from_numpy(sqsl).to(dev)
+            mql = int(max(np.diff(sqsl))) if sqsl is not None else 1
+            if t_qsl is not None and mql == 1:
+                t_qsl = None
+            parts[name] = {"ms": time_graph(lambda: cache.attend(
+                sq, t_bt, t_cl, wl.scale, out=sout, query_start_loc=t_qsl, max_query_len=mql,
+                max_context_len=int(scl.max())))}
+        if "decode_rows" in parts:
+            dbytes, _, _ = seq_bytes(wl, batch, dec_ids)
+            parts["decode_rows"]["GBps"] = dbytes / (parts["decode_rows"]["ms"] * 1e-3) / 1e9
+        if "chunk_rows" in parts:
+            fl = chunk_flops(batch) * wl.num_heads * wl.head_dim * 4
+            parts["chunk_rows"]["flops"] = fl
+            parts["chunk_rows"]["TFLOPs"] = fl / (parts["chunk_rows"]["ms"] * 1e-3) / 1e12
+
     # ---- end to end through the public API, host (pinned) buffers ----------
     hq = vals["q"].pin_memory()
     hkey = vals["new_key"].pin_memory()
@@ -471,6 +538,7 @@ def run_ours(args, rank, world, local_rank):
         "kernels_ms": {"pa_decode": dec_avg, "pa_reshape_and_cache": res_avg},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        **({"parts": parts} if parts else {}),
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
