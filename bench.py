@@ -37,7 +37,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import workloads  # noqa: E402
-from paged_kv_cache_388_b200.batch import build_batch  # noqa: E402
+from paged_kv_cache_388_b200.batch import build_batch, shared_prefix_groups  # noqa: E402
 
 METRIC = "paged decode attention: achieved HBM GB/s (% of peak) and decode tokens/s"
 UNIT = "GB/s"
@@ -342,6 +342,26 @@ def run_ours(args, rank, world, local_rank):
     cache.workspace(batch.num_seqs, wl.num_heads, mcl)
     stream = torch.cuda.current_stream(dev)
 
+    # Batches whose sequences share prompt blocks (parallel sampling) attend
+    # through the shared-prefix entry point unless --plain-decode is given.
+    shared = wl.kind == "shared_prefix" and not args.plain_decode
+    if shared:
+        gs_np, gb_np = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)
+        gs = torch.from_numpy(gs_np).to(dev)
+        gb = torch.from_numpy(gb_np).to(dev)
+        max_group = int(np.diff(gs_np).max())
+
+    def attend_plain():
+        cache.attend(q, bt, cl, wl.scale, out=out, query_start_loc=qsl,
+                     max_query_len=batch.max_query_len, max_context_len=mcl)
+
+    def attend():
+        if shared:
+            cache.attend_shared_prefix(q, bt, cl, gs, gb, wl.scale, max_group_size=max_group,
+                                       out=out, max_context_len=mcl)
+        else:
+            attend_plain()
+
     K = args.steps
 
     def step(evs=None):
@@ -352,8 +372,7 @@ def run_ours(args, rank, world, local_rank):
         cache.write(key, value, slot)
         if evs:
             evs[1].record(stream)
-        cache.attend(q, bt, cl, wl.scale, out=out, query_start_loc=qsl,
-                     max_query_len=batch.max_query_len, max_context_len=mcl)
+        attend()
         if evs:
             evs[2].record(stream)
 
@@ -411,13 +430,22 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1) / K
 
-    dec_avg = time_graph(lambda: cache.attend(q, bt, cl, wl.scale, out=out, query_start_loc=qsl,
-                                              max_query_len=batch.max_query_len,
-                                              max_context_len=mcl))
+    dec_avg = time_graph(attend)
     res_avg = time_graph(lambda: cache.write(key, value, slot))
 
     # Mixed batches: the decode rows and the chunked-query rows, each timed alone
     parts = {}
+    if shared:  # the same batch through plain decode (every shared block read per sequence)
+        plain_ms = time_graph(attend_plain)
+        logical = sum(int(batch.context_lens[i]) for i in range(batch.num_seqs)) * 2 * \
+            wl.num_kv_heads * wl.head_dim * elem_bytes(wl.dtype)
+        parts["plain_decode"] = {"ms": plain_ms,
+                                 "GBps_unique": nbytes["decode"] / (plain_ms * 1e-3) / 1e9}
+        parts["shared_prefix"] = {"ms": dec_avg,
+                                  "GBps_unique": nbytes["decode"] / (dec_avg * 1e-3) / 1e9,
+                                  "groups": int(gb_np.shape[0]),
+                                  "shared_blocks": int(gb_np.max()),
+                                  "logical_kv_bytes": logical}
     if batch.query_start_loc is not None:
         qsl_np = batch.query_start_loc
         dec_ids = [i for i in range(batch.num_seqs) if qsl_np[i + 1] - qsl_np[i] == 1]
@@ -455,7 +483,7 @@ def run_ours(args, rank, world, local_rank):
     hout = torch.empty_like(hq).pin_memory()
     h2d = PagedKVCache.host_bytes(hq, hkey, hval, hslot, hbt, hcl)
     d2h = PagedKVCache.host_bytes(hout)
-    e2e_ok = batch.query_start_loc is None and cow.shape[0] == 0
+    e2e_ok = batch.query_start_loc is None and cow.shape[0] == 0 and not shared
     e2e = None
     if e2e_ok:
         # the public API's captured host step: copy in, write K/V, attend, copy out
@@ -489,7 +517,7 @@ def run_ours(args, rank, world, local_rank):
 
     splits = ws_bytes > 0  # the decode call also launches its merge kernel
     launches_per_step = 1 + 1 + (1 if splits else 0) + (1 if cow.shape[0] else 0) + \
-        (1 if batch.max_query_len > 1 else 0)
+        (1 if batch.max_query_len > 1 else 0) + (1 if shared else 0)
     peak, peak_kind = hbm_peak()
     achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
     value = job_bytes / (ms * 1e-3) / 1e9
@@ -521,7 +549,9 @@ def run_ours(args, rank, world, local_rank):
         "decode_tokens_per_s": batch.num_seqs * world * K / (ms * 1e-3),
         "pct_of_nominal_8TBps": 100.0 * value / NOMINAL_HBM_GBS,
         "roofline": {
-            "kernel": "pa_decode (paged_decode_mma_kernel + balanced_merge_kernel)",
+            "kernel": ("pa_decode_shared_prefix (shared_prefix_kernel + paged_decode_mma_kernel + "
+                       "balanced_merge_kernel)") if shared else
+                      "pa_decode (paged_decode_mma_kernel + balanced_merge_kernel)",
             "bound": "hbm",
             "achieved": achieved,
             "peak": peak,
@@ -535,7 +565,8 @@ def run_ours(args, rank, world, local_rank):
             "algorithmic_bytes": nbytes["decode"],
             "avg_ms": dec_avg,
         },
-        "kernels_ms": {"pa_decode": dec_avg, "pa_reshape_and_cache": res_avg},
+        "kernels_ms": {("pa_decode_shared_prefix" if shared else "pa_decode"): dec_avg,
+                       "pa_reshape_and_cache": res_avg},
         "cpu_baseline": cpu,
         "e2e": e2e,
         **({"parts": parts} if parts else {}),
@@ -556,6 +587,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plain-decode", action="store_true",
+                    help="attend shared-prefix batches with pa_decode instead of "
+                         "pa_decode_shared_prefix")
     ap.add_argument("--memory-report", action="store_true",
                     help="host only: KV slots held by paged blocks vs max-length reservation")
     args = ap.parse_args()

@@ -62,6 +62,11 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
 #define PA_DEVERR_CONTEXT_LEN 0x4u /* context_len < 0 or > max_blocks_per_seq*block_size */
 #define PA_DEVERR_QUERY_LEN 0x8u   /* query rows of a sequence exceed its context */
 #define PA_DEVERR_TIMEOUT 0x10u    /* a bounded wait inside a kernel expired */
+#define PA_DEVERR_PREFIX 0x20u     /* pa_decode_shared_prefix: malformed group arrays,
+                                      a member whose context is shorter than the
+                                      group's shared prefix, or a member whose block
+                                      table differs from the group's first sequence
+                                      over the shared range */
 
 /*
  * pa_reshape_and_cache -- write this step's new K/V into their cache slots.
@@ -197,6 +202,63 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache,
 
 /* Size of the static scratch array pa_decode_noalloc uses, in bytes. */
 size_t pa_noalloc_scratch_bytes(void);
+
+/*
+ * pa_decode_shared_prefix -- decode attention for batches in which groups of
+ * sequences share the leading blocks of their block tables.
+ *
+ * Defined by: sequences forked from one prompt (parallel sampling, beam
+ * search) map the prompt's logical blocks to the same physical blocks and
+ * own only the blocks written after the fork ("理解 vLLM PagedAttention",
+ * section 六; "核心概念", section 内存共享; "PagedAttention 实战", section
+ * PagedAttention 的核心, item 3).  The result is exactly pa_decode's (the
+ * sharing changes where the keys live, not the attention): for every
+ * sequence i and head h, out = softmax(scale * q . K_i^T) V_i over all
+ * context_lens[i] keys.  Only the work differs: the shared blocks of a group
+ * are read once for all of its sequences' query rows (members x GROUP heads
+ * of one KV head form one matrix product), the private tails are read per
+ * sequence, and the two partial softmax results are merged.
+ *
+ *   out, q, k_cache, v_cache, block_tables, context_lens, scale,
+ *   max_context_len: as for pa_decode with one query row per sequence
+ *                    (num_q_tokens == num_seqs, no query_start_loc).
+ *   group_start      int32 [num_groups + 1], device: group j is sequences
+ *                    group_start[j] .. group_start[j+1]-1.  Nondecreasing,
+ *                    within [0, num_seqs]; sequences outside every group
+ *                    are plain decode sequences.
+ *   group_shared_blocks int32 [num_groups], device: P_j, the number of
+ *                    leading block-table entries that every member of group
+ *                    j holds in common (the ids of the group's first
+ *                    sequence are used); those blocks must be full
+ *                    (P_j * block_size <= every member's context length).
+ *                    P_j = 0 makes the group plain decode sequences.
+ *   max_group_size   host-side upper bound of any group's size (<= 0: num_seqs)
+ *   workspace        >= pa_decode_shared_prefix_workspace_size(...) bytes;
+ *                    contents need no initialisation.
+ * Supported: 16-bit caches (PA_F16, PA_BF16), num_seqs <= 2048, and the
+ * head_dim / block_size / group list above.
+ * Device checks: malformed group arrays (decreasing or out of range) make
+ * every sequence plain decode -- results stay correct -- and set
+ * PA_DEVERR_PREFIX; a member whose context is shorter than P_j * block_size
+ * or whose table differs from the first sequence's in the shared range gets
+ * zero output and PA_DEVERR_PREFIX.
+ */
+int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_tables,
+                            int max_blocks_per_seq, const int32_t *context_lens,
+                            int num_seqs, const int32_t *group_start,
+                            const int32_t *group_shared_blocks, int num_groups,
+                            int max_group_size, int num_heads, int num_kv_heads,
+                            int head_dim, int block_size, int num_blocks,
+                            float scale, int max_context_len, int dtype,
+                            void *workspace, size_t workspace_bytes,
+                            struct CUstream_st *stream);
+
+/* Workspace bytes pa_decode_shared_prefix needs (current device). */
+size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_heads,
+                                              int num_kv_heads, int head_dim,
+                                              int block_size,
+                                              int max_context_len);
 
 /*
  * pa_get_device_error -- synchronise `stream`, then read and clear the

@@ -38,6 +38,11 @@ _lib.pa_decode.restype = I
 _lib.pa_decode.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, I, I, P, SZ, P]
 _lib.pa_decode_noalloc.restype = I
 _lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, I, I, P]
+_lib.pa_decode_shared_prefix.restype = I
+_lib.pa_decode_shared_prefix.argtypes = [P, P, P, P, P, I, P, I, P, P, I, I, I, I, I, I, I, F, I, I,
+                                         P, SZ, P]
+_lib.pa_decode_shared_prefix_workspace_size.restype = SZ
+_lib.pa_decode_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I]
 _lib.pa_noalloc_scratch_bytes.restype = SZ
 _lib.pa_noalloc_scratch_bytes.argtypes = []
 _lib.pa_get_device_error.restype = I
@@ -55,6 +60,7 @@ PA_DEVERR_SLOT = 0x2
 PA_DEVERR_CONTEXT_LEN = 0x4
 PA_DEVERR_QUERY_LEN = 0x8
 PA_DEVERR_TIMEOUT = 0x10
+PA_DEVERR_PREFIX = 0x20
 
 
 class PAError(RuntimeError):
@@ -181,6 +187,48 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scal
                                 int(max_context_len), int(kv_split_tokens), _DT[q.dtype],
                                 _stream(stream))
     _check(rc, "pa_decode_noalloc")
+
+
+def pa_decode_shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                           max_context_len) -> int:
+    return int(_lib.pa_decode_shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads,
+                                                           head_dim, block_size, max_context_len))
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                            group_shared_blocks, scale, max_group_size=0, max_context_len=0,
+                            workspace=None, stream=None):
+    """Decode with shared-prefix groups.  out/q [S, H, D]; group_start int32
+    [G+1] and group_shared_blocks int32 [G] on the device; workspace: uint8
+    CUDA tensor of >= pa_decode_shared_prefix_workspace_size(...) bytes."""
+    _dev(q, "q")
+    _dev(out, "out", q.dtype)
+    _dev(k_cache, "k_cache", q.dtype)
+    _dev(v_cache, "v_cache", q.dtype)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    _dev(group_start, "group_start", torch.int32)
+    _dev(group_shared_blocks, "group_shared_blocks", torch.int32)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+    s, h, d = q.shape
+    nb, hk, bs, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    s2, mbps = block_tables.shape
+    if s2 != s or context_lens.shape[0] != s:
+        raise ValueError("q, block_tables and context_lens disagree on the number of sequences")
+    g = group_shared_blocks.shape[0]
+    if group_start.shape[0] != g + 1:
+        raise ValueError("group_start must have one more entry than group_shared_blocks")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.pa_decode_shared_prefix(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(block_tables), mbps, _ptr(context_lens), s,
+                                      _ptr(group_start), _ptr(group_shared_blocks), g,
+                                      int(max_group_size), h, hk, d, bs, nb, float(scale),
+                                      int(max_context_len), _DT[q.dtype], _ptr(workspace),
+                                      ws_bytes, _stream(stream))
+    _check(rc, "pa_decode_shared_prefix")
 
 
 def pa_noalloc_scratch_bytes() -> int:

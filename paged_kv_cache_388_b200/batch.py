@@ -86,3 +86,38 @@ def build_batch(wl) -> Batch:
         max_query_len=max(qlens) if qlens else 0,
         allocator=alloc,
     )
+
+
+def shared_prefix_groups(block_tables: np.ndarray, context_lens: np.ndarray, block_size: int,
+                         min_shared_blocks: int = 1):
+    """Group consecutive sequences whose block tables start with the same
+    physical blocks (forks of one prompt share them until they diverge).
+
+    Returns ``(group_start, group_shared_blocks)``, int32 arrays of G+1 and G
+    entries covering every sequence: group j is sequences
+    group_start[j] .. group_start[j+1]-1, which share their first
+    group_shared_blocks[j] block-table entries.  Only blocks that every member
+    has filled count (shared blocks * block_size <= each member's context).
+    A sequence that shares fewer than ``min_shared_blocks`` blocks with the
+    sequence before it starts a new group; groups of one sequence get 0.
+    """
+    bt = np.asarray(block_tables)
+    lens = np.asarray(context_lens, dtype=np.int64)
+    n = lens.shape[0]
+    starts, shared = [0], []
+    s = 0
+    while s < n:
+        p = int(lens[s] // block_size)
+        e = s + 1
+        while e < n:
+            lim = min(p, int(lens[e] // block_size))
+            same = bt[s, :lim] == bt[e, :lim]
+            c = lim if same.all() else int(np.argmin(same))
+            if c < min_shared_blocks:
+                break
+            p = c
+            e += 1
+        shared.append(p if e - s > 1 else 0)
+        starts.append(e)
+        s = e
+    return np.asarray(starts, dtype=np.int32), np.asarray(shared, dtype=np.int32)

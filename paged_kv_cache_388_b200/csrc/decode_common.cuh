@@ -39,7 +39,8 @@ struct Item {
   int nsplit;
   int kvh;
   int b0, b1;  // KV blocks [b0, b1) of the sequence
-  int L;       // keys visible to the row
+  int L;       // keys visible to the row, counted from block boff
+  int boff;    // leading blocks of the sequence left to the shared-prefix kernel
   unsigned int bad_bits;  // PA_DEVERR_* of an invalid sequence (0: ok)
 };
 
@@ -48,23 +49,56 @@ struct BatchSmem {
   int *len;     // [n] context length
   int *q0;      // [n] first query row
   int *ql;      // [n] query rows
+  int *pre;     // [n] leading blocks shared with the sequence's group (0: none)
   int *prefix;  // [n+1] items before sequence s (in units of KV-head groups)
   int *scan;    // [32] scratch
-  static constexpr int bytes(int n) { return 4 * (4 * n + 1) + 4 * 32 + 16; }
+  static constexpr int bytes(int n) { return 4 * (5 * n + 1) + 4 * 32 + 16; }
   __device__ void carve(unsigned char *base, int n) {
     len = reinterpret_cast<int *>(base);
     q0 = len + n;
     ql = q0 + n;
-    prefix = ql + n;
-    scan = reinterpret_cast<int *>(base + align_up(4 * (4 * n + 1), 16));
+    pre = ql + n;
+    prefix = pre + n;
+    scan = reinterpret_cast<int *>(base + align_up(4 * (5 * n + 1), 16));
   }
 };
 
-// KV blocks of a decode sequence (one query row, valid length), else 0: the
-// unit of the balanced partition.
-__device__ __forceinline__ int unit_blocks(const AttnArgs &a, int L, int qlen) {
+// KV blocks of a decode sequence (one query row, valid length) after its
+// `pre` shared-prefix blocks, else 0: the unit of the balanced partition.
+__device__ __forceinline__ int unit_blocks(const AttnArgs &a, int L, int qlen, int pre) {
   if (qlen != 1 || L <= 0 || L > a.max_context_len) return 0;
-  return ceil_div(L, a.block_size);
+  const int tail = L - pre * a.block_size;
+  return tail > 0 ? ceil_div(tail, a.block_size) : 0;
+}
+
+// Shared-prefix groups -> b.pre[s], the leading KV blocks of sequence s that
+// the prefix kernel attends (0 outside every group and when the call has no
+// groups).  The group arrays are one list of boundaries, so checking that
+// every group is an in-range, nondecreasing range [start_j, start_j+1) with a
+// block count inside the table proves that the groups are disjoint.  When any
+// group fails, no sequence takes the shared path: each is attended in full by
+// the decode kernel (the result is the same) and PA_DEVERR_PREFIX is raised.
+// Called by every thread of the CTA; ends with a barrier.
+__device__ __forceinline__ void scan_groups(const AttnArgs &a, const BatchSmem &b, int n) {
+  for (int s = threadIdx.x; s < n; s += blockDim.x) b.pre[s] = 0;
+  bool ok = true;
+  if (a.pre_rec) {
+    for (int j = threadIdx.x; j < a.num_groups; j += blockDim.x) {
+      const int s0 = a.grp_start[j], s1 = a.grp_start[j + 1], nb = a.grp_blocks[j];
+      ok = ok && 0 <= s0 && s0 <= s1 && s1 <= n && 0 <= nb && nb <= a.max_blocks_per_seq;
+    }
+  }
+  const bool all_ok = __syncthreads_and(ok) != 0;
+  if (!a.pre_rec) return;
+  if (!all_ok) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_error(a.err, PA_DEVERR_PREFIX);
+    return;
+  }
+  for (int j = threadIdx.x; j < a.num_groups; j += blockDim.x) {
+    const int s0 = a.grp_start[j], s1 = a.grp_start[j + 1], nb = a.grp_blocks[j];
+    for (int s = s0; s < s1; ++s) b.pre[s] = nb;
+  }
+  __syncthreads();
 }
 
 // Called by every thread of the CTA; ends with __syncthreads().  prefix[s]
@@ -72,6 +106,7 @@ __device__ __forceinline__ int unit_blocks(const AttnArgs &a, int L, int qlen) {
 // sequences before s.
 template <bool BAL = false>
 __device__ __forceinline__ void scan_batch(const AttnArgs &a, const BatchSmem &b, int n) {
+  scan_groups(a, b, n);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
   const int per = ceil_div(n, nthreads);
   const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
@@ -91,7 +126,7 @@ __device__ __forceinline__ void scan_batch(const AttnArgs &a, const BatchSmem &b
     b.len[s] = L;
     b.q0[s] = q0;
     b.ql[s] = q1 - q0;
-    local += BAL ? unit_blocks(a, L, q1 - q0) : seq_items(a, L, q1 - q0);
+    local += BAL ? unit_blocks(a, L, q1 - q0, b.pre[s]) : seq_items(a, L, q1 - q0);
   }
   int x = local;  // block exclusive scan of `local`
 #pragma unroll
@@ -115,7 +150,7 @@ __device__ __forceinline__ void scan_batch(const AttnArgs &a, const BatchSmem &b
   int run = (warp ? b.scan[warp - 1] : 0) + x - local;
   for (int s = s0; s < s1; ++s) {
     b.prefix[s] = run;
-    run += BAL ? unit_blocks(a, b.len[s], b.ql[s]) : seq_items(a, b.len[s], b.ql[s]);
+    run += BAL ? unit_blocks(a, b.len[s], b.ql[s], b.pre[s]) : seq_items(a, b.len[s], b.ql[s]);
   }
   if (tid == nthreads - 1) b.prefix[n] = run;
   __syncthreads();
@@ -135,6 +170,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs &a, const BatchSmem &
   const int q0 = b.q0[lo];
   const int qlen = b.ql[lo];
   it.bad_bits = 0;
+  it.boff = 0;
   if (L < 0 || L > a.max_context_len) it.bad_bits = PA_DEVERR_CONTEXT_LEN;
   else if (qlen > L && L > 0) it.bad_bits = PA_DEVERR_QUERY_LEN;
   if (qlen > 1) {  // row mode: one item per query row, never split
@@ -238,7 +274,8 @@ struct SegIter {
     it.kvh = kvh;
     it.b0 = b0;
     it.b1 = b1;
-    it.L = b.len[lo];
+    it.boff = b.pre[lo];
+    it.L = b.len[lo] - it.boff * a.block_size;
     it.bad_bits = 0;
     const bool complete = b0 == 0 && b1 == nb;
     seg->out = complete ? kOutDirect : kOutRecord;
@@ -270,6 +307,27 @@ __device__ __forceinline__ void store4<__half>(__half *dst, float4 v) {
   u.x = *reinterpret_cast<uint32_t *>(&lo);
   u.y = *reinterpret_cast<uint32_t *>(&hi);
   *reinterpret_cast<uint2 *>(dst) = u;
+}
+
+// Merge one partial softmax result (accumulator slice x, running max m in
+// base 2, running sum l; l = NaN marks a poisoned record) into (M, Lsum, o).
+__device__ __forceinline__ void fold_record(const float *x4, float m, float l, float *M,
+                                            float *Lsum, float4 *o, bool *bad) {
+  if (isnan(l)) {
+    *bad = true;
+    return;
+  }
+  const float Mn = fmaxf(*M, m);
+  if (Mn == -INFINITY) return;
+  const float sa = *M == -INFINITY ? 0.f : fast_exp2(*M - Mn);
+  const float sb = m == -INFINITY ? 0.f : fast_exp2(m - Mn);
+  const float4 x = *reinterpret_cast<const float4 *>(x4);
+  o->x = o->x * sa + x.x * sb;
+  o->y = o->y * sa + x.y * sb;
+  o->z = o->z * sa + x.z * sb;
+  o->w = o->w * sa + x.w * sb;
+  *Lsum = *Lsum * sa + l * sb;
+  *M = Mn;
 }
 
 // Merge area written by the consumer warps at the end of an item: warp w, its
@@ -311,6 +369,11 @@ __device__ __forceinline__ void merge_store(const AttnArgs &a, const Seg &seg,
       o.w += wgt * x.w;
     }
     const int head = item.kvh * a.group + hg;
+    if (seg.out == kOutDirect && item.boff > 0) {
+      // the sequence's shared prefix: fold in the prefix kernel's partial
+      const float *pr = a.pre_rec + ((int64_t)item.seq * a.num_heads + head) * (D + 4);
+      fold_record(pr + d4 * 4, pr[D], pr[D + 1], &M, &Lsum, &o, &anybad);
+    }
     if (seg.out == kOutDirect) {
       const float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
       T *dst = static_cast<T *>(a.out) + ((int64_t)item.qrow * a.num_heads + head) * D + d4 * 4;

@@ -35,14 +35,23 @@ namespace {
 
 using namespace dec;
 
+// CTA shape: PA_MMA_WARPS consumer warps + 1 producer, a K/V ring of
+// PA_MMA_RING_KB KiB, register budget for PA_MMA_MIN_CTAS resident CTAs per
+// SM.  Many small CTAs (2 consumer warps, 3 blocks of 16 tokens in flight
+// each, 5 per SM) keep more independent (sequence, KV head) pieces streaming
+// per SM than a few large ones: each piece ends with a cross-warp merge and
+// starts with a dependent block-table read, and short contexts have many
+// pieces.  Measured on B200: decode of 256 x U[1,512]-token sequences 105 ->
+// 75 us, the Llama-3-8B-shaped batch 178 -> 172 us against 4 warps / 48 KiB /
+// 3 per SM.
 #ifndef PA_MMA_RING_KB
-#define PA_MMA_RING_KB 48
+#define PA_MMA_RING_KB 24
 #endif
 #ifndef PA_MMA_MIN_CTAS
-#define PA_MMA_MIN_CTAS 3
+#define PA_MMA_MIN_CTAS 5
 #endif
 #ifndef PA_MMA_WARPS
-#define PA_MMA_WARPS 4
+#define PA_MMA_WARPS 2
 #endif
 
 constexpr int kMaxSeqsPerLaunch = 2048;
@@ -191,18 +200,37 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
   if (a.balanced && tid == 0) a.bal_desc[4 * blockIdx.x] = -1;  // no cut pair starts here (yet)
   if (a.balanced) {
     scan_batch<true>(a, bsm, n);
-    if (blockIdx.x == 0)  // block prefix for the merge kernel
+    if (blockIdx.x == 0) {  // block prefix (and shared blocks) for the merge kernel
       for (int s = tid; s <= n; s += blockDim.x) a.bal_prefix[s] = bsm.prefix[s];
-    // Decode sequences with no KV blocks (empty or invalid context) own no
-    // part of the partition: their rows are written as zeros here.
+      if (a.seq_pre)
+        for (int s = tid; s < n; s += blockDim.x) a.seq_pre[s] = bsm.pre[s];
+    }
+    // Decode sequences with no KV blocks of their own (empty or invalid
+    // context, or every key inside the group's shared prefix) own no part of
+    // the partition: their rows are written here, from the prefix kernel's
+    // partial when all keys are shared, else as zeros.
     if (warp < NCW) {
       for (int s = blockIdx.x; s < n; s += gridDim.x) {
         if (bsm.ql[s] != 1 || bsm.prefix[s + 1] != bsm.prefix[s]) continue;
         const int L = bsm.len[s];
-        if (L != 0 && tid == 0) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
+        const int pre = bsm.pre[s];
+        const bool valid = L >= 0 && L <= a.max_context_len;
+        const bool shared_only = valid && pre > 0 && L >= pre * a.block_size;
+        if (tid == 0 && !shared_only && (L != 0 || pre > 0))
+          raise_error(a.err, valid && pre > 0 ? PA_DEVERR_PREFIX : PA_DEVERR_CONTEXT_LEN);
         T *row = static_cast<T *>(a.out) + (int64_t)bsm.q0[s] * a.num_heads * D;
-        for (int i = tid; i < a.num_heads * D / 4; i += NCW * 32)
-          store4<T>(row + 4 * i, make_float4(0.f, 0.f, 0.f, 0.f));
+        for (int i = tid; i < a.num_heads * D / 4; i += NCW * 32) {
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (shared_only) {
+            const int h = i / (D / 4), d4 = i - h * (D / 4);
+            const float *r = a.pre_rec + ((int64_t)(a.seq_begin + s) * a.num_heads + h) * (D + 4);
+            const float l = r[D + 1];
+            const float inv = (l > 0.f && !isnan(l)) ? 1.f / l : 0.f;
+            const float4 x = *reinterpret_cast<const float4 *>(r + d4 * 4);
+            v = make_float4(x.x * inv, x.y * inv, x.z * inv, x.w * inv);
+          }
+          store4<T>(row + 4 * i, v);
+        }
       }
     }
   } else {
@@ -240,7 +268,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
         }
         __syncwarp();
       }
-      const int32_t *table = a.block_tables + (int64_t)item.seq * a.max_blocks_per_seq;
+      const int32_t *table = a.block_tables + (int64_t)item.seq * a.max_blocks_per_seq + item.boff;
       for (int b = item.b0; b < item.b1; b += 32) {
         const int cnt = min(32, item.b1 - b);
         const int my_id = lane < cnt ? table[b + lane] : 0;
@@ -561,6 +589,25 @@ __global__ void __launch_bounds__(256) balanced_merge_kernel(const AttnArgs a) {
     for (int e = 0; e < PER; ++e) o[e] = o[e] * sa + x[e] * sb;
     M = Mn;
   }
+  if (a.seq_pre && a.seq_pre[qrow] > 0) {
+    // the sequence's shared prefix: fold in the prefix kernel's partial
+    // (one decode row per sequence here, so the query row is the sequence)
+    const float *r = a.pre_rec + ((int64_t)qrow * a.num_heads + kvh * grp + hg) * (D + 4);
+    const float m = r[D], l = r[D + 1];
+    if (isnan(l)) {
+      poisoned = true;
+    } else {
+      const float Mn = fmaxf(M, m);
+      if (Mn != -INFINITY) {
+        const float sa = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+        const float sb = m == -INFINITY ? 0.f : fast_exp2(m - Mn);
+        Lsum = Lsum * sa + l * sb;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o[e] = o[e] * sa + r[lane * PER + e] * sb;
+        M = Mn;
+      }
+    }
+  }
   const float inv = (Lsum > 0.f && !poisoned) ? 1.f / Lsum : 0.f;
   T *dst = static_cast<T *>(a.out) + ((int64_t)qrow * a.num_heads + kvh * grp + hg) * D + lane * PER;
 #pragma unroll
@@ -593,6 +640,27 @@ bool make_map(CUtensorMap *map, const void *base, int num_blocks, int num_kv_hea
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+bool make_cache_map(CUtensorMap *map, const void *base, int num_blocks, int num_kv_heads,
+                    int head_dim, int block_size, int dtype) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return false;
+  const bool bf = dtype == PA_BF16;
+  if (head_dim == 64)
+    return block_size == 16
+               ? (bf ? make_map<__nv_bfloat16, 64, 16>(map, base, num_blocks, num_kv_heads)
+                     : make_map<__half, 64, 16>(map, base, num_blocks, num_kv_heads))
+               : (bf ? make_map<__nv_bfloat16, 64, 32>(map, base, num_blocks, num_kv_heads)
+                     : make_map<__half, 64, 32>(map, base, num_blocks, num_kv_heads));
+  return block_size == 16
+             ? (bf ? make_map<__nv_bfloat16, 128, 16>(map, base, num_blocks, num_kv_heads)
+                   : make_map<__half, 128, 16>(map, base, num_blocks, num_kv_heads))
+             : (bf ? make_map<__nv_bfloat16, 128, 32>(map, base, num_blocks, num_kv_heads)
+                   : make_map<__half, 128, 32>(map, base, num_blocks, num_kv_heads));
+}
+
+namespace {
 
 template <typename T, int D, int BS, int NT>
 cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {

@@ -266,6 +266,151 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
   return PA_OK;
 }
 
+namespace {
+
+// Workspace of pa_decode_shared_prefix: the balanced decode scheme's records,
+// descriptors and block prefix, then the per-sequence shared block counts and
+// the prefix kernel's records [num_seqs][num_heads][head_dim + 4].
+struct SharedPrefixWs {
+  size_t desc, prefix, seq_pre, pre_rec, total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+SharedPrefixWs shared_prefix_ws(int num_seqs, int num_heads, int head_dim, int group, int grid) {
+  SharedPrefixWs w;
+  size_t off = balanced_record_bytes(grid, group, head_dim);
+  w.desc = off;
+  off += balanced_desc_bytes(grid);
+  w.prefix = off;
+  off += align256((size_t)(num_seqs + 1) * sizeof(int));
+  w.seq_pre = off;
+  off += align256((size_t)num_seqs * sizeof(int));
+  w.pre_rec = off;
+  off += align256((size_t)num_seqs * num_heads * (head_dim + 4) * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+// CTAs per cluster of the prefix kernel (ranges of the shared blocks per
+// (group, chunk, KV head)): 1 while there are at least 0.4 units per SM,
+// doubled (up to 8) until there are.  Measured on B200 (256 units of 64 blocks): prefix
+// kernel 55 us with 1, 81 us with 4.  PA_PREFIX_CLUSTER = 1, 2, 4 or 8
+// overrides.
+int prefix_cluster(int64_t units, int sm_count) {
+  const char *env = getenv("PA_PREFIX_CLUSTER");
+  if (env) {
+    const int c = atoi(env);
+    if (c == 1 || c == 2 || c == 4 || c == 8) return c;
+  }
+  // one CTA per unit while the units alone give a wave of work: a CTA's
+  // fixed cost (Q gather, first loads, merge) then is paid once
+  int c = 1;
+  while (c < 8 && units * c * 5 < (int64_t)2 * sm_count) c *= 2;
+  return c;
+}
+
+}  // namespace
+
+size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                              int head_dim, int block_size, int max_context_len) {
+  (void)block_size;
+  (void)max_context_len;
+  if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      num_heads % num_kv_heads != 0)
+    return 0;
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return 0;
+  // the decode grid is at most 8 resident CTAs per SM
+  return shared_prefix_ws(num_seqs, num_heads, head_dim, num_heads / num_kv_heads,
+                          dev.sm_count * 8).total;
+}
+
+int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *context_lens, int num_seqs,
+                            const int32_t *group_start, const int32_t *group_shared_blocks,
+                            int num_groups, int max_group_size, int num_heads, int num_kv_heads,
+                            int head_dim, int block_size, int num_blocks, float scale,
+                            int max_context_len, int dtype, void *workspace,
+                            size_t workspace_bytes, struct CUstream_st *stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || !dtype_ok(dtype) || num_groups < 0)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_heads / num_kv_heads;
+  if (!group_supported(group)) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > decode_max_seqs_per_launch()) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (num_groups > 0 && (!group_start || !group_shared_blocks)) return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (out == q) return PA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30) return PA_ERR_UNSUPPORTED;
+  const int cap = max_blocks_per_seq * block_size;
+  if (max_context_len <= 0 || max_context_len > cap) max_context_len = cap;
+  if (max_group_size <= 0 || max_group_size > num_seqs) max_group_size = num_seqs;
+
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  AttnArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start_loc = nullptr;
+  a.err = dev.err;
+  a.num_seqs = num_seqs;
+  a.seq_begin = 0;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.split_blocks = 1;
+  a.max_splits = 1;
+  a.max_query_len = 1;
+  a.max_context_len = max_context_len;
+  a.num_q_tokens = num_seqs;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.balanced = 1;
+  if (!decode_mma_supported(a, dtype) || !prefix_supported(a, dtype)) return PA_ERR_UNSUPPORTED;
+  a.grid = decode_mma_grid(a, dtype, dev.sm_count);
+  if (a.grid <= 0) return PA_ERR_CUDA;
+  const SharedPrefixWs w = shared_prefix_ws(num_seqs, num_heads, head_dim, group, a.grid);
+  if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+  char *ws = static_cast<char *>(workspace);
+  a.part_o = reinterpret_cast<float *>(ws);
+  a.bal_desc = reinterpret_cast<int *>(ws + w.desc);
+  a.bal_prefix = reinterpret_cast<int *>(ws + w.prefix);
+  a.seq_pre = reinterpret_cast<int *>(ws + w.seq_pre);
+  a.pre_rec = reinterpret_cast<float *>(ws + w.pre_rec);
+  a.grp_start = group_start;
+  a.grp_blocks = group_shared_blocks;
+  a.num_groups = num_groups;
+  const int mpc = kPrefixRows / group;
+  a.grp_chunks = (max_group_size + mpc - 1) / mpc;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (num_groups > 0) {
+    const int64_t units = (int64_t)num_groups * a.grp_chunks * num_kv_heads;
+    e = launch_prefix(a, dtype, prefix_cluster(units, dev.sm_count), s);
+  }
+  if (e == cudaSuccess) e = launch_decode_mma(a, dtype, dev.sm_count, s);
+  if (e == cudaSuccess) e = launch_balanced_reduce(a, dtype, s);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int pa_get_device_error(unsigned int *code_out, struct CUstream_st *stream) {
   if (!code_out) return PA_ERR_INVALID_ARG;
   DevInfo dev;

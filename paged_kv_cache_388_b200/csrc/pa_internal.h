@@ -1,6 +1,7 @@
 // pa_internal.h -- host-side declarations shared by the libpa translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -40,6 +41,15 @@ struct AttnArgs {
   int *bal_prefix;    // balanced: [num_seqs + 1] block prefix written by CTA 0
   int *bal_desc;      // balanced: [grid][4] cut-pair descriptors written by the decode kernel
   float scale_log2;   // scale * log2(e)
+  // Shared-prefix decode (all null / 0 otherwise).  The decode kernels read
+  // only the blocks after a sequence's shared prefix and fold in the prefix
+  // partial that the prefix kernel left in pre_rec.
+  const int32_t *grp_start;   // [num_groups + 1] first sequence of each group
+  const int32_t *grp_blocks;  // [num_groups] leading blocks the group's members share
+  int num_groups;
+  int grp_chunks;             // prefix kernel: member chunks per group
+  float *pre_rec;             // [num_seqs][num_heads][D + 4]: o (unnormalised), m, l
+  int *seq_pre;               // [num_seqs] shared blocks per sequence (decode kernel CTA 0)
 };
 
 struct DevInfo {
@@ -65,6 +75,17 @@ inline size_t balanced_record_bytes(int grid, int group, int head_dim) {
   return ((size_t)grid * 2 * group * (head_dim + 4) * sizeof(float) + 255) / 256 * 256;
 }
 inline size_t balanced_desc_bytes(int grid) { return ((size_t)grid * 4 * sizeof(int) + 255) / 256 * 256; }
+
+// 2-D tensor map of a 16-bit cache (rows = blocks * kv heads * block_size,
+// columns = head_dim; boxes of 64 columns x block_size rows, 128-byte
+// swizzle).  Implemented in decode_mma.cu.
+bool make_cache_map(CUtensorMap *map, const void *base, int num_blocks, int num_kv_heads,
+                    int head_dim, int block_size, int dtype);
+
+// Implemented in cascade.cu (shared-prefix kernel)
+constexpr int kPrefixRows = 64;  // query rows (members x group heads) per prefix CTA
+bool prefix_supported(const AttnArgs &a, int dtype);
+cudaError_t launch_prefix(const AttnArgs &a, int dtype, int cluster, cudaStream_t stream);
 
 // Implemented in decode.cu (CUDA-core kernel, fixed-split scheme)
 cudaError_t launch_decode(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream);

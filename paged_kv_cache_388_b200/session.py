@@ -53,6 +53,27 @@ class PagedKVCache:
                        max_context_len=mcl, kv_split_tokens=kv_split_tokens, workspace=ws)
         return out
 
+    def attend_shared_prefix(self, q, block_tables, context_lens, group_start, group_shared_blocks,
+                             scale, max_group_size=0, out=None, max_context_len=0):
+        """Decode (one query row per sequence) where groups of consecutive
+        sequences share the leading blocks of their tables: group j is
+        sequences group_start[j] .. group_start[j+1]-1 sharing
+        group_shared_blocks[j] blocks (see ``batch.shared_prefix_groups``).
+        Same result as ``attend``; the shared blocks are read once per group."""
+        if out is None:
+            out = torch.empty_like(q)
+        mcl = max_context_len or block_tables.shape[1] * self.block_size
+        need = _lib.pa_decode_shared_prefix_workspace_size(block_tables.shape[0], q.shape[1],
+                                                           self.num_kv_heads, self.head_dim,
+                                                           self.block_size, mcl)
+        if self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        _lib.pa_decode_shared_prefix(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
+                                     group_start, group_shared_blocks, scale,
+                                     max_group_size=max_group_size, max_context_len=mcl,
+                                     workspace=self._ws)
+        return out
+
     # ---- one step from host memory ------------------------------------------
     def _dev_like(self, name, t):
         buf = self._staging.get(name)
