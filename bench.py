@@ -579,6 +579,68 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+def run_swap(args):
+    """Swap-out / swap-in of KV blocks between the device pool and a pinned
+    host pool (pa_swap_blocks), against the host link's DMA copy rate."""
+    from paged_kv_cache_388_b200.session import PagedKVCache
+
+    dev = torch.device("cuda", 0)
+    wl = workloads.make(args.config)
+    batch = build_batch(wl)
+    vals = workloads.values(wl)
+    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                         k_cache=vals["k_pool"].to(dev), v_cache=vals["v_pool"].to(dev))
+    # preempt the first half of the sequences: every block they hold goes out
+    half = batch.num_seqs // 2
+    blocks = []
+    for i in range(half):
+        n = -(-int(batch.context_lens[i]) // wl.block_size)
+        blocks.extend(int(b) for b in batch.block_tables[i, :n])
+    blocks = np.unique(np.asarray(blocks, dtype=np.int64))
+    nb = blocks.shape[0]
+    host_k, host_v = cache.host_pool(nb)
+    out_map = torch.from_numpy(np.stack([blocks, np.arange(nb)], 1)).to(dev)
+    in_map = out_map.flip(1).contiguous()
+    block_bytes = 2 * wl.num_kv_heads * wl.block_size * wl.head_dim * elem_bytes(wl.dtype)
+    nbytes = nb * block_bytes
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    ms_out = timed(lambda: cache.swap_out(host_k, host_v, out_map))
+    ms_in = timed(lambda: cache.swap_in(host_k, host_v, in_map))
+    # the host link's DMA rate on the same bytes (one contiguous copy each way)
+    hbuf = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dbuf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    ms_h2d = timed(lambda: dbuf.copy_(hbuf, non_blocking=True))
+    ms_d2h = timed(lambda: hbuf.copy_(dbuf, non_blocking=True))
+    gb = lambda ms: nbytes / (ms * 1e-3) / 1e9  # noqa: E731
+    return {
+        "metric": "KV block swap between device pool and pinned host pool (pa_swap_blocks)",
+        "value": gb(ms_out + ms_in) * 2, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "blocks": int(nb), "bytes_per_direction": int(nbytes),
+                   "block_bytes": block_bytes, "pairs_scattered": True},
+        "swap_out": {"ms": ms_out, "GBps": gb(ms_out)},
+        "swap_in": {"ms": ms_in, "GBps": gb(ms_in)},
+        "roofline": {"bound": "host link", "peak_d2h_GBps": gb(ms_d2h), "peak_h2d_GBps": gb(ms_h2d),
+                     "peak_kind": "measured contiguous DMA copy of the same bytes (cudaMemcpyAsync)",
+                     "frac_out": ms_d2h / ms_out, "frac_in": ms_h2d / ms_in},
+        "gpu_launches": 2 * args.steps,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -592,8 +654,13 @@ def main():
                          "pa_decode_shared_prefix")
     ap.add_argument("--memory-report", action="store_true",
                     help="host only: KV slots held by paged blocks vs max-length reservation")
+    ap.add_argument("--swap", action="store_true",
+                    help="time pa_swap_blocks (device <-> pinned host) instead of the decode step")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.swap:
+        print(json.dumps(run_swap(args)), flush=True)
+        return
     if args.memory_report:
         from paged_kv_cache_388_b200.memory import pool_usage, waste_report
         for cfg, max_len in (("1", 100), ("2", 2048), ("3", 4096), ("4", 1536), ("4cow", 1528),

@@ -109,6 +109,36 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping,
                    struct CUstream_st *stream);
 
 /*
+ * pa_swap_blocks -- move whole blocks from one pool to another, either of
+ * which may live in page-locked host memory: swap-out (device pool -> host
+ * pool) and swap-in (host -> device) of the blocks of preempted or inactive
+ * sequences.
+ *
+ * Defined by: the KV cache is tiered -- device memory holds the blocks of
+ * active requests, host memory the blocks that overflow, and blocks move
+ * between the tiers ("核心概念", section 内存层次结构); preemption frees device
+ * blocks when memory runs short ("理解 vLLM PagedAttention", section 五).
+ *
+ *   dst_k, dst_v    [num_dst_blocks][num_kv_heads][block_size][head_dim], written
+ *   src_k, src_v    [num_src_blocks][num_kv_heads][block_size][head_dim]
+ *   block_mapping   int64 [num_pairs][2] = {src block, dst block}
+ * Each of the five pointers may be device memory, managed memory or
+ * page-locked host memory (cudaHostAlloc / cudaHostRegister, or a pinned
+ * PyTorch tensor); the kernel reads and writes host memory directly over the
+ * host link.  Pageable host memory is rejected (PA_ERR_INVALID_ARG, nothing
+ * launched).  All five must be 16-byte aligned.  A dst block must not appear
+ * twice; when both pools are the same arrays, a dst must also not be a src
+ * of the same call.  Byte-exact copy.
+ * Device checks: a pair with src outside [0, num_src_blocks) or dst outside
+ * [0, num_dst_blocks) is skipped and PA_DEVERR_BLOCK_ID is set.
+ */
+int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k,
+                   const void *src_v, const int64_t *block_mapping,
+                   int num_pairs, int num_kv_heads, int head_dim,
+                   int block_size, int num_src_blocks, int num_dst_blocks,
+                   int dtype, struct CUstream_st *stream);
+
+/*
  * pa_decode_workspace_size -- bytes of device scratch pa_decode needs for
  * split-KV partial results (0 when no sequence is split).  Arguments as for
  * pa_decode; depends on the current device's SM count.

@@ -8,7 +8,7 @@ the two share nothing but the seeded input generators in ``workloads/``.
 Contents
 --------
 ``pa_oracle.c``   plain C, fp64, OpenMP over (query row, head): paged
-                  attention, reshape_and_cache, copy_blocks.
+                  attention, reshape_and_cache, copy_blocks, swap_blocks.
 ``brute.py``      NumPy attention over *contiguous* per-sequence K/V, for tiny
                   inputs (pins the paged gather).
 ``alloc_model.py`` the block-allocation rules written as plain definitions.
@@ -76,6 +76,8 @@ def _bind(lib):
     lib.oracle_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I]
     lib.oracle_copy_blocks.restype = I
     lib.oracle_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I]
+    lib.oracle_swap_blocks.restype = I
+    lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I]
     lib.oracle_max_threads.restype = I
     lib.oracle_max_threads.argtypes = []
     return lib
@@ -162,6 +164,21 @@ def copy_blocks(k_cache, v_cache, block_mapping, dtype, lib=None):
     rc = lib.oracle_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(bm), bm.shape[0],
                                 hk, d, bs, nb, DTYPES[dtype])
     _check(rc, "copy_blocks")
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, dtype, lib=None):
+    """Copy whole blocks (src, dst) from the (src_k, src_v) pool into the
+    (dst_k, dst_v) pool, in place."""
+    lib = lib or load()
+    for t in (dst_k, dst_v, src_k, src_v):
+        assert t.flags.c_contiguous
+    bm = _c(np.asarray(block_mapping).reshape(-1, 2), np.int64)
+    nd, hk, bs, d = dst_k.shape
+    ns = src_k.shape[0]
+    assert src_k.shape[1:] == dst_k.shape[1:] and src_v.shape == src_k.shape and dst_v.shape == dst_k.shape
+    rc = lib.oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), _ptr(bm),
+                                bm.shape[0], hk, d, bs, ns, nd, DTYPES[dtype])
+    _check(rc, "swap_blocks")
 
 
 def max_threads(lib=None) -> int:

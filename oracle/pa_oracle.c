@@ -335,6 +335,32 @@ int oracle_copy_blocks(void *k_cache, void *v_cache,
   return ORACLE_OK;
 }
 
+/*
+ * swap_blocks: move whole blocks from one pool to another (the GPU tier and
+ * the CPU tier of a tiered KV cache, "核心概念", section 内存层次结构).  For
+ * pair i, destination block dst_i of (dst_k, dst_v) receives the bytes of
+ * source block src_i of (src_k, src_v).  Every pair is checked before anything
+ * is written.  The two pools are distinct arrays, so the order of the pairs
+ * does not matter.
+ */
+int oracle_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                       const int64_t *block_mapping, int num_pairs, int num_kv_heads,
+                       int head_dim, int block_size, int num_src_blocks, int num_dst_blocks,
+                       int dtype) {
+  int64_t blk_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_bytes(dtype);
+  int i;
+  for (i = 0; i < num_pairs; ++i) {
+    int64_t s = block_mapping[2 * i], d = block_mapping[2 * i + 1];
+    if (s < 0 || s >= num_src_blocks || d < 0 || d >= num_dst_blocks) return ORACLE_BAD_BLOCK;
+  }
+  for (i = 0; i < num_pairs; ++i) {
+    int64_t s = block_mapping[2 * i], d = block_mapping[2 * i + 1];
+    memcpy((char *)dst_k + d * blk_bytes, (const char *)src_k + s * blk_bytes, (size_t)blk_bytes);
+    memcpy((char *)dst_v + d * blk_bytes, (const char *)src_v + s * blk_bytes, (size_t)blk_bytes);
+  }
+  return ORACLE_OK;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

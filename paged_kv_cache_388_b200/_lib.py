@@ -32,6 +32,8 @@ _lib.pa_reshape_and_cache.restype = I
 _lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
 _lib.pa_copy_blocks.restype = I
 _lib.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P]
+_lib.pa_swap_blocks.restype = I
+_lib.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P]
 _lib.pa_decode_workspace_size.restype = SZ
 _lib.pa_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
 _lib.pa_decode.restype = I
@@ -122,6 +124,30 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
                              block_mapping.shape[0], hk, d, bs, nb, _DT[k_cache.dtype],
                              _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None):
+    """Copy blocks (src, dst) of block_mapping int64 [P, 2] from the
+    (src_k, src_v) pool into the (dst_k, dst_v) pool.  Pools and mapping may
+    be CUDA tensors or pinned CPU tensors (not pageable ones)."""
+    for name, t in (("dst_k", dst_k), ("dst_v", dst_v), ("src_k", src_k), ("src_v", src_v),
+                    ("block_mapping", block_mapping)):
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if block_mapping.dtype != torch.int64:
+        raise ValueError("block_mapping must be int64")
+    if not (dst_k.dtype == dst_v.dtype == src_k.dtype == src_v.dtype):
+        raise ValueError("pools must share one dtype")
+    nd, hk, bs, d = dst_k.shape
+    ns = src_k.shape[0]
+    if tuple(src_k.shape[1:]) != (hk, bs, d) or src_v.shape != src_k.shape or dst_v.shape != dst_k.shape:
+        raise ValueError("pool shapes disagree")
+    rc = _lib.pa_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
+                             _ptr(block_mapping), block_mapping.shape[0], hk, d, bs, ns, nd,
+                             _DT[dst_k.dtype], _stream(stream))
+    _check(rc, "pa_swap_blocks")
 
 
 def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,

@@ -35,6 +35,24 @@ class PagedKVCache:
         if block_mapping.shape[0]:
             _lib.pa_copy_blocks(self.k_cache, self.v_cache, block_mapping)
 
+    def host_pool(self, num_blocks):
+        """A (K, V) pair of page-locked host pools of ``num_blocks`` blocks with
+        this cache's block shape: the CPU tier that blocks are swapped to."""
+        shape = (num_blocks,) + tuple(self.k_cache.shape[1:])
+        return (torch.empty(shape, dtype=self.dtype, pin_memory=True),
+                torch.empty(shape, dtype=self.dtype, pin_memory=True))
+
+    def swap_out(self, host_k, host_v, block_mapping):
+        """Copy device blocks to host blocks: block_mapping int64 [P, 2] of
+        (device block, host block), on the device or pinned."""
+        if block_mapping.shape[0]:
+            _lib.pa_swap_blocks(host_k, host_v, self.k_cache, self.v_cache, block_mapping)
+
+    def swap_in(self, host_k, host_v, block_mapping):
+        """Copy host blocks back into device blocks: (host block, device block)."""
+        if block_mapping.shape[0]:
+            _lib.pa_swap_blocks(self.k_cache, self.v_cache, host_k, host_v, block_mapping)
+
     def workspace(self, num_seqs, num_heads, max_context_len, kv_split_tokens=0):
         need = _lib.pa_decode_workspace_size(num_seqs, num_heads, self.num_kv_heads, self.head_dim,
                                              self.block_size, max_context_len, kv_split_tokens)

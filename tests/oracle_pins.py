@@ -416,10 +416,47 @@ def pin_copy_blocks(lib):
             assert np.array_equal(kp[b], k0[b]) and np.array_equal(vp[b], v0[b])
 
 
+def pin_swap_blocks(lib):
+    """Moving blocks between two pools (device tier <-> host tier): every
+    destination block named by a pair holds its source block's bytes, K from K
+    and V from V, every other destination block is untouched, the source pool
+    is not modified, and swapping out then back in restores the original
+    bytes at the original block ids."""
+    rng = np.random.default_rng(21)
+    Hk, bs, D = 2, 16, 64
+    for dt in ("f32", "bf16"):
+        dev_k = _bits(rng.standard_normal((12, Hk, bs, D)), dt)
+        dev_v = _bits(rng.standard_normal((12, Hk, bs, D)), dt)
+        host_k = _bits(rng.standard_normal((5, Hk, bs, D)), dt)
+        host_v = _bits(rng.standard_normal((5, Hk, bs, D)), dt)
+        d0k, d0v, h0k, h0v = dev_k.copy(), dev_v.copy(), host_k.copy(), host_v.copy()
+        out_pairs = [(3, 0), (11, 4), (7, 2)]    # device block -> host block
+        oracle.swap_blocks(host_k, host_v, dev_k, dev_v, out_pairs, dt, lib=lib)
+        assert np.array_equal(dev_k, d0k) and np.array_equal(dev_v, d0v)
+        for s, d in out_pairs:
+            assert np.array_equal(host_k[d], d0k[s]) and np.array_equal(host_v[d], d0v[s])
+        for d in (1, 3):
+            assert np.array_equal(host_k[d], h0k[d]) and np.array_equal(host_v[d], h0v[d])
+        # the device blocks are reused by others, then the sequence comes back
+        dev_k[[3, 11, 7]] = 0
+        dev_v[[3, 11, 7]] = 0
+        oracle.swap_blocks(dev_k, dev_v, host_k, host_v, [(d, s) for s, d in out_pairs], dt, lib=lib)
+        assert np.array_equal(dev_k, d0k) and np.array_equal(dev_v, d0v)
+        # against the definition by array indexing, on a random mapping
+        src = rng.permutation(12)[:6]
+        dst = rng.permutation(5)[:4]
+        pairs = list(zip(src[:4].tolist(), dst.tolist()))
+        want_k, want_v = host_k.copy(), host_v.copy()
+        want_k[dst] = dev_k[src[:4]]
+        want_v[dst] = dev_v[src[:4]]
+        oracle.swap_blocks(host_k, host_v, dev_k, dev_v, pairs, dt, lib=lib)
+        assert np.array_equal(host_k, want_k) and np.array_equal(host_v, want_v)
+
+
 ALL_PINS = [
     pin_brute_force, pin_decode_without_qsl, pin_identical_keys_mean, pin_single_key,
     pin_dominant_logit, pin_v_linearity, pin_scale_zero_mean, pin_hand_example,
     pin_gqa_equals_replicated_mha, pin_placement_invariance, pin_shared_equals_duplicated,
     pin_causal_truncation, pin_empty_context, pin_dtype_decoding, pin_worked_block_table,
-    pin_block_counts, pin_reshape_then_gather, pin_copy_blocks,
+    pin_block_counts, pin_reshape_then_gather, pin_copy_blocks, pin_swap_blocks,
 ]

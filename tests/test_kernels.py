@@ -269,8 +269,11 @@ def test_nan_in_unused_slots_does_not_leak(lib, decode_kernel):
     kc, vc, q, bt, cl = _tiny_decode(lib, lens=(20, 37))
     nan = torch.tensor(float("nan"), dtype=kc.dtype, device="cuda")
     ref_out = torch.empty_like(q)
+    ref_bal = torch.empty_like(q)
     ws = _ws(lib, 2)
     lib.pa_decode(ref_out, q, kc, vc, bt, cl, 0.1, kv_split_tokens=1 << 20, workspace=ws)
+    # the balanced partition sums in another order: its own reference
+    lib.pa_decode(ref_bal, q, kc, vc, bt, cl, 0.1, workspace=ws)
     kc[bt[0, 1], :, 4:] = nan  # seq 0: tokens 20.. of block 1 are unused
     vc[bt[0, 1], :, 4:] = nan
     kc[bt[1, 2], :, 5:] = nan  # seq 1: tokens 37.. of block 2
@@ -281,4 +284,4 @@ def test_nan_in_unused_slots_does_not_leak(lib, decode_kernel):
     assert torch.equal(out, ref_out)
     lib.pa_decode(out, q, kc, vc, bt, cl, 0.1, workspace=ws)  # balanced partition
     assert lib.pa_get_device_error() == 0
-    assert torch.equal(out, ref_out)
+    assert torch.equal(out, ref_bal)

@@ -32,6 +32,12 @@ MUTANTS = {
     "copy_without_staging": (
         "memcpy(stage_k + i * blk_bytes, (const char *)k_cache + s * blk_bytes, (size_t)blk_bytes);",
         "memcpy((char *)k_cache + block_mapping[2 * i + 1] * blk_bytes, (const char *)k_cache + s * blk_bytes, (size_t)blk_bytes); memcpy(stage_k + i * blk_bytes, (const char *)k_cache + s * blk_bytes, (size_t)blk_bytes);"),
+    "swap_k_and_v_crossed": (
+        "memcpy((char *)dst_k + d * blk_bytes, (const char *)src_k + s * blk_bytes, (size_t)blk_bytes);",
+        "memcpy((char *)dst_k + d * blk_bytes, (const char *)src_v + s * blk_bytes, (size_t)blk_bytes);"),
+    "swap_half_block": (
+        "memcpy((char *)dst_v + d * blk_bytes, (const char *)src_v + s * blk_bytes, (size_t)blk_bytes);",
+        "memcpy((char *)dst_v + d * blk_bytes, (const char *)src_v + s * blk_bytes, (size_t)(blk_bytes / 2));"),
     "f16_exponent_bias": ("v = ldexp((double)(mant | 0x400), expo - 25);",
                           "v = ldexp((double)(mant | 0x400), expo - 24);"),
     "f16_subnormal_scale": ("v = ldexp((double)mant, -24);", "v = ldexp((double)mant, -25);"),
