@@ -124,10 +124,12 @@ def elem_bytes(dtype):
     return {"f32": 4, "f16": 2, "bf16": 2}[dtype]
 
 
-def seq_bytes(wl, batch, seqs):
+def seq_bytes(wl, batch, seqs, kv_elem=None):
     """Algorithmic bytes of the step restricted to sequences `seqs`: every
-    byte the method has to move, once (shared physical blocks once)."""
+    byte the method has to move, once (shared physical blocks once).
+    kv_elem: bytes per cached element when it differs from q's (FP8 cache)."""
     e = elem_bytes(wl.dtype)
+    ekv = e if kv_elem is None else kv_elem
     H, Hk, D, bs = wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
     seen = set()
     kv_tokens = 0
@@ -144,17 +146,18 @@ def seq_bytes(wl, batch, seqs):
                 kv_tokens += min(bs, L - j * bs)
         qsl = batch.query_start_loc
         qrows += 1 if qsl is None else int(qsl[i + 1] - qsl[i])
-    decode = kv_tokens * 2 * Hk * D * e + 2 * qrows * H * D * e + nblk_total * 4 + len(seqs) * 4
+    decode = kv_tokens * 2 * Hk * D * ekv + 2 * qrows * H * D * e + nblk_total * 4 + len(seqs) * 4
     return decode, kv_tokens, qrows
 
 
-def step_bytes(wl, batch):
+def step_bytes(wl, batch, kv_elem=None):
     e = elem_bytes(wl.dtype)
+    ekv = e if kv_elem is None else kv_elem
     Hk, D, bs = wl.num_kv_heads, wl.head_dim, wl.block_size
-    decode, kv_tokens, qrows = seq_bytes(wl, batch, range(batch.num_seqs))
+    decode, kv_tokens, qrows = seq_bytes(wl, batch, range(batch.num_seqs), kv_elem)
     t_new = wl.num_new_tokens
-    reshape = 2 * (2 * t_new * Hk * D * e) + t_new * 8
-    copy = int(batch.cow_pairs.shape[0]) * 2 * (2 * Hk * bs * D * e)
+    reshape = 2 * (t_new * Hk * D * (e + ekv)) + t_new * 8
+    copy = int(batch.cow_pairs.shape[0]) * 2 * (2 * Hk * bs * D * ekv)
     return {"decode": decode, "reshape": reshape, "copy_blocks": copy,
             "step": decode + reshape + copy, "kv_tokens": kv_tokens, "q_rows": qrows}
 
@@ -323,10 +326,26 @@ def run_ours(args, rank, world, local_rank):
     wl = workloads.make(args.config, replica=rank)
     batch = build_batch(wl)
     vals = workloads.values(wl)
-    nbytes = step_bytes(wl, batch)
+    nbytes = step_bytes(wl, batch, 1 if args.kv_fp8 else None)
 
-    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
-                         k_cache=vals["k_pool"].to(dev), v_cache=vals["v_pool"].to(dev))
+    if args.kv_fp8:
+        # FP8 (E4M3) cache: one scale per tensor, the pool's history quantised
+        # on the host, this step's K/V quantised by pa_reshape_and_cache_fp8
+        def fp8_scale(*ts):
+            return float(np.float32(max(float(t.float().abs().max()) for t in ts) / 448.0 * 1.25))
+
+        def quant(t, sc):
+            return (t.float() / torch.tensor(sc, dtype=torch.float32)).to(
+                torch.float8_e4m3fn).view(torch.uint8)
+
+        ks = fp8_scale(vals["k_pool"], vals["new_key"])
+        vs = fp8_scale(vals["v_pool"], vals["new_value"])
+        cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                             dtype=torch.uint8, k_cache=quant(vals["k_pool"], ks).to(dev),
+                             v_cache=quant(vals["v_pool"], vs).to(dev), kv_scales=(ks, vs))
+    else:
+        cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                             k_cache=vals["k_pool"].to(dev), v_cache=vals["v_pool"].to(dev))
     q = vals["q"].to(dev)
     key = vals["new_key"].to(dev)
     value = vals["new_value"].to(dev)
@@ -344,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
 
     # Batches whose sequences share prompt blocks (parallel sampling) attend
     # through the shared-prefix entry point unless --plain-decode is given.
-    shared = wl.kind == "shared_prefix" and not args.plain_decode
+    shared = wl.kind == "shared_prefix" and not args.plain_decode and not args.kv_fp8
     if shared:
         gs_np, gb_np = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)
         gs = torch.from_numpy(gs_np).to(dev)
@@ -506,7 +525,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1) -----------
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and batch.query_start_loc is None:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and batch.query_start_loc is None
+            and not args.kv_fp8):
         run, cores = oracle_runner(wl, vals, batch)
         n = size_sample(run, batch.num_seqs, target_s=12.0)
         dt, ob, _ = run(n)
@@ -532,10 +552,10 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": wl.dtype,
+        "dtype": ("fp8_e4m3 KV cache, " + wl.dtype + " q/out") if args.kv_fp8 else wl.dtype,
         "data": "synthetic",
         "config": {
-            "workload": wl.name,
+            "workload": wl.name + ("_kv_fp8_e4m3" if args.kv_fp8 else ""),
             "global_batch": batch.num_seqs * world,
             "heads": f"{wl.num_heads}q/{wl.num_kv_heads}kv",
             "head_dim": wl.head_dim,
@@ -559,7 +579,7 @@ def run_ours(args, rank, world, local_rank):
             "unit": "GB/s",
             "frac": achieved / peak,
             "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
-            "traffic": profiled_traffic(args.config),
+            "traffic": None if args.kv_fp8 else profiled_traffic(args.config),
             "traffic_source": "profiles/paged_decode_mma_kernel_cfg3.md (ncu dram__bytes_read+write "
                               "of the decode kernel; null when the kernel sources changed since)",
             "algorithmic_bytes": nbytes["decode"],
@@ -654,6 +674,8 @@ def main():
                          "pa_decode_shared_prefix")
     ap.add_argument("--memory-report", action="store_true",
                     help="host only: KV slots held by paged blocks vs max-length reservation")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="FP8 (E4M3) KV cache: pa_reshape_and_cache_fp8 + pa_decode_fp8")
     ap.add_argument("--swap", action="store_true",
                     help="time pa_swap_blocks (device <-> pinned host) instead of the decode step")
     args = ap.parse_args()

@@ -54,7 +54,10 @@ typedef enum {
   PA_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+/* PA_FP8_E4M3: 1-byte E4M3 codes with one scale per cache tensor; only the
+ * caches of the *_fp8 entry points and the byte movers (pa_copy_blocks,
+ * pa_swap_blocks) take it. */
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
 
 /* Bits of the device error word. */
 #define PA_DEVERR_BLOCK_ID 0x1u    /* block id outside [0, num_blocks) */
@@ -98,7 +101,8 @@ int pa_reshape_and_cache(const void *key, const void *value, void *k_cache,
  * 的核心, item 3).
  *
  *   block_mapping  int64 [num_pairs][2] = {src, dst}; copies K and V of all
- *                  KV heads of block src onto block dst.  A dst must not
+ *                  KV heads of block src onto block dst.  dtype may also be
+ *                  PA_FP8_E4M3 (1-byte elements).  A dst must not
  *                  appear twice nor also be a src in the same call (the
  *                  result would depend on ordering).
  * Byte-exact copy.
@@ -137,6 +141,52 @@ int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k,
                    int num_pairs, int num_kv_heads, int head_dim,
                    int block_size, int num_src_blocks, int num_dst_blocks,
                    int dtype, struct CUstream_st *stream);
+
+/*
+ * pa_reshape_and_cache_fp8 -- pa_reshape_and_cache into an FP8 (E4M3) cache.
+ *
+ * Defined by: KV-cache quantisation ("理解 vLLM PagedAttention", 版本矩阵:
+ * 量化 FP8 ... 权重 KV cache 量化); slots as pa_reshape_and_cache.  Element x of
+ * a new key is stored as the E4M3 code (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, no infinities, largest magnitude 448) of the IEEE binary32
+ * quotient x / k_scale, rounded to nearest with ties to even and saturated
+ * to +-448 (NaN -> NaN); values likewise with v_scale.
+ *
+ *   key, value       [num_tokens][num_kv_heads][head_dim] of in_dtype
+ *                    (PA_F32, PA_F16 or PA_BF16)
+ *   k_cache, v_cache uint8 [num_blocks][num_kv_heads][block_size][head_dim]
+ *   k_scale, v_scale positive finite per-tensor scales
+ * The codes are bit-exact functions of the inputs (no other arithmetic).
+ */
+int pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache,
+                             void *v_cache, const int64_t *slot_mapping,
+                             int num_tokens, int num_kv_heads, int head_dim,
+                             int block_size, int num_blocks, int in_dtype,
+                             float k_scale, float v_scale,
+                             struct CUstream_st *stream);
+
+/*
+ * pa_decode_fp8 -- pa_decode (one query row per sequence) over FP8 (E4M3)
+ * caches written by pa_reshape_and_cache_fp8: key element = code * k_scale,
+ * value element = code * v_scale, and out = softmax(scale * q . K^T) V in
+ * fp32 accumulation.  The cache holds one byte per element, so decode reads
+ * half the bytes of a 16-bit cache.
+ *
+ *   q, out           [num_seqs][num_heads][head_dim] of q_dtype (PA_F16 or PA_BF16)
+ *   k_cache, v_cache uint8 codes as above
+ *   workspace        >= pa_decode_workspace_size(num_seqs, num_heads,
+ *                    num_kv_heads, head_dim, block_size, max_context_len, 0) bytes
+ * Other arguments, checks and device error reporting as for pa_decode.
+ * Supported: num_seqs <= 2048 and group = num_heads / num_kv_heads <= 16.
+ */
+int pa_decode_fp8(void *out, const void *q, const void *k_cache,
+                  const void *v_cache, const int32_t *block_tables,
+                  int max_blocks_per_seq, const int32_t *context_lens,
+                  int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                  int block_size, int num_blocks, float scale, float k_scale,
+                  float v_scale, int max_context_len, int q_dtype,
+                  void *workspace, size_t workspace_bytes,
+                  struct CUstream_st *stream);
 
 /*
  * pa_decode_workspace_size -- bytes of device scratch pa_decode needs for

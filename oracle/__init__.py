@@ -8,7 +8,8 @@ the two share nothing but the seeded input generators in ``workloads/``.
 Contents
 --------
 ``pa_oracle.c``   plain C, fp64, OpenMP over (query row, head): paged
-                  attention, reshape_and_cache, copy_blocks, swap_blocks.
+                  attention, reshape_and_cache, copy_blocks, swap_blocks, and the
+                  FP8 (E4M3) codec with quantising reshape and FP8-cache decode.
 ``brute.py``      NumPy attention over *contiguous* per-sequence K/V, for tiny
                   inputs (pins the paged gather).
 ``alloc_model.py`` the block-allocation rules written as plain definitions.
@@ -32,7 +33,7 @@ _SO = os.path.join(_HERE, "_pa_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-DTYPES = {"f32": 0, "f16": 1, "bf16": 2}
+DTYPES = {"f32": 0, "f16": 1, "bf16": 2, "fp8": 3}  # "fp8": E4M3 codes, for the byte movers
 _STATUS = {
     0: "ok",
     1: "bad argument",
@@ -78,6 +79,16 @@ def _bind(lib):
     lib.oracle_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I]
     lib.oracle_swap_blocks.restype = I
     lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_reshape_and_cache_fp8.restype = I
+    lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, I, P, I, I, I, I, I,
+                                                 ctypes.c_float, ctypes.c_float]
+    lib.oracle_decode_fp8.restype = I
+    lib.oracle_decode_fp8.argtypes = [P, P, I, P, P, ctypes.c_double, ctypes.c_double, P, I, P,
+                                      P, I, I, I, I, I, I, ctypes.c_double, P, I]
     lib.oracle_max_threads.restype = I
     lib.oracle_max_threads.argtypes = []
     return lib
@@ -140,6 +151,58 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
                            _ptr(sel), int(threads))
     _check(rc, "decode")
     return out
+
+
+def decode_fp8(q, q_dtype, k_codes, v_codes, k_scale, v_scale, block_tables, context_lens,
+               scale, query_start_loc=None, rows=None, threads=0, lib=None):
+    """Paged attention in fp64 over E4M3 caches (uint8 codes [NB, Hk, bs, D])
+    whose elements are code value * k_scale / v_scale; q in q_dtype."""
+    lib = lib or load()
+    q = _raw(q)
+    kc = _c(k_codes, np.uint8)
+    vc = _c(v_codes, np.uint8)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    qsl = _c(query_start_loc, np.int32)
+    tq, h, d = q.shape
+    nb, hk, bs, d2 = kc.shape
+    assert d2 == d and vc.shape == kc.shape
+    out = np.full((tq, h, d), np.nan, dtype=np.float64)
+    sel = None
+    if rows is not None:
+        sel = np.zeros(tq, dtype=np.uint8)
+        sel[np.asarray(list(rows), dtype=np.int64)] = 1
+    rc = lib.oracle_decode_fp8(_ptr(out), _ptr(q), DTYPES[q_dtype], _ptr(kc), _ptr(vc),
+                               float(k_scale), float(v_scale), _ptr(bt),
+                               bt.shape[1] if bt.ndim == 2 else 0, _ptr(cl), _ptr(qsl),
+                               cl.shape[0], h, hk, d, bs, nb, float(scale), _ptr(sel), int(threads))
+    _check(rc, "decode_fp8")
+    return out
+
+
+def reshape_and_cache_fp8(k_codes, v_codes, key, value, in_dtype, slot_mapping, k_scale, v_scale,
+                          lib=None):
+    """Quantise key/value [T, Hk, D] (in_dtype) to E4M3 codes of x / scale and
+    scatter them into the uint8 caches in place."""
+    lib = lib or load()
+    assert k_codes.dtype == np.uint8 and v_codes.dtype == np.uint8
+    assert k_codes.flags.c_contiguous and v_codes.flags.c_contiguous
+    key = _raw(key)
+    value = _raw(value)
+    sm = _c(slot_mapping, np.int64)
+    nb, hk, bs, d = k_codes.shape
+    rc = lib.oracle_reshape_and_cache_fp8(_ptr(k_codes), _ptr(v_codes), _ptr(key), _ptr(value),
+                                          DTYPES[in_dtype], _ptr(sm), sm.shape[0], hk, d, bs, nb,
+                                          float(k_scale), float(v_scale))
+    _check(rc, "reshape_and_cache_fp8")
+
+
+def e4m3_decode(code, lib=None) -> float:
+    return float((lib or load()).oracle_e4m3_decode(int(code)))
+
+
+def e4m3_encode(x, lib=None) -> int:
+    return int((lib or load()).oracle_e4m3_encode(float(x)))
 
 
 def reshape_and_cache(k_cache, v_cache, key, value, slot_mapping, dtype, lib=None):

@@ -51,7 +51,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
+enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2, ORACLE_FP8_E4M3 = 3 };
 
 enum {
   ORACLE_OK = 0,
@@ -85,21 +85,99 @@ static double bf16_to_double(uint16_t b) {
   return (double)f;
 }
 
+/*
+ * FP8 E4M3 (the "FN" variant: no infinities): 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits.  Exponent field 0 holds subnormals
+ * m * 2^-9; S.1111.111 is NaN; the largest finite magnitude is
+ * 1.75 * 2^8 = 448.  Code -> exact double.
+ */
+static double e4m3_to_double(uint8_t c) {
+  int sign = (c >> 7) & 1;
+  int expo = (c >> 3) & 0xf;
+  int mant = c & 7;
+  double v;
+  if (expo == 0xf && mant == 7)
+    v = NAN;
+  else if (expo == 0)
+    v = ldexp((double)mant, -9);                /* subnormal: mant * 2^-9 */
+  else
+    v = ldexp((double)(8 + mant), expo - 10);   /* 1.mant * 2^(expo-7) */
+  return sign ? -v : v;
+}
+
+/*
+ * float -> E4M3 code: round to nearest, ties to the even code, magnitudes
+ * beyond 448 saturated to +-448, NaN -> 0x7f.  Written as the plain
+ * definition: of all finite non-negative codes (0x00 .. 0x7e, increasing in
+ * value) take the one nearest |f|; on a tie the even one (its mantissa's low
+ * bit is the code's low bit).  The sign bit is copied (so -0 -> 0x80).
+ */
+static uint8_t e4m3_from_float(float f) {
+  uint8_t sign = signbit(f) ? 0x80 : 0x00;
+  double a = fabs((double)f);
+  int best = 0, c;
+  double best_d;
+  if (isnan(f)) return 0x7f;
+  if (a >= 448.0) return (uint8_t)(sign | 0x7e);
+  best_d = a;
+  for (c = 1; c <= 0x7e; ++c) {
+    double d = fabs(e4m3_to_double((uint8_t)c) - a);
+    if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
 static double elem(const void *base, int64_t idx, int dtype) {
   if (dtype == ORACLE_F32) return (double)((const float *)base)[idx];
   if (dtype == ORACLE_F16) return f16_to_double(((const uint16_t *)base)[idx]);
+  if (dtype == ORACLE_FP8_E4M3) return e4m3_to_double(((const uint8_t *)base)[idx]);
   return bf16_to_double(((const uint16_t *)base)[idx]);
 }
 
-static int elem_bytes(int dtype) { return dtype == ORACLE_F32 ? 4 : 2; }
+static int elem_bytes(int dtype) {
+  return dtype == ORACLE_F32 ? 4 : (dtype == ORACLE_FP8_E4M3 ? 1 : 2);
+}
+
+/*
+ * Layout of an FP8 cache tile (one block, one KV head), fixed by this project
+ * (the pages give none) so that each thread of the device's products loads
+ * its operands with one 16-byte (K) or 4/8-byte (V) read:
+ *   K [block_size][head_dim] bytes: in every row r, column d = 64j + 16k + c
+ *     (c < 16) is stored at byte (C ^ (r mod head_dim/16)) * 16 + 4k + i of
+ *     the row, with t = (c mod 8) / 2, i = c mod 2 + 2 * (c / 8), C = 4j + t.
+ *   V [head_dim][block_size] bytes (transposed): key r = 16k + c of column d
+ *     is stored at byte d * block_size + 4t + i (block_size 16) or
+ *     d * block_size + 8t + 4k + i (block_size 32), t and i from c as above.
+ */
+static int64_t fp8_k_pos(int r, int d, int head_dim) {
+  int j = d / 64, w = d % 64, k = w / 16, c = w % 16;
+  int t = (c % 8) / 2, i = c % 2 + 2 * (c / 8);
+  int chunk = (4 * j + t) ^ (r % (head_dim / 16));
+  return (int64_t)r * head_dim + chunk * 16 + 4 * k + i;
+}
+
+static int64_t fp8_v_pos(int r, int d, int block_size) {
+  int k = r / 16, c = r % 16;
+  int t = (c % 8) / 2, i = c % 2 + 2 * (c / 8);
+  int pos = block_size == 16 ? 4 * t + i : 8 * t + 4 * k + i;
+  return (int64_t)d * block_size + pos;
+}
+
+/* Exported for the pins: the codec alone. */
+double oracle_e4m3_decode(uint8_t c) { return e4m3_to_double(c); }
+uint8_t oracle_e4m3_encode(float f) { return e4m3_from_float(f); }
 
 /*
  * One output row: query token `row` of sequence `seq`, query head `h`.
  * Writes head_dim doubles to out_row.  `kbuf`/`vbuf` are caller scratch of
  * n_vis * head_dim doubles and `sbuf` of n_vis doubles.
  */
-static int attend_one(double *out_row, const void *q, const void *k_cache,
-                      const void *v_cache, int dtype, const int32_t *table,
+static int attend_one(double *out_row, const void *q, int q_dtype, const void *k_cache,
+                      const void *v_cache, int dtype, double k_scale, double v_scale,
+                      const int32_t *table,
                       int n_vis, int64_t row, int h, int num_heads,
                       int num_kv_heads, int head_dim, int block_size,
                       int num_blocks, double scale, double *kbuf, double *vbuf,
@@ -121,9 +199,19 @@ static int attend_one(double *out_row, const void *q, const void *k_cache,
     int64_t base;
     if (pb < 0 || pb >= num_blocks) return ORACLE_BAD_BLOCK;
     base = (((int64_t)pb * num_kv_heads + h_kv) * block_size + off) * head_dim;
+    if (dtype == ORACLE_FP8_E4M3) { /* tile-internal layout above */
+      int64_t tile = ((int64_t)pb * num_kv_heads + h_kv) * block_size * head_dim;
+      for (d = 0; d < head_dim; ++d) {
+        kbuf[(int64_t)p * head_dim + d] =
+            elem(k_cache, tile + fp8_k_pos(off, d, head_dim), dtype) * k_scale;
+        vbuf[(int64_t)p * head_dim + d] =
+            elem(v_cache, tile + fp8_v_pos(off, d, block_size), dtype) * v_scale;
+      }
+      continue;
+    }
     for (d = 0; d < head_dim; ++d) {
-      kbuf[(int64_t)p * head_dim + d] = elem(k_cache, base + d, dtype);
-      vbuf[(int64_t)p * head_dim + d] = elem(v_cache, base + d, dtype);
+      kbuf[(int64_t)p * head_dim + d] = elem(k_cache, base + d, dtype) * k_scale;
+      vbuf[(int64_t)p * head_dim + d] = elem(v_cache, base + d, dtype) * v_scale;
     }
   }
 
@@ -134,7 +222,7 @@ static int attend_one(double *out_row, const void *q, const void *k_cache,
     for (p = 0; p < n_vis; ++p) {
       double s = 0.0;
       for (d = 0; d < head_dim; ++d)
-        s += elem(q, qbase + d, dtype) * kbuf[(int64_t)p * head_dim + d];
+        s += elem(q, qbase + d, q_dtype) * kbuf[(int64_t)p * head_dim + d];
       s *= scale;
       sbuf[p] = s;
       if (s > m) m = s;
@@ -162,13 +250,14 @@ static int attend_one(double *out_row, const void *q, const void *k_cache,
  *                    computed (their output is left untouched)
  *   num_threads      <= 0: library default
  */
-int oracle_decode(double *out, const void *q, const void *k_cache,
-                  const void *v_cache, int dtype, const int32_t *block_tables,
-                  int max_blocks_per_seq, const int32_t *context_lens,
-                  const int32_t *query_start_loc, int num_seqs, int num_heads,
-                  int num_kv_heads, int head_dim, int block_size,
-                  int num_blocks, double scale, const uint8_t *row_select,
-                  int num_threads) {
+static int decode_impl(double *out, const void *q, int q_dtype, const void *k_cache,
+                       const void *v_cache, int dtype, double k_scale, double v_scale,
+                       const int32_t *block_tables,
+                       int max_blocks_per_seq, const int32_t *context_lens,
+                       const int32_t *query_start_loc, int num_seqs, int num_heads,
+                       int num_kv_heads, int head_dim, int block_size,
+                       int num_blocks, double scale, const uint8_t *row_select,
+                       int num_threads) {
   int64_t num_q_tokens;
   int64_t *task_row;
   int32_t *task_seq;
@@ -179,7 +268,10 @@ int oracle_decode(double *out, const void *q, const void *k_cache,
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_heads % num_kv_heads != 0)
     return ORACLE_BAD_ARG;
-  if (dtype != ORACLE_F32 && dtype != ORACLE_F16 && dtype != ORACLE_BF16)
+  if (dtype != ORACLE_F32 && dtype != ORACLE_F16 && dtype != ORACLE_BF16 &&
+      dtype != ORACLE_FP8_E4M3)
+    return ORACLE_BAD_ARG;
+  if (q_dtype != ORACLE_F32 && q_dtype != ORACLE_F16 && q_dtype != ORACLE_BF16)
     return ORACLE_BAD_ARG;
 
   num_q_tokens = query_start_loc ? query_start_loc[num_seqs] : num_seqs;
@@ -250,8 +342,8 @@ int oracle_decode(double *out, const void *q, const void *k_cache,
         cap = -1;
         continue;
       }
-      rc = attend_one(out + (row * num_heads + h) * (int64_t)head_dim, q, k_cache,
-                      v_cache, dtype,
+      rc = attend_one(out + (row * num_heads + h) * (int64_t)head_dim, q, q_dtype, k_cache,
+                      v_cache, dtype, k_scale, v_scale,
                       block_tables + (int64_t)seq * max_blocks_per_seq, n_vis,
                       row, h, num_heads, num_kv_heads, head_dim, block_size,
                       num_blocks, scale, kbuf, vbuf, sbuf);
@@ -267,6 +359,38 @@ int oracle_decode(double *out, const void *q, const void *k_cache,
   free(task_row);
   free(task_seq);
   return status;
+}
+
+int oracle_decode(double *out, const void *q, const void *k_cache,
+                  const void *v_cache, int dtype, const int32_t *block_tables,
+                  int max_blocks_per_seq, const int32_t *context_lens,
+                  const int32_t *query_start_loc, int num_seqs, int num_heads,
+                  int num_kv_heads, int head_dim, int block_size,
+                  int num_blocks, double scale, const uint8_t *row_select,
+                  int num_threads) {
+  return decode_impl(out, q, dtype, k_cache, v_cache, dtype, 1.0, 1.0, block_tables,
+                     max_blocks_per_seq, context_lens, query_start_loc, num_seqs, num_heads,
+                     num_kv_heads, head_dim, block_size, num_blocks, scale, row_select,
+                     num_threads);
+}
+
+/*
+ * Paged attention over an FP8 (E4M3) cache with one scale per cache tensor:
+ * key element = code value * k_scale, value element = code value * v_scale
+ * (KV-cache quantisation, "理解 vLLM PagedAttention", 版本矩阵: 量化 FP8 ...
+ * 权重 KV cache 量化).  q (q_dtype) and everything else as oracle_decode.
+ */
+int oracle_decode_fp8(double *out, const void *q, int q_dtype, const uint8_t *k_codes,
+                      const uint8_t *v_codes, double k_scale, double v_scale,
+                      const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *context_lens, const int32_t *query_start_loc,
+                      int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, double scale,
+                      const uint8_t *row_select, int num_threads) {
+  return decode_impl(out, q, q_dtype, k_codes, v_codes, ORACLE_FP8_E4M3, k_scale, v_scale,
+                     block_tables, max_blocks_per_seq, context_lens, query_start_loc, num_seqs,
+                     num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                     row_select, num_threads);
 }
 
 /*
@@ -292,6 +416,43 @@ int oracle_reshape_and_cache(void *k_cache, void *v_cache, const void *key,
       int64_t src = ((int64_t)t * num_kv_heads + h) * row_bytes;
       memcpy((char *)k_cache + dst, (const char *)key + src, (size_t)row_bytes);
       memcpy((char *)v_cache + dst, (const char *)value + src, (size_t)row_bytes);
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
+ * reshape_and_cache into an FP8 (E4M3) cache: the element x of key token t
+ * (in_dtype) is stored as the code of x / k_scale, values likewise with
+ * v_scale (KV-cache quantisation, "理解 vLLM PagedAttention", 版本矩阵).  The
+ * division is one IEEE binary32 division (float / float) and the rounding to
+ * E4M3 is done from that binary32 result, which is the precision the device
+ * quantiser works in; slots as oracle_reshape_and_cache, positions inside the
+ * (block, head) tile as fp8_k_pos / fp8_v_pos.
+ */
+int oracle_reshape_and_cache_fp8(uint8_t *k_codes, uint8_t *v_codes, const void *key,
+                                 const void *value, int in_dtype, const int64_t *slot_mapping,
+                                 int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                 int num_blocks, float k_scale, float v_scale) {
+  int t, h, d;
+  if (in_dtype != ORACLE_F32 && in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16)
+    return ORACLE_BAD_ARG;
+  for (t = 0; t < num_tokens; ++t) {
+    int64_t slot = slot_mapping[t];
+    int64_t blk, off;
+    if (slot < 0) continue;
+    if (slot >= (int64_t)num_blocks * block_size) return ORACLE_BAD_SLOT;
+    blk = slot / block_size;
+    off = slot - blk * block_size;
+    for (h = 0; h < num_kv_heads; ++h) {
+      int64_t tile = (blk * num_kv_heads + h) * block_size * head_dim;
+      int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+      for (d = 0; d < head_dim; ++d) {
+        float kx = (float)elem(key, src + d, in_dtype);
+        float vx = (float)elem(value, src + d, in_dtype);
+        k_codes[tile + fp8_k_pos((int)off, d, head_dim)] = e4m3_from_float(kx / k_scale);
+        v_codes[tile + fp8_v_pos((int)off, d, block_size)] = e4m3_from_float(vx / v_scale);
+      }
     }
   }
   return ORACLE_OK;

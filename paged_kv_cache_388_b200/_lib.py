@@ -32,6 +32,10 @@ _lib.pa_reshape_and_cache.restype = I
 _lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
 _lib.pa_copy_blocks.restype = I
 _lib.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P]
+_lib.pa_reshape_and_cache_fp8.restype = I
+_lib.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, P]
+_lib.pa_decode_fp8.restype = I
+_lib.pa_decode_fp8.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, I, F, F, F, I, I, P, SZ, P]
 _lib.pa_swap_blocks.restype = I
 _lib.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P]
 _lib.pa_decode_workspace_size.restype = SZ
@@ -54,8 +58,9 @@ _lib.pa_status_string.argtypes = [I]
 _lib.pa_abi_version.restype = I
 _lib.pa_abi_version.argtypes = []
 
-PA_F32, PA_F16, PA_BF16 = 0, 1, 2
-_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
+_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
+       torch.uint8: PA_FP8_E4M3, torch.float8_e4m3fn: PA_FP8_E4M3}
 
 PA_DEVERR_BLOCK_ID = 0x1
 PA_DEVERR_SLOT = 0x2
@@ -124,6 +129,48 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
                              block_mapping.shape[0], hk, d, bs, nb, _DT[k_cache.dtype],
                              _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             stream=None):
+    """key/value [T, Hk, D] (fp32/fp16/bf16); caches uint8 [NB, Hk, bs, D] of
+    E4M3 codes; slot_mapping int64 [T]."""
+    _dev(key, "key")
+    _dev(value, "value", key.dtype)
+    _dev(k_cache, "k_cache", torch.uint8)
+    _dev(v_cache, "v_cache", torch.uint8)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    nb, hk, bs, d = k_cache.shape
+    rc = _lib.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(slot_mapping), key.shape[0], hk, d, bs, nb,
+                                       _DT[key.dtype], float(k_scale), float(v_scale),
+                                       _stream(stream))
+    _check(rc, "pa_reshape_and_cache_fp8")
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale,
+                  max_context_len=0, workspace=None, stream=None):
+    """out/q [S, H, D] fp16/bf16; caches uint8 E4M3 codes [NB, Hk, bs, D];
+    workspace: uint8 CUDA tensor of >= pa_decode_workspace_size(...) bytes."""
+    _dev(q, "q")
+    _dev(out, "out", q.dtype)
+    _dev(k_cache, "k_cache", torch.uint8)
+    _dev(v_cache, "v_cache", torch.uint8)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+    s, h, d = q.shape
+    nb, hk, bs, d2 = k_cache.shape
+    if d2 != d or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    s2, mbps = block_tables.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                            mbps, _ptr(context_lens), s, h, hk, d, bs, nb, float(scale),
+                            float(k_scale), float(v_scale), int(max_context_len), _DT[q.dtype],
+                            _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "pa_decode_fp8")
 
 
 def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None):

@@ -27,6 +27,9 @@
 // CUDA-core kernel (decode_common.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp8.h>
+
+#include <type_traits>
 
 #include "decode_common.cuh"
 
@@ -121,6 +124,24 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+// Two E4M3 codes (low byte first) -> an fp16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
 // A staged tile is BS rows x D columns of 16-bit values held as D/64 boxes of
 // BS rows x 128 bytes, each written by TMA with the 128-byte swizzle: the
 // 16-byte chunk c of row r sits at chunk position c ^ (r % 8).  Box bases are
@@ -131,9 +152,13 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int r, int c8) {
   return tile + box * (BS * 128) + r * 128 + ((chunk ^ (r & 7)) << 4);
 }
 
-template <int D, int BS, int NT, int NCW>
+// F8: the cache holds FP8 E4M3 codes (1 byte) in the tile layout of
+// pa_reshape_and_cache_fp8; consumer warps convert them straight into fp16
+// mma fragments.
+template <int D, int BS, int NT, int NCW, bool F8 = false>
 struct MmaLayout {
-  static constexpr int kTile = BS * D * 2;   // bytes of one (block, kv-head) K or V tile
+  static constexpr int kElem = F8 ? 1 : 2;        // bytes per cached element
+  static constexpr int kTile = BS * D * kElem;    // bytes of one (block, kv-head) K or V tile
   static constexpr int kStage = 2 * kTile;
   static constexpr int kStages = (PA_MMA_RING_KB * 1024) / kStage < 2 ? 2 : (PA_MMA_RING_KB * 1024) / kStage;
   static constexpr int kPbuf = NT * 2 * 8 * 16 * 2;  // per warp: P^T hi+lo [nt][8 heads][16 keys]
@@ -156,11 +181,16 @@ struct MmaLayout {
   }
 };
 
-template <typename T, int D, int BS, int NT, int NCW>
+// T is the type of q and out.  With F8 the cache holds E4M3 codes and the
+// products run in fp16 (Tc): every E4M3 value is exact in fp16, and a bf16 q
+// row is scaled by a power of two into fp16 range (the scale is divided out
+// of its logits).
+template <typename T, int D, int BS, int NT, int NCW, bool F8 = false>
 __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
     paged_decode_mma_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv) {
-  using L = MmaLayout<D, BS, NT, NCW>;
+  using L = MmaLayout<D, BS, NT, NCW, F8>;
+  using Tc = typename std::conditional<F8, __half, T>::type;
   constexpr int KS = D / 16;    // k-steps of the QK product (head dim)
   constexpr int MT = D / 16;    // m-tiles of the PV product (head dim)
   extern __shared__ unsigned char smem_raw[];
@@ -294,10 +324,18 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
               const int row = (pb * a.num_kv_heads + item.kvh) * BS;
               const uint32_t dst = ring + slot * L::kStage;
               mbar_arrive_expect_tx(&full[slot], L::kStage);
+              if constexpr (F8) {  // each E4M3 tile is one contiguous run of BS * D bytes
+                const int64_t off = (int64_t)row * D;
+                bulk_load(smem + lay.ring + slot * L::kStage,
+                          static_cast<const unsigned char *>(a.k_cache) + off, L::kTile, &full[slot]);
+                bulk_load(smem + lay.ring + slot * L::kStage + L::kTile,
+                          static_cast<const unsigned char *>(a.v_cache) + off, L::kTile, &full[slot]);
+              } else {
 #pragma unroll
-              for (int bx = 0; bx < D / 64; ++bx) {
-                tma_load_2d(dst + bx * (BS * 128), &tmk, bx * 64, row, &full[slot]);
-                tma_load_2d(dst + L::kTile + bx * (BS * 128), &tmv, bx * 64, row, &full[slot]);
+                for (int bx = 0; bx < D / 64; ++bx) {
+                  tma_load_2d(dst + bx * (BS * 128), &tmk, bx * 64, row, &full[slot]);
+                  tma_load_2d(dst + L::kTile + bx * (BS * 128), &tmv, bx * 64, row, &full[slot]);
+                }
               }
             }
           }
@@ -352,6 +390,43 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&qempty[qs]);
     }
+    // Logit factor of heads 2t, 2t+1 of each n-tile: scale * log2(e) (times
+    // k_scale for an FP8 cache), divided by the power of two that brought a
+    // bf16 q row into fp16 range for the fp16 products.
+    float qf[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) qf[nt][0] = qf[nt][1] = sl2;
+    if constexpr (F8 && std::is_same<T, __nv_bfloat16>::value) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float mx = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+          for (int j2 = 0; j2 < 2; ++j2) {
+            const uint32_t u = qb[nt][ks][j2];
+            mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(u << 16)), fabsf(__uint_as_float(u & 0xffff0000u))));
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        int e = 0;
+        if (mx > 0.f && isfinite(mx)) frexpf(mx, &e);  // mx < 2^e
+        const int sh = max(-100, min(100, 15 - e));     // |q| * 2^sh < 2^15 < fp16 max
+        const float up = ldexpf(1.f, sh);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+          for (int j2 = 0; j2 < 2; ++j2) {
+            const uint32_t u = qb[nt][ks][j2];
+            __half2 h = __floats2half2_rn(__uint_as_float(u << 16) * up,
+                                          __uint_as_float(u & 0xffff0000u) * up);
+            qb[nt][ks][j2] = *reinterpret_cast<uint32_t *>(&h);
+          }
+        const float down = sl2 * ldexpf(1.f, -sh);
+        qf[nt][0] = __shfl_sync(0xffffffffu, down, (2 * t) * 4);
+        qf[nt][1] = __shfl_sync(0xffffffffu, down, (2 * t + 1) * 4);
+      }
+    }
 
     float o[NT][MT][4];
     float m[NT][2], l[NT][2];
@@ -405,7 +480,27 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
             float s[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-            {
+            if constexpr (F8) {
+              // E4M3 tile: the codes of this thread's fragment (rows g, g+8;
+              // columns 2t, 2t+1, 2t+8, 2t+9 of four k-steps) are one 16-byte
+              // chunk per row; each pair of codes converts to an fp16 pair.
+              const int ra = r0 + g, rb = ra + 8;
+#pragma unroll
+              for (int j = 0; j < D / 64; ++j) {
+                const uint4 wa = ld_shared_v4(ktile + ra * D + (((4 * j + t) ^ (ra & (D / 16 - 1))) << 4));
+                const uint4 wb = ld_shared_v4(ktile + rb * D + (((4 * j + t) ^ (rb & (D / 16 - 1))) << 4));
+                const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w};
+                const uint32_t xb[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq) {
+                  const uint32_t af[4] = {e4m3x2_to_f16x2(xa[kq] & 0xffffu), e4m3x2_to_f16x2(xb[kq] & 0xffffu),
+                                          e4m3x2_to_f16x2(xa[kq] >> 16), e4m3x2_to_f16x2(xb[kq] >> 16)};
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+                    MmaT<Tc>::mma(s[nt], af, qb[nt][4 * j + kq][0], qb[nt][4 * j + kq][1]);
+                }
+              }
+            } else {
               const int mi = lane >> 3;
               const int kr = r0 + (lane & 7) + (mi & 1) * 8;
 #pragma unroll
@@ -413,7 +508,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
                 uint32_t af[4];
                 ldsm_x4(af, swz<BS>(ktile, kr, ks * 2 + (mi >> 1)));
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) MmaT<T>::mma(s[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+                for (int nt = 0; nt < NT; ++nt) MmaT<Tc>::mma(s[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
               }
             }
             // ---- online softmax: thread holds keys r0+g, r0+g+8 of heads 2t, 2t+1 ----
@@ -424,8 +519,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
               float p[4];
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
-                const float x0 = v0 ? s[nt][hh] * sl2 : -INFINITY;
-                const float x1 = v1 ? s[nt][2 + hh] * sl2 : -INFINITY;
+                const float x0 = v0 ? s[nt][hh] * qf[nt][hh] : -INFINITY;
+                const float x1 = v1 ? s[nt][2 + hh] * qf[nt][hh] : -INFINITY;
                 float mx = fmaxf(x0, x1);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -448,14 +543,14 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 const int head = 2 * t + (c & 1), key = g + (c >> 1) * 8;
-                const uint16_t hi = MmaT<T>::bits(p[c]);
+                const uint16_t hi = MmaT<Tc>::bits(p[c]);
                 ph[head * 16 + key] = hi;
-                if constexpr (MmaT<T>::kSplitP) pl[head * 16 + key] = MmaT<T>::bits(p[c] - MmaT<T>::back(hi));
+                if constexpr (MmaT<Tc>::kSplitP) pl[head * 16 + key] = MmaT<Tc>::bits(p[c] - MmaT<Tc>::back(hi));
               }
               __syncwarp();
               pb_hi[nt][0] = *reinterpret_cast<const uint32_t *>(ph + g * 16 + 2 * t);
               pb_hi[nt][1] = *reinterpret_cast<const uint32_t *>(ph + g * 16 + 8 + 2 * t);
-              if constexpr (MmaT<T>::kSplitP) {
+              if constexpr (MmaT<Tc>::kSplitP) {
                 pb_lo[nt][0] = *reinterpret_cast<const uint32_t *>(pl + g * 16 + 2 * t);
                 pb_lo[nt][1] = *reinterpret_cast<const uint32_t *>(pl + g * 16 + 8 + 2 * t);
               }
@@ -463,7 +558,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
             }
             // ---- rows past the context end may hold anything (even NaN):
             //      zero them in the staged V tile, as P is 0 there ----
-            if (r0 + 16 > nvalid) {
+            if (!F8 && r0 + 16 > nvalid) {
               const int z0 = nvalid;
               const int nz = (r0 + 16 - z0) * (D / 8);
               for (int c = lane; c < nz; c += 32) {
@@ -476,7 +571,27 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
               __syncwarp();
             }
             // ---- O^T += V^T P^T ----
-            {
+            if constexpr (F8) {
+              // E4M3 V tile is stored transposed: the thread's keys 2t, 2t+1,
+              // 2t+8, 2t+9 of one head-dim row are one word; keys past the
+              // context end are masked to zero (P is 0 there, codes may be NaN)
+              const int kb = r0 + 2 * t;
+              const uint32_t mlo = (kb < nvalid ? 0xffffu : 0u) | (kb + 1 < nvalid ? 0xffff0000u : 0u);
+              const uint32_t mhi = (kb + 8 < nvalid ? 0xffffu : 0u) | (kb + 9 < nvalid ? 0xffff0000u : 0u);
+              const int voff = BS == 16 ? 4 * t : 8 * t + 4 * (r0 >> 4);
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                const uint32_t wa = ld_shared_u32(vtile + (16 * mt + g) * BS + voff);
+                const uint32_t wb = ld_shared_u32(vtile + (16 * mt + g + 8) * BS + voff);
+                const uint32_t af[4] = {e4m3x2_to_f16x2(wa & 0xffffu) & mlo, e4m3x2_to_f16x2(wb & 0xffffu) & mlo,
+                                        e4m3x2_to_f16x2(wa >> 16) & mhi, e4m3x2_to_f16x2(wb >> 16) & mhi};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  MmaT<Tc>::mma(o[nt][mt], af, pb_hi[nt][0], pb_hi[nt][1]);
+                  if constexpr (MmaT<Tc>::kSplitP) MmaT<Tc>::mma(o[nt][mt], af, pb_lo[nt][0], pb_lo[nt][1]);
+                }
+              }
+            } else {
               const int mi = lane >> 3;
               const int vr = r0 + (lane & 7) + (mi >> 1) * 8;
 #pragma unroll
@@ -485,8 +600,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
                 ldsm_x4_t(af, swz<BS>(vtile, vr, mt * 2 + (mi & 1)));
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                  MmaT<T>::mma(o[nt][mt], af, pb_hi[nt][0], pb_hi[nt][1]);
-                  if constexpr (MmaT<T>::kSplitP) MmaT<T>::mma(o[nt][mt], af, pb_lo[nt][0], pb_lo[nt][1]);
+                  MmaT<Tc>::mma(o[nt][mt], af, pb_hi[nt][0], pb_hi[nt][1]);
+                  if constexpr (MmaT<Tc>::kSplitP) MmaT<Tc>::mma(o[nt][mt], af, pb_lo[nt][0], pb_lo[nt][1]);
                 }
               }
             }
@@ -520,7 +635,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
           }
           if (g == 0) {
             mw[head * (D + 4) + D] = m[nt][hh];
-            mw[head * (D + 4) + D + 1] = lt;
+            // an FP8 cache's values are codes * v_scale: the sum is stored
+            // divided by v_scale, so that every later o / l carries it
+            mw[head * (D + 4) + D + 1] = F8 ? lt * a.v_inv : lt;
             mw[head * (D + 4) + D + 2] = item_bad ? 1.f : 0.f;
           }
         }
@@ -662,14 +779,14 @@ bool make_cache_map(CUtensorMap *map, const void *base, int num_blocks, int num_
 
 namespace {
 
-template <typename T, int D, int BS, int NT>
+template <typename T, int D, int BS, int NT, bool F8>
 cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
   constexpr int NCW = PA_MMA_WARPS;
-  using L = MmaLayout<D, BS, NT, NCW>;
-  auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW>;
-  CUtensorMap tmk, tmv;
-  if (!make_map<T, D, BS>(&tmk, a.k_cache, a.num_blocks, a.num_kv_heads) ||
-      !make_map<T, D, BS>(&tmv, a.v_cache, a.num_blocks, a.num_kv_heads))
+  using L = MmaLayout<D, BS, NT, NCW, F8>;
+  auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW, F8>;
+  CUtensorMap tmk{}, tmv{};  // E4M3 tiles are moved with plain bulk copies
+  if (!F8 && !(make_map<T, D, BS>(&tmk, a.k_cache, a.num_blocks, a.num_kv_heads) &&
+               make_map<T, D, BS>(&tmv, a.v_cache, a.num_blocks, a.num_kv_heads)))
     return cudaErrorInvalidValue;
   const L lay(a.num_seqs, a.group);
   static bool attr_set[64] = {};
@@ -709,11 +826,11 @@ cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a, tmk, tmv);
 }
 
-template <typename T, int D, int BS, int NT>
+template <typename T, int D, int BS, int NT, bool F8>
 int grid_mma_t(const AttnArgs &a, int sm_count) {
   constexpr int NCW = PA_MMA_WARPS;
-  using L = MmaLayout<D, BS, NT, NCW>;
-  auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW>;
+  using L = MmaLayout<D, BS, NT, NCW, F8>;
+  auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW, F8>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -730,13 +847,13 @@ int grid_mma_t(const AttnArgs &a, int sm_count) {
   return sm_count * (occ < 1 ? 1 : occ);
 }
 
-template <typename T>
+template <typename T, bool F8 = false>
 int grid_mma_d(const AttnArgs &a, int sm_count) {
   if (a.head_dim == 64)
-    return a.block_size == 16 ? (a.group <= 8 ? grid_mma_t<T, 64, 16, 1>(a, sm_count) : grid_mma_t<T, 64, 16, 2>(a, sm_count))
-                              : (a.group <= 8 ? grid_mma_t<T, 64, 32, 1>(a, sm_count) : grid_mma_t<T, 64, 32, 2>(a, sm_count));
-  return a.block_size == 16 ? (a.group <= 8 ? grid_mma_t<T, 128, 16, 1>(a, sm_count) : grid_mma_t<T, 128, 16, 2>(a, sm_count))
-                            : (a.group <= 8 ? grid_mma_t<T, 128, 32, 1>(a, sm_count) : grid_mma_t<T, 128, 32, 2>(a, sm_count));
+    return a.block_size == 16 ? (a.group <= 8 ? grid_mma_t<T, 64, 16, 1, F8>(a, sm_count) : grid_mma_t<T, 64, 16, 2, F8>(a, sm_count))
+                              : (a.group <= 8 ? grid_mma_t<T, 64, 32, 1, F8>(a, sm_count) : grid_mma_t<T, 64, 32, 2, F8>(a, sm_count));
+  return a.block_size == 16 ? (a.group <= 8 ? grid_mma_t<T, 128, 16, 1, F8>(a, sm_count) : grid_mma_t<T, 128, 16, 2, F8>(a, sm_count))
+                            : (a.group <= 8 ? grid_mma_t<T, 128, 32, 1, F8>(a, sm_count) : grid_mma_t<T, 128, 32, 2, F8>(a, sm_count));
 }
 
 template <typename T>
@@ -757,20 +874,20 @@ cudaError_t launch_bal_reduce_t(const AttnArgs &a, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, balanced_merge_kernel<T, 128>, a);
 }
 
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, bool F8>
 cudaError_t mma_nt(const AttnArgs &a, int sm_count, cudaStream_t s) {
-  return a.group <= 8 ? launch_mma_t<T, D, BS, 1>(a, sm_count, s)
-                      : launch_mma_t<T, D, BS, 2>(a, sm_count, s);
+  return a.group <= 8 ? launch_mma_t<T, D, BS, 1, F8>(a, sm_count, s)
+                      : launch_mma_t<T, D, BS, 2, F8>(a, sm_count, s);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool F8>
 cudaError_t mma_bs(const AttnArgs &a, int sm_count, cudaStream_t s) {
-  return a.block_size == 16 ? mma_nt<T, D, 16>(a, sm_count, s) : mma_nt<T, D, 32>(a, sm_count, s);
+  return a.block_size == 16 ? mma_nt<T, D, 16, F8>(a, sm_count, s) : mma_nt<T, D, 32, F8>(a, sm_count, s);
 }
 
-template <typename T>
+template <typename T, bool F8 = false>
 cudaError_t mma_d(const AttnArgs &a, int sm_count, cudaStream_t s) {
-  return a.head_dim == 64 ? mma_bs<T, 64>(a, sm_count, s) : mma_bs<T, 128>(a, sm_count, s);
+  return a.head_dim == 64 ? mma_bs<T, 64, F8>(a, sm_count, s) : mma_bs<T, 128, F8>(a, sm_count, s);
 }
 
 }  // namespace
@@ -792,6 +909,17 @@ bool decode_mma_supported(const AttnArgs &a, int dtype) {
 cudaError_t launch_decode_mma(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream) {
   if (dtype == PA_F16) return mma_d<__half>(a, sm_count, stream);
   return mma_d<__nv_bfloat16>(a, sm_count, stream);
+}
+
+int decode_mma_grid_fp8(const AttnArgs &a, int q_dtype, int sm_count) {
+  return q_dtype == PA_F16 ? grid_mma_d<__half, true>(a, sm_count)
+                           : grid_mma_d<__nv_bfloat16, true>(a, sm_count);
+}
+
+cudaError_t launch_decode_mma_fp8(const AttnArgs &a, int q_dtype, int sm_count,
+                                  cudaStream_t stream) {
+  if (q_dtype == PA_F16) return mma_d<__half, true>(a, sm_count, stream);
+  return mma_d<__nv_bfloat16, true>(a, sm_count, stream);
 }
 
 }  // namespace pa

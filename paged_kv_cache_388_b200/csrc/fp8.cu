@@ -1,0 +1,272 @@
+// fp8.cu -- FP8 (E4M3) KV cache: quantising reshape_and_cache and decode over
+// the quantised cache.
+//
+// KV-cache quantisation halves the bytes decode has to read ("理解 vLLM
+// PagedAttention", 版本矩阵: 量化 FP8 ... 权重 KV cache 量化; decode is bound by
+// the KV history it reads, "PagedAttention 实战", section 先理解 KV Cache).  One
+// scale per cache tensor: an element x of a new key is stored as the E4M3
+// code of x / k_scale (one IEEE binary32 division, round to nearest even,
+// magnitudes beyond 448 saturated), values likewise with v_scale.  Decode
+// reads the codes (one byte each) and computes with code * scale: k_scale is
+// folded into the logit scale, v_scale into the softmax sum.
+#include <cuda_fp8.h>
+
+#include "../../include/pa.h"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ void load8(const T *p, float (&x)[8]);
+
+template <>
+__device__ __forceinline__ void load8<float>(const float *p, float (&x)[8]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldcs(reinterpret_cast<const float4 *>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[8]) {
+  const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(p));
+  float2 f[4];
+  Elem<__nv_bfloat16>::to_f2(v, f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = f[i].x;
+    x[2 * i + 1] = f[i].y;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<__half>(const __half *p, float (&x)[8]) {
+  const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(p));
+  float2 f[4];
+  Elem<__half>::to_f2(v, f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = f[i].x;
+    x[2 * i + 1] = f[i].y;
+  }
+}
+
+// Two elements -> two E4M3 codes of x / scale (the first in the low byte).
+__device__ __forceinline__ uint32_t quant2(float a, float b, float scale) {
+  const float2 q = make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale));
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+}
+
+// One thread per (token, kv head, group of 16 columns).  The cache tile of a
+// (block, kv head) is laid out for the decode kernel's fragment loads:
+//   K [BS][D]: column d = 64j + 16k + c of row r goes to byte
+//     ((4j + t) ^ (r mod D/16)) * 16 + 4k + i of the row, t = (c mod 8) / 2,
+//     i = c mod 2 + 2 (c / 8): the four codes a thread's mma fragment needs
+//     for k-step 4j + k sit in one word, its four k-steps in one 16-byte
+//     chunk, and the chunk swizzle keeps the warp's loads off shared banks.
+//   V [D][BS] (transposed): key r = 16k + c of column d goes to byte
+//     d * BS + (BS == 16 ? 4t + i : 8t + 4k + i).
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
+    const T *__restrict__ key, const T *__restrict__ value, unsigned char *__restrict__ k_cache,
+    unsigned char *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping, int num_tokens,
+    int num_kv_heads, int64_t num_slots, float k_scale, float v_scale, unsigned int *err) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  constexpr int G16 = D / 16;
+  const int64_t per_token = (int64_t)num_kv_heads * G16;
+  const int64_t total = (int64_t)num_tokens * per_token;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tok = i / per_token;
+    const int64_t rest = i - tok * per_token;
+    const int64_t slot = slot_mapping[tok];
+    if (slot < 0) continue;  // padding token
+    if (slot >= num_slots) {
+      if (rest == 0) raise_error(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int h = (int)(rest / G16);
+    const int g16 = (int)(rest - (int64_t)h * G16);
+    const int j = g16 >> 2, k = g16 & 3;
+    const int64_t blk = slot / BS;
+    const int r = (int)(slot - blk * BS);
+    const int64_t tile = (blk * num_kv_heads + h) * (int64_t)(BS * D);
+    const int64_t src = (tok * num_kv_heads + h) * D + g16 * 16;
+    float x[16];
+    load8<T>(key + src, *reinterpret_cast<float(*)[8]>(x));
+    load8<T>(key + src + 8, *reinterpret_cast<float(*)[8]>(x + 8));
+    unsigned char *krow = k_cache + tile + (int64_t)r * D;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t w = quant2(x[2 * t], x[2 * t + 1], k_scale) |
+                         (quant2(x[2 * t + 8], x[2 * t + 9], k_scale) << 16);
+      const int chunk = (4 * j + t) ^ (r & (G16 - 1));
+      *reinterpret_cast<uint32_t *>(krow + chunk * 16 + 4 * k) = w;
+    }
+    load8<T>(value + src, *reinterpret_cast<float(*)[8]>(x));
+    load8<T>(value + src + 8, *reinterpret_cast<float(*)[8]>(x + 8));
+    const int kk = r >> 4, c = r & 15;
+    const int vpos = BS == 16 ? 4 * ((c & 7) >> 1) + (c & 1) + 2 * (c >> 3)
+                              : 8 * ((c & 7) >> 1) + 4 * kk + (c & 1) + 2 * (c >> 3);
+    unsigned char *vcol = v_cache + tile + (int64_t)(g16 * 16) * BS + vpos;
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const uint32_t two = quant2(x[e], x[e + 1], v_scale);
+      vcol[(int64_t)e * BS] = (unsigned char)(two & 0xffu);
+      vcol[(int64_t)(e + 1) * BS] = (unsigned char)(two >> 8);
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t reshape_fp8_bs(int block_size, const cudaLaunchConfig_t &cfg, const void *key,
+                           const void *value, void *kc, void *vc, const int64_t *slots,
+                           int num_tokens, int num_kv_heads, int64_t num_slots, float ks,
+                           float vs, unsigned int *err) {
+  if (block_size == 16)
+    return cudaLaunchKernelEx(&cfg, reshape_and_cache_fp8_kernel<T, D, 16>, (const T *)key,
+                              (const T *)value, (unsigned char *)kc, (unsigned char *)vc, slots,
+                              num_tokens, num_kv_heads, num_slots, ks, vs, err);
+  return cudaLaunchKernelEx(&cfg, reshape_and_cache_fp8_kernel<T, D, 32>, (const T *)key,
+                            (const T *)value, (unsigned char *)kc, (unsigned char *)vc, slots,
+                            num_tokens, num_kv_heads, num_slots, ks, vs, err);
+}
+
+template <typename T>
+cudaError_t reshape_fp8_d(int head_dim, int block_size, const cudaLaunchConfig_t &cfg,
+                          const void *key, const void *value, void *kc, void *vc,
+                          const int64_t *slots, int num_tokens, int num_kv_heads,
+                          int64_t num_slots, float ks, float vs, unsigned int *err) {
+  if (head_dim == 64)
+    return reshape_fp8_bs<T, 64>(block_size, cfg, key, value, kc, vc, slots, num_tokens,
+                                 num_kv_heads, num_slots, ks, vs, err);
+  return reshape_fp8_bs<T, 128>(block_size, cfg, key, value, kc, vc, slots, num_tokens,
+                                num_kv_heads, num_slots, ks, vs, err);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool scale_ok(float s) { return s > 0.f && s < 3.0e38f; }
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+int pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache, void *v_cache,
+                             const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                             int head_dim, int block_size, int num_blocks, int in_dtype,
+                             float k_scale, float v_scale, struct CUstream_st *stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+  if (in_dtype != PA_F32 && in_dtype != PA_F16 && in_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (!scale_ok(k_scale) || !scale_ok(v_scale)) return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const int64_t total = (int64_t)num_tokens * num_kv_heads * (head_dim / 16);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > (int64_t)dev.sm_count * 16) blocks = (int64_t)dev.sm_count * 16;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int64_t slots = (int64_t)num_blocks * block_size;
+  cudaError_t e;
+  if (in_dtype == PA_F32)
+    e = reshape_fp8_d<float>(head_dim, block_size, cfg, key, value, k_cache, v_cache, slot_mapping,
+                             num_tokens, num_kv_heads, slots, k_scale, v_scale, dev.err);
+  else if (in_dtype == PA_F16)
+    e = reshape_fp8_d<__half>(head_dim, block_size, cfg, key, value, k_cache, v_cache,
+                              slot_mapping, num_tokens, num_kv_heads, slots, k_scale, v_scale,
+                              dev.err);
+  else
+    e = reshape_fp8_d<__nv_bfloat16>(head_dim, block_size, cfg, key, value, k_cache, v_cache,
+                                     slot_mapping, num_tokens, num_kv_heads, slots, k_scale,
+                                     v_scale, dev.err);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, int max_blocks_per_seq,
+                  const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                  int head_dim, int block_size, int num_blocks, float scale, float k_scale,
+                  float v_scale, int max_context_len, int q_dtype, void *workspace,
+                  size_t workspace_bytes, struct CUstream_st *stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!scale_ok(k_scale) || !scale_ok(v_scale)) return PA_ERR_INVALID_ARG;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > decode_max_seqs_per_launch()) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (out == q) return PA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30) return PA_ERR_UNSUPPORTED;
+  const int cap = max_blocks_per_seq * block_size;
+  if (max_context_len <= 0 || max_context_len > cap) max_context_len = cap;
+
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  AttnArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.err = dev.err;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.split_blocks = 1;
+  a.max_splits = 1;
+  a.max_query_len = 1;
+  a.max_context_len = max_context_len;
+  a.num_q_tokens = num_seqs;
+  a.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  a.v_inv = 1.f / v_scale;
+  a.balanced = 1;
+  a.grid = decode_mma_grid_fp8(a, q_dtype, dev.sm_count);
+  if (a.grid <= 0) return PA_ERR_CUDA;
+  const size_t rec = balanced_record_bytes(a.grid, group, head_dim);
+  const size_t desc = balanced_desc_bytes(a.grid);
+  const size_t need = rec + desc + (size_t)(num_seqs + 1) * sizeof(int);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+  a.part_o = static_cast<float *>(workspace);
+  a.bal_desc = reinterpret_cast<int *>(static_cast<char *>(workspace) + rec);
+  a.bal_prefix = reinterpret_cast<int *>(static_cast<char *>(workspace) + rec + desc);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_decode_mma_fp8(a, q_dtype, dev.sm_count, s);
+  if (e == cudaSuccess) e = launch_balanced_reduce(a, q_dtype, s);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -24,9 +24,12 @@ bool g_dev_ok[kMaxDevices];
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : (dtype == PA_FP8_E4M3 ? 1 : 2); }
 
 bool dtype_ok(int dtype) { return dtype == PA_F32 || dtype == PA_F16 || dtype == PA_BF16; }
+
+// Byte movers (copy_blocks) also take FP8 caches.
+bool byte_dtype_ok(int dtype) { return dtype_ok(dtype) || dtype == PA_FP8_E4M3; }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
@@ -126,7 +129,7 @@ int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void
 int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                    struct CUstream_st *stream) {
-  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !dtype_ok(dtype))
+  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0 || !byte_dtype_ok(dtype))
     return PA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;

@@ -50,6 +50,9 @@ struct AttnArgs {
   int grp_chunks;             // prefix kernel: member chunks per group
   float *pre_rec;             // [num_seqs][num_heads][D + 4]: o (unnormalised), m, l
   int *seq_pre;               // [num_seqs] shared blocks per sequence (decode kernel CTA 0)
+  // FP8 (E4M3) cache: key elements are codes * k_scale (folded into
+  // scale_log2), value elements codes * v_scale; v_inv = 1 / v_scale.
+  float v_inv;
 };
 
 struct DevInfo {
@@ -69,6 +72,10 @@ bool decode_mma_supported(const AttnArgs &a, int dtype);
 cudaError_t launch_decode_mma(const AttnArgs &a, int dtype, int sm_count, cudaStream_t stream);
 int decode_mma_grid(const AttnArgs &a, int dtype, int sm_count);  // CTAs of a balanced launch
 cudaError_t launch_balanced_reduce(const AttnArgs &a, int dtype, cudaStream_t stream);
+// FP8 (E4M3) caches, q/out of q_dtype (PA_F16 or PA_BF16), balanced scheme only
+int decode_mma_grid_fp8(const AttnArgs &a, int q_dtype, int sm_count);
+cudaError_t launch_decode_mma_fp8(const AttnArgs &a, int q_dtype, int sm_count,
+                                  cudaStream_t stream);
 // Workspace of the balanced scheme: per-CTA partial records, the per-CTA
 // cut-pair descriptors, then the block prefix.
 inline size_t balanced_record_bytes(int grid, int group, int head_dim) {

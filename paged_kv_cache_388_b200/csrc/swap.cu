@@ -101,7 +101,8 @@ extern "C" int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const
                               int num_dst_blocks, int dtype, struct CUstream_st *stream) {
   if (num_pairs < 0 || num_kv_heads <= 0 || num_src_blocks <= 0 || num_dst_blocks <= 0)
     return PA_ERR_INVALID_ARG;
-  if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16 && dtype != PA_FP8_E4M3)
+    return PA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
   if (num_pairs == 0) return PA_OK;
@@ -114,7 +115,8 @@ extern "C" int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const
   }
   DevInfo di;
   if (device_info(&di) != cudaSuccess) return PA_ERR_CUDA;
-  const int64_t tile_bytes = (int64_t)block_size * head_dim * (dtype == PA_F32 ? 4 : 2);
+  const int64_t tile_bytes =
+      (int64_t)block_size * head_dim * (dtype == PA_F32 ? 4 : (dtype == PA_FP8_E4M3 ? 1 : 2));
   const int64_t tiles = (int64_t)num_pairs * 2 * num_kv_heads;
   const int64_t warps_per_cta = kSwapThreads / 32;
   int64_t grid = (tiles + warps_per_cta - 1) / warps_per_cta;
@@ -129,8 +131,8 @@ extern "C" int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // a tile is 2, 4 or 8 KiB (16-bit) or twice that (fp32); 4 vectors per
-  // lane move 2 KiB per warp pass
+  // a tile is 1 to 16 KiB (a multiple of 16 bytes); 4 vectors per lane move
+  // 2 KiB per warp pass
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, swap_blocks_kernel<4>, (unsigned char *)dev[0], (unsigned char *)dev[1],
       (const unsigned char *)dev[2], (const unsigned char *)dev[3], (const int64_t *)dev[4],

@@ -16,7 +16,9 @@ from . import _lib
 
 class PagedKVCache:
     def __init__(self, num_blocks, num_kv_heads, head_dim, block_size, dtype=torch.bfloat16,
-                 device="cuda", k_cache=None, v_cache=None):
+                 device="cuda", k_cache=None, v_cache=None, kv_scales=None):
+        """dtype torch.uint8 with kv_scales=(k_scale, v_scale) makes an FP8
+        (E4M3) cache: ``write`` quantises, ``attend`` decodes the codes."""
         shape = (num_blocks, num_kv_heads, block_size, head_dim)
         self.k_cache = k_cache if k_cache is not None else torch.empty(shape, dtype=dtype, device=device)
         self.v_cache = v_cache if v_cache is not None else torch.empty(shape, dtype=dtype, device=device)
@@ -24,12 +26,20 @@ class PagedKVCache:
         self.num_blocks, self.num_kv_heads, self.head_dim, self.block_size = shape[0], shape[1], shape[3], shape[2]
         self.dtype = self.k_cache.dtype
         self.device = self.k_cache.device
+        self.fp8 = self.dtype == torch.uint8
+        if self.fp8 and kv_scales is None:
+            raise ValueError("an FP8 cache needs kv_scales=(k_scale, v_scale)")
+        self.k_scale, self.v_scale = kv_scales if kv_scales is not None else (1.0, 1.0)
         self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
         self._staging = {}
 
     # ---- the three device operations --------------------------------------
     def write(self, key, value, slot_mapping):
-        _lib.pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slot_mapping)
+        if self.fp8:
+            _lib.pa_reshape_and_cache_fp8(key, value, self.k_cache, self.v_cache, slot_mapping,
+                                          self.k_scale, self.v_scale)
+        else:
+            _lib.pa_reshape_and_cache(key, value, self.k_cache, self.v_cache, slot_mapping)
 
     def copy_blocks(self, block_mapping):
         if block_mapping.shape[0]:
@@ -66,6 +76,12 @@ class PagedKVCache:
             out = torch.empty_like(q)
         mcl = max_context_len or block_tables.shape[1] * self.block_size
         ws = self.workspace(block_tables.shape[0], q.shape[1], mcl, kv_split_tokens)
+        if self.fp8:
+            if query_start_loc is not None or kv_split_tokens:
+                raise ValueError("an FP8 cache serves decode rows (one per sequence) only")
+            _lib.pa_decode_fp8(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
+                               self.k_scale, self.v_scale, max_context_len=mcl, workspace=ws)
+            return out
         _lib.pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
                        query_start_loc=query_start_loc, max_query_len=max_query_len,
                        max_context_len=mcl, kv_split_tokens=kv_split_tokens, workspace=ws)

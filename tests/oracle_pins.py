@@ -453,10 +453,159 @@ def pin_swap_blocks(lib):
         assert np.array_equal(host_k, want_k) and np.array_equal(host_v, want_v)
 
 
+def _torch_e4m3(x32):
+    """float32 array -> E4M3 codes by torch's own float8_e4m3fn conversion
+    (round to nearest even; inputs kept within +-448, where it saturates
+    nothing)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_e4m3_codec(lib):
+    """The E4M3 codec against torch's float8_e4m3fn: every one of the 256
+    codes decodes to torch's value, and quantisation of random magnitudes
+    across the whole range, of exact ties (ties go to the even code) and of
+    subnormals gives torch's code; beyond 448 the oracle saturates."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    got = np.array([oracle.e4m3_decode(c, lib=lib) for c in codes])
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    assert np.array_equal(got[~np.isnan(got)], want[~np.isnan(want)])
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal(4000) * rng.choice([1e-3, 3e-2, 1.0, 30.0, 200.0], 4000)
+    finite = want[np.isfinite(want)]
+    mids = (np.unique(finite)[1:] + np.unique(finite)[:-1]) / 2  # every tie between neighbours
+    x = np.concatenate([x, mids, -mids[:50], [0.0, -0.0, 2.0 ** -9, 2.0 ** -10, 447.0]])
+    x = x[np.abs(x) <= 448].astype(np.float32)
+    mine = np.array([oracle.e4m3_encode(v, lib=lib) for v in x], dtype=np.uint8)
+    assert np.array_equal(mine, _torch_e4m3(x))
+    assert oracle.e4m3_encode(1e6, lib=lib) == 0x7E and oracle.e4m3_encode(-500.0, lib=lib) == 0xFE
+
+
+def pin_fp8_layout_examples(lib):
+    """Where one element lands inside an FP8 (block, head) tile, against
+    positions worked out by hand from the layout contract (K columns
+    interleaved in groups of 16 and 16-byte chunks swizzled by the row; V
+    stored transposed with keys interleaved): a single token whose element d
+    is 1.0 (code 0x38) and every other element 0."""
+    cases_k = {(16, 128): [((0, 0), 0), ((0, 1), 1), ((0, 8), 2), ((0, 9), 3), ((0, 2), 16),
+                           ((0, 16), 4), ((0, 64), 64), ((3, 0), 432), ((5, 18), 708)],
+               (32, 64): [((0, 2), 16), ((1, 0), 64 + 16), ((6, 33), 6 * 64 + 16 * (0 ^ 2) + 4 * 2 + 1)]}
+    cases_v = {(16, 128): [((0, 0), 0), ((1, 0), 1), ((8, 0), 2), ((2, 0), 4), ((10, 0), 6),
+                           ((3, 5), 85)],
+               (32, 64): [((17, 2), 69), ((31, 0), 8 * 3 + 4 + 3)]}
+    for (bs, D), cases in cases_k.items():
+        for (r, d), want in cases:
+            kc = np.zeros((1, 1, bs, D), np.uint8)
+            vc = np.zeros((1, 1, bs, D), np.uint8)
+            key = np.zeros((1, 1, D), np.float32)
+            key[0, 0, d] = 1.0
+            oracle.reshape_and_cache_fp8(kc, vc, key, np.zeros_like(key), "f32",
+                                         np.array([r], np.int64), 1.0, 1.0, lib=lib)
+            assert np.flatnonzero(kc.reshape(-1)).tolist() == [want], (bs, D, r, d)
+            assert kc.reshape(-1)[want] == 0x38
+    for (bs, D), cases in cases_v.items():
+        for (r, d), want in cases:
+            kc = np.zeros((1, 1, bs, D), np.uint8)
+            vc = np.zeros((1, 1, bs, D), np.uint8)
+            val = np.zeros((1, 1, D), np.float32)
+            val[0, 0, d] = 1.0
+            oracle.reshape_and_cache_fp8(kc, vc, np.zeros_like(val), val, "f32",
+                                         np.array([r], np.int64), 1.0, 1.0, lib=lib)
+            assert np.flatnonzero(vc.reshape(-1)).tolist() == [want], (bs, D, r, d)
+
+
+def pin_fp8_reshape(lib):
+    """Quantising scatter: each token's K row lands in row (slot mod
+    block_size) of its slot's (block, head) tile as exactly torch's E4M3
+    codes of the float32 quotients x / k_scale -- the same bytes, in the
+    tile's column order; tiles that no slot addresses keep their bytes, and a
+    padding slot writes nothing.  (Where V bytes land is pinned by the worked
+    layout examples and by attention over the written codes.)"""
+    import torch
+    rng = np.random.default_rng(23)
+    nb, Hk, bs, D = 6, 2, 16, 64
+    for dt in ("f32", "bf16"):
+        key = _bits(rng.standard_normal((5, Hk, D)) * 3, dt)
+        val = _bits(rng.standard_normal((5, Hk, D)) * 3, dt)
+        kc = rng.integers(0, 256, (nb, Hk, bs, D), dtype=np.uint8)
+        vc = rng.integers(0, 256, (nb, Hk, bs, D), dtype=np.uint8)
+        k0, v0 = kc.copy(), vc.copy()
+        slots = np.array([5, -1, 40, 95, 33], dtype=np.int64)   # blocks 0, -, 2, 5, 2
+        ks, vs = 0.0517, 0.0391
+        oracle.reshape_and_cache_fp8(kc, vc, key, val, dt, slots, ks, vs, lib=lib)
+        kf = _as_f64(key, dt).astype(np.float32)
+        qk = _torch_e4m3(torch.from_numpy(kf).div(np.float32(ks)).numpy())
+        for b in (1, 3, 4):
+            assert np.array_equal(kc[b], k0[b]) and np.array_equal(vc[b], v0[b])
+        for t, sl in enumerate(slots):
+            if sl < 0:
+                continue
+            for h in range(Hk):
+                row = kc[sl // bs, h, sl % bs]
+                assert sorted(row.tolist()) == sorted(qk[t, h].tolist())
+        for b, used in ((0, {5}), (2, {8, 1}), (5, {15})):   # rows other than the written ones
+            for r in set(range(bs)) - used:
+                assert np.array_equal(kc[b, :, r], k0[b, :, r])
+
+
+def pin_fp8_decode(lib):
+    """Write tokens with the E4M3 reshape, then attend over the codes: the
+    result is bit-identical to the pinned float32 path (natural layout) over
+    the dequantised values code * scale written by the plain reshape -- for
+    scales whose products are exact in float32 (powers of two, 3/8, 5/16) --
+    with q in bf16; a one-key context returns that key's dequantised value
+    row exactly; the value scale enters linearly."""
+    import torch
+    rng = np.random.default_rng(24)
+    Hk, H = 2, 8
+    deq = np.array([oracle.e4m3_decode(c, lib=lib) for c in range(256)])
+    for bs, D in ((16, 64), (32, 128)):
+        nb = 10
+        lens = np.array([1, 16, 33, 70], dtype=np.int32)
+        need = [-(-int(L) // bs) for L in lens]
+        perm = rng.permutation(nb)
+        bt = np.zeros((len(lens), 5), np.int32)
+        pos = 0
+        for i, n in enumerate(need):            # distinct physical blocks per sequence
+            bt[i, :n] = perm[pos:pos + n]
+            pos += n
+        slots = []
+        for i, L in enumerate(lens):
+            for p in range(L):
+                slots.append(int(bt[i, p // bs]) * bs + p % bs)
+        slots = np.asarray(slots, np.int64)
+        T = slots.shape[0]
+        key = _bits(rng.standard_normal((T, Hk, D)) * 2, "bf16")
+        val = _bits(rng.standard_normal((T, Hk, D)) * 2, "bf16")
+        for ks, vs in ((0.25, 4.0), (0.375, 0.3125)):
+            kc = rng.integers(0, 256, (nb, Hk, bs, D), dtype=np.uint8)
+            vc = rng.integers(0, 256, (nb, Hk, bs, D), dtype=np.uint8)
+            oracle.reshape_and_cache_fp8(kc, vc, key, val, "bf16", slots, ks, vs, lib=lib)
+            kq = _torch_e4m3(torch.from_numpy(_as_f64(key, "bf16").astype(np.float32)).div(np.float32(ks)).numpy())
+            vq = _torch_e4m3(torch.from_numpy(_as_f64(val, "bf16").astype(np.float32)).div(np.float32(vs)).numpy())
+            kf = np.zeros((nb, Hk, bs, D), np.float32)
+            vf = np.zeros((nb, Hk, bs, D), np.float32)
+            oracle.reshape_and_cache(kf, vf, (deq[kq] * ks).astype(np.float32),
+                                     (deq[vq] * vs).astype(np.float32), slots, "f32", lib=lib)
+            q = _bits(rng.standard_normal((4, H, D)), "bf16")
+            qf = _as_f64(q, "bf16").astype(np.float32)
+            got = oracle.decode_fp8(q, "bf16", kc, vc, ks, vs, bt, lens, 0.125, lib=lib)
+            want = oracle.decode(qf, kf, vf, bt, lens, 0.125, "f32", lib=lib)
+            assert np.array_equal(got, want)
+            one = deq[vq[0]] * vs                    # sequence 0 holds token 0 only
+            assert np.array_equal(got[0].reshape(H, D), np.repeat(one, H // Hk, axis=0))
+            got2 = oracle.decode_fp8(q, "bf16", kc, vc, ks, 2 * vs, bt, lens, 0.125, lib=lib)
+            assert np.allclose(got2, 2 * got, rtol=1e-12, atol=0)
+
+
 ALL_PINS = [
     pin_brute_force, pin_decode_without_qsl, pin_identical_keys_mean, pin_single_key,
     pin_dominant_logit, pin_v_linearity, pin_scale_zero_mean, pin_hand_example,
     pin_gqa_equals_replicated_mha, pin_placement_invariance, pin_shared_equals_duplicated,
     pin_causal_truncation, pin_empty_context, pin_dtype_decoding, pin_worked_block_table,
     pin_block_counts, pin_reshape_then_gather, pin_copy_blocks, pin_swap_blocks,
+    pin_e4m3_codec, pin_fp8_layout_examples, pin_fp8_reshape, pin_fp8_decode,
 ]

@@ -38,6 +38,16 @@ MUTANTS = {
     "swap_half_block": (
         "memcpy((char *)dst_v + d * blk_bytes, (const char *)src_v + s * blk_bytes, (size_t)blk_bytes);",
         "memcpy((char *)dst_v + d * blk_bytes, (const char *)src_v + s * blk_bytes, (size_t)(blk_bytes / 2));"),
+    "e4m3_exponent_bias": ("v = ldexp((double)(8 + mant), expo - 10);",
+                           "v = ldexp((double)(8 + mant), expo - 9);"),
+    "e4m3_ties_to_odd": ("(d == best_d && (c & 1) == 0 && (best & 1) == 1)",
+                         "(d == best_d && (c & 1) == 1 && (best & 1) == 0)"),
+    "fp8_value_scale_from_key": ("elem(v_cache, tile + fp8_v_pos(off, d, block_size), dtype) * v_scale;",
+                                 "elem(v_cache, tile + fp8_v_pos(off, d, block_size), dtype) * k_scale;"),
+    "fp8_quantise_value_with_key_scale": ("fp8_v_pos((int)off, d, block_size)] = e4m3_from_float(vx / v_scale);",
+                                          "fp8_v_pos((int)off, d, block_size)] = e4m3_from_float(vx / k_scale);"),
+    "fp8_key_layout_unswizzled": ("int chunk = (4 * j + t) ^ (r % (head_dim / 16));",
+                                  "int chunk = (4 * j + t);"),
     "f16_exponent_bias": ("v = ldexp((double)(mant | 0x400), expo - 25);",
                           "v = ldexp((double)(mant | 0x400), expo - 24);"),
     "f16_subnormal_scale": ("v = ldexp((double)mant, -24);", "v = ldexp((double)mant, -25);"),
