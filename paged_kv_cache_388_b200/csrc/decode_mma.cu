@@ -136,10 +136,15 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
-// Two E4M3 codes (low byte first) -> an fp16 pair (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four E4M3 codes (byte i = code i) -> two fp16 pairs (exact): lo = codes
+// 0, 1 and hi = codes 2, 3, the lower code in the lower half.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
 }
 
 // A staged tile is BS rows x D columns of 16-bit values held as D/64 boxes of
@@ -493,8 +498,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
                 const uint32_t xb[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
                 for (int kq = 0; kq < 4; ++kq) {
-                  const uint32_t af[4] = {e4m3x2_to_f16x2(xa[kq] & 0xffffu), e4m3x2_to_f16x2(xb[kq] & 0xffffu),
-                                          e4m3x2_to_f16x2(xa[kq] >> 16), e4m3x2_to_f16x2(xb[kq] >> 16)};
+                  uint32_t af[4];  // rows g / g+8 x columns 2t.. / 2t+8..
+                  e4m3x4_to_f16x2x2(xa[kq], af[0], af[2]);
+                  e4m3x4_to_f16x2x2(xb[kq], af[1], af[3]);
 #pragma unroll
                   for (int nt = 0; nt < NT; ++nt)
                     MmaT<Tc>::mma(s[nt], af, qb[nt][4 * j + kq][0], qb[nt][4 * j + kq][1]);
@@ -576,6 +582,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
               // 2t+8, 2t+9 of one head-dim row are one word; keys past the
               // context end are masked to zero (P is 0 there, codes may be NaN)
               const int kb = r0 + 2 * t;
+              const bool partial = r0 + 16 > nvalid;  // warp-uniform
               const uint32_t mlo = (kb < nvalid ? 0xffffu : 0u) | (kb + 1 < nvalid ? 0xffff0000u : 0u);
               const uint32_t mhi = (kb + 8 < nvalid ? 0xffffu : 0u) | (kb + 9 < nvalid ? 0xffff0000u : 0u);
               const int voff = BS == 16 ? 4 * t : 8 * t + 4 * (r0 >> 4);
@@ -583,8 +590,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
               for (int mt = 0; mt < MT; ++mt) {
                 const uint32_t wa = ld_shared_u32(vtile + (16 * mt + g) * BS + voff);
                 const uint32_t wb = ld_shared_u32(vtile + (16 * mt + g + 8) * BS + voff);
-                const uint32_t af[4] = {e4m3x2_to_f16x2(wa & 0xffffu) & mlo, e4m3x2_to_f16x2(wb & 0xffffu) & mlo,
-                                        e4m3x2_to_f16x2(wa >> 16) & mhi, e4m3x2_to_f16x2(wb >> 16) & mhi};
+                uint32_t af[4];  // head-dim rows g / g+8 x keys 2t.. / 2t+8..
+                e4m3x4_to_f16x2x2(wa, af[0], af[2]);
+                e4m3x4_to_f16x2x2(wb, af[1], af[3]);
+                if (partial) {
+                  af[0] &= mlo;
+                  af[1] &= mlo;
+                  af[2] &= mhi;
+                  af[3] &= mhi;
+                }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                   MmaT<Tc>::mma(o[nt][mt], af, pb_hi[nt][0], pb_hi[nt][1]);
