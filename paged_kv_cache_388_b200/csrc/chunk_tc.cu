@@ -8,15 +8,18 @@
 // (128x64x128) and O += P V (128x128x64) run as tcgen05.mma with fp32
 // accumulators in tensor memory.
 //
-// CTA = (sequence, KV head, 128 query rows); 6 warps:
-//   warps 0-3  softmax: thread r owns row r (TMEM lane r).  Reads S from TMEM,
-//              masks, keeps a running max that is only moved (and O rescaled
-//              in TMEM) when the tile max exceeds it by more than 2^8, writes
-//              P = 2^(s - m) as bf16 hi + lo (or fp16) into swizzled shared
-//              memory, and at the end writes O / l.
-//   warp 4     producer: TMA loads of Q (once) and of each 64-key K/V tile,
-//              block by block through the block table (128-byte swizzle).
-//   warp 5     MMA issue (one elected thread) and TMEM allocation.
+// CTA = (sequence, KV head, 128 query rows); 4 * kHalves + 2 warps:
+//   softmax    warps w (and w + 4 when kHalves = 2) own rows 32w .. 32w+31
+//              (TMEM lane quadrant w), each taking 64 / kHalves of every
+//              tile's keys and 128 / kHalves of O's columns.  Reads S from
+//              TMEM, masks, exchanges the tile row max with its partner (two
+//              halves), keeps a running max that is only
+//              moved (and O rescaled in TMEM) when the tile max exceeds it by
+//              more than 2^8, writes P = 2^(s - m) as bf16 hi + lo (or fp16)
+//              into swizzled shared memory, and at the end writes O / l.
+//   producer   (warp 4 * kHalves) TMA loads of Q (once) and of each 64-key K/V
+//              tile, block by block through the block table (128-byte swizzle).
+//   MMA        (the last warp) MMA issue (one elected thread) and TMEM allocation.
 // TMEM: S double buffer (2 x 64 columns) and O (128 columns).
 // Shared memory: Q 32 KB, kStagesTC K/V stages of 32 KB, 2 P buffers of 32 KB.
 #include <cuda.h>
@@ -35,7 +38,34 @@ constexpr int kHeadDim = 128;
 #define PA_CHUNK_TC_STAGES 3
 #endif
 constexpr int kStagesTC = PA_CHUNK_TC_STAGES;  // K/V tiles in flight
-constexpr int kThreadsTC = 192;
+// Softmax warps per row quadrant: each of the kHalves warps that share 32 rows
+// (TMEM lanes) takes kKeysTC / kHalves keys of every tile and kHeadDim /
+// kHalves columns of O; with two, the pair exchanges its tile row maxima and,
+// at the end, its row sums through shared memory.  Measured on B200 (long
+// mixed batch, 4 chunks of 512 rows over 16K-token prefixes): 2.06 ms with
+// one warp per quadrant, 2.10 ms with two -- the softmax warps are not what
+// bounds the kernel -- so one is the default.
+#ifndef PA_CHUNK_TC_HALVES
+#define PA_CHUNK_TC_HALVES 1
+#endif
+constexpr int kHalves = PA_CHUNK_TC_HALVES;
+constexpr int kSoftWarps = 4 * kHalves;
+constexpr int kProdWarp = kSoftWarps;       // TMA producer
+constexpr int kMmaWarp = kSoftWarps + 1;    // MMA issue + TMEM allocation
+constexpr int kThreadsTC = 32 * (kSoftWarps + 2);
+constexpr int kKeysPerHalf = kKeysTC / kHalves;
+constexpr int kOColsPerHalf = kHeadDim / kHalves;
+static_assert(kHalves == 1 || kHalves == 2, "one or two softmax warps per row quadrant");
+// P buffers in shared memory: tile j's softmax writes buffer j % kPBufs once
+// tile j - kPBufs's P.V has read it.  Measured on B200 (long mixed batch): a
+// third buffer, a fourth K/V stage and a second softmax warp per row quadrant
+// each change nothing -- per-SM K/V tile loads (about 32 KB per 2300 cycles,
+// their latency growing with every stage added) bound the kernel once the
+// block ids are prefetched.
+#ifndef PA_CHUNK_TC_PBUFS
+#define PA_CHUNK_TC_PBUFS 2
+#endif
+constexpr int kPBufs = PA_CHUNK_TC_PBUFS;
 constexpr uint32_t kTmemCols = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between rescales
 
@@ -83,7 +113,11 @@ struct TcLayout {
   static constexpr int kStageBytes = 2 * kKeysTC * kHeadDim * 2;
   static constexpr int kP = kKV + kStagesTC * kStageBytes;       // 2 buffers x (hi, lo) x [128 x 128 B]
   static constexpr int kPBuf = 2 * kRowsTC * kKeysTC * 2;
-  static constexpr int kBar = kP + 2 * kPBuf;
+  // row-max exchange [2 buffers][kHalves][128] and row-sum exchange [kHalves][128] floats
+  static constexpr int kX = kP + kPBufs * kPBuf;
+  static constexpr int kXBytes = 3 * kHalves * kRowsTC * 4;
+  static constexpr int kBar = kX + kXBytes;
+  static_assert(kBar + 256 + 1024 <= 227 * 1024, "shared memory per CTA");
   static constexpr int kBytes = kBar + 256 + 1024;               // barriers etc. + alignment slack
 };
 
@@ -94,10 +128,12 @@ enum {
   kKvEmpty = kKvFull + kStagesTC,    // [kStagesTC]
   kSFull = kKvEmpty + kStagesTC,     // [2]
   kSFree = kSFull + 2,               // [2]
-  kPFull = kSFree + 2,               // [2]
-  kPvDone = kPFull + 2,              // [2]
-  kDone = kPvDone + 2,
-  kNumBars = kDone + 1
+  kPFull = kSFree + 2,               // [kPBufs]
+  kPvDone = kPFull + kPBufs,         // [kPBufs]
+  kDone = kPvDone + kPBufs,
+  kXFull = kDone + 1,                // [4 quadrants][2 buffers] row maxima written
+  kLFull = kXFull + 8,               // [4 quadrants] row sums written
+  kNumBars = kLFull + 4
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -250,16 +286,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[kSFull + b], 1);
-      mbar_init(&bars[kSFree + b], 4);
-      mbar_init(&bars[kPFull + b], 4);
+      mbar_init(&bars[kSFree + b], kSoftWarps);
+    }
+    for (int b = 0; b < kPBufs; ++b) {
+      mbar_init(&bars[kPFull + b], kSoftWarps);
       mbar_init(&bars[kPvDone + b], 1);
     }
     mbar_init(&bars[kDone], 1);
+    for (int b = 0; b < 8; ++b) mbar_init(&bars[kXFull + b], 32 * kHalves);
+    for (int b = 0; b < 4; ++b) mbar_init(&bars[kLFull + b], 32 * kHalves);
     flags[0] = 0;
     flags[1] = 0;
     mbar_init_fence();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kTmemCols)
@@ -277,25 +317,49 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     flags[0] = 1;
   };
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ======================= producer =======================================
+    // The whole warp reads the block table 32 ids at a time (one coalesced
+    // load, the next group fetched while the current one is issued); lane 0
+    // issues the TMA loads.
+    const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
     if (lane == 0) {
-      const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
       // Q: 128 rows (token, head) of this CTA, two 64-column boxes
       mbar_arrive_expect_tx(&bars[kQFull], kRowsTC * D * 2);
       for (int h = 0; h < 2; ++h)
         tma_load_4d(sbase + TcLayout::kQ + h * kRowsTC * 128, &tmq, h * 64, 0, kvh, q0 + t0,
                     &bars[kQFull]);
-      for (int j = 0; j < ntiles && !flags[0]; ++j) {
-        const int st = j % kStagesTC;
-        if (!mbar_wait(&bars[kKvEmpty + st], ((j / kStagesTC) & 1) ^ 1)) { fail(); break; }
-        const int b0 = j * (kKeysTC / BS);
-        const int nb = min(kKeysTC / BS, nblk - b0);  // blocks of this tile inside the sequence
+    }
+    constexpr int kBpt = kKeysTC / BS;  // blocks per tile
+    int grp = 0;                        // first block of the group held in `ids`
+    int ids = lane < nblk ? table[lane] : 0;
+    int ids_next = 32 + lane < nblk ? table[32 + lane] : 0;
+    bool aborted = false;
+    for (int j = 0; j < ntiles && !aborted; ++j) {
+      const int st = j % kStagesTC;
+      const int b0 = j * kBpt;
+      if (b0 >= grp + 32) {  // next group of 32 block ids
+        grp += 32;
+        ids = ids_next;
+        ids_next = grp + 32 + lane < nblk ? table[grp + 32 + lane] : 0;
+      }
+      const int nb = min(kBpt, nblk - b0);  // blocks of this tile inside the sequence
+      int pbs[kBpt];
+#pragma unroll
+      for (int b = 0; b < kBpt; ++b) pbs[b] = __shfl_sync(0xffffffffu, ids, (b0 - grp + b) & 31);
+      bool ok = !flags[0] && mbar_wait(&bars[kKvEmpty + st], ((j / kStagesTC) & 1) ^ 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) fail();
+        aborted = true;
+        continue;
+      }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&bars[kKvFull + st], nb * 2 * BS * D * 2);
         const uint32_t kdst = sbase + TcLayout::kKV + st * TcLayout::kStageBytes;
         const uint32_t vdst = kdst + TcLayout::kStageBytes / 2;
         for (int b = 0; b < nb; ++b) {
-          int pb = table[b0 + b];
+          int pb = pbs[b];
           if (pb < 0 || pb >= a.num_blocks) {
             raise_error(a.err, PA_DEVERR_BLOCK_ID);
             flags[1] = 1;
@@ -308,8 +372,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
         }
       }
+      __syncwarp();
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ======================= MMA issue ======================================
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc(TT::kFmt, 0, 0, kRowsTC, kKeysTC);
@@ -317,8 +382,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bool ok = mbar_wait(&bars[kQFull], 0);
       if (!ok) fail();
       auto issue_pv = [&](int jj) {
-        const int pbuf = jj & 1;
-        if (!mbar_wait(&bars[kPFull + pbuf], (jj >> 1) & 1)) { fail(); return false; }
+        const int pbuf = jj % kPBufs;
+        if (!mbar_wait(&bars[kPFull + pbuf], (jj / kPBufs) & 1)) { fail(); return false; }
         tc_fence_after();
         const uint32_t vst = sbase + TcLayout::kKV + (jj % kStagesTC) * TcLayout::kStageBytes +
                              TcLayout::kStageBytes / 2;
@@ -355,9 +420,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (!mbar_wait(&bars[kDone], 0)) fail();
     }
   } else {
-    // ======================= softmax warps (row r = tid) ======================
-    const int r = tid;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ======================= softmax warps =================================
+    // Warp w: rows 32 (w mod 4) .. +31 (its TMEM lane quadrant), keys
+    // hf * kKeysPerHalf .. of every tile and O columns hf * kOColsPerHalf ..
+    const int qd = warp & 3, hf = warp >> 2;
+    const int r = qd * 32 + lane;              // query row = TMEM lane
+    const int sid = hf * kRowsTC + r;          // 0 .. kSoftWarps * 32 - 1
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    float *xmax = reinterpret_cast<float *>(smem + TcLayout::kX);  // [2][kHalves][128]
+    float *xl = xmax + 2 * kHalves * kRowsTC;                      // [kHalves][128]
     const int tok = r / G;
     const int limit = L - Q + t0 + tok;  // last key this row may see
     const float sl2 = a.scale_log2;
@@ -367,24 +438,41 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bool ok = !flags[0] && mbar_wait(&bars[kSFull + sb], (j >> 1) & 1);
       if (!__all_sync(0xffffffffu, ok)) { fail(); break; }  // warp-uniform: tcgen05.ld is collective
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tmem_s0 + lane_off + sb * kKeysTC, sr[0]);
-      tmem_ld32(tmem_s0 + lane_off + sb * kKeysTC + 32, sr[1]);
-      tmem_wait_ld();
+      uint32_t sr[kKeysPerHalf];
+      {
+        uint32_t part[32];
+#pragma unroll
+        for (int q32 = 0; q32 < kKeysPerHalf / 32; ++q32) {
+          tmem_ld32(tmem_s0 + lane_off + sb * kKeysTC + hf * kKeysPerHalf + q32 * 32, part);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sr[q32 * 32 + i] = part[i];
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kSFree + sb]);
-      // scale and causal mask in place (as float bits), tile max
+      // scale and causal mask in place (as float bits), max over this warp's keys
       float mx = -INFINITY;
-      const int k0 = j * kKeysTC;
+      const int k0 = j * kKeysTC + hf * kKeysPerHalf;
 #pragma unroll
-      for (int c = 0; c < kKeysTC; ++c) {
-        const float v = (k0 + c <= limit) ? __uint_as_float(sr[c >> 5][c & 31]) * sl2 : -INFINITY;
-        sr[c >> 5][c & 31] = __float_as_uint(v);
+      for (int c = 0; c < kKeysPerHalf; ++c) {
+        const float v = (k0 + c <= limit) ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
+        sr[c] = __float_as_uint(v);
         mx = fmaxf(mx, v);
       }
+      if constexpr (kHalves > 1) {
+        // the tile max of the row: exchange with the other warp of the quadrant
+        const int xb = j & 1;
+        xmax[(xb * kHalves + hf) * kRowsTC + r] = mx;
+        mbar_arrive(&bars[kXFull + qd * 2 + xb]);
+        const bool got = mbar_wait(&bars[kXFull + qd * 2 + xb], (j >> 1) & 1);
+        if (!__all_sync(0xffffffffu, got)) { fail(); break; }
+#pragma unroll
+        for (int h2 = 0; h2 < kHalves; ++h2) mx = fmaxf(mx, xmax[(xb * kHalves + h2) * kRowsTC + r]);
+      }
       // lazy rescale: move the reference max only when the tile max exceeds it
-      // by more than 2^8 (first tile: always)
+      // by more than 2^8 (first tile: always); both warps of a row decide alike
       const bool need = mx > m_used + kRescaleThreshold;
       float alpha = 1.f;
       if (need) {
@@ -394,34 +482,36 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O (in TMEM) is complete up to tile j-1 once that tile's P.V is done
-        const bool done = mbar_wait(&bars[kPvDone + ((j - 1) & 1)], ((j - 1) >> 1) & 1);
+        const bool done = mbar_wait(&bars[kPvDone + ((j - 1) % kPBufs)], ((j - 1) / kPBufs) & 1);
         if (!__all_sync(0xffffffffu, done)) { fail(); break; }
         tc_fence_after();
 #pragma unroll 1
-        for (int cblk = 0; cblk < D / 32; ++cblk) {
+        for (int cblk = 0; cblk < kOColsPerHalf / 32; ++cblk) {
+          const uint32_t col = hf * kOColsPerHalf + cblk * 32;
           uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off + cblk * 32, o);
+          tmem_ld32(tmem_o + lane_off + col, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem_o + lane_off + cblk * 32, o);
+          tmem_st32(tmem_o + lane_off + col, o);
         }
         tmem_wait_st();
         tc_fence_before();
       }
-      // the P buffer of tile j was last read by tile j-2's P.V
-      if (j >= 2 && !mbar_wait(&bars[kPvDone + sb], ((j - 2) >> 1) & 1)) { fail(); break; }
+      // the P buffer of tile j was last read by tile j - kPBufs's P.V
+      const int pb = j % kPBufs;
+      if (j >= kPBufs && !mbar_wait(&bars[kPvDone + pb], ((j - kPBufs) / kPBufs) & 1)) { fail(); break; }
       // P = 2^(x - m_used) -> shared memory (K-major, 128-byte swizzle), hi and lo
-      const uint32_t prow = sbase + TcLayout::kP + sb * TcLayout::kPBuf + r * 128;
+      const uint32_t prow = sbase + TcLayout::kP + pb * TcLayout::kPBuf + r * 128;
       float psum = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < kKeysTC / 8; ++c8) {
+      for (int c8 = 0; c8 < kKeysPerHalf / 8; ++c8) {
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int c = c8 * 8 + 2 * i;
-          const float p0 = fast_exp2(__uint_as_float(sr[c >> 5][c & 31]) - m_used);
-          const float p1 = fast_exp2(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]) - m_used);
+          const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_used);
+          const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_used);
           psum += p0 + p1;
           hi[i] = TT::pack(p0, p1);
           if constexpr (TT::kSplitP) {
@@ -429,7 +519,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             lo[i] = TT::pack(p0 - h.x, p1 - h.y);
           }
         }
-        const uint32_t addr = prow + ((c8 ^ (r & 7)) << 4);
+        const int cg = hf * (kKeysPerHalf / 8) + c8;  // 16-byte chunk of the row
+        const uint32_t addr = prow + ((cg ^ (r & 7)) << 4);
         st_shared_v4(addr, hi[0], hi[1], hi[2], hi[3]);
         if constexpr (TT::kSplitP) st_shared_v4(addr + kRowsTC * 128, lo[0], lo[1], lo[2], lo[3]);
       }
@@ -443,7 +534,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int nz = (kKeysTC - z0) * 16;  // 16-byte chunks over both halves
         // all of the tile's K/V bytes must have landed before they are overwritten
         if (mbar_wait(&bars[kKvFull + (j % kStagesTC)], (j / kStagesTC) & 1)) {
-          for (int c = r; c < nz; c += kRowsTC) {
+          for (int c = sid; c < nz; c += kSoftWarps * 32) {
             const int row = z0 + c / 16, ch = c % 16;
             const int h = ch >> 3, cc = ch & 7;
             st_shared_v4(vst + h * kKeysTC * 128 + row * 128 + ((cc ^ (row & 7)) << 4), 0, 0, 0, 0);
@@ -454,21 +545,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kPFull + sb]);
+      if (lane == 0) mbar_arrive(&bars[kPFull + pb]);
     }
     // ---- epilogue: O / l -> out ----
     bool ok = !flags[0] && ntiles > 0 &&
-              mbar_wait(&bars[kPvDone + ((ntiles - 1) & 1)], ((ntiles - 1) >> 1) & 1);
+              mbar_wait(&bars[kPvDone + ((ntiles - 1) % kPBufs)], ((ntiles - 1) / kPBufs) & 1);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok && ntiles > 0) fail();
+    if constexpr (kHalves > 1) {  // the row's sum over both warps' keys
+      xl[hf * kRowsTC + r] = l;
+      mbar_arrive(&bars[kLFull + qd]);
+      if (mbar_wait(&bars[kLFull + qd], 0)) {
+        l = 0.f;
+#pragma unroll
+        for (int h2 = 0; h2 < kHalves; ++h2) l += xl[h2 * kRowsTC + r];
+      } else {
+        fail();
+        ok = false;
+      }
+      ok = __all_sync(0xffffffffu, ok);
+    }
     tc_fence_after();
     const bool write = tok < ntok && r < TPT * G;
     const float inv = (ok && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
     T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * D;
 #pragma unroll 1
-    for (int cblk = 0; cblk < D / 32; ++cblk) {
+    for (int cblk = 0; cblk < kOColsPerHalf / 32; ++cblk) {
+      const int col = hf * kOColsPerHalf + cblk * 32;
       uint32_t o[32];
-      tmem_ld32(tmem_o + lane_off + cblk * 32, o);
+      tmem_ld32(tmem_o + lane_off + col, o);
       tmem_wait_ld();
       if (write) {
 #pragma unroll
@@ -478,14 +583,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           v.y = TT::pack(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
           v.z = TT::pack(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
           v.w = TT::pack(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-          *reinterpret_cast<uint4 *>(dst + cblk * 32 + i) = v;
+          *reinterpret_cast<uint4 *>(dst + col + i) = v;
         }
       }
     }
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
