@@ -116,7 +116,8 @@ struct TcLayout {
   // row-max exchange [2 buffers][kHalves][128] and row-sum exchange [kHalves][128] floats
   static constexpr int kX = kP + kPBufs * kPBuf;
   static constexpr int kXBytes = 3 * kHalves * kRowsTC * 4;
-  static constexpr int kBar = kX + kXBytes;
+  static constexpr int kMemBad = kX + kXBytes;   // prefix mode: [128] member-table mismatch flags
+  static constexpr int kBar = kMemBad + 128;
   static_assert(kBar + 256 + 1024 <= 227 * 1024, "shared memory per CTA");
   static constexpr int kBytes = kBar + 256 + 1024;               // barriers etc. + alignment slack
 };
@@ -228,7 +229,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-template <typename T, int BS>
+// PREFIX: the shared-prefix pass of pa_decode_shared_prefix.  The CTA is
+// (group, chunk of 128/GROUP members, KV head); its rows are the members'
+// decode rows (consecutive sequences, so the same 4-D view of q serves), its
+// keys the group's shared blocks read through the group's first table, with
+// no causal mask; the softmax warps check every member's table against those
+// ids while the first tile loads; the
+// output is one record (o unnormalised, reference max in base 2, sum) per
+// (member, head) for the decode kernel to fold in.
+template <typename T, int BS, bool PREFIX = false>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     chunk_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -246,36 +255,59 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  const int tile = blockIdx.x % tiles_per_seq;
-  const int rest = blockIdx.x / tiles_per_seq;
-  const int kvh = rest % a.num_kv_heads;
-  const int seq = a.seq_begin + rest / a.num_kv_heads;
-  const int q0 = a.query_start_loc[seq];
-  const int Q = a.query_start_loc[seq + 1] - q0;
-  if (Q <= 1 || q0 < 0 || q0 + Q > a.num_q_tokens) return;  // CTA-uniform exits, before any barrier
-  if (Q > a.max_query_len) {
-    if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
-    return;
-  }
   const int G = a.group;
   const int TPT = kRowsTC / G;
-  const int t0 = tile * TPT;
-  if (t0 >= Q) return;
-  const int ntok = min(TPT, Q - t0);
-  const int L = a.context_lens[seq];
-  if (L < Q || L > a.max_context_len) {
-    if (tid == 0 && tile == 0 && kvh == 0)
-      raise_error(a.err, (L < 0 || L > a.max_context_len) ? PA_DEVERR_CONTEXT_LEN : PA_DEVERR_QUERY_LEN);
-    for (int idx = tid; idx < ntok * G * D; idx += blockDim.x) {
-      const int r = idx / D, dd = idx - r * D;
-      static_cast<T *>(a.out)[((int64_t)(q0 + t0 + r / G) * a.num_heads + kvh * G + r % G) * D + dd] =
-          Elem<T>::from_f(0.f);
+  // The CTA's work: rows (query token or member, head) q0 + t0 .., the
+  // sequence whose table holds the keys, the keys [0, kend) some row sees.
+  int kvh, seq, q0, Q, t0, ntok, L, kend;
+  if constexpr (PREFIX) {
+    const int chunk = blockIdx.x % tiles_per_seq;  // member chunk
+    const int rest = blockIdx.x / tiles_per_seq;
+    kvh = rest % a.num_kv_heads;
+    const int jg = rest / a.num_kv_heads;
+    const int s0 = a.grp_start[jg], s1 = a.grp_start[jg + 1], P = a.grp_blocks[jg];
+    const int m0 = s0 + chunk * TPT;
+    // CTA-uniform exits, before any barrier
+    if (!(0 <= s0 && s0 <= s1 && s1 <= a.num_seqs && 0 < P && P <= a.max_blocks_per_seq && m0 < s1))
+      return;
+    seq = s0;        // the group's first sequence: its table holds the shared blocks
+    q0 = m0;         // one decode row per member: q row = sequence index
+    Q = 1;
+    t0 = 0;
+    ntok = min(TPT, s1 - m0);
+    L = P * BS;      // every row sees every shared key
+    kend = L;
+  } else {
+    const int tile = blockIdx.x % tiles_per_seq;
+    const int rest = blockIdx.x / tiles_per_seq;
+    kvh = rest % a.num_kv_heads;
+    seq = a.seq_begin + rest / a.num_kv_heads;
+    q0 = a.query_start_loc[seq];
+    Q = a.query_start_loc[seq + 1] - q0;
+    if (Q <= 1 || q0 < 0 || q0 + Q > a.num_q_tokens) return;  // CTA-uniform exits, before any barrier
+    if (Q > a.max_query_len) {
+      if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
+      return;
     }
-    return;
+    t0 = tile * TPT;
+    if (t0 >= Q) return;
+    ntok = min(TPT, Q - t0);
+    L = a.context_lens[seq];
+    if (L < Q || L > a.max_context_len) {
+      if (tid == 0 && tile == 0 && kvh == 0)
+        raise_error(a.err, (L < 0 || L > a.max_context_len) ? PA_DEVERR_CONTEXT_LEN : PA_DEVERR_QUERY_LEN);
+      for (int idx = tid; idx < ntok * G * D; idx += blockDim.x) {
+        const int r = idx / D, dd = idx - r * D;
+        static_cast<T *>(a.out)[((int64_t)(q0 + t0 + r / G) * a.num_heads + kvh * G + r % G) * D + dd] =
+            Elem<T>::from_f(0.f);
+      }
+      return;
+    }
+    kend = L - Q + t0 + ntok;                      // keys [0, kend) visible to some row
   }
-  const int kend = L - Q + t0 + ntok;              // keys [0, kend) visible to some row
   const int ntiles = (kend + kKeysTC - 1) / kKeysTC;
-  const int nblk = (L + BS - 1) / BS;              // blocks that hold the sequence
+  const int nblk = (L + BS - 1) / BS;              // blocks that hold the keys
+  volatile unsigned char *bad_member = smem + TcLayout::kMemBad;
 
   // ---- set-up: barriers, TMEM ------------------------------------------------
   if (tid == 0) {
@@ -296,6 +328,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int b = 0; b < 8; ++b) mbar_init(&bars[kXFull + b], 32 * kHalves);
     for (int b = 0; b < 4; ++b) mbar_init(&bars[kLFull + b], 32 * kHalves);
     flags[0] = 0;
+    for (int i = 0; i < 128; ++i) bad_member[i] = 0;
     flags[1] = 0;
     mbar_init_fence();
   }
@@ -429,9 +462,36 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     float *xmax = reinterpret_cast<float *>(smem + TcLayout::kX);  // [2][kHalves][128]
     float *xl = xmax + 2 * kHalves * kRowsTC;                      // [kHalves][128]
+    (void)xl;
     const int tok = r / G;
-    const int limit = L - Q + t0 + tok;  // last key this row may see
+    const int limit = PREFIX ? L - 1 : L - Q + t0 + tok;  // last key this row may see
     const float sl2 = a.scale_log2;
+    if constexpr (PREFIX) {
+      // Every member's table must hold the group's ids over the shared range.
+      // All of the checks' loads are issued together here, while the first
+      // tile is still in flight, instead of one dependent round trip per tile
+      // on the producer's path.
+      const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
+      for (int x0 = sid; x0 < ntok * nblk; x0 += kSoftWarps * 32 * 8) {
+        int mine[8], ref[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int x = x0 + u * kSoftWarps * 32;
+          const int i = x / nblk, b = x - i * nblk;
+          mine[u] = x < ntok * nblk ? a.block_tables[(int64_t)(q0 + i) * a.max_blocks_per_seq + b] : 0;
+          ref[u] = x < ntok * nblk ? table[b] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int x = x0 + u * kSoftWarps * 32;
+          if (x < ntok * nblk && mine[u] != ref[u]) {
+            const int i = x / nblk;
+            if (!bad_member[i]) raise_error(a.err, PA_DEVERR_PREFIX);
+            bad_member[i] = 1;
+          }
+        }
+      }
+    }
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
@@ -567,23 +627,50 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     tc_fence_after();
     const bool write = tok < ntok && r < TPT * G;
-    const float inv = (ok && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
-    T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * D;
+    if constexpr (PREFIX) {
+      // the member flags of every softmax warp (named barrier 1)
+      asm volatile("bar.sync 1, %0;" ::"n"(kSoftWarps * 32) : "memory");
+      // record of (member q0 + tok, head): o unnormalised, the reference max
+      // (base 2) o and l are relative to, l; NaN l marks a poisoned record
+      const bool poison = !ok || flags[1] || (write && bad_member[tok]);
+      float *rec = a.pre_rec + ((int64_t)(q0 + tok) * a.num_heads + kvh * G + r % G) * (D + 4);
 #pragma unroll 1
-    for (int cblk = 0; cblk < kOColsPerHalf / 32; ++cblk) {
-      const int col = hf * kOColsPerHalf + cblk * 32;
-      uint32_t o[32];
-      tmem_ld32(tmem_o + lane_off + col, o);
-      tmem_wait_ld();
-      if (write) {
+      for (int cblk = 0; cblk < kOColsPerHalf / 32; ++cblk) {
+        const int col = hf * kOColsPerHalf + cblk * 32;
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_off + col, o);
+        tmem_wait_ld();
+        if (write) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 v;
-          v.x = TT::pack(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
-          v.y = TT::pack(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-          v.z = TT::pack(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-          v.w = TT::pack(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-          *reinterpret_cast<uint4 *>(dst + col + i) = v;
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4 *>(rec + col + i) =
+                make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]), __uint_as_float(o[i + 2]),
+                            __uint_as_float(o[i + 3]));
+        }
+      }
+      if (write && hf == 0) {
+        rec[D] = m_used;
+        rec[D + 1] = poison ? __int_as_float(0x7fc00000) : l;
+      }
+    } else {
+      const float inv = (ok && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
+      T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * D;
+#pragma unroll 1
+      for (int cblk = 0; cblk < kOColsPerHalf / 32; ++cblk) {
+        const int col = hf * kOColsPerHalf + cblk * 32;
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_off + col, o);
+        tmem_wait_ld();
+        if (write) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = TT::pack(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+            v.y = TT::pack(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            v.z = TT::pack(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            v.w = TT::pack(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *reinterpret_cast<uint4 *>(dst + col + i) = v;
+          }
         }
       }
     }
@@ -609,7 +696,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_tc() {
   return fn;
 }
 
-template <typename T, int BS>
+template <typename T, int BS, bool PREFIX = false>
 cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
   auto fn = encode_fn_tc();
   if (!fn) return cudaErrorNotSupported;
@@ -638,7 +725,7 @@ cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = chunk_tc_kernel<T, BS>;
+  auto kern = chunk_tc_kernel<T, BS, PREFIX>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -647,8 +734,10 @@ cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int tiles = (a.max_query_len + TPT - 1) / TPT;
-  const int64_t grid = (int64_t)a.num_seqs * a.num_kv_heads * tiles;
+  // chunk rows: (sequence, KV head, tile of TPT tokens); prefix: (group, KV
+  // head, chunk of TPT members)
+  const int tiles = PREFIX ? (a.max_group + TPT - 1) / TPT : (a.max_query_len + TPT - 1) / TPT;
+  const int64_t grid = (int64_t)(PREFIX ? a.num_groups : a.num_seqs) * a.num_kv_heads * tiles;
   if (grid == 0) return cudaSuccess;
   kern<<<(unsigned)grid, kThreadsTC, TcLayout::kBytes, stream>>>(a, tmq, tmk, tmv, tiles);
   return cudaGetLastError();
@@ -659,6 +748,14 @@ cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
 bool chunk_tc_supported(const AttnArgs &a, int dtype) {
   return (dtype == PA_BF16 || dtype == PA_F16) && a.head_dim == kHeadDim && a.group >= 1 &&
          a.group <= kRowsTC && kRowsTC % a.group == 0 && encode_fn_tc() != nullptr;
+}
+
+cudaError_t launch_prefix_tc(const AttnArgs &a, int dtype, cudaStream_t stream) {
+  if (dtype == PA_BF16)
+    return a.block_size == 16 ? launch_tc_t<__nv_bfloat16, 16, true>(a, stream)
+                              : launch_tc_t<__nv_bfloat16, 32, true>(a, stream);
+  return a.block_size == 16 ? launch_tc_t<__half, 16, true>(a, stream)
+                            : launch_tc_t<__half, 32, true>(a, stream);
 }
 
 cudaError_t launch_chunk_tc(const AttnArgs &a, int dtype, cudaStream_t stream) {

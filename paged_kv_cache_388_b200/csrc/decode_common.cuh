@@ -311,7 +311,7 @@ __device__ __forceinline__ void store4<__half>(__half *dst, float4 v) {
 
 // Merge one partial softmax result (accumulator slice x, running max m in
 // base 2, running sum l; l = NaN marks a poisoned record) into (M, Lsum, o).
-__device__ __forceinline__ void fold_record(const float *x4, float m, float l, float *M,
+__device__ __forceinline__ void fold_record(float4 x, float m, float l, float *M,
                                             float *Lsum, float4 *o, bool *bad) {
   if (isnan(l)) {
     *bad = true;
@@ -321,7 +321,6 @@ __device__ __forceinline__ void fold_record(const float *x4, float m, float l, f
   if (Mn == -INFINITY) return;
   const float sa = *M == -INFINITY ? 0.f : fast_exp2(*M - Mn);
   const float sb = m == -INFINITY ? 0.f : fast_exp2(m - Mn);
-  const float4 x = *reinterpret_cast<const float4 *>(x4);
   o->x = o->x * sa + x.x * sb;
   o->y = o->y * sa + x.y * sb;
   o->z = o->z * sa + x.z * sb;
@@ -337,13 +336,29 @@ __device__ __forceinline__ void fold_record(const float *x4, float m, float l, f
 // Warp w = bl*hsplit + hs handled heads hs*gw .. hs*gw+gw-1 of the group for
 // the blocks j = bl (mod nbl).  All consumer threads (ncw*32) call this;
 // direct items go to `out`, split items to the workspace.
-template <typename T, int D>
+// The prefix kernel's partial (o, m, l) of head hg of a shared-prefix item,
+// read from the workspace.
+struct PreFromGlobal {
+  const float *rec;  // the item's first group head: [group heads][D + 4]
+  int D;
+  __device__ __forceinline__ void operator()(int hg, int d4, float4 *x, float *m, float *l) const {
+    const float *r = rec + hg * (D + 4);
+    *x = *reinterpret_cast<const float4 *>(r + d4 * 4);
+    *m = r[D];
+    *l = r[D + 1];
+  }
+};
+
+// `pre` gives the prefix partial of a direct item of a shared-prefix
+// sequence (item.boff > 0), which is folded in before the store.
+template <typename T, int D, typename Pre>
 __device__ __forceinline__ void merge_store(const AttnArgs &a, const Seg &seg,
                                             const float *merge, int mstride, int gw,
-                                            int hsplit, int nbl, int ncw, int tid) {
+                                            int hsplit, int nbl, int ncw, int tid, const Pre &pre) {
   const Item &item = seg.it;
   constexpr int D4 = D / 4;
   const int total4 = a.group * D4;
+  const bool fold = seg.out == kOutDirect && item.boff > 0;
   for (int idx = tid; idx < total4; idx += ncw * 32) {
     const int hg = idx / D4;  // head within the group
     const int d4 = idx - hg * D4;
@@ -362,17 +377,18 @@ __device__ __forceinline__ void merge_store(const AttnArgs &a, const Seg &seg,
       const float mb = src[D];
       const float wgt = mb == -INFINITY ? 0.f : fast_exp2(mb - M);
       Lsum += wgt * src[D + 1];
-      const float4 x = *reinterpret_cast<const float4 *>(src + d4 * 4);
-      o.x += wgt * x.x;
-      o.y += wgt * x.y;
-      o.z += wgt * x.z;
-      o.w += wgt * x.w;
+      const float4 y = *reinterpret_cast<const float4 *>(src + d4 * 4);
+      o.x += wgt * y.x;
+      o.y += wgt * y.y;
+      o.z += wgt * y.z;
+      o.w += wgt * y.w;
     }
     const int head = item.kvh * a.group + hg;
-    if (seg.out == kOutDirect && item.boff > 0) {
-      // the sequence's shared prefix: fold in the prefix kernel's partial
-      const float *pr = a.pre_rec + ((int64_t)item.seq * a.num_heads + head) * (D + 4);
-      fold_record(pr + d4 * 4, pr[D], pr[D + 1], &M, &Lsum, &o, &anybad);
+    if (fold) {  // the sequence's shared prefix: fold in the prefix kernel's partial
+      float4 x;
+      float xm, xl;
+      pre(hg, d4, &x, &xm, &xl);
+      fold_record(x, xm, xl, &M, &Lsum, &o, &anybad);
     }
     if (seg.out == kOutDirect) {
       const float inv = (Lsum > 0.f && !anybad) ? 1.f / Lsum : 0.f;
@@ -396,6 +412,15 @@ __device__ __forceinline__ void merge_store(const AttnArgs &a, const Seg &seg,
       }
     }
   }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void merge_store(const AttnArgs &a, const Seg &seg,
+                                            const float *merge, int mstride, int gw,
+                                            int hsplit, int nbl, int ncw, int tid) {
+  const PreFromGlobal pre{
+      a.pre_rec + ((int64_t)seg.it.seq * a.num_heads + seg.it.kvh * a.group) * (D + 4), D};
+  merge_store<T, D>(a, seg, merge, mstride, gw, hsplit, nbl, ncw, tid, pre);
 }
 
 }  // namespace dec

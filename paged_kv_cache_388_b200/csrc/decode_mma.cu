@@ -196,6 +196,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
                             const __grid_constant__ CUtensorMap tmv) {
   using L = MmaLayout<D, BS, NT, NCW, F8>;
   using Tc = typename std::conditional<F8, __half, T>::type;
+  // a prefix partial of up to NT * 8 heads must fit the ring at once
+  static_assert((NT * 8 * (D + 4) * 4 + L::kStage - 1) / L::kStage <= L::kStages, "ring too small");
   constexpr int KS = D / 16;    // k-steps of the QK product (head dim)
   constexpr int MT = D / 16;    // m-tiles of the PV product (head dim)
   extern __shared__ unsigned char smem_raw[];
@@ -342,6 +344,37 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
                   tma_load_2d(dst + L::kTile + bx * (BS * 128), &tmv, bx * 64, row, &full[slot]);
                 }
               }
+            }
+          }
+          __syncwarp();
+        }
+      }
+      if (seg.out == kOutDirect && item.boff > 0) {
+        // The prefix kernel's partial that this item folds in at its end
+        // ([group heads][D + 4] floats) comes through the next ring stages,
+        // kStage bytes each: issued behind the item's last block, it lands
+        // while that block is computed, where a global read at the fold
+        // would wait a full round trip of a saturated memory system.
+        const int rec_bytes = a.group * (D + 4) * 4;
+        const unsigned char *pr = reinterpret_cast<const unsigned char *>(
+            a.pre_rec + ((int64_t)item.seq * a.num_heads + item.kvh * a.group) * (D + 4));
+        for (int c = 0; c * L::kStage < rec_bytes; ++c) {
+          const uint32_t slot = it % L::kStages;
+          const uint32_t par = ((it / L::kStages) & 1u) ^ 1u;
+          ++it;
+          bool ok = !*abort_flag;
+          if (ok) ok = mbar_wait(&empty[slot], par);
+          if (lane == 0) {
+            if (!ok) {
+              if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+              *abort_flag = 1;
+              bad[slot] = 1;
+              mbar_arrive(&full[slot]);
+            } else {
+              bad[slot] = 0;
+              const int bytes = min(L::kStage, rec_bytes - c * L::kStage);
+              mbar_arrive_expect_tx(&full[slot], bytes);
+              bulk_load(smem + lay.ring + slot * L::kStage, pr + c * L::kStage, bytes, &full[slot]);
             }
           }
           __syncwarp();
@@ -657,8 +690,27 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
         }
       }
     }
+    // the prefix partial of a shared-prefix item, from the ring stages the
+    // producer loaded it into (a failed stage poisons the row: NaN sum)
+    const int nrec = (seg.out == kOutDirect && item.boff > 0)
+                         ? (a.group * (D + 4) * 4 + L::kStage - 1) / L::kStage : 0;
+    bool rec_ok = true;
+    for (int c = 0; c < nrec; ++c) rec_ok &= wait_stage(it_base + c);
+    const unsigned char *ring_g = smem + lay.ring;
+    const uint32_t rec_first = it_base;
+    auto pre = [&](int hg, int d4, float4 *x, float *pm, float *pl) {
+      const int f = (hg * (D + 4) + d4 * 4) * 4;  // byte offsets inside the record:
+      const int fm = (hg * (D + 4) + D) * 4;      // each 16-byte run lies in one stage
+      const unsigned char *px = ring_g + ((rec_first + f / L::kStage) % L::kStages) * L::kStage + f % L::kStage;
+      const unsigned char *pmp = ring_g + ((rec_first + fm / L::kStage) % L::kStages) * L::kStage + fm % L::kStage;
+      *x = *reinterpret_cast<const float4 *>(px);
+      *pm = reinterpret_cast<const float *>(pmp)[0];
+      *pl = rec_ok ? reinterpret_cast<const float *>(pmp)[1] : __int_as_float(0x7fc00000);
+    };
     named_sync(1, NCW * 32);
-    merge_store<T, D>(a, seg, merge, mstride, a.group, 1, NCW, NCW, tid);
+    merge_store<T, D>(a, seg, merge, mstride, a.group, 1, NCW, NCW, tid, pre);
+    for (int c = 0; c < nrec; ++c) release_stage(it_base + c);
+    it_base += nrec;
     if (seg.out == kOutRecord && item.b0 == 0 && tid == 0) {
       // This CTA holds the first piece of a pair cut at its range end: leave
       // the merge kernel a descriptor {record slot, kv head, last covering

@@ -402,12 +402,22 @@ int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const
   a.num_groups = num_groups;
   const int mpc = kPrefixRows / group;
   a.grp_chunks = (max_group_size + mpc - 1) / mpc;
+  a.max_group = max_group_size;
 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
   if (num_groups > 0) {
-    const int64_t units = (int64_t)num_groups * a.grp_chunks * num_kv_heads;
-    e = launch_prefix(a, dtype, prefix_cluster(units, dev.sm_count), s);
+    // the shared blocks on the 5th-generation tensor cores (head_dim 128,
+    // group dividing 128) unless PA_PREFIX_KERNEL=mma asks for the mma.sync
+    // cluster kernel, which serves every other shape
+    const char *sel = getenv("PA_PREFIX_KERNEL");
+    const bool want_mma = sel && strcmp(sel, "mma") == 0;
+    if (!want_mma && chunk_tc_supported(a, dtype)) {
+      e = launch_prefix_tc(a, dtype, s);
+    } else {
+      const int64_t units = (int64_t)num_groups * a.grp_chunks * num_kv_heads;
+      e = launch_prefix(a, dtype, prefix_cluster(units, dev.sm_count), s);
+    }
   }
   if (e == cudaSuccess) e = launch_decode_mma(a, dtype, dev.sm_count, s);
   if (e == cudaSuccess) e = launch_balanced_reduce(a, dtype, s);

@@ -48,6 +48,7 @@ struct AttnArgs {
   const int32_t *grp_blocks;  // [num_groups] leading blocks the group's members share
   int num_groups;
   int grp_chunks;             // prefix kernel: member chunks per group
+  int max_group;              // host bound of any group's size
   float *pre_rec;             // [num_seqs][num_heads][D + 4]: o (unnormalised), m, l
   int *seq_pre;               // [num_seqs] shared blocks per sequence (decode kernel CTA 0)
   // FP8 (E4M3) cache: key elements are codes * k_scale (folded into
@@ -102,6 +103,8 @@ int decode_max_seqs_per_launch();
 // Implemented in chunk_tc.cu (tcgen05 chunked-query kernel, head_dim 128)
 bool chunk_tc_supported(const AttnArgs &a, int dtype);
 cudaError_t launch_chunk_tc(const AttnArgs &a, int dtype, cudaStream_t stream);
+// The same kernel as the shared-prefix pass (group rows, records out)
+cudaError_t launch_prefix_tc(const AttnArgs &a, int dtype, cudaStream_t stream);
 
 // Implemented in chunk.cu
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int num_q_tokens, cudaStream_t stream);
