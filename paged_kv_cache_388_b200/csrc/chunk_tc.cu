@@ -34,8 +34,17 @@ namespace {
 constexpr int kRowsTC = 128;   // query rows per CTA (MMA M)
 constexpr int kKeysTC = 64;    // keys per tile (MMA N of S, K of P.V)
 constexpr int kHeadDim = 128;
+// P in tensor memory: the softmax writes P (bf16 hi + lo, or fp16) over its
+// tile's S columns and P V reads it from there as the A operand, instead of
+// P going through shared memory (generic stores, a proxy fence, and the
+// tensor core reading it back).  Three S/P buffers in TMEM then let S(j) be
+// issued while P(j-1) and P(j-2) are still to be consumed.
+#ifndef PA_CHUNK_TC_PTMEM
+#define PA_CHUNK_TC_PTMEM 1
+#endif
+constexpr bool kPTmem = PA_CHUNK_TC_PTMEM != 0;
 #ifndef PA_CHUNK_TC_STAGES
-#define PA_CHUNK_TC_STAGES 3
+#define PA_CHUNK_TC_STAGES (PA_CHUNK_TC_PTMEM ? 4 : 3)
 #endif
 constexpr int kStagesTC = PA_CHUNK_TC_STAGES;  // K/V tiles in flight
 // Softmax warps per row quadrant: each of the kHalves warps that share 32 rows
@@ -56,17 +65,23 @@ constexpr int kThreadsTC = 32 * (kSoftWarps + 2);
 constexpr int kKeysPerHalf = kKeysTC / kHalves;
 constexpr int kOColsPerHalf = kHeadDim / kHalves;
 static_assert(kHalves == 1 || kHalves == 2, "one or two softmax warps per row quadrant");
-// P buffers in shared memory: tile j's softmax writes buffer j % kPBufs once
-// tile j - kPBufs's P.V has read it.  Measured on B200 (long mixed batch): a
-// third buffer, a fourth K/V stage and a second softmax warp per row quadrant
-// each change nothing -- per-SM K/V tile loads (about 32 KB per 2300 cycles,
-// their latency growing with every stage added) bound the kernel once the
-// block ids are prefetched.
+// P buffers in shared memory (PA_CHUNK_TC_PTMEM=0): tile j's softmax writes
+// buffer j % kPBufs once tile j - kPBufs's P.V has read it.  Measured on B200
+// (long mixed batch, whole call): P in TMEM 1.717 ms vs 1.742 ms through
+// shared memory; 3 / 4 / 5 K/V stages 1.729 / 1.717 / 1.717 ms; a second
+// softmax warp per row quadrant 1.735 ms; separate K and V rings (V trailing
+// K by a tile) 2.05-2.18 ms.  A tile takes about 2300 cycles, of which the
+// MMA thread spends about 1550 issuing its 16 tcgen05.mma (the tensor pipe
+// runs these M=128, N=64/128, K=16 shapes at about half its peak rate) and
+// the softmax warps about 1700: the chain S -> softmax -> P V, not the
+// loads, sets the pace.
 #ifndef PA_CHUNK_TC_PBUFS
 #define PA_CHUNK_TC_PBUFS 2
 #endif
-constexpr int kPBufs = PA_CHUNK_TC_PBUFS;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kSBufs = kPTmem ? 3 : 2;                   // S (and with kPTmem P) buffers in TMEM
+constexpr int kPBufs = kPTmem ? kSBufs : PA_CHUNK_TC_PBUFS;
+constexpr uint32_t kTmemCols = kPTmem ? 512 : 256;     // allocation: a power of two
+constexpr uint32_t kTmemO = kPTmem ? 256 : 128;        // O's first column
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between rescales
 
 template <typename T>
@@ -114,12 +129,12 @@ struct TcLayout {
   static constexpr int kP = kKV + kStagesTC * kStageBytes;       // 2 buffers x (hi, lo) x [128 x 128 B]
   static constexpr int kPBuf = 2 * kRowsTC * kKeysTC * 2;
   // row-max exchange [2 buffers][kHalves][128] and row-sum exchange [kHalves][128] floats
-  static constexpr int kX = kP + kPBufs * kPBuf;
+  static constexpr int kX = kP + (kPTmem ? 0 : kPBufs * kPBuf);
   static constexpr int kXBytes = 3 * kHalves * kRowsTC * 4;
   static constexpr int kMemBad = kX + kXBytes;   // prefix mode: [128] member-table mismatch flags
   static constexpr int kBar = kMemBad + 128;
-  static_assert(kBar + 256 + 1024 <= 227 * 1024, "shared memory per CTA");
-  static constexpr int kBytes = kBar + 256 + 1024;               // barriers etc. + alignment slack
+  static_assert(kBar + 512 + 1024 <= 227 * 1024, "shared memory per CTA");
+  static constexpr int kBytes = kBar + 512 + 1024;               // barriers etc. + alignment slack
 };
 
 // barrier indices within the barrier block
@@ -127,9 +142,9 @@ enum {
   kQFull = 0,
   kKvFull = 1,                       // [kStagesTC]
   kKvEmpty = kKvFull + kStagesTC,    // [kStagesTC]
-  kSFull = kKvEmpty + kStagesTC,     // [2]
-  kSFree = kSFull + 2,               // [2]
-  kPFull = kSFree + 2,               // [kPBufs]
+  kSFull = kKvEmpty + kStagesTC,     // [kSBufs]
+  kSFree = kSFull + kSBufs,          // [kSBufs] (P in shared memory only)
+  kPFull = kSFree + kSBufs,          // [kPBufs]
   kPvDone = kPFull + kPBufs,         // [kPBufs]
   kDone = kPvDone + kPBufs,
   kXFull = kDone + 1,                // [4 quadrants][2 buffers] row maxima written
@@ -181,6 +196,16 @@ __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t da, uint64_t db, 
       : "memory");
 }
 
+// A from tensor memory (lane = row, 16 K elements in 8 consecutive columns).
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
                    "r"(smem_addr(bar))
@@ -214,6 +239,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
       "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
       "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -316,7 +348,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&bars[kKvFull + s], 1);
       mbar_init(&bars[kKvEmpty + s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSBufs; ++b) {
       mbar_init(&bars[kSFull + b], 1);
       mbar_init(&bars[kSFree + b], kSoftWarps);
     }
@@ -343,7 +375,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s0 = tmem, tmem_o = tmem + 128;
+  const uint32_t tmem_s0 = tmem, tmem_o = tmem + kTmemO;
 
   auto fail = [&](void) {
     if (!flags[0]) raise_error(a.err, PA_DEVERR_TIMEOUT);
@@ -420,13 +452,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tc_fence_after();
         const uint32_t vst = sbase + TcLayout::kKV + (jj % kStagesTC) * TcLayout::kStageBytes +
                              TcLayout::kStageBytes / 2;
-        const uint32_t pbase = sbase + TcLayout::kP + pbuf * TcLayout::kPBuf;
         const int nparts = TT::kSplitP ? 2 : 1;
         for (int part = 0; part < nparts; ++part) {
           for (int ks = 0; ks < kKeysTC / 16; ++ks) {
-            const uint64_t da = umma_desc(pbase + part * (kRowsTC * 128) + ks * 32, 16, 1024);
             const uint64_t db = umma_desc(vst + ks * 16 * 128, kKeysTC * 128, 1024);
-            umma(tmem_o, da, db, idesc_pv, (jj > 0 || part > 0 || ks > 0) ? 1u : 0u);
+            const uint32_t acc = (jj > 0 || part > 0 || ks > 0) ? 1u : 0u;
+            if constexpr (kPTmem) {
+              // P of tile jj: hi in the first half of its S columns, lo in the second
+              const uint32_t pa = tmem_s0 + (jj % kSBufs) * kKeysTC + part * (kKeysTC / 2) + ks * 8;
+              umma_ts(tmem_o, pa, db, idesc_pv, acc);
+            } else {
+              const uint32_t pbase = sbase + TcLayout::kP + pbuf * TcLayout::kPBuf;
+              const uint64_t da = umma_desc(pbase + part * (kRowsTC * 128) + ks * 32, 16, 1024);
+              umma(tmem_o, da, db, idesc_pv, acc);
+            }
           }
         }
         umma_commit(&bars[kPvDone + pbuf]);
@@ -434,9 +473,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         return true;
       };
       for (int j = 0; ok && j < ntiles && !flags[0]; ++j) {
-        const int st = j % kStagesTC, sb = j & 1;
+        const int st = j % kStagesTC, sb = j % kSBufs;
         if (!mbar_wait(&bars[kKvFull + st], (j / kStagesTC) & 1)) { fail(); break; }
-        if (!mbar_wait(&bars[kSFree + sb], ((j >> 1) & 1) ^ 1)) { fail(); break; }
+        if constexpr (kPTmem) {
+          // S(j) overwrites P(j - kSBufs): its P V must be done
+          if (j >= kSBufs && !mbar_wait(&bars[kPvDone + sb], ((j / kSBufs) - 1) & 1)) { fail(); break; }
+        } else {
+          if (!mbar_wait(&bars[kSFree + sb], ((j / kSBufs) & 1) ^ 1)) { fail(); break; }
+        }
         tc_fence_after();
         const uint32_t kst = sbase + TcLayout::kKV + st * TcLayout::kStageBytes;
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -494,8 +538,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < ntiles; ++j) {
-      const int sb = j & 1;
-      bool ok = !flags[0] && mbar_wait(&bars[kSFull + sb], (j >> 1) & 1);
+      const int sb = j % kSBufs;
+      bool ok = !flags[0] && mbar_wait(&bars[kSFull + sb], (j / kSBufs) & 1);
       if (!__all_sync(0xffffffffu, ok)) { fail(); break; }  // warp-uniform: tcgen05.ld is collective
       tc_fence_after();
       uint32_t sr[kKeysPerHalf];
@@ -509,9 +553,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           for (int i = 0; i < 32; ++i) sr[q32 * 32 + i] = part[i];
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kSFree + sb]);
+      if constexpr (!kPTmem) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kSFree + sb]);
+      }
       // scale and causal mask in place (as float bits), max over this warp's keys
       float mx = -INFINITY;
       const int k0 = j * kKeysTC + hf * kKeysPerHalf;
@@ -558,20 +604,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tmem_wait_st();
         tc_fence_before();
       }
-      // the P buffer of tile j was last read by tile j - kPBufs's P.V
       const int pb = j % kPBufs;
-      if (j >= kPBufs && !mbar_wait(&bars[kPvDone + pb], ((j - kPBufs) / kPBufs) & 1)) { fail(); break; }
-      // P = 2^(x - m_used) -> shared memory (K-major, 128-byte swizzle), hi and lo
-      const uint32_t prow = sbase + TcLayout::kP + pb * TcLayout::kPBuf + r * 128;
       float psum = 0.f;
+      if constexpr (kPTmem) {
+        // P = 2^(x - m_used) over this tile's S columns: hi words at
+        // columns [0, 32), lo words at [32, 64) of the buffer, two keys a word
+        constexpr int W = kKeysPerHalf / 2;  // words of this warp per part
+        uint32_t hi[W], lo[W];
 #pragma unroll
-      for (int c8 = 0; c8 < kKeysPerHalf / 8; ++c8) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = c8 * 8 + 2 * i;
-          const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_used);
-          const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_used);
+        for (int i = 0; i < W; ++i) {
+          const float p0 = fast_exp2(__uint_as_float(sr[2 * i]) - m_used);
+          const float p1 = fast_exp2(__uint_as_float(sr[2 * i + 1]) - m_used);
           psum += p0 + p1;
           hi[i] = TT::pack(p0, p1);
           if constexpr (TT::kSplitP) {
@@ -579,10 +622,38 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             lo[i] = TT::pack(p0 - h.x, p1 - h.y);
           }
         }
-        const int cg = hf * (kKeysPerHalf / 8) + c8;  // 16-byte chunk of the row
-        const uint32_t addr = prow + ((cg ^ (r & 7)) << 4);
-        st_shared_v4(addr, hi[0], hi[1], hi[2], hi[3]);
-        if constexpr (TT::kSplitP) st_shared_v4(addr + kRowsTC * 128, lo[0], lo[1], lo[2], lo[3]);
+        const uint32_t pcol = tmem_s0 + lane_off + sb * kKeysTC + hf * W;
+#pragma unroll
+        for (int w16 = 0; w16 < W / 16; ++w16) {
+          tmem_st16(pcol + w16 * 16, hi + w16 * 16);
+          if constexpr (TT::kSplitP) tmem_st16(pcol + kKeysTC / 2 + w16 * 16, lo + w16 * 16);
+        }
+        tmem_wait_st();
+      } else {
+        // the P buffer of tile j was last read by tile j - kPBufs's P.V
+        if (j >= kPBufs && !mbar_wait(&bars[kPvDone + pb], ((j - kPBufs) / kPBufs) & 1)) { fail(); break; }
+        // P = 2^(x - m_used) -> shared memory (K-major, 128-byte swizzle), hi and lo
+        const uint32_t prow = sbase + TcLayout::kP + pb * TcLayout::kPBuf + r * 128;
+#pragma unroll
+        for (int c8 = 0; c8 < kKeysPerHalf / 8; ++c8) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = c8 * 8 + 2 * i;
+            const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_used);
+            const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_used);
+            psum += p0 + p1;
+            hi[i] = TT::pack(p0, p1);
+            if constexpr (TT::kSplitP) {
+              const float2 h = TT::unpack(hi[i]);
+              lo[i] = TT::pack(p0 - h.x, p1 - h.y);
+            }
+          }
+          const int cg = hf * (kKeysPerHalf / 8) + c8;  // 16-byte chunk of the row
+          const uint32_t addr = prow + ((cg ^ (r & 7)) << 4);
+          st_shared_v4(addr, hi[0], hi[1], hi[2], hi[3]);
+          if constexpr (TT::kSplitP) st_shared_v4(addr + kRowsTC * 128, lo[0], lo[1], lo[2], lo[3]);
+        }
       }
       l += psum;
       // keys past the context end in the last tile: zero their V rows (P is 0
@@ -604,6 +675,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
       fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+      if constexpr (kPTmem) tc_fence_before();  // the tcgen05.st of P -> the MMA thread
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kPFull + pb]);
     }
