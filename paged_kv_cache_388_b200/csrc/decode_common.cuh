@@ -234,8 +234,10 @@ struct SegIter {
   int w;             // fixed scheme: next item
   int64_t pos, end;  // balanced scheme: flat block range still to do
   bool first;
+  int s;             // balanced scheme: sequence holding pos (-1 before the first)
   __device__ void init(const AttnArgs &a, const BatchSmem &b, int n) {
     w = blockIdx.x;
+    s = -1;
     if (a.balanced) {
       const int64_t W = (int64_t)b.prefix[n] * a.num_kv_heads;
       pos = bal_start(blockIdx.x, W, gridDim.x);
@@ -253,17 +255,26 @@ struct SegIter {
       return true;
     }
     if (pos >= end) return false;
-    // sequence s holding flat position pos: prefix[s]*Hk <= pos < prefix[s+1]*Hk
+    // sequence holding flat position pos: prefix[lo]*Hk <= pos < prefix[lo+1]*Hk.
+    // A binary search for the first segment; after that pos only grows, so
+    // the sequence is the current one or a later one (usually the next).
     const int Hk = a.num_kv_heads;
-    int lo = 0, hi = n;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if ((int64_t)b.prefix[mid] * Hk <= pos) lo = mid; else hi = mid;
+    int lo = 0;
+    if (s < 0) {
+      int hi = n;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)b.prefix[mid] * Hk <= pos) lo = mid; else hi = mid;
+      }
+    } else {
+      lo = s;
+      while (lo + 1 < n && (int64_t)b.prefix[lo + 1] * Hk <= pos) ++lo;
     }
+    s = lo;
     const int nb = b.prefix[lo + 1] - b.prefix[lo];  // > 0: empty sequences own no range
-    const int64_t off = pos - (int64_t)b.prefix[lo] * Hk;
-    const int kvh = (int)(off / nb);
-    const int b0 = (int)(off - (int64_t)kvh * nb);
+    const int off = (int)(pos - (int64_t)b.prefix[lo] * Hk);  // < nb * Hk
+    const int kvh = off / nb;
+    const int b0 = off - kvh * nb;
     const int64_t left = end - pos;
     const int b1 = left < nb - b0 ? b0 + (int)left : nb;
     Item &it = seg->it;

@@ -283,8 +283,20 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
     uint32_t it = 0, k = 0;
     SegIter iter;
     iter.init(a, bsm, n);
-    Seg seg;
-    for (; iter.next(a, bsm, n, &seg); ++k) {
+    // Block ids are read 32 at a time, one group ahead: the ids of the
+    // following group (the rest of this item, else the next item's first) are
+    // loaded while the current group's tiles are issued, so that no dependent
+    // table read stalls the ring at an item boundary (a balanced CTA can hold
+    // a dozen short items).
+    Seg seg, nxt;
+    bool have = iter.next(a, bsm, n, &seg);
+    bool have_nxt = have && iter.next(a, bsm, n, &nxt);
+    auto load_ids = [&](const Seg &sg, int b) -> int {
+      const int32_t *tb = a.block_tables + (int64_t)sg.it.seq * a.max_blocks_per_seq + sg.it.boff;
+      return lane < min(32, sg.it.b1 - b) ? tb[b + lane] : 0;
+    };
+    int ids = have ? load_ids(seg, seg.it.b0) : 0;
+    for (; have; ++k) {
       const Item &item = seg.it;
       {  // the segment's GROUP query rows -> qbuf[k & 1]
         const uint32_t qs = k & 1u;
@@ -305,10 +317,10 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
         }
         __syncwarp();
       }
-      const int32_t *table = a.block_tables + (int64_t)item.seq * a.max_blocks_per_seq + item.boff;
       for (int b = item.b0; b < item.b1; b += 32) {
         const int cnt = min(32, item.b1 - b);
-        const int my_id = lane < cnt ? table[b + lane] : 0;
+        const int my_id = ids;
+        ids = b + 32 < item.b1 ? load_ids(seg, b + 32) : (have_nxt ? load_ids(nxt, nxt.it.b0) : 0);
         for (int j = 0; j < cnt; ++j) {
           const int pb = __shfl_sync(0xffffffffu, my_id, j);
           const uint32_t slot = it % L::kStages;
@@ -380,6 +392,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
           __syncwarp();
         }
       }
+      seg = nxt;
+      have = have_nxt;
+      if (have) have_nxt = iter.next(a, bsm, n, &nxt);
     }
     return;
   }
