@@ -730,13 +730,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
       // This CTA holds the first piece of a pair cut at its range end: leave
       // the merge kernel a descriptor {record slot, kv head, last covering
       // CTA, query row}.
-      const int nb = ceil_div(item.L, a.block_size);
+      const int nu = ceil_div(item.L, a.block_size) + kItemUnits;  // the pair's units
       const int64_t W = (int64_t)bsm.prefix[n] * a.num_kv_heads;
       const int64_t ps = (int64_t)bsm.prefix[item.seq - a.seq_begin] * a.num_kv_heads +
-                         (int64_t)item.kvh * nb;
+                         (int64_t)item.kvh * nu;
       int *d = a.bal_desc + 4 * blockIdx.x;
       d[1] = item.kvh;
-      d[2] = bal_owner(ps + nb - 1, W, gridDim.x);
+      d[2] = bal_owner(ps + nu - 1, W, gridDim.x);
       d[3] = item.qrow;
       d[0] = seg.index;  // record slot of this piece in this CTA
     }
