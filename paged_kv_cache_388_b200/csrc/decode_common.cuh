@@ -67,7 +67,14 @@ struct BatchSmem {
 // its KV blocks: the fixed cost of an item (q load, cross-warp merge, output
 // store, next-item set-up) measured on B200 at 1.3-2.4 us against ~0.9 us per
 // block, so a CTA that holds many short items is given fewer blocks.
-constexpr int kItemUnits = 2;
+// Measured (pa_decode, CUDA graphs): 1 / 2 / 3 / 4 units -> Llama-3-8B-shaped
+// batch 0.1700 / 0.1680 / 0.1677 / 0.1691 ms, Llama-2-7B-shaped MHA batch
+// 0.1719 / 0.1700 / 0.1681 / 0.1681 ms, parallel-sampling shared-prefix call
+// 0.1345 / 0.1266 / 0.1211 / 0.1170 ms.
+#ifndef PA_ITEM_UNITS
+#define PA_ITEM_UNITS 3
+#endif
+constexpr int kItemUnits = PA_ITEM_UNITS;
 
 // Partition units of a decode sequence (one query row, valid length) per KV
 // head: its KV blocks after the `pre` shared-prefix blocks plus kItemUnits,
