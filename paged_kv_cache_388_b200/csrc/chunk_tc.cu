@@ -8,20 +8,25 @@
 // (128x64x128) and O += P V (128x128x64) run as tcgen05.mma with fp32
 // accumulators in tensor memory.
 //
-// CTA = (sequence, KV head, 128 query rows); 4 * kHalves + 2 warps:
-//   softmax    warps w (and w + 4 when kHalves = 2) own rows 32w .. 32w+31
-//              (TMEM lane quadrant w), each taking 64 / kHalves of every
-//              tile's keys and 128 / kHalves of O's columns.  Reads S from
-//              TMEM, masks, exchanges the tile row max with its partner (two
-//              halves), keeps a running max that is only
-//              moved (and O rescaled in TMEM) when the tile max exceeds it by
-//              more than 2^8, writes P = 2^(s - m) as bf16 hi + lo (or fp16)
-//              into swizzled shared memory, and at the end writes O / l.
-//   producer   (warp 4 * kHalves) TMA loads of Q (once) and of each 64-key K/V
-//              tile, block by block through the block table (128-byte swizzle).
-//   MMA        (the last warp) MMA issue (one elected thread) and TMEM allocation.
-// TMEM: S double buffer (2 x 64 columns) and O (128 columns).
-// Shared memory: Q 32 KB, kStagesTC K/V stages of 32 KB, 2 P buffers of 32 KB.
+// CTA = (sequence, KV head, NQ tiles of 128 query rows); 4 * kHalves * NQ + 2
+// warps (NQ = 2 for chunk rows: the two Q tiles share every K/V tile, which
+// halves the TMA boxes per row -- a B200 SM's TMA unit spends ~100 cycles per
+// 2 KB box, and a 64-key bs-16 tile is 16 of them):
+//   softmax    warps of Q tile t (and w + 4 when kHalves = 2) own rows 32w ..
+//              32w+31 of the tile (TMEM lane quadrant w), each taking
+//              64 / kHalves of every K tile's keys and 128 / kHalves of O's
+//              columns.  Reads S from TMEM, masks, exchanges the tile row max
+//              with its partner (two halves), keeps a running max that is
+//              only moved (and O rescaled in TMEM) when the tile max exceeds
+//              it by more than 2^8, writes P = 2^(s - m) as bf16 hi + lo (or
+//              fp16) over its S columns in TMEM, and at the end writes O / l.
+//   producer   TMA loads of Q (once) and of each 64-key K/V tile, block by
+//              block through the block table (128-byte swizzle).
+//   MMA        (the last warp) MMA issue (one elected thread) and TMEM
+//              allocation.
+// TMEM per Q tile: S/P buffers of 64 columns (3 with one Q tile, 2 with two)
+// and O (128 columns).  Shared memory: Q 32 KB per tile, kStagesTC K/V stages
+// of 32 KB.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -58,10 +63,13 @@ constexpr int kStagesTC = PA_CHUNK_TC_STAGES;  // K/V tiles in flight
 #define PA_CHUNK_TC_HALVES 1
 #endif
 constexpr int kHalves = PA_CHUNK_TC_HALVES;
-constexpr int kSoftWarps = 4 * kHalves;
-constexpr int kProdWarp = kSoftWarps;       // TMA producer
-constexpr int kMmaWarp = kSoftWarps + 1;    // MMA issue + TMEM allocation
-constexpr int kThreadsTC = 32 * (kSoftWarps + 2);
+// Warps of a CTA (see chunk_tc_kernel): 4 * kHalves softmax warps per Q tile,
+// then one TMA producer warp and one MMA-issue / TMEM-allocation warp.
+// Q tiles of 128 rows per chunk-row CTA (1 or 2; see chunk_tc_kernel)
+#ifndef PA_CHUNK_TC_NQ
+#define PA_CHUNK_TC_NQ 2
+#endif
+constexpr int kChunkQTiles = PA_CHUNK_TC_NQ;
 constexpr int kKeysPerHalf = kKeysTC / kHalves;
 constexpr int kOColsPerHalf = kHeadDim / kHalves;
 static_assert(kHalves == 1 || kHalves == 2, "one or two softmax warps per row quadrant");
@@ -78,10 +86,16 @@ static_assert(kHalves == 1 || kHalves == 2, "one or two softmax warps per row qu
 #ifndef PA_CHUNK_TC_PBUFS
 #define PA_CHUNK_TC_PBUFS 2
 #endif
-constexpr int kSBufs = kPTmem ? 3 : 2;                   // S (and with kPTmem P) buffers in TMEM
+#ifndef PA_CHUNK_TC_SBUFS
+#define PA_CHUNK_TC_SBUFS (PA_CHUNK_TC_PTMEM ? 3 : 2)
+#endif
+constexpr int kSBufs = PA_CHUNK_TC_SBUFS;                // S (and with kPTmem P) buffers in TMEM
+#ifndef PA_CHUNK_TC_MIN_CTAS
+#define PA_CHUNK_TC_MIN_CTAS 1
+#endif
 constexpr int kPBufs = kPTmem ? kSBufs : PA_CHUNK_TC_PBUFS;
-constexpr uint32_t kTmemCols = kPTmem ? 512 : 256;     // allocation: a power of two
-constexpr uint32_t kTmemO = kPTmem ? 256 : 128;        // O's first column
+constexpr uint32_t kTmemO = kSBufs * 64 <= 128 ? 128 : 256;  // O's first column
+constexpr uint32_t kTmemCols = kTmemO + 128 <= 256 ? 256 : 512;  // allocation: a power of two
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between rescales
 
 template <typename T>
@@ -122,9 +136,10 @@ struct TcType<__half> {
 };
 
 // ---- shared-memory layout (offsets from a 1024-byte aligned base) ---------
-struct TcLayout {
-  static constexpr int kQ = 0;                                   // 2 halves x [128 rows x 128 B]
-  static constexpr int kKV = kQ + kRowsTC * kHeadDim * 2;        // stages: K (2x8 KB) + V (2x8 KB)
+template <int NQ>
+struct TcLayoutT {
+  static constexpr int kQ = 0;                                   // NQ tiles x 2 halves x [128 rows x 128 B]
+  static constexpr int kKV = kQ + NQ * kRowsTC * kHeadDim * 2;   // stages: K (2x8 KB) + V (2x8 KB)
   static constexpr int kStageBytes = 2 * kKeysTC * kHeadDim * 2;
   static constexpr int kP = kKV + kStagesTC * kStageBytes;       // 2 buffers x (hi, lo) x [128 x 128 B]
   static constexpr int kPBuf = 2 * kRowsTC * kKeysTC * 2;
@@ -137,16 +152,18 @@ struct TcLayout {
   static constexpr int kBytes = kBar + 512 + 1024;               // barriers etc. + alignment slack
 };
 
-// barrier indices within the barrier block
+// barrier indices within the barrier block; per-(Q tile, buffer) arrays hold
+// up to two Q tiles of kSBufs buffers
+constexpr int kSlots = 2 * (kSBufs > kPBufs ? kSBufs : kPBufs);
 enum {
   kQFull = 0,
   kKvFull = 1,                       // [kStagesTC]
   kKvEmpty = kKvFull + kStagesTC,    // [kStagesTC]
-  kSFull = kKvEmpty + kStagesTC,     // [kSBufs]
-  kSFree = kSFull + kSBufs,          // [kSBufs] (P in shared memory only)
-  kPFull = kSFree + kSBufs,          // [kPBufs]
-  kPvDone = kPFull + kPBufs,         // [kPBufs]
-  kDone = kPvDone + kPBufs,
+  kSFull = kKvEmpty + kStagesTC,     // [Q tile][buffer] (kSlots)
+  kSFree = kSFull + kSlots,          // (P in shared memory only)
+  kPFull = kSFree + kSlots,          // [Q tile][buffer]
+  kPvDone = kPFull + kSlots,         // [Q tile][buffer]
+  kDone = kPvDone + kSlots,
   kXFull = kDone + 1,                // [4 quadrants][2 buffers] row maxima written
   kLFull = kXFull + 8,               // [4 quadrants] row sums written
   kNumBars = kLFull + 4
@@ -269,18 +286,34 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // ids while the first tile loads; the
 // output is one record (o unnormalised, reference max in base 2, sum) per
 // (member, head) for the decode kernel to fold in.
-template <typename T, int BS, bool PREFIX = false>
-__global__ void __launch_bounds__(kThreadsTC, 1)
+//
+// NQ = 2 (chunk rows): the CTA holds two 128-row Q tiles of the same
+// (sequence, KV head) against one stream of K/V tiles, so every K/V box the
+// TMA unit moves serves 256 rows; each Q tile has its own 4 softmax warps,
+// its own 2 S/P buffers and O in TMEM (2 x 128 + 2 x 128 = 512 columns).
+template <typename T, int BS, bool PREFIX = false, int NQ = 1>
+__global__ void __launch_bounds__(32 * (4 * kHalves * NQ + 2), PA_CHUNK_TC_MIN_CTAS)
     chunk_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                     int tiles_per_seq) {
   using TT = TcType<T>;
+  using LY = TcLayoutT<NQ>;
+  static_assert(NQ == 1 || (NQ == 2 && kHalves == 1 && kPTmem && !PREFIX),
+                "two Q tiles: chunk rows, P in TMEM, one softmax warp per lane quadrant");
+  constexpr int SWT = 4 * kHalves;                      // softmax warps per Q tile
+  constexpr int SW = SWT * NQ;                          // softmax warps
+  constexpr int PW = SW, MW = SW + 1;                   // producer, MMA warps
+  constexpr int SB = NQ == 1 ? kSBufs : 2;              // S (/P) buffers per Q tile
+  constexpr int PB = kPTmem ? SB : kPBufs;              // P buffers per Q tile
+  constexpr uint32_t OB = NQ == 1 ? kTmemO : 256;       // first O column (tile t: OB + 128 t)
+  constexpr uint32_t TCOLS = NQ == 1 ? kTmemCols : 512;
+  static_assert(NQ * SB <= kSlots && NQ * PB <= kSlots, "barrier slots");
   constexpr int D = kHeadDim;
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TcLayout::kBar);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TcLayout::kBar + 8 * kNumBars);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LY::kBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + LY::kBar + 8 * kNumBars);
   volatile int *flags = reinterpret_cast<volatile int *>(tmem_slot + 1);  // [0] abort, [1] bad block
   const uint32_t sbase = smem_addr(smem);
 
@@ -321,9 +354,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
       return;
     }
-    t0 = tile * TPT;
+    t0 = tile * NQ * TPT;
     if (t0 >= Q) return;
-    ntok = min(TPT, Q - t0);
+    ntok = min(NQ * TPT, Q - t0);  // rows of all Q tiles
     L = a.context_lens[seq];
     if (L < Q || L > a.max_context_len) {
       if (tid == 0 && tile == 0 && kvh == 0)
@@ -339,7 +372,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   }
   const int ntiles = (kend + kKeysTC - 1) / kKeysTC;
   const int nblk = (L + BS - 1) / BS;              // blocks that hold the keys
-  volatile unsigned char *bad_member = smem + TcLayout::kMemBad;
+  volatile unsigned char *bad_member = smem + LY::kMemBad;
 
   // ---- set-up: barriers, TMEM ------------------------------------------------
   if (tid == 0) {
@@ -348,12 +381,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&bars[kKvFull + s], 1);
       mbar_init(&bars[kKvEmpty + s], 1);
     }
-    for (int b = 0; b < kSBufs; ++b) {
+    for (int b = 0; b < NQ * SB; ++b) {
       mbar_init(&bars[kSFull + b], 1);
-      mbar_init(&bars[kSFree + b], kSoftWarps);
+      mbar_init(&bars[kSFree + b], SWT);
     }
-    for (int b = 0; b < kPBufs; ++b) {
-      mbar_init(&bars[kPFull + b], kSoftWarps);
+    for (int b = 0; b < NQ * PB; ++b) {
+      mbar_init(&bars[kPFull + b], SWT);
       mbar_init(&bars[kPvDone + b], 1);
     }
     mbar_init(&bars[kDone], 1);
@@ -364,10 +397,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     flags[1] = 0;
     mbar_init_fence();
   }
-  if (warp == kMmaWarp) {
+  if (warp == MW) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
-                 "r"(kTmemCols)
+                 "r"(TCOLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -375,25 +408,26 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s0 = tmem, tmem_o = tmem + kTmemO;
+  // TMEM: Q tile t's S/P buffers at columns t*SB*64 .., its O at OB + 128 t
 
   auto fail = [&](void) {
     if (!flags[0]) raise_error(a.err, PA_DEVERR_TIMEOUT);
     flags[0] = 1;
   };
 
-  if (warp == kProdWarp) {
+  if (warp == PW) {
     // ======================= producer =======================================
     // The whole warp reads the block table 32 ids at a time (one coalesced
     // load, the next group fetched while the current one is issued); lane 0
     // issues the TMA loads.
     const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
     if (lane == 0) {
-      // Q: 128 rows (token, head) of this CTA, two 64-column boxes
-      mbar_arrive_expect_tx(&bars[kQFull], kRowsTC * D * 2);
-      for (int h = 0; h < 2; ++h)
-        tma_load_4d(sbase + TcLayout::kQ + h * kRowsTC * 128, &tmq, h * 64, 0, kvh, q0 + t0,
-                    &bars[kQFull]);
+      // Q: 128 rows (token, head) per Q tile, two 64-column boxes each
+      mbar_arrive_expect_tx(&bars[kQFull], NQ * kRowsTC * D * 2);
+      for (int t = 0; t < NQ; ++t)
+        for (int h = 0; h < 2; ++h)
+          tma_load_4d(sbase + LY::kQ + t * kRowsTC * D * 2 + h * kRowsTC * 128, &tmq, h * 64, 0, kvh,
+                      q0 + t0 + t * TPT, &bars[kQFull]);
     }
     constexpr int kBpt = kKeysTC / BS;  // blocks per tile
     int grp = 0;                        // first block of the group held in `ids`
@@ -421,8 +455,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(&bars[kKvFull + st], nb * 2 * BS * D * 2);
-        const uint32_t kdst = sbase + TcLayout::kKV + st * TcLayout::kStageBytes;
-        const uint32_t vdst = kdst + TcLayout::kStageBytes / 2;
+        const uint32_t kdst = sbase + LY::kKV + st * LY::kStageBytes;
+        const uint32_t vdst = kdst + LY::kStageBytes / 2;
         for (int b = 0; b < nb; ++b) {
           int pb = pbs[b];
           if (pb < 0 || pb >= a.num_blocks) {
@@ -439,7 +473,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       __syncwarp();
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == MW) {
     // ======================= MMA issue ======================================
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc(TT::kFmt, 0, 0, kRowsTC, kKeysTC);
@@ -447,49 +481,66 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bool ok = mbar_wait(&bars[kQFull], 0);
       if (!ok) fail();
       auto issue_pv = [&](int jj) {
-        const int pbuf = jj % kPBufs;
-        if (!mbar_wait(&bars[kPFull + pbuf], (jj / kPBufs) & 1)) { fail(); return false; }
-        tc_fence_after();
-        const uint32_t vst = sbase + TcLayout::kKV + (jj % kStagesTC) * TcLayout::kStageBytes +
-                             TcLayout::kStageBytes / 2;
-        const int nparts = TT::kSplitP ? 2 : 1;
-        for (int part = 0; part < nparts; ++part) {
-          for (int ks = 0; ks < kKeysTC / 16; ++ks) {
-            const uint64_t db = umma_desc(vst + ks * 16 * 128, kKeysTC * 128, 1024);
-            const uint32_t acc = (jj > 0 || part > 0 || ks > 0) ? 1u : 0u;
-            if constexpr (kPTmem) {
-              // P of tile jj: hi in the first half of its S columns, lo in the second
-              const uint32_t pa = tmem_s0 + (jj % kSBufs) * kKeysTC + part * (kKeysTC / 2) + ks * 8;
-              umma_ts(tmem_o, pa, db, idesc_pv, acc);
-            } else {
-              const uint32_t pbase = sbase + TcLayout::kP + pbuf * TcLayout::kPBuf;
-              const uint64_t da = umma_desc(pbase + part * (kRowsTC * 128) + ks * 32, 16, 1024);
-              umma(tmem_o, da, db, idesc_pv, acc);
+        const int pbuf = jj % PB;
+        const uint32_t vst = sbase + LY::kKV + (jj % kStagesTC) * LY::kStageBytes +
+                             LY::kStageBytes / 2;
+        for (int t = 0; t < NQ; ++t) {
+          if (!mbar_wait(&bars[kPFull + t * PB + pbuf], (jj / PB) & 1)) { fail(); return false; }
+          tc_fence_after();
+          const uint32_t tmem_o = tmem + OB + t * 128;
+          const int nparts = TT::kSplitP ? 2 : 1;
+          for (int part = 0; part < nparts; ++part) {
+            for (int ks = 0; ks < kKeysTC / 16; ++ks) {
+              const uint64_t db = umma_desc(vst + ks * 16 * 128, kKeysTC * 128, 1024);
+              const uint32_t acc = (jj > 0 || part > 0 || ks > 0) ? 1u : 0u;
+              if constexpr (kPTmem) {
+                // P of tile jj: hi in the first half of its S columns, lo in the second
+                const uint32_t pa =
+                    tmem + (t * SB + jj % SB) * kKeysTC + part * (kKeysTC / 2) + ks * 8;
+                umma_ts(tmem_o, pa, db, idesc_pv, acc);
+              } else {
+                const uint32_t pbase = sbase + LY::kP + pbuf * LY::kPBuf;
+                const uint64_t da = umma_desc(pbase + part * (kRowsTC * 128) + ks * 32, 16, 1024);
+                umma(tmem_o, da, db, idesc_pv, acc);
+              }
             }
           }
+          umma_commit(&bars[kPvDone + t * PB + pbuf]);
         }
-        umma_commit(&bars[kPvDone + pbuf]);
-        umma_commit(&bars[kKvEmpty + (jj % kStagesTC)]);
+        umma_commit(&bars[kKvEmpty + (jj % kStagesTC)]);  // after every Q tile's P V
         return true;
       };
       for (int j = 0; ok && j < ntiles && !flags[0]; ++j) {
-        const int st = j % kStagesTC, sb = j % kSBufs;
+        const int st = j % kStagesTC, sb = j % SB;
         if (!mbar_wait(&bars[kKvFull + st], (j / kStagesTC) & 1)) { fail(); break; }
-        if constexpr (kPTmem) {
-          // S(j) overwrites P(j - kSBufs): its P V must be done
-          if (j >= kSBufs && !mbar_wait(&bars[kPvDone + sb], ((j / kSBufs) - 1) & 1)) { fail(); break; }
-        } else {
-          if (!mbar_wait(&bars[kSFree + sb], ((j / kSBufs) & 1) ^ 1)) { fail(); break; }
+        const uint32_t kst = sbase + LY::kKV + st * LY::kStageBytes;
+        bool go = true;
+        for (int t = 0; t < NQ && go; ++t) {
+          if constexpr (kPTmem) {
+            // S(j) overwrites P(j - SB) of this Q tile: its P V must be done
+            if (j >= SB && !mbar_wait(&bars[kPvDone + t * PB + sb], ((j / SB) - 1) & 1)) {
+              fail();
+              go = false;
+              break;
+            }
+          } else {
+            if (!mbar_wait(&bars[kSFree + sb], ((j / SB) & 1) ^ 1)) {
+              fail();
+              go = false;
+              break;
+            }
+          }
+          tc_fence_after();
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const int h = ks >> 2, kk = ks & 3;
+            const uint64_t da =
+                umma_desc(sbase + LY::kQ + t * kRowsTC * D * 2 + h * kRowsTC * 128 + kk * 32, 16, 1024);
+            const uint64_t db = umma_desc(kst + h * kKeysTC * 128 + kk * 32, 16, 1024);
+            umma(tmem + (t * SB + sb) * kKeysTC, da, db, idesc_qk, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars[kSFull + t * SB + sb]);
         }
-        tc_fence_after();
-        const uint32_t kst = sbase + TcLayout::kKV + st * TcLayout::kStageBytes;
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int h = ks >> 2, kk = ks & 3;
-          const uint64_t da = umma_desc(sbase + TcLayout::kQ + h * kRowsTC * 128 + kk * 32, 16, 1024);
-          const uint64_t db = umma_desc(kst + h * kKeysTC * 128 + kk * 32, 16, 1024);
-          umma(tmem_s0 + sb * kKeysTC, da, db, idesc_qk, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars[kSFull + sb]);
+        if (!go) break;
         if (j > 0 && !issue_pv(j - 1)) break;
       }
       if (ok && !flags[0] && ntiles > 0) issue_pv(ntiles - 1);
@@ -498,16 +549,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
   } else {
     // ======================= softmax warps =================================
-    // Warp w: rows 32 (w mod 4) .. +31 (its TMEM lane quadrant), keys
-    // hf * kKeysPerHalf .. of every tile and O columns hf * kOColsPerHalf ..
-    const int qd = warp & 3, hf = warp >> 2;
-    const int r = qd * 32 + lane;              // query row = TMEM lane
-    const int sid = hf * kRowsTC + r;          // 0 .. kSoftWarps * 32 - 1
+    // Warp w: Q tile qt = w / SWT; within it rows 32 (w mod 4) .. +31 (its
+    // TMEM lane quadrant), keys hf * kKeysPerHalf .. of every tile and O
+    // columns hf * kOColsPerHalf ..
+    const int qt = warp / SWT, wl = warp - qt * SWT;
+    const int qd = wl & 3, hf = wl >> 2;
+    const int r = qd * 32 + lane;              // query row of the Q tile = TMEM lane
+    const int sid = hf * kRowsTC + r;          // 0 .. SWT * 32 - 1
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    float *xmax = reinterpret_cast<float *>(smem + TcLayout::kX);  // [2][kHalves][128]
+    const uint32_t tmem_s0 = tmem + qt * SB * kKeysTC;  // this Q tile's S/P buffers
+    const uint32_t tmem_o = tmem + OB + qt * 128;       // and its O
+    float *xmax = reinterpret_cast<float *>(smem + LY::kX);  // [2][kHalves][128]
     float *xl = xmax + 2 * kHalves * kRowsTC;                      // [kHalves][128]
     (void)xl;
-    const int tok = r / G;
+    const int tok = qt * TPT + r / G;          // token (member) among the CTA's rows
     const int limit = PREFIX ? L - 1 : L - Q + t0 + tok;  // last key this row may see
     const float sl2 = a.scale_log2;
     if constexpr (PREFIX) {
@@ -516,18 +571,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // tile is still in flight, instead of one dependent round trip per tile
       // on the producer's path.
       const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
-      for (int x0 = sid; x0 < ntok * nblk; x0 += kSoftWarps * 32 * 8) {
+      for (int x0 = sid; x0 < ntok * nblk; x0 += SWT * 32 * 8) {
         int mine[8], ref[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int x = x0 + u * kSoftWarps * 32;
+          const int x = x0 + u * SWT * 32;
           const int i = x / nblk, b = x - i * nblk;
           mine[u] = x < ntok * nblk ? a.block_tables[(int64_t)(q0 + i) * a.max_blocks_per_seq + b] : 0;
           ref[u] = x < ntok * nblk ? table[b] : 0;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int x = x0 + u * kSoftWarps * 32;
+          const int x = x0 + u * SWT * 32;
           if (x < ntok * nblk && mine[u] != ref[u]) {
             const int i = x / nblk;
             if (!bad_member[i]) raise_error(a.err, PA_DEVERR_PREFIX);
@@ -538,8 +593,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < ntiles; ++j) {
-      const int sb = j % kSBufs;
-      bool ok = !flags[0] && mbar_wait(&bars[kSFull + sb], (j / kSBufs) & 1);
+      const int sb = j % SB;
+      bool ok = !flags[0] && mbar_wait(&bars[kSFull + qt * SB + sb], (j / SB) & 1);
       if (!__all_sync(0xffffffffu, ok)) { fail(); break; }  // warp-uniform: tcgen05.ld is collective
       tc_fence_after();
       uint32_t sr[kKeysPerHalf];
@@ -588,7 +643,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O (in TMEM) is complete up to tile j-1 once that tile's P.V is done
-        const bool done = mbar_wait(&bars[kPvDone + ((j - 1) % kPBufs)], ((j - 1) / kPBufs) & 1);
+        const bool done = mbar_wait(&bars[kPvDone + qt * PB + ((j - 1) % PB)], ((j - 1) / PB) & 1);
         if (!__all_sync(0xffffffffu, done)) { fail(); break; }
         tc_fence_after();
 #pragma unroll 1
@@ -604,7 +659,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tmem_wait_st();
         tc_fence_before();
       }
-      const int pb = j % kPBufs;
+      const int pb = j % PB;
       float psum = 0.f;
       if constexpr (kPTmem) {
         // P = 2^(x - m_used) over this tile's S columns: hi words at
@@ -630,10 +685,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         tmem_wait_st();
       } else {
-        // the P buffer of tile j was last read by tile j - kPBufs's P.V
-        if (j >= kPBufs && !mbar_wait(&bars[kPvDone + pb], ((j - kPBufs) / kPBufs) & 1)) { fail(); break; }
+        // the P buffer of tile j was last read by tile j - PB's P.V
+        if (j >= PB && !mbar_wait(&bars[kPvDone + qt * PB + pb], ((j - PB) / PB) & 1)) { fail(); break; }
         // P = 2^(x - m_used) -> shared memory (K-major, 128-byte swizzle), hi and lo
-        const uint32_t prow = sbase + TcLayout::kP + pb * TcLayout::kPBuf + r * 128;
+        const uint32_t prow = sbase + LY::kP + pb * LY::kPBuf + r * 128;
 #pragma unroll
         for (int c8 = 0; c8 < kKeysPerHalf / 8; ++c8) {
           uint32_t hi[4], lo[4];
@@ -659,13 +714,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // keys past the context end in the last tile: zero their V rows (P is 0
       // there, but the slots may hold anything and 0 * NaN is NaN)
       if (j == ntiles - 1 && (j + 1) * kKeysTC > L) {
-        const uint32_t vst = sbase + TcLayout::kKV + (j % kStagesTC) * TcLayout::kStageBytes +
-                             TcLayout::kStageBytes / 2;
+        const uint32_t vst = sbase + LY::kKV + (j % kStagesTC) * LY::kStageBytes +
+                             LY::kStageBytes / 2;
         const int z0 = L - j * kKeysTC;  // first stale row of the tile
         const int nz = (kKeysTC - z0) * 16;  // 16-byte chunks over both halves
         // all of the tile's K/V bytes must have landed before they are overwritten
         if (mbar_wait(&bars[kKvFull + (j % kStagesTC)], (j / kStagesTC) & 1)) {
-          for (int c = sid; c < nz; c += kSoftWarps * 32) {
+          for (int c = sid; c < nz; c += SWT * 32) {  // each Q tile's warps zero all of them
             const int row = z0 + c / 16, ch = c % 16;
             const int h = ch >> 3, cc = ch & 7;
             st_shared_v4(vst + h * kKeysTC * 128 + row * 128 + ((cc ^ (row & 7)) << 4), 0, 0, 0, 0);
@@ -677,11 +732,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
       if constexpr (kPTmem) tc_fence_before();  // the tcgen05.st of P -> the MMA thread
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kPFull + pb]);
+      if (lane == 0) mbar_arrive(&bars[kPFull + qt * PB + pb]);
     }
     // ---- epilogue: O / l -> out ----
     bool ok = !flags[0] && ntiles > 0 &&
-              mbar_wait(&bars[kPvDone + ((ntiles - 1) % kPBufs)], ((ntiles - 1) / kPBufs) & 1);
+              mbar_wait(&bars[kPvDone + qt * PB + ((ntiles - 1) % PB)], ((ntiles - 1) / PB) & 1);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok && ntiles > 0) fail();
     if constexpr (kHalves > 1) {  // the row's sum over both warps' keys
@@ -701,7 +756,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const bool write = tok < ntok && r < TPT * G;
     if constexpr (PREFIX) {
       // the member flags of every softmax warp (named barrier 1)
-      asm volatile("bar.sync 1, %0;" ::"n"(kSoftWarps * 32) : "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(SW * 32) : "memory");
       // record of (member q0 + tok, head): o unnormalised, the reference max
       // (base 2) o and l are relative to, l; NaN l marks a poisoned record
       const bool poison = !ok || flags[1] || (write && bad_member[tok]);
@@ -749,9 +804,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == MW) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS)
                  : "memory");
   }
 }
@@ -768,7 +823,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_tc() {
   return fn;
 }
 
-template <typename T, int BS, bool PREFIX = false>
+template <typename T, int BS, bool PREFIX = false, int NQ = 1>
 cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
   auto fn = encode_fn_tc();
   if (!fn) return cudaErrorNotSupported;
@@ -797,21 +852,23 @@ cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = chunk_tc_kernel<T, BS, PREFIX>;
+  auto kern = chunk_tc_kernel<T, BS, PREFIX, NQ>;
+  constexpr int kBytes = TcLayoutT<NQ>::kBytes;
+  constexpr int kThreads = 32 * (4 * kHalves * NQ + 2);
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcLayout::kBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   // chunk rows: (sequence, KV head, tile of TPT tokens); prefix: (group, KV
   // head, chunk of TPT members)
-  const int tiles = PREFIX ? (a.max_group + TPT - 1) / TPT : (a.max_query_len + TPT - 1) / TPT;
+  const int tiles = PREFIX ? (a.max_group + TPT - 1) / TPT : (a.max_query_len + NQ * TPT - 1) / (NQ * TPT);
   const int64_t grid = (int64_t)(PREFIX ? a.num_groups : a.num_seqs) * a.num_kv_heads * tiles;
   if (grid == 0) return cudaSuccess;
-  kern<<<(unsigned)grid, kThreadsTC, TcLayout::kBytes, stream>>>(a, tmq, tmk, tmv, tiles);
+  kern<<<(unsigned)grid, kThreads, kBytes, stream>>>(a, tmq, tmk, tmv, tiles);
   return cudaGetLastError();
 }
 
@@ -832,9 +889,10 @@ cudaError_t launch_prefix_tc(const AttnArgs &a, int dtype, cudaStream_t stream) 
 
 cudaError_t launch_chunk_tc(const AttnArgs &a, int dtype, cudaStream_t stream) {
   if (dtype == PA_BF16)
-    return a.block_size == 16 ? launch_tc_t<__nv_bfloat16, 16>(a, stream)
-                              : launch_tc_t<__nv_bfloat16, 32>(a, stream);
-  return a.block_size == 16 ? launch_tc_t<__half, 16>(a, stream) : launch_tc_t<__half, 32>(a, stream);
+    return a.block_size == 16 ? launch_tc_t<__nv_bfloat16, 16, false, kChunkQTiles>(a, stream)
+                              : launch_tc_t<__nv_bfloat16, 32, false, kChunkQTiles>(a, stream);
+  return a.block_size == 16 ? launch_tc_t<__half, 16, false, kChunkQTiles>(a, stream)
+                            : launch_tc_t<__half, 32, false, kChunkQTiles>(a, stream);
 }
 
 }  // namespace pa
