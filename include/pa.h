@@ -33,6 +33,35 @@
  *    a bit is OR-ed into a per-device error word (PA_DEVERR_*), which
  *    pa_get_device_error() reads and clears.  Kernels never trap and every
  *    wait inside them is bounded in time.
+ *
+ * Departures from the boundary as first planned
+ * ----------------------------------------------
+ * The planned prototypes were pa_reshape_and_cache, pa_decode,
+ * pa_copy_blocks, a four-argument pa_decode_workspace_size(num_q_tokens,
+ * num_heads, head_dim, max_context_len), pa_get_device_error(int *, stream)
+ * and pa_status_string, with the element type as a pa_dtype.  What ships
+ * differs as follows, each for the reason given:
+ *  - dtype is an `int` holding a pa_dtype value in every entry point: the
+ *    size of a C enum is up to the compiler, an int is not, and the byte
+ *    movers take one more value (PA_FP8_E4M3) than the attention calls.
+ *  - pa_decode adds num_q_tokens (rows of q/out; with query_start_loc ==
+ *    NULL it must equal num_seqs), max_query_len (host bound of any
+ *    sequence's query rows: sequences with more than one row go to the
+ *    chunked-prefill kernel, whose grid it sizes) and kv_split_tokens (0 =
+ *    the library's balanced partition; > 0 forces fixed splits of that many
+ *    tokens, used to test the split path on small inputs).
+ *  - pa_decode_workspace_size takes (num_seqs, num_heads, num_kv_heads,
+ *    head_dim, block_size, max_context_len, kv_split_tokens): the split
+ *    policy depends on num_seqs * num_kv_heads and on block_size, the
+ *    balanced partition's per-CTA records on group = num_heads /
+ *    num_kv_heads and on the device's SM count, and a forced split on
+ *    kv_split_tokens; num_q_tokens does not enter.
+ *  - pa_get_device_error writes an `unsigned int`: the word is a set of
+ *    PA_DEVERR_* bits that kernels OR in atomically.
+ *  - Added entry points for the rows after the core path:
+ *    pa_decode_shared_prefix (+ its workspace size), pa_reshape_and_cache_fp8,
+ *    pa_decode_fp8, pa_swap_blocks, pa_decode_noalloc (+
+ *    pa_noalloc_scratch_bytes) and pa_abi_version.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -260,9 +289,16 @@ int pa_decode(void *out, const void *q, const void *k_cache,
  *
  * Arguments and results are those of pa_decode (without workspace).
  * PA_ERR_WORKSPACE (nothing launched) if the batch needs more scratch than
- * the array holds; pa_decode_workspace_size() tells how much a batch may
- * need (16-bit caches with kv_split_tokens = 0 need about
- * 8 * SMs * 2 * group * (head_dim + 4) * 4 bytes, well inside the array).
+ * the array holds.  The call checks what its own launch needs, which can be
+ * less than pa_decode_workspace_size() reports: that function is an upper
+ * bound sized for 8 resident CTAs per SM.  16-bit caches with
+ * kv_split_tokens = 0 need at most 8 * SMs * 2 * group * (head_dim + 4) * 4
+ * bytes plus a few KiB, so on a 148-SM B200 every group <= 8 at head_dim
+ * 128 and every group <= 16 at head_dim 64 fits whatever the occupancy;
+ * group 16 at head_dim 128 fits at the occupancy the decode kernel reaches
+ * (5 CTAs per SM, about 12.5 MiB) but not at the bound.  Fixed splits
+ * (kv_split_tokens > 0) need num_seqs * num_heads * splits * (head_dim + 2)
+ * * 4 bytes.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
  * All calls share the one array and it keeps the last call's contents:

@@ -91,13 +91,60 @@ def _stream(stream):
 
 
 def _dev(t, name, dtype=None):
+    """A contiguous CUDA tensor on the current device (the library launches on
+    the current device and would otherwise dereference another GPU's memory)."""
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current device is cuda:{cur}; "
+                         "call under torch.cuda.device(...) of the tensors' device")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     return t
+
+
+def _shape(cond, what):
+    if not cond:
+        raise ValueError(what)
+
+
+def _cache_shapes(k_cache, v_cache):
+    """(num_blocks, num_kv_heads, block_size, head_dim) of a pair of caches."""
+    _shape(k_cache.dim() == 4, "k_cache must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    _shape(tuple(v_cache.shape) == tuple(k_cache.shape), "k_cache and v_cache shapes disagree")
+    return tuple(k_cache.shape)
+
+
+def _new_token_shapes(key, value, k_cache, v_cache, slot_mapping):
+    nb, hk, bs, d = _cache_shapes(k_cache, v_cache)
+    _shape(key.dim() == 3 and tuple(key.shape[1:]) == (hk, d),
+           f"key must be [num_tokens, {hk}, {d}] to match the caches, got {tuple(key.shape)}")
+    _shape(tuple(value.shape) == tuple(key.shape), "key and value shapes disagree")
+    _shape(slot_mapping.dim() == 1 and slot_mapping.shape[0] == key.shape[0],
+           "slot_mapping must hold one slot per key/value token")
+    return nb, hk, bs, d
+
+
+def _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc=None):
+    """Shapes of a decode call; every tensor must agree with the others."""
+    nb, hk, bs, d = _cache_shapes(k_cache, v_cache)
+    _shape(q.dim() == 3 and q.shape[2] == d, f"q must be [tokens, heads, {d}] to match the caches")
+    _shape(tuple(out.shape) == tuple(q.shape), "out and q shapes disagree")
+    tq, h, _ = q.shape
+    _shape(h % hk == 0, "num_heads must be a multiple of num_kv_heads")
+    _shape(block_tables.dim() == 2, "block_tables must be [num_seqs, max_blocks_per_seq]")
+    s, mbps = block_tables.shape
+    _shape(context_lens.dim() == 1 and context_lens.shape[0] == s,
+           "block_tables and context_lens disagree on the number of sequences")
+    if query_start_loc is None:
+        _shape(tq == s, "without query_start_loc q must hold one row per sequence")
+    else:
+        _shape(query_start_loc.dim() == 1 and query_start_loc.shape[0] == s + 1,
+               "query_start_loc must have num_seqs + 1 entries")
+    return tq, h, d, nb, hk, bs, s, mbps
 
 
 def _check(rc, what):
@@ -107,12 +154,12 @@ def _check(rc, what):
 
 def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
     """key/value [T, Hk, D]; caches [NB, Hk, bs, D]; slot_mapping int64 [T]."""
+    nb, hk, bs, d = _new_token_shapes(key, value, k_cache, v_cache, slot_mapping)
     _dev(key, "key")
     _dev(value, "value", key.dtype)
     _dev(k_cache, "k_cache", key.dtype)
     _dev(v_cache, "v_cache", key.dtype)
     _dev(slot_mapping, "slot_mapping", torch.int64)
-    nb, hk, bs, d = k_cache.shape
     rc = _lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
                                    _ptr(slot_mapping), key.shape[0], hk, d, bs, nb,
                                    _DT[key.dtype], _stream(stream))
@@ -121,10 +168,12 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
     """block_mapping int64 [P, 2] of (src, dst) physical block ids."""
+    nb, hk, bs, d = _cache_shapes(k_cache, v_cache)
+    _shape(block_mapping.dim() == 2 and block_mapping.shape[1] == 2,
+           "block_mapping must be [num_pairs, 2]")
     _dev(k_cache, "k_cache")
     _dev(v_cache, "v_cache", k_cache.dtype)
     _dev(block_mapping, "block_mapping", torch.int64)
-    nb, hk, bs, d = k_cache.shape
     rc = _lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping),
                              block_mapping.shape[0], hk, d, bs, nb, _DT[k_cache.dtype],
                              _stream(stream))
@@ -135,12 +184,12 @@ def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale
                              stream=None):
     """key/value [T, Hk, D] (fp32/fp16/bf16); caches uint8 [NB, Hk, bs, D] of
     E4M3 codes; slot_mapping int64 [T]."""
+    nb, hk, bs, d = _new_token_shapes(key, value, k_cache, v_cache, slot_mapping)
     _dev(key, "key")
     _dev(value, "value", key.dtype)
     _dev(k_cache, "k_cache", torch.uint8)
     _dev(v_cache, "v_cache", torch.uint8)
     _dev(slot_mapping, "slot_mapping", torch.int64)
-    nb, hk, bs, d = k_cache.shape
     rc = _lib.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
                                        _ptr(slot_mapping), key.shape[0], hk, d, bs, nb,
                                        _DT[key.dtype], float(k_scale), float(v_scale),
@@ -152,6 +201,8 @@ def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k
                   max_context_len=0, workspace=None, stream=None):
     """out/q [S, H, D] fp16/bf16; caches uint8 E4M3 codes [NB, Hk, bs, D];
     workspace: uint8 CUDA tensor of >= pa_decode_workspace_size(...) bytes."""
+    s, h, d, nb, hk, bs, _, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                  context_lens)
     _dev(q, "q")
     _dev(out, "out", q.dtype)
     _dev(k_cache, "k_cache", torch.uint8)
@@ -160,11 +211,6 @@ def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k
     _dev(context_lens, "context_lens", torch.int32)
     if workspace is not None:
         _dev(workspace, "workspace")
-    s, h, d = q.shape
-    nb, hk, bs, d2 = k_cache.shape
-    if d2 != d or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("shape mismatch between q, out and the caches")
-    s2, mbps = block_tables.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = _lib.pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                             mbps, _ptr(context_lens), s, h, hk, d, bs, nb, float(scale),
@@ -179,7 +225,9 @@ def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None):
     be CUDA tensors or pinned CPU tensors (not pageable ones)."""
     for name, t in (("dst_k", dst_k), ("dst_v", dst_v), ("src_k", src_k), ("src_v", src_v),
                     ("block_mapping", block_mapping)):
-        if not (t.is_cuda or t.is_pinned()):
+        if t.is_cuda:
+            _dev(t, name)
+        elif not t.is_pinned():
             raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
@@ -210,6 +258,8 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
     context_lens int32 [S]; query_start_loc int32 [S+1] or None; workspace: a
     uint8 CUDA tensor of >= pa_decode_workspace_size(...) bytes (or None when
     that size is 0)."""
+    tq, h, d, nb, hk, bs, s, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                   context_lens, query_start_loc)
     _dev(q, "q")
     _dev(out, "out", q.dtype)
     _dev(k_cache, "k_cache", q.dtype)
@@ -220,11 +270,6 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
         _dev(query_start_loc, "query_start_loc", torch.int32)
     if workspace is not None:
         _dev(workspace, "workspace")
-    tq, h, d = q.shape
-    nb, hk, bs, d2 = k_cache.shape
-    if d2 != d or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("shape mismatch between q, out and the caches")
-    s, mbps = block_tables.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = _lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                         mbps, _ptr(context_lens), _ptr(query_start_loc), s, tq,
@@ -241,6 +286,8 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scal
     callers that cannot allocate device memory.  Calls must not overlap on
     the GPU (they share the scratch); make the first call on a device before
     any stream capture."""
+    tq, h, d, nb, hk, bs, s, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                   context_lens, query_start_loc)
     _dev(q, "q")
     _dev(out, "out", q.dtype)
     _dev(k_cache, "k_cache", q.dtype)
@@ -249,11 +296,6 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scal
     _dev(context_lens, "context_lens", torch.int32)
     if query_start_loc is not None:
         _dev(query_start_loc, "query_start_loc", torch.int32)
-    tq, h, d = q.shape
-    nb, hk, bs, d2 = k_cache.shape
-    if d2 != d or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("shape mismatch between q, out and the caches")
-    s, mbps = block_tables.shape
     rc = _lib.pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                 _ptr(block_tables), mbps, _ptr(context_lens), _ptr(query_start_loc),
                                 s, tq, int(max_query_len), h, hk, d, bs, nb, float(scale),
@@ -274,6 +316,11 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
     """Decode with shared-prefix groups.  out/q [S, H, D]; group_start int32
     [G+1] and group_shared_blocks int32 [G] on the device; workspace: uint8
     CUDA tensor of >= pa_decode_shared_prefix_workspace_size(...) bytes."""
+    s, h, d, nb, hk, bs, _, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                  context_lens)
+    _shape(group_start.dim() == 1 and group_shared_blocks.dim() == 1 and
+           group_start.shape[0] == group_shared_blocks.shape[0] + 1,
+           "group_start must have one more entry than group_shared_blocks")
     _dev(q, "q")
     _dev(out, "out", q.dtype)
     _dev(k_cache, "k_cache", q.dtype)
@@ -284,16 +331,7 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
     _dev(group_shared_blocks, "group_shared_blocks", torch.int32)
     if workspace is not None:
         _dev(workspace, "workspace")
-    s, h, d = q.shape
-    nb, hk, bs, d2 = k_cache.shape
-    if d2 != d or tuple(out.shape) != tuple(q.shape):
-        raise ValueError("shape mismatch between q, out and the caches")
-    s2, mbps = block_tables.shape
-    if s2 != s or context_lens.shape[0] != s:
-        raise ValueError("q, block_tables and context_lens disagree on the number of sequences")
     g = group_shared_blocks.shape[0]
-    if group_start.shape[0] != g + 1:
-        raise ValueError("group_start must have one more entry than group_shared_blocks")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = _lib.pa_decode_shared_prefix(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                       _ptr(block_tables), mbps, _ptr(context_lens), s,

@@ -481,13 +481,9 @@ cudaError_t launch_prefix_t(const AttnArgs &a, int dtype, int cluster, cudaStrea
   if (!make_cache_map(&tmk, a.k_cache, a.num_blocks, a.num_kv_heads, D, BS, dtype) ||
       !make_cache_map(&tmv, a.v_cache, a.num_blocks, a.num_kv_heads, D, BS, dtype))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kBytes);
+  {
+    cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), Lay::kBytes);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
   }
   const int64_t grid = (int64_t)a.num_groups * a.grp_chunks * a.num_kv_heads * cluster;
   if (grid == 0) return cudaSuccess;

@@ -280,12 +280,8 @@ cudaError_t launch_chunk_t(const AttnArgs &a, cudaStream_t stream) {
   constexpr int LD = D + kPad;
   const int smem = (kRows * LD + 4 * kKT * LD) * (int)sizeof(T);
   auto kern = chunk_kernel<T, D, BS>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), smem);
+  if (e != cudaSuccess) return e;
   const int tpt = kRows / a.group;
   const int tiles = (a.max_query_len + tpt - 1) / tpt;
   const int64_t grid = (int64_t)a.num_seqs * a.num_kv_heads * tiles;

@@ -812,14 +812,15 @@ __global__ void __launch_bounds__(32 * (4 * kHalves * NQ + 2), PA_CHUNK_TC_MIN_C
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn_tc() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // looked up once; a function-local static is initialised thread-safely
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     cudaDriverEntryPointQueryResult q;
     void *p = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -855,13 +856,9 @@ cudaError_t launch_tc_t(const AttnArgs &a, cudaStream_t stream) {
   auto kern = chunk_tc_kernel<T, BS, PREFIX, NQ>;
   constexpr int kBytes = TcLayoutT<NQ>::kBytes;
   constexpr int kThreads = 32 * (4 * kHalves * NQ + 2);
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+  {
+    cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kBytes);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
   }
   // chunk rows: (sequence, KV head, tile of TPT tokens); prefix: (group, KV
   // head, chunk of TPT members)

@@ -552,18 +552,11 @@ cudaError_t launch_variant(const AttnArgs &a, int sm_count, int ncw, int hsplit,
   auto kern = paged_decode_kernel<T, D, BS, GW, MAXW>;
   const Layout<C> lay(a.num_seqs, ncw, a.group);
   // Opt in to the largest layout once; resident CTAs per SM for this launch.
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    const Layout<C> big(kMaxSeqsPerLaunch, MAXW, 32);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         big.bytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  const Layout<C> big(kMaxSeqsPerLaunch, MAXW, 32);
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes);
+  if (e != cudaSuccess) return e;
   int occ = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (ncw + 1),
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (ncw + 1),
                                                                 lay.bytes);
   if (e != cudaSuccess) return e;
   if (occ < 1) occ = 1;

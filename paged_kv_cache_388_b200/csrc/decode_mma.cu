@@ -813,14 +813,15 @@ __global__ void __launch_bounds__(256) balanced_merge_kernel(const AttnArgs a) {
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // looked up once; a function-local static is initialised thread-safely
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     cudaDriverEntryPointQueryResult q;
     void *p = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -870,17 +871,11 @@ cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
                make_map<T, D, BS>(&tmv, a.v_cache, a.num_blocks, a.num_kv_heads)))
     return cudaErrorInvalidValue;
   const L lay(a.num_seqs, a.group);
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    const L big(kMaxSeqsPerLaunch, 8 * NT);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, big.bytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  const L big(kMaxSeqsPerLaunch, 8 * NT);
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes);
+  if (e != cudaSuccess) return e;
   int occ = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1), lay.bytes);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1), lay.bytes);
   if (e != cudaSuccess) return e;
   if (occ < 1) occ = 1;
   int64_t grid = (int64_t)sm_count * occ;
@@ -912,15 +907,8 @@ int grid_mma_t(const AttnArgs &a, int sm_count) {
   constexpr int NCW = PA_MMA_WARPS;
   using L = MmaLayout<D, BS, NT, NCW, F8>;
   auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW, F8>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    const L big(kMaxSeqsPerLaunch, 8 * NT);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, big.bytes) != cudaSuccess)
-      return 0;
-    attr_set[dev] = true;
-  }
+  const L big(kMaxSeqsPerLaunch, 8 * NT);
+  if (set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes) != cudaSuccess) return 0;
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1),
                                                     L(a.num_seqs, a.group).bytes) != cudaSuccess)

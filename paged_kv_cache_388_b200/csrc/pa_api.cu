@@ -6,7 +6,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "../../include/pa.h"
 #include "pa_internal.h"
@@ -61,6 +63,21 @@ cudaError_t device_info(DevInfo *info) {
   }
   *info = g_dev[dev];
   return cudaSuccess;
+}
+
+cudaError_t set_smem_limit_once(const void *func, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, cudaError_t> done;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(func, dev);
+  const auto it = done.find(key);
+  if (it != done.end()) return it->second;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace(key, e);  // failures are retried on the next call
+  return e;
 }
 
 void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_context_len,

@@ -64,6 +64,11 @@ struct DevInfo {
 // Implemented in pa_api.cu
 cudaError_t device_info(DevInfo *info);
 
+// Raise the dynamic shared-memory limit of kernel `func` to `bytes` on the
+// current device, once per (kernel, device); thread-safe.  Later calls for the
+// same pair return the first call's result without touching the runtime.
+cudaError_t set_smem_limit_once(const void *func, int bytes);
+
 // Split policy: KV blocks per split and the largest split count per sequence.
 void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
                   int kv_split_tokens, int sm_count, int *split_blocks, int *max_splits);

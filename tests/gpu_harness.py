@@ -3,6 +3,9 @@ device (copy_blocks -> reshape_and_cache -> decode) and the same step in the
 CPU oracle, on the same seeded inputs."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -65,7 +68,22 @@ def raw_cpu(t):
     return workloads.to_numpy_raw(t.cpu())
 
 
+def _log_errors(what, dtype, rows_checked, max_abs, max_rel):
+    """Append the comparison's error figures to $PA_PARITY_LOG (JSON lines)
+    when that variable is set, and print them (visible with pytest -s)."""
+    rec = {"what": what, "dtype": dtype, "rows_checked": rows_checked, "max_abs": max_abs,
+           "max_rel_ref_gt_1e-3": max_rel}
+    print("parity", json.dumps(rec))
+    path = os.environ.get("PA_PARITY_LOG")
+    if path:
+        with open(path, "a", encoding="utf-8") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
 def assert_close(got, want, dtype, rows=None, what=""):
+    """Element-wise |got - want| <= atol + rtol*|want| at the dtype's
+    tolerance; returns the max absolute error and logs it together with the
+    max relative error over elements with |want| > 1e-3."""
     atol, rtol = TOL[dtype]
     g = got.float().cpu().numpy().astype(np.float64)
     if rows is not None:
@@ -74,9 +92,12 @@ def assert_close(got, want, dtype, rows=None, what=""):
     err = np.abs(g - want)
     bound = atol + rtol * np.abs(want)
     bad = err > bound
+    big = np.abs(want) > 1e-3
+    max_rel = float((err[big] / np.abs(want[big])).max()) if big.any() else 0.0
+    _log_errors(what, dtype, int(g.shape[0]), float(err.max()) if err.size else 0.0, max_rel)
     if bad.any():
         idx = np.argwhere(bad)[:5]
         raise AssertionError(
             f"{what}: {int(bad.sum())} of {bad.size} elements outside |d| <= {atol} + {rtol}|ref|; "
             f"max abs {err.max():.3g}; first bad {idx.tolist()} got {g[bad][:5]} want {want[bad][:5]}")
-    return float(err.max())
+    return float(err.max()) if err.size else 0.0

@@ -82,12 +82,9 @@ def test_small_configs(lib, cfg):
 
 
 @pytest.mark.parametrize("cfg", ["2", "3"])
-def test_full_configs_sampled(lib, cfg):
-    wl = workloads.make(cfg)
-    rng = np.random.default_rng(31)
-    rows = sorted(set(rng.choice(wl.num_seqs, size=20, replace=False).tolist()) |
-                  {0, wl.num_seqs - 1, int(np.argmax(wl.seq_context_lens()))})
-    _run(lib, wl, rows=rows)
+def test_full_configs(lib, cfg):
+    """Full-size batches in the benchmark's launch configuration, every row."""
+    _run(lib, workloads.make(cfg))
 
 
 @pytest.mark.parametrize("q_mul", [1000.0, 1e-3, 3e4])

@@ -88,12 +88,9 @@ def test_small_configs(lib, cfg):
 
 
 @pytest.mark.parametrize("cfg", ["4", "4cow"])
-def test_full_configs_sampled(lib, cfg):
-    wl = workloads.make(cfg)
-    rng = np.random.default_rng(91)
-    rows = sorted(set(rng.choice(wl.num_seqs, size=24, replace=False).tolist()) |
-                  {0, 7, 8, wl.num_seqs - 1})
-    _run(lib, wl, rows=rows)
+def test_full_configs(lib, cfg):
+    """Full-size parallel-sampling batches, every row."""
+    _run(lib, workloads.make(cfg))
 
 
 def test_agrees_with_plain_decode(lib):
