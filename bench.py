@@ -1,16 +1,29 @@
 #!/usr/bin/env python
-"""Benchmark: one decode step of paged attention on the Llama-3-8B-shaped GQA batch.
+"""Benchmark: one decode step of paged attention on the Llama-3-8B-shaped GQA batch,
+then every other workload of the build measured call by call.
 
-A step is the whole hot path over one batch: copy-on-write block copies (none
-in this batch), reshape_and_cache of the step's 256 new tokens, then paged
-decode attention of the 256 query tokens over their block-table KV cache
-(32 query heads / 8 KV heads, head_dim 128, block size 16, bf16, context
-lengths lognormal with median 800 capped at 4096, shuffled pool).
+Headline (the JSON line's ``value``): a step is the whole hot path over one
+batch -- copy-on-write block copies (none in this batch), reshape_and_cache of
+the step's 256 new tokens, then paged decode attention of the 256 query tokens
+over their block-table KV cache (32 query heads / 8 KV heads, head_dim 128,
+block size 16, bf16, context lengths lognormal with median 800 capped at 4096,
+shuffled pool); achieved HBM GB/s of the step (algorithmic bytes / device
+time) and decode tokens/s.
 
-Printed (rank 0, one JSON line): achieved HBM GB/s of the step (algorithmic
-bytes / device time), decode tokens/s, the dominant kernel's roofline, an
-end-to-end figure through the public API with host buffers, and the CPU oracle
-timed on a bounded sample as a baseline.
+``configs`` (N = 1): every workload -- Llama-2-7B-shaped MHA fp16, the
+Llama-3-8B-shaped batch in bf16 and with an FP8 (E4M3) cache, the
+parallel-sampling shared-prefix batch (shared-prefix call and plain decode,
+also with copy-on-write), the long-context batch with chunked-prefill rows at
+block size 16 and 32 (whole call, decode rows alone, chunk rows alone), the
+tiny fp32 batch -- each call timed as the median (min, max) of 50 calls with
+the L2 flushed before every one, against its roofline (HBM copy bandwidth for
+decode, the bf16 tensor peak for chunk rows, the larger of the two bounds for
+a mixed call).
+
+``cpu_baseline``: the CPU oracle (fp64) on the machine's host cores on bounded
+samples: the headline step, and per workload a sample of query rows timed
+with all threads (and one thread for the first three workloads), with the
+largest absolute and relative differences between those rows and the GPU's.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -21,6 +34,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import gc
 import json
 import os
 import statistics
@@ -43,15 +57,32 @@ METRIC = "paged decode attention: achieved HBM GB/s (% of peak) and decode token
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
+FLUSH_BYTES = 256 * 2 ** 20          # >= 2x L2: a memset of this evicts every cached line
+EXTRA_CONFIGS = ("2", "3fp8", "4", "4cow", "5", "5bs32", "1")
 
 
-def hbm_peak():
+def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
+            return json.load(f)
+    return None
+
+
+def hbm_peak():
+    pk = _peaks()
+    if pk and "hbm_gbs" in pk:
+        return float(pk["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    pk = _peaks()
+    if pk and "bf16_tflops" in pk:
+        return float(pk["bf16_tflops"]), "measured"
+    return FALLBACK_TFLOPS, "fallback"
 
 
 KERNEL_SOURCES = ("paged_kv_cache_388_b200/csrc/decode_mma.cu",
@@ -82,22 +113,17 @@ def profiled_traffic(config):
     return int(fields["traffic_bytes_per_launch"])
 
 
-def tensor_peak():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured"
-    return 1590.0, "fallback"
-
-
-def chunk_flops(batch):
+def chunk_flops(batch, seqs=None):
     """Multiply-add FLOPs of the chunked-query rows (QK^T and PV over the keys
-    each row may see): sum over rows of visible keys * H * D * 4."""
+    each row may see), per head and head_dim unit: sum over rows of visible
+    keys (multiply by H * D * 4 for FLOPs)."""
     qsl = batch.query_start_loc
     if qsl is None:
         return 0
     total = 0
     for i, L in enumerate(batch.context_lens.tolist()):
+        if seqs is not None and i not in seqs:
+            continue
         Q = int(qsl[i + 1] - qsl[i])
         if Q <= 1:
             continue
@@ -224,9 +250,6 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-# --------------------------------------------------------------------------
-# CPU oracle legs (cpu_baseline and --impl reference)
-# --------------------------------------------------------------------------
 def aggregate(local_bytes, local_ms, device):
     """Whole-job totals over ranks: bytes summed, time = the slowest rank's.
     No-op without an initialised process group."""
@@ -240,6 +263,237 @@ def aggregate(local_bytes, local_ms, device):
     return float(b.item()), float(t.item())
 
 
+# --------------------------------------------------------------------------
+# device timing
+# --------------------------------------------------------------------------
+class Timer:
+    """CUDA-event timing on the launching stream.  Calls are captured into
+    CUDA graphs so that host launch cost stays out of the device time."""
+
+    def __init__(self, dev):
+        self.dev = dev
+        self.stream = torch.cuda.current_stream(dev)
+        self._flush = None
+
+    def _graph(self, fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                fn()
+        return g
+
+    def back_to_back(self, fn, k):
+        """Average ms of one call over k calls replayed back to back."""
+        g = self._graph(fn, k)
+        g.replay()
+        torch.cuda.synchronize(self.dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        g.replay()
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        del g
+        return e0.elapsed_time(e1) / k
+
+    def flushed(self, fn, warm=10, iters=50):
+        """Median (min, max) ms of `iters` single calls, each preceded by a
+        memset of FLUSH_BYTES that evicts the L2, after `warm` calls."""
+        if self._flush is None:
+            self._flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=self.dev)
+        g = self._graph(fn, 1)
+        for _ in range(warm):
+            g.replay()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(iters)]
+        torch.cuda.synchronize(self.dev)
+        for e0, e1 in evs:
+            self._flush.zero_()  # ~40-80 us on the device: the replay below is enqueued meanwhile
+            e0.record(self.stream)
+            g.replay()
+            e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        ts = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+        del g
+        return {"median_ms": statistics.median(ts), "min_ms": ts[0], "max_ms": ts[-1],
+                "calls": iters, "l2": "flushed before every call"}
+
+
+# --------------------------------------------------------------------------
+# one workload resident on the device
+# --------------------------------------------------------------------------
+def fp8_scale(*ts):
+    return float(np.float32(max(float(t.float().abs().max()) for t in ts) / 448.0 * 1.25))
+
+
+def fp8_quant(t, sc):
+    return (t.float() / torch.tensor(sc, dtype=torch.float32)).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+class DeviceBatch:
+    """A workload's batch on the device with the calls of its step."""
+
+    def __init__(self, cfg, dev, replica=0, kv_fp8=False, plain_decode=False):
+        from paged_kv_cache_388_b200.session import PagedKVCache
+        self.cfg = cfg
+        self.wl = wl = workloads.make(cfg, replica=replica)
+        self.batch = batch = build_batch(wl)
+        self.vals = vals = workloads.values(wl)
+        self.dev = dev
+        self.kv_fp8 = kv_fp8
+        if kv_fp8:
+            # FP8 (E4M3) cache: one scale per tensor, the pool's history quantised
+            # on the host, this step's K/V quantised by pa_reshape_and_cache_fp8
+            self.ks = fp8_scale(vals["k_pool"], vals["new_key"])
+            self.vs = fp8_scale(vals["v_pool"], vals["new_value"])
+            self.k_codes = fp8_quant(vals["k_pool"], self.ks)
+            self.v_codes = fp8_quant(vals["v_pool"], self.vs)
+            self.cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                      dtype=torch.uint8, k_cache=self.k_codes.to(dev),
+                                      v_cache=self.v_codes.to(dev), kv_scales=(self.ks, self.vs))
+        else:
+            self.cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                      k_cache=vals["k_pool"].to(dev), v_cache=vals["v_pool"].to(dev))
+        self.q = vals["q"].to(dev)
+        self.key = vals["new_key"].to(dev)
+        self.value = vals["new_value"].to(dev)
+        self.slot = torch.from_numpy(batch.slot_mapping).to(dev)
+        self.bt = torch.from_numpy(batch.block_tables).to(dev)
+        self.cl = torch.from_numpy(batch.context_lens).to(dev)
+        self.qsl = None if batch.query_start_loc is None else torch.from_numpy(batch.query_start_loc).to(dev)
+        self.cow = torch.from_numpy(np.ascontiguousarray(batch.cow_pairs)).to(dev)
+        self.out = torch.empty_like(self.q)
+        self.mcl = batch.max_context_len
+        self.cache.workspace(batch.num_seqs, wl.num_heads, self.mcl)
+        self.shared = wl.kind == "shared_prefix" and not plain_decode and not kv_fp8
+        if self.shared:
+            gs_np, gb_np = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)
+            self.gs = torch.from_numpy(gs_np).to(dev)
+            self.gb = torch.from_numpy(gb_np).to(dev)
+            self.gb_np = gb_np
+            self.max_group = int(np.diff(gs_np).max())
+        self.bytes = step_bytes(wl, batch, 1 if kv_fp8 else None)
+
+    def attend_plain(self):
+        self.cache.attend(self.q, self.bt, self.cl, self.wl.scale, out=self.out,
+                          query_start_loc=self.qsl, max_query_len=self.batch.max_query_len,
+                          max_context_len=self.mcl)
+
+    def attend(self):
+        if self.shared:
+            self.cache.attend_shared_prefix(self.q, self.bt, self.cl, self.gs, self.gb,
+                                            self.wl.scale, max_group_size=self.max_group,
+                                            out=self.out, max_context_len=self.mcl)
+        else:
+            self.attend_plain()
+
+    def write(self):
+        self.cache.write(self.key, self.value, self.slot)
+
+    def copy_blocks(self):
+        self.cache.copy_blocks(self.cow)
+
+    def step(self):
+        if self.cow.shape[0]:
+            self.copy_blocks()
+        self.write()
+        self.attend()
+
+    def launches_per_step(self):
+        from paged_kv_cache_388_b200 import _lib
+        b = self.batch
+        splits = _lib.pa_decode_workspace_size(b.num_seqs, self.wl.num_heads, self.wl.num_kv_heads,
+                                               self.wl.head_dim, self.wl.block_size, self.mcl, 0) > 0
+        return 1 + 1 + (1 if splits else 0) + (1 if self.cow.shape[0] else 0) + \
+            (1 if b.max_query_len > 1 else 0) + (1 if self.shared else 0)
+
+    def rows_callable(self, ids):
+        """A call attending only the query rows of sequences `ids` (the decode
+        rows or the chunk rows of a mixed batch), into its own output."""
+        sbt, scl, sqsl, srows = sub_batch(self.batch, ids)
+        sq = self.q[torch.from_numpy(srows).to(self.dev)].contiguous()
+        sout = torch.empty_like(sq)
+        t_bt = torch.from_numpy(np.ascontiguousarray(sbt)).to(self.dev)
+        t_cl = torch.from_numpy(np.ascontiguousarray(scl)).to(self.dev)
+        t_qsl = None if sqsl is None else torch.from_numpy(sqsl).to(self.dev)
+        mql = int(max(np.diff(sqsl))) if sqsl is not None else 1
+        if t_qsl is not None and mql == 1:
+            t_qsl = None
+        mcl = int(scl.max())
+        return lambda: self.cache.attend(sq, t_bt, t_cl, self.wl.scale, out=sout,
+                                         query_start_loc=t_qsl, max_query_len=mql,
+                                         max_context_len=mcl)
+
+
+def _rate(nbytes, ms):
+    return nbytes / (ms * 1e-3) / 1e9
+
+
+def measure_config(db, timer, k):
+    """Per-call timings of one workload against its rooflines."""
+    wl, batch = db.wl, db.batch
+    peak, peak_kind = hbm_peak()
+    tc, tc_kind = tensor_peak()
+    for _ in range(3):
+        db.step()
+    torch.cuda.synchronize(db.dev)
+    res = {"workload": wl.name, "dtype": ("fp8_e4m3 KV, " + wl.dtype + " q/out") if db.kv_fp8
+           else wl.dtype, "seqs": batch.num_seqs, "q_rows": db.bytes["q_rows"],
+           "kv_tokens": db.bytes["kv_tokens"], "decode_bytes": db.bytes["decode"]}
+    name = "pa_decode_shared_prefix" if db.shared else ("pa_decode_fp8" if db.kv_fp8 else "pa_decode")
+    call = timer.flushed(db.attend)
+    call["avg_ms_back_to_back"] = timer.back_to_back(db.attend, k)
+    call["GBps"] = _rate(db.bytes["decode"], call["median_ms"])
+    call["frac_of_hbm_peak"] = call["GBps"] / peak
+    call["tokens_per_s"] = db.bytes["q_rows"] / (call["median_ms"] * 1e-3)
+    res[name] = call
+    res["hbm_peak_GBps"] = {"value": peak, "kind": f"{peak_kind} copy bandwidth"}
+    w = timer.flushed(db.write)
+    w["GBps"] = _rate(db.bytes["reshape"], w["median_ms"])
+    res["pa_reshape_and_cache_fp8" if db.kv_fp8 else "pa_reshape_and_cache"] = w
+    if db.cow.shape[0]:
+        c = timer.flushed(db.copy_blocks)
+        c["pairs"] = int(db.cow.shape[0])
+        c["GBps"] = _rate(db.bytes["copy_blocks"], c["median_ms"])
+        res["pa_copy_blocks"] = c
+    if db.shared:
+        plain = timer.flushed(db.attend_plain)
+        plain["GBps_unique"] = _rate(db.bytes["decode"], plain["median_ms"])
+        res["pa_decode_plain"] = plain
+        logical = int(batch.context_lens.astype(np.int64).sum()) * 2 * wl.num_kv_heads * \
+            wl.head_dim * elem_bytes(wl.dtype)
+        res[name]["logical_kv_bytes"] = logical
+        res[name]["GBps_logical"] = _rate(logical, call["median_ms"])
+        res[name]["groups"] = int(db.gb_np.shape[0])
+        res[name]["shared_blocks"] = int(db.gb_np.max())
+    if batch.query_start_loc is not None:
+        qsl = batch.query_start_loc
+        dec_ids = [i for i in range(batch.num_seqs) if qsl[i + 1] - qsl[i] == 1]
+        chk_ids = [i for i in range(batch.num_seqs) if qsl[i + 1] - qsl[i] > 1]
+        flops = chunk_flops(batch) * wl.num_heads * wl.head_dim * 4
+        dbytes, _, _ = seq_bytes(wl, batch, dec_ids)
+        if dec_ids:
+            d = timer.flushed(db.rows_callable(dec_ids))
+            d["GBps"] = _rate(dbytes, d["median_ms"])
+            d["frac_of_hbm_peak"] = d["GBps"] / peak
+            d["bytes"] = dbytes
+            res["decode_rows"] = d
+        if chk_ids:
+            c = timer.flushed(db.rows_callable(chk_ids))
+            c["flops"] = flops
+            c["TFLOPs"] = flops / (c["median_ms"] * 1e-3) / 1e12
+            c["frac_of_tensor_peak"] = c["TFLOPs"] / tc
+            res["chunk_rows"] = c
+        bound_ms = max(db.bytes["decode"] / (peak * 1e9), flops / (tc * 1e12)) * 1e3
+        res["mixed_bound"] = {"ms": bound_ms, "rule": "max(all bytes / HBM peak, chunk flops / "
+                              "bf16 tensor peak)", "tensor_peak_TFLOPs": tc,
+                              "tensor_peak_kind": tc_kind,
+                              "frac": bound_ms / call["median_ms"]}
+    return res
+
+
+# --------------------------------------------------------------------------
+# CPU oracle legs (cpu_baseline and --impl reference)
+# --------------------------------------------------------------------------
 def oracle_runner(wl, vals, batch):
     """Returns run(n_seqs) -> (seconds, bytes, n_seqs): the oracle doing the
     step for the first n_seqs sequences (their new tokens' writes into a copy
@@ -278,6 +532,85 @@ def size_sample(run, total, target_s):
     return n
 
 
+def oracle_config_leg(db, gpu_out, target_s=1.5):
+    """The oracle on a sample of one workload's query rows, on the same
+    inputs as the GPU call (copy-on-write copies and this step's K/V applied
+    to a host copy of the pool first): seconds with all threads (and with one
+    thread for the first three workloads), the equivalent GB/s, and the largest
+    differences between the sampled rows and the GPU's output."""
+    import oracle
+    wl, batch, vals = db.wl, db.batch, db.vals
+    if db.kv_fp8:
+        kp, vp = db.k_codes.numpy(), db.v_codes.numpy()   # host arrays, not on the device
+        if batch.cow_pairs.shape[0]:
+            oracle.copy_blocks(kp, vp, batch.cow_pairs, "fp8")
+        oracle.reshape_and_cache_fp8(kp, vp, workloads.to_numpy_raw(vals["new_key"]),
+                                     workloads.to_numpy_raw(vals["new_value"]), wl.dtype,
+                                     batch.slot_mapping, db.ks, db.vs)
+    else:
+        kp = workloads.to_numpy_raw(vals["k_pool"])  # in place: the device pool is a copy
+        vp = workloads.to_numpy_raw(vals["v_pool"])
+        if batch.cow_pairs.shape[0]:
+            oracle.copy_blocks(kp, vp, batch.cow_pairs, wl.dtype)
+        oracle.reshape_and_cache(kp, vp, workloads.to_numpy_raw(vals["new_key"]),
+                                 workloads.to_numpy_raw(vals["new_value"]), batch.slot_mapping,
+                                 wl.dtype)
+    q = workloads.to_numpy_raw(vals["q"])
+    qsl = batch.query_start_loc
+
+    def decode(rows, threads):
+        t0 = time.perf_counter()
+        if db.kv_fp8:
+            ref = oracle.decode_fp8(q, wl.dtype, kp, vp, db.ks, db.vs, batch.block_tables,
+                                    batch.context_lens, wl.scale, rows=rows, threads=threads)
+        else:
+            ref = oracle.decode(q, kp, vp, batch.block_tables, batch.context_lens, wl.scale,
+                                wl.dtype, query_start_loc=qsl, rows=rows, threads=threads)
+        return time.perf_counter() - t0, ref
+
+    # visible keys of every query row, to size the sample by work
+    lens = batch.context_lens.astype(np.int64)
+    if qsl is None:
+        keys = lens
+        row_seq = np.arange(batch.num_seqs)
+    else:
+        keys, row_seq = [], []
+        for i in range(batch.num_seqs):
+            Q = int(qsl[i + 1] - qsl[i])
+            keys.extend(int(lens[i]) - Q + t + 1 for t in range(Q))
+            row_seq.extend([i] * Q)
+        keys, row_seq = np.asarray(keys), np.asarray(row_seq)
+    order = np.random.default_rng(7).permutation(keys.shape[0])
+    probe = order[: max(1, min(8, keys.shape[0]))]
+    dt, _ = decode(probe.tolist(), 0)
+    per_key = dt / max(1, int(keys[probe].sum()))
+    csum = np.cumsum(keys[order])
+    n = int(np.searchsorted(csum, target_s / max(per_key, 1e-12))) + 1
+    rows = np.sort(order[: max(1, min(n, keys.shape[0]))])
+    dt, ref = decode(rows.tolist(), 0)
+    e = elem_bytes(wl.dtype)
+    ekv = 1 if db.kv_fp8 else e
+    kv_bytes = int(keys[rows].sum()) * 2 * wl.num_kv_heads * wl.head_dim * ekv
+    nbytes = kv_bytes + 2 * rows.shape[0] * wl.num_heads * wl.head_dim * e
+    g = gpu_out.float().cpu().numpy().astype(np.float64)[rows]
+    r = ref[rows]
+    err = np.abs(g - r)
+    big = np.abs(r) > 1e-3
+    leg = {"rows": int(rows.shape[0]), "of_rows": int(keys.shape[0]),
+           "sample": "query rows drawn uniformly at random (seed 7), all heads; GB/s counts the "
+                     "KV bytes each sampled row reads (no sharing between rows)",
+           "threads_all": {"cores": oracle.max_threads(), "s": dt, "GBps": nbytes / dt / 1e9},
+           "max_abs_err_vs_gpu": float(err.max()),
+           "max_rel_err_vs_gpu_ref_gt_1e-3": float((err[big] / np.abs(r[big])).max()) if big.any() else 0.0}
+    if db.cfg in ("1", "2", "3"):
+        rows1 = rows[: max(1, rows.shape[0] // 8)]
+        dt1, _ = decode(rows1.tolist(), 1)
+        kb1 = int(keys[rows1].sum()) * 2 * wl.num_kv_heads * wl.head_dim * ekv + \
+            2 * rows1.shape[0] * wl.num_heads * wl.head_dim * e
+        leg["threads_1"] = {"rows": int(rows1.shape[0]), "s": dt1, "GBps": kb1 / dt1 / 1e9}
+    return leg
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle, as it stands, on the host cores."""
     wl = workloads.make(args.config)
@@ -310,93 +643,63 @@ def run_reference(args):
 # --------------------------------------------------------------------------
 # GPU leg
 # --------------------------------------------------------------------------
+def e2e_pipelined(db, k, warmup, barrier):
+    """The step through the public API from page-locked host buffers: every
+    step copies its inputs in (q, new K/V, slots, context lengths and the
+    block-table entries the step appended) and its output back; copies of
+    neighbouring steps overlap the kernels (PagedKVCache
+    .capture_pipelined_steps_from_host)."""
+    from paged_kv_cache_388_b200.session import PagedKVCache
+    wl, batch, vals = db.wl, db.batch, db.vals
+    idx, ids = PagedKVCache.appended_table_entries(batch.block_tables, batch.context_lens,
+                                                   wl.block_size)
+    host = {"q": vals["q"].pin_memory(), "key": vals["new_key"].pin_memory(),
+            "value": vals["new_value"].pin_memory(),
+            "slot_mapping": torch.from_numpy(batch.slot_mapping).pin_memory(),
+            "context_lens": torch.from_numpy(batch.context_lens).pin_memory(),
+            "bt_index": idx.pin_memory(), "bt_ids": ids.pin_memory()}
+    outs = [torch.empty_like(host["q"]).pin_memory() for _ in range(2)]
+    steps = [dict(host, out=outs[i % 2]) for i in range(k)]
+    replay = db.cache.capture_pipelined_steps_from_host(steps, db.bt, wl.scale,
+                                                        max_context_len=db.mcl, warmup=1)
+    for _ in range(max(1, warmup // 2)):
+        replay()
+    stream = torch.cuda.current_stream(db.dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    barrier()
+    h2d = PagedKVCache.host_bytes(*host.values())
+    d2h = PagedKVCache.host_bytes(outs[0])
+    ms = e0.elapsed_time(e1)
+    assert torch.equal(outs[(k - 1) % 2], db.out.cpu()), "end-to-end output differs from the device step"
+    return ms, h2d, d2h
+
+
 def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from paged_kv_cache_388_b200 import _lib
-    from paged_kv_cache_388_b200.session import PagedKVCache
 
     if world > 1:
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-
-    # weak scaling: every rank runs its own batch of the workload's shape
-    wl = workloads.make(args.config, replica=rank)
-    batch = build_batch(wl)
-    vals = workloads.values(wl)
-    nbytes = step_bytes(wl, batch, 1 if args.kv_fp8 else None)
-
-    if args.kv_fp8:
-        # FP8 (E4M3) cache: one scale per tensor, the pool's history quantised
-        # on the host, this step's K/V quantised by pa_reshape_and_cache_fp8
-        def fp8_scale(*ts):
-            return float(np.float32(max(float(t.float().abs().max()) for t in ts) / 448.0 * 1.25))
-
-        def quant(t, sc):
-            return (t.float() / torch.tensor(sc, dtype=torch.float32)).to(
-                torch.float8_e4m3fn).view(torch.uint8)
-
-        ks = fp8_scale(vals["k_pool"], vals["new_key"])
-        vs = fp8_scale(vals["v_pool"], vals["new_value"])
-        cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
-                             dtype=torch.uint8, k_cache=quant(vals["k_pool"], ks).to(dev),
-                             v_cache=quant(vals["v_pool"], vs).to(dev), kv_scales=(ks, vs))
-    else:
-        cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, wl.block_size,
-                             k_cache=vals["k_pool"].to(dev), v_cache=vals["v_pool"].to(dev))
-    q = vals["q"].to(dev)
-    key = vals["new_key"].to(dev)
-    value = vals["new_value"].to(dev)
-    slot = torch.from_numpy(batch.slot_mapping).to(dev)
-    bt = torch.from_numpy(batch.block_tables).to(dev)
-    cl = torch.from_numpy(batch.context_lens).to(dev)
-    qsl = None if batch.query_start_loc is None else torch.from_numpy(batch.query_start_loc).to(dev)
-    cow = torch.from_numpy(np.ascontiguousarray(batch.cow_pairs)).to(dev)
-    out = torch.empty_like(q)
-    mcl = batch.max_context_len
-    ws_bytes = _lib.pa_decode_workspace_size(batch.num_seqs, wl.num_heads, wl.num_kv_heads,
-                                             wl.head_dim, wl.block_size, mcl, 0)
-    cache.workspace(batch.num_seqs, wl.num_heads, mcl)
-    stream = torch.cuda.current_stream(dev)
-
-    # Batches whose sequences share prompt blocks (parallel sampling) attend
-    # through the shared-prefix entry point unless --plain-decode is given.
-    shared = wl.kind == "shared_prefix" and not args.plain_decode and not args.kv_fp8
-    if shared:
-        gs_np, gb_np = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)
-        gs = torch.from_numpy(gs_np).to(dev)
-        gb = torch.from_numpy(gb_np).to(dev)
-        max_group = int(np.diff(gs_np).max())
-
-    def attend_plain():
-        cache.attend(q, bt, cl, wl.scale, out=out, query_start_loc=qsl,
-                     max_query_len=batch.max_query_len, max_context_len=mcl)
-
-    def attend():
-        if shared:
-            cache.attend_shared_prefix(q, bt, cl, gs, gb, wl.scale, max_group_size=max_group,
-                                       out=out, max_context_len=mcl)
-        else:
-            attend_plain()
-
+    timer = Timer(dev)
+    stream = timer.stream
     K = args.steps
 
-    def step(evs=None):
-        if cow.shape[0]:
-            cache.copy_blocks(cow)
-        if evs:
-            evs[0].record(stream)
-        cache.write(key, value, slot)
-        if evs:
-            evs[1].record(stream)
-        attend()
-        if evs:
-            evs[2].record(stream)
+    # weak scaling: every rank runs its own batch of the workload's shape
+    db = DeviceBatch(args.config, dev, replica=rank, kv_fp8=args.kv_fp8,
+                     plain_decode=args.plain_decode)
+    wl, batch, nbytes = db.wl, db.batch, db.bytes
+    launches_per_step = db.launches_per_step()
 
     for _ in range(args.warmup):  # eager warm-up: one-time library set-up
-        step()
+        db.step()
     torch.cuda.synchronize(dev)
     assert _lib.pa_get_device_error() == 0
 
@@ -405,10 +708,10 @@ def run_ours(args, rank, world, local_rank):
     g_steps = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_steps):
         for _ in range(K):
-            step()
+            db.step()
     g_warm = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_warm):
-        step()
+        db.step()
     for _ in range(args.warmup):
         g_warm.replay()
     torch.cuda.synchronize(dev)
@@ -432,115 +735,68 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.summary()
     del g_steps, g_warm
 
-    # Per-call device time of the step's two calls, each timed as K back-to-back
-    # calls in its own CUDA graph (CUDA events on the launching stream).
-    def time_graph(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for _ in range(K):
-                fn()
-        g.replay()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / K
-
-    dec_avg = time_graph(attend)
-    res_avg = time_graph(lambda: cache.write(key, value, slot))
-
-    # Mixed batches: the decode rows and the chunked-query rows, each timed alone
-    parts = {}
-    if shared:  # the same batch through plain decode (every shared block read per sequence)
-        plain_ms = time_graph(attend_plain)
-        logical = sum(int(batch.context_lens[i]) for i in range(batch.num_seqs)) * 2 * \
-            wl.num_kv_heads * wl.head_dim * elem_bytes(wl.dtype)
-        parts["plain_decode"] = {"ms": plain_ms,
-                                 "GBps_unique": nbytes["decode"] / (plain_ms * 1e-3) / 1e9}
-        parts["shared_prefix"] = {"ms": dec_avg,
-                                  "GBps_unique": nbytes["decode"] / (dec_avg * 1e-3) / 1e9,
-                                  "groups": int(gb_np.shape[0]),
-                                  "shared_blocks": int(gb_np.max()),
-                                  "logical_kv_bytes": logical}
-    if batch.query_start_loc is not None:
-        qsl_np = batch.query_start_loc
-        dec_ids = [i for i in range(batch.num_seqs) if qsl_np[i + 1] - qsl_np[i] == 1]
-        chk_ids = [i for i in range(batch.num_seqs) if qsl_np[i + 1] - qsl_np[i] > 1]
-        for name, ids in (("decode_rows", dec_ids), ("chunk_rows", chk_ids)):
-            if not ids:
-                continue
-            sbt, scl, sqsl, srows = sub_batch(batch, ids)
-            sq = q[torch.from_numpy(srows).to(dev)].contiguous()
-            sout = torch.empty_like(sq)
-            t_bt = torch.from_numpy(np.ascontiguousarray(sbt)).to(dev)
-            t_cl = torch.from_numpy(np.ascontiguousarray(scl)).to(dev)
-            t_qsl = None if sqsl is None else torch.from_numpy(sqsl).to(dev)
-            mql = int(max(np.diff(sqsl))) if sqsl is not None else 1
-            if t_qsl is not None and mql == 1:
-                t_qsl = None
-            parts[name] = {"ms": time_graph(lambda: cache.attend(
-                sq, t_bt, t_cl, wl.scale, out=sout, query_start_loc=t_qsl, max_query_len=mql,
-                max_context_len=int(scl.max())))}
-        if "decode_rows" in parts:
-            dbytes, _, _ = seq_bytes(wl, batch, dec_ids)
-            parts["decode_rows"]["GBps"] = dbytes / (parts["decode_rows"]["ms"] * 1e-3) / 1e9
-        if "chunk_rows" in parts:
-            fl = chunk_flops(batch) * wl.num_heads * wl.head_dim * 4
-            parts["chunk_rows"]["flops"] = fl
-            parts["chunk_rows"]["TFLOPs"] = fl / (parts["chunk_rows"]["ms"] * 1e-3) / 1e12
+    # per-call device time of the step's calls: K back-to-back calls in one
+    # graph (inputs larger than L2) and 50 single calls after an L2 flush
+    dec_avg = timer.back_to_back(db.attend, K)
+    res_avg = timer.back_to_back(db.write, K)
+    dec_flushed = timer.flushed(db.attend)
 
     # ---- end to end through the public API, host (pinned) buffers ----------
-    hq = vals["q"].pin_memory()
-    hkey = vals["new_key"].pin_memory()
-    hval = vals["new_value"].pin_memory()
-    hslot = torch.from_numpy(batch.slot_mapping).pin_memory()
-    hbt = torch.from_numpy(batch.block_tables).pin_memory()
-    hcl = torch.from_numpy(batch.context_lens).pin_memory()
-    hout = torch.empty_like(hq).pin_memory()
-    h2d = PagedKVCache.host_bytes(hq, hkey, hval, hslot, hbt, hcl)
-    d2h = PagedKVCache.host_bytes(hout)
-    e2e_ok = batch.query_start_loc is None and cow.shape[0] == 0 and not shared
     e2e = None
-    if e2e_ok:
-        # the public API's captured host step: copy in, write K/V, attend, copy out
-        replay = cache.capture_step_from_host(hq, hkey, hval, hslot, hbt, hcl, hout, wl.scale,
-                                              max_context_len=mcl, warmup=args.warmup)
-        for _ in range(args.warmup):
-            replay()
-        barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(K):
-            replay()
-        e1.record(stream)
-        barrier()
-        e2e_bytes, e2e_ms = aggregate(nbytes["step"] * K, e0.elapsed_time(e1), dev)
+    if batch.query_start_loc is None and db.cow.shape[0] == 0 and not db.shared:
+        e2e_ms, h2d, d2h = e2e_pipelined(db, K, args.warmup, barrier)
+        e2e_bytes, e2e_ms = aggregate(nbytes["step"] * K, e2e_ms, dev)
         e2e = {"value": e2e_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / K, "path": "PagedKVCache.capture_step_from_host (CUDA graph)"}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
+               "path": "PagedKVCache.capture_pipelined_steps_from_host (CUDA graph of K steps; "
+                       "H2D and D2H copies on their own streams overlap the neighbouring steps' "
+                       "kernels; block tables resident, appended entries sent per step)"}
+
+    # ---- every other workload, call by call (one GPU) ----------------------
+    configs = {}
+    if world == 1 and not args.headline_only:
+        configs[args.config + ("fp8" if args.kv_fp8 else "")] = measure_config(db, timer, K)
+    head_out = db.out.clone()
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1) -----------
     cpu = None
     if (rank == 0 and world == 1 and not args.no_cpu_baseline and batch.query_start_loc is None
-            and not args.kv_fp8):
-        run, cores = oracle_runner(wl, vals, batch)
-        n = size_sample(run, batch.num_seqs, target_s=12.0)
+            and not args.kv_fp8 and batch.cow_pairs.shape[0] == 0):
+        run, cores = oracle_runner(wl, db.vals, batch)
+        n = size_sample(run, batch.num_seqs, target_s=8.0)
         dt, ob, _ = run(n)
         cpu = {"value": ob / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"first {n} of {batch.num_seqs} sequences (reshape_and_cache of their "
                          f"new tokens + decode rows over all {wl.num_heads} heads), "
                          f"one run of {dt:.1f} s"}
+        cpu["per_config"] = {}
+        if configs:
+            cpu["per_config"][args.config] = oracle_config_leg(db, head_out)
 
-    splits = ws_bytes > 0  # the decode call also launches its merge kernel
-    launches_per_step = 1 + 1 + (1 if splits else 0) + (1 if cow.shape[0] else 0) + \
-        (1 if batch.max_query_len > 1 else 0) + (1 if shared else 0)
+    if world == 1 and not args.headline_only:
+        del db
+        gc.collect()
+        torch.cuda.empty_cache()
+        for cfg in (args.extra_configs.split(",") if args.extra_configs else EXTRA_CONFIGS):
+            if not cfg or cfg == args.config:
+                continue
+            fp8 = cfg.endswith("fp8")
+            xdb = DeviceBatch(cfg[:-3] if fp8 else cfg, dev, kv_fp8=fp8)
+            configs[cfg] = measure_config(xdb, timer, K)
+            assert _lib.pa_get_device_error() == 0
+            if cpu is not None:
+                cpu["per_config"][cfg] = oracle_config_leg(xdb, xdb.out)
+            del xdb
+            gc.collect()
+            torch.cuda.empty_cache()
+    else:
+        del db
+
     peak, peak_kind = hbm_peak()
     achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
     value = job_bytes / (ms * 1e-3) / 1e9
+    call_name = ("pa_decode_shared_prefix" if args.config.startswith("4") and not args.plain_decode
+                 else ("pa_decode_fp8" if args.kv_fp8 else "pa_decode"))
     res = {
         "metric": METRIC,
         "value": value,
@@ -563,15 +819,14 @@ def run_ours(args, rank, world, local_rank):
             "kv_tokens": nbytes["kv_tokens"],
             "step_bytes": nbytes["step"],
             "l2": f"inputs larger than L2 ({nbytes['decode'] / 1e9:.2f} GB of KV per step vs "
-                  f"{L2_BYTES / 2**20:.0f} MiB L2); no flush",
+                  f"{L2_BYTES / 2**20:.0f} MiB L2); no flush in the timed steps; per-call "
+                  f"medians flush L2 before every call",
             "parallelism": f"dp{world} (independent batches)",
         },
         "decode_tokens_per_s": batch.num_seqs * world * K / (ms * 1e-3),
         "pct_of_nominal_8TBps": 100.0 * value / NOMINAL_HBM_GBS,
         "roofline": {
-            "kernel": ("pa_decode_shared_prefix (shared_prefix_kernel + paged_decode_mma_kernel + "
-                       "balanced_merge_kernel)") if shared else
-                      "pa_decode (paged_decode_mma_kernel + balanced_merge_kernel)",
+            "kernel": f"{call_name} (paged_decode_mma_kernel + balanced_merge_kernel)",
             "bound": "hbm",
             "achieved": achieved,
             "peak": peak,
@@ -584,12 +839,12 @@ def run_ours(args, rank, world, local_rank):
                               "of the decode kernel; null when the kernel sources changed since)",
             "algorithmic_bytes": nbytes["decode"],
             "avg_ms": dec_avg,
+            "flushed_calls": dec_flushed,
         },
-        "kernels_ms": {("pa_decode_shared_prefix" if shared else "pa_decode"): dec_avg,
-                       "pa_reshape_and_cache": res_avg},
+        "kernels_ms": {call_name: dec_avg, "pa_reshape_and_cache": res_avg},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        **({"parts": parts} if parts else {}),
+        **({"configs": configs} if configs else {}),
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
     }
@@ -669,6 +924,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the per-workload call timings (the `configs` block)")
+    ap.add_argument("--extra-configs", default="",
+                    help="comma-separated workloads for the `configs` block (default: all)")
     ap.add_argument("--plain-decode", action="store_true",
                     help="attend shared-prefix batches with pa_decode instead of "
                          "pa_decode_shared_prefix")

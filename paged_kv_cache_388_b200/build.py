@@ -35,11 +35,19 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src, verbose=False):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+# The test build of the decode kernel: a 50 ms wait limit and one ring use of
+# CTA 0 announced but never copied, so that a test can watch a wait expire and
+# the kernel unwind with PA_DEVERR_TIMEOUT (tests/test_wait_timeout.py).
+WAITTEST_LIB = os.path.join(PKG, "libpa_waittest.so")
+WAITTEST_SRC = "decode_mma.cu"
+WAITTEST_DEFINES = ["-DPA_WAIT_LIMIT_NS=50000000ull", "-DPA_TEST_LOST_COPY=3"]
+
+
+def _compile(src, verbose=False, defines=(), tag=""):
+    obj = os.path.join(BUILD, os.path.basename(src) + tag + ".o")
     if not _stale(obj, [src] + _headers()):
         return obj
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+    cmd = [NVCC, *ARCH, *FLAGS, *defines, "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,16 +64,24 @@ def build(verbose: bool = False, force: bool = False) -> str:
     if force:
         for o in glob.glob(os.path.join(BUILD, "*.o")):
             os.remove(o)
+    wt_src = os.path.join(CSRC, WAITTEST_SRC)
+    jobs = [(s, (), "") for s in srcs] + [(wt_src, WAITTEST_DEFINES, ".waittest")]
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    if _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        built = list(ex.map(lambda j: _compile(j[0], verbose, j[1], j[2]), jobs))
+    objs, wt_obj = built[:-1], built[-1]
+    _link(LIB, objs)
+    _link(WAITTEST_LIB, [o for o in objs if os.path.basename(o) != WAITTEST_SRC + ".o"] + [wt_obj])
+    return LIB
+
+
+def _link(out, objs):
+    if _stale(out, objs):
+        tmp = out + f".tmp{os.getpid()}"
         cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, out)
 
 
 if __name__ == "__main__":

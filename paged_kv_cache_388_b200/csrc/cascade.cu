@@ -239,6 +239,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();
     if (lane == 0 && *mbad) raise_error(a.err, PA_DEVERR_PREFIX);
+    // the copies this warp started land before the CTA may exit
+    if (lane == 0 && !(drain_ring(full, Lay::kStages, nstage) & drain_ring(qbar, 1, 1))) {
+      if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
   } else {
     // ============================ consumer warps ===========================
     const int g8 = lane >> 2, tig = lane & 3;

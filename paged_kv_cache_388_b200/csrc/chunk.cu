@@ -303,10 +303,13 @@ cudaError_t chunk_d(const AttnArgs &a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int /*num_q_tokens*/, cudaStream_t stream) {
-  // head_dim 128: tcgen05 kernel (chunk_tc.cu) unless PA_CHUNK_KERNEL=mma asks
-  // for this mma.sync kernel, which also serves head_dim 64.
+  // head_dim 128: the tcgen05 ping-pong kernel (chunk_pp.cu); PA_CHUNK_KERNEL=tc64
+  // selects the earlier tcgen05 kernel over 64-key tiles (chunk_tc.cu) and
+  // PA_CHUNK_KERNEL=mma this mma.sync kernel, which also serves head_dim 64.
   const char *sel = getenv("PA_CHUNK_KERNEL");
   const bool want_mma = sel && strcmp(sel, "mma") == 0;
+  const bool want_tc64 = sel && strcmp(sel, "tc64") == 0;
+  if (!want_mma && !want_tc64 && chunk_pp_supported(a, dtype)) return launch_chunk_pp(a, dtype, stream);
   if (!want_mma && chunk_tc_supported(a, dtype)) return launch_chunk_tc(a, dtype, stream);
   if (dtype == PA_F16) return chunk_d<__half>(a, stream);
   if (dtype == PA_BF16) return chunk_d<__nv_bfloat16>(a, stream);

@@ -1,0 +1,530 @@
+// chunk_pp.cu -- chunked-prefill attention on the 5th-generation tensor cores:
+// two query tiles in ping-pong over 128-key K/V tiles.
+//
+// A chunk of Q > 1 query tokens of one sequence attends causally over the
+// sequence's paged KV: row t sees keys 0 .. L-Q+t ("PagedAttention 实战",
+// section Chunked Prefill).  The GROUP query heads of a token read the same
+// K/V, so 128 rows (128/GROUP tokens x GROUP heads) against a tile of keys
+// form a dense contraction.
+//
+// CTA = (sequence, KV head, 256 query rows held as two Q tiles of 128).  Per
+// 128-key tile j and Q tile t the tensor cores compute S_t = Q_t K_j^T
+// (M 128, N 128, K = head_dim 128) and O_t += P_t V_j (M 128, N 128, K 128)
+// with fp32 accumulators in tensor memory: S_t in 128 columns, O_t in the next
+// 128 -- the four regions fill the SM's 512 columns.  P_t overwrites S_t in
+// place (bf16 hi + lo words, or one fp16 word, two keys a word) and is read
+// from there as the A operand of P V.
+//
+// Ping-pong: the MMA issue order per tile is PV_0(j), S_0(j+1), PV_1(j),
+// S_1(j+1), so the softmax of one Q tile runs while the tensor cores work on
+// the other's products.  S_t(j+1) overwrites P_t(j): the MMA thread waits for
+// P V of tile j to complete before issuing it.
+//
+// K/V tiles arrive by TMA through the block table, one box per (block, KV
+// head) and K or V: a 5-D tensor map splits every block's rows into groups of
+// 8 and each row into two 64-column halves, so a box lands as [row group]
+// [half][8 rows][64 columns] -- the 128-byte-swizzle atom layout the UMMA
+// descriptors want, with a uniform 2 KB stride per 8 keys across the blocks
+// of a tile.  One 4 KB (block size 16) or 8 KB (32) box per block instead of
+// two 2 KB boxes halves the boxes the SM's TMA unit issues per key.
+//
+// Warps: 8 softmax (4 per Q tile; thread = row = TMEM lane), 1 TMA producer,
+// 1 MMA issuer (one elected thread) that also owns the TMEM allocation.
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "tc_common.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kRows = 128;   // rows per Q tile (MMA M)
+constexpr int kKeys = 128;   // keys per K/V tile (N of S = Q K^T, K of P V)
+constexpr int kD = 128;      // head_dim
+constexpr int kQTiles = 2;
+#ifndef PA_CHUNK_PP_STAGES
+#define PA_CHUNK_PP_STAGES 2
+#endif
+constexpr int kStages = PA_CHUNK_PP_STAGES;  // K/V tiles in flight
+constexpr float kRescaleThreshold = 8.0f;    // log2 units: P stays <= 2^8 between rescales
+constexpr int kSoftmaxWarps = 4 * kQTiles;
+constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+
+// shared memory (offsets from a 1024-byte aligned base)
+constexpr int kQBytes = kRows * kD * 2;           // one Q tile: 2 halves x [128 rows][128 B]
+constexpr int kOffQ = 0;
+constexpr int kHalfStage = kKeys * kD * 2;        // K (or V) of one tile: 32 KB
+constexpr int kStageBytes = 2 * kHalfStage;
+constexpr int kOffKV = kOffQ + kQTiles * kQBytes;
+constexpr int kOffBar = kOffKV + kStages * kStageBytes;
+enum {
+  kQFull = 0,
+  kKFull = 1,                      // [kStages] the K half of a stage landed
+  kVFull = kKFull + kStages,       // [kStages] the V half landed
+  kKvEmpty = kVFull + kStages,     // [kStages] both Q tiles' products of the stage done
+  kSFull = kKvEmpty + kStages,     // [Q tile] S in TMEM
+  kPFull = kSFull + kQTiles,       // [Q tile] P written over S (4 softmax warps)
+  kPvDone = kPFull + kQTiles,      // [Q tile] P V complete
+  kDone = kPvDone + kQTiles,
+  kNumBars = kDone + 1
+};
+constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 64 + 1024;  // + TMEM slot, flags, alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+
+// TMEM columns: Q tile t's S/P at t*256, its O at t*256 + 128.
+__device__ __forceinline__ uint32_t tmem_s_col(int t) { return (uint32_t)t * 256u; }
+__device__ __forceinline__ uint32_t tmem_o_col(int t) { return (uint32_t)t * 256u + 128u; }
+
+template <typename T, int BS>
+__global__ void __maxnreg__(200)
+    chunk_pp_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmq,
+                    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                    int tiles_per_seq) {
+  using TT = TcType<T>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * kNumBars);
+  volatile int *flags = reinterpret_cast<volatile int *>(tmem_slot + 1);  // [0] abort, [1] bad block
+  const uint32_t sbase = smem_addr(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- the CTA's rows: tokens t0 .. t0 + ntok - 1 of the sequence's chunk --
+  const int G = a.group;
+  const int TPT = kRows / G;  // tokens per Q tile
+  const int tile = blockIdx.x % tiles_per_seq;
+  const int rest = blockIdx.x / tiles_per_seq;
+  const int kvh = rest % a.num_kv_heads;
+  const int seq = a.seq_begin + rest / a.num_kv_heads;
+  const int q0 = a.query_start_loc[seq];
+  const int Q = a.query_start_loc[seq + 1] - q0;
+  if (Q <= 1 || q0 < 0 || q0 + Q > a.num_q_tokens) return;  // CTA-uniform exits, before any barrier
+  if (Q > a.max_query_len) {
+    if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
+    return;
+  }
+  const int t0 = tile * kQTiles * TPT;
+  if (t0 >= Q) return;
+  const int ntok = min(kQTiles * TPT, Q - t0);
+  const int nq = ntok > TPT ? 2 : 1;  // Q tiles holding rows of this chunk
+  const int L = a.context_lens[seq];
+  if (L < Q || L > a.max_context_len) {
+    if (tid == 0 && tile == 0 && kvh == 0)
+      raise_error(a.err, (L < 0 || L > a.max_context_len) ? PA_DEVERR_CONTEXT_LEN : PA_DEVERR_QUERY_LEN);
+    for (int idx = tid; idx < ntok * G * kD; idx += blockDim.x) {
+      const int r = idx / kD, dd = idx - r * kD;
+      static_cast<T *>(a.out)[((int64_t)(q0 + t0 + r / G) * a.num_heads + kvh * G + r % G) * kD + dd] =
+          Elem<T>::from_f(0.f);
+    }
+    return;
+  }
+  const int kend = L - Q + t0 + ntok;  // keys [0, kend) are visible to some row
+  const int ntiles = (kend + kKeys - 1) / kKeys;
+  const int nblk = (L + BS - 1) / BS;
+
+  // ---- set-up: barriers, TMEM ---------------------------------------------
+  if (tid == 0) {
+    mbar_init(&bars[kQFull], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars[kKFull + s], 1);
+      mbar_init(&bars[kVFull + s], 1);
+      mbar_init(&bars[kKvEmpty + s], 1);
+    }
+    for (int t = 0; t < kQTiles; ++t) {
+      mbar_init(&bars[kSFull + t], 1);
+      mbar_init(&bars[kPFull + t], 4);
+      mbar_init(&bars[kPvDone + t], 1);
+    }
+    mbar_init(&bars[kDone], 1);
+    flags[0] = 0;
+    flags[1] = 0;
+    mbar_init_fence();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&](void) {
+    if (!flags[0]) raise_error(a.err, PA_DEVERR_TIMEOUT);
+    flags[0] = 1;
+  };
+
+  if (warp == kProducerWarp) {
+    // ======================= producer =======================================
+    // The warp reads the block table 32 ids at a time (one coalesced load, the
+    // next group fetched while the current one is issued); lane 0 issues the
+    // TMA loads: Q once, then per tile one K box and one V box per block.
+    const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[kQFull], nq * kQBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int h = 0; h < 2; ++h)
+          tma_load_4d(sbase + kOffQ + t * kQBytes + h * (kQBytes / 2), &tmq, h * 64, 0, kvh,
+                      q0 + t0 + t * TPT, &bars[kQFull]);
+    }
+    constexpr int kBpt = kKeys / BS;  // blocks per tile (8 or 4; divides 32)
+    int grp = 0;
+    int ids = lane < nblk ? table[lane] : 0;
+    int ids_next = 32 + lane < nblk ? table[32 + lane] : 0;
+    int last_issued[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_issued[s] = -1;
+    bool aborted = false;
+    for (int j = 0; j < ntiles && !aborted; ++j) {
+      const int st = j % kStages;
+      const int b0 = j * kBpt;
+      if (b0 >= grp + 32) {
+        grp += 32;
+        ids = ids_next;
+        ids_next = grp + 32 + lane < nblk ? table[grp + 32 + lane] : 0;
+      }
+      const int nb = min(kBpt, nblk - b0);  // blocks of this tile inside the sequence
+      int pbs[kBpt];
+#pragma unroll
+      for (int b = 0; b < kBpt; ++b) pbs[b] = __shfl_sync(0xffffffffu, ids, (b0 - grp + b) & 31);
+      bool ok = !flags[0] && mbar_wait(&bars[kKvEmpty + st], ((j / kStages) & 1) ^ 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) fail();
+        aborted = true;
+        continue;
+      }
+      if (lane == 0) {
+        const uint32_t kdst = sbase + kOffKV + st * kStageBytes;
+        const uint32_t vdst = kdst + kHalfStage;
+        const uint32_t bytes = nb * BS * kD * 2;
+        mbar_arrive_expect_tx(&bars[kKFull + st], bytes);
+        mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
+#pragma unroll
+        for (int b = 0; b < kBpt; ++b) {
+          if (b < nb && (pbs[b] < 0 || pbs[b] >= a.num_blocks)) {
+            raise_error(a.err, PA_DEVERR_BLOCK_ID);
+            flags[1] = 1;
+            pbs[b] = 0;  // load a valid block; the CTA's rows are written as zeros
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kBpt; ++b)
+          if (b < nb)
+            tma_load_5d(kdst + b * BS * kD * 2, &tmk, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
+                        &bars[kKFull + st]);
+#pragma unroll
+        for (int b = 0; b < kBpt; ++b)
+          if (b < nb)
+            tma_load_5d(vdst + b * BS * kD * 2, &tmv, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
+                        &bars[kVFull + st]);
+#pragma unroll
+        for (int s2 = 0; s2 < kStages; ++s2)
+          if (s2 == st) last_issued[s2] = j;
+      }
+      __syncwarp();
+    }
+    // Before the CTA can exit, every copy this warp started must have landed
+    // (an unwinding CTA's shared memory may be handed to the next CTA).
+    if (lane == 0) {
+      mbar_wait(&bars[kQFull], 0);
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) {
+        if (last_issued[s] < 0) continue;
+        const uint32_t par = (last_issued[s] / kStages) & 1;
+        if (!mbar_wait(&bars[kKFull + s], par) || !mbar_wait(&bars[kVFull + s], par)) fail();
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ======================= MMA issue ======================================
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc(TT::kFmt, 0, 0, kRows, kKeys);
+      constexpr uint32_t idesc_pv = umma_idesc(TT::kFmt, 0, 1, kRows, kD);
+      // S_t(j) = Q_t K_j^T: both operands K-major; K rows of 8-key group g at
+      // 2 KB steps (SBO), the two 64-column halves 1 KB apart
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kst = sbase + kOffKV + (j % kStages) * kStageBytes;
+        const uint32_t qst = sbase + kOffQ + t * kQBytes;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const int h = ks >> 2, kk = ks & 3;
+          const uint64_t da = umma_desc(qst + h * (kQBytes / 2) + kk * 32, 16, 1024);
+          const uint64_t db = umma_desc(kst + h * 1024 + kk * 32, 16, 2048);
+          umma(tmem + tmem_s_col(t), da, db, idesc_s, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars[kSFull + t]);
+      };
+      // O_t += P_t(j) V_j: A = P from tensor memory (16 keys in 8 columns per
+      // word kind), B = V MN-major (64-column atoms 1 KB apart, 8-key groups 2 KB)
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vst = sbase + kOffKV + (j % kStages) * kStageBytes + kHalfStage;
+#pragma unroll
+        for (int ks = 0; ks < kKeys / 16; ++ks) {
+          const uint64_t db = umma_desc(vst + ks * 4096, 1024, 2048);
+          if constexpr (TT::kSplitP) {
+            umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + ks * 16, db, idesc_pv,
+                    (j > 0 || ks > 0) ? 1u : 0u);
+            umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + ks * 16 + 8, db, idesc_pv, 1u);
+          } else {
+            umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + ks * 8, db, idesc_pv,
+                    (j > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&bars[kPvDone + t]);
+      };
+      bool ok = mbar_wait(&bars[kQFull], 0) && mbar_wait(&bars[kKFull], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (nq > 1) issue_s(1, 0);
+      } else {
+        fail();
+      }
+      for (int j = 0; ok && j < ntiles && !flags[0]; ++j) {
+        const int st = j % kStages;
+        const uint32_t par = (uint32_t)(j & 1);
+        const int jn = j + 1;
+        const bool more = jn < ntiles;
+        for (int t = 0; t < nq && ok; ++t) {
+          // P V of this Q tile (V of the stage must have landed)
+          ok = mbar_wait(&bars[kPFull + t], par) && (t > 0 || mbar_wait(&bars[kVFull + st], (j / kStages) & 1));
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          if (t == nq - 1) umma_commit(&bars[kKvEmpty + st]);  // the stage is free once these finish
+          if (more) {
+            // S(j+1) overwrites P(j) of this Q tile: its P V must be complete
+            ok = mbar_wait(&bars[kPvDone + t], par) &&
+                 (t > 0 || mbar_wait(&bars[kKFull + (jn % kStages)], (jn / kStages) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, jn);
+          }
+        }
+        if (!ok) fail();
+      }
+      umma_commit(&bars[kDone]);  // completes when every MMA above has finished
+      if (!mbar_wait(&bars[kDone], 0)) fail();
+    }
+  } else {
+    // ======================= softmax warps =================================
+    const int qt = warp >> 2, qd = warp & 3;
+    const int r = qd * 32 + lane;  // row of the Q tile = TMEM lane
+    if (qt < nq) {
+      const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+      const uint32_t ts = tmem + tmem_s_col(qt) + lane_off;
+      const uint32_t to = tmem + tmem_o_col(qt) + lane_off;
+      const int tok = qt * TPT + r / G;                     // token among the CTA's rows
+      const int limit = min(L - Q + t0 + tok, L - 1);       // last key this row may see
+      const int limit_lo = L - Q + t0 + qt * TPT;           // the tile's smallest limit
+      const float sl2 = a.scale_log2;
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < ntiles; ++j) {
+        ok = !flags[0] && mbar_wait(&bars[kSFull + qt], (uint32_t)(j & 1));
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; fail(); break; }  // tcgen05.ld is collective
+        tc_fence_after();
+        uint32_t s[kKeys];
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) {
+          uint32_t (&part)[32] = *reinterpret_cast<uint32_t (*)[32]>(&s[32 * c]);
+          tmem_ld32(ts + 32 * c, part);
+        }
+        tmem_wait_ld();
+        // causal mask (only tiles reaching past the tile's first limit), row max
+        float mx = -INFINITY;
+        const int k0 = j * kKeys;
+        if (k0 + kKeys - 1 > limit_lo) {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c) {
+            const float v = (k0 + c <= limit) ? __uint_as_float(s[c]) : -INFINITY;
+            s[c] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        }
+        mx *= sl2;
+        // lazy rescale: move the reference max only when the tile max exceeds
+        // it by more than 2^8 (first tile: always).  O_t is quiescent here: S_t(j)
+        // was issued after P V of tile j-1 completed.
+        const bool need = mx > m_used + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = m_used == -INFINITY ? 0.f : fast_exp2(m_used - mx);
+          m_used = mx;
+          l *= alpha;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(to + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(to + 32 * c, o);
+          }
+        }
+        // P = 2^(s*scale*log2e - m) over this tile's S columns
+        const float neg = -m_used;
+        float psum = 0.f;
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) {
+          uint32_t w[32];
+#pragma unroll
+          for (int g2 = 0; g2 < 2; ++g2) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int k = 32 * c + 16 * g2 + 2 * i;
+              const float p0 = fast_exp2(fmaf(__uint_as_float(s[k]), sl2, neg));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(s[k + 1]), sl2, neg));
+              psum += p0 + p1;
+              const uint32_t hi = TT::pack(p0, p1);
+              if constexpr (TT::kSplitP) {
+                // 16 keys: 8 hi words then 8 lo words (columns 16g .. 16g+15)
+                const float2 hv = TT::unpack(hi);
+                w[16 * g2 + i] = hi;
+                w[16 * g2 + 8 + i] = TT::pack(p0 - hv.x, p1 - hv.y);
+              } else {
+                w[8 * g2 + i] = hi;  // 16 keys: 8 words (columns 8g .. 8g+7)
+              }
+            }
+          }
+          if constexpr (TT::kSplitP) {
+            tmem_st32(ts + 32 * c, w);
+          } else {
+            tmem_st16(ts + 16 * c, w);
+          }
+        }
+        tmem_wait_st();
+        l += psum;
+        // keys past the context end in the sequence's last tile: zero their V
+        // rows (P is 0 there, but the slots may hold anything and 0 * NaN is
+        // NaN).  Q tile 0's warps do it before P V of either tile is issued;
+        // the stage's bytes have all landed (S(j) waited for K, and V is
+        // waited for below).
+        if (qt == 0 && (j + 1) * kKeys > L) {
+          const int st = j % kStages;
+          if (mbar_wait(&bars[kVFull + st], (uint32_t)((j / kStages) & 1))) {
+            const uint32_t vst = sbase + kOffKV + st * kStageBytes + kHalfStage;
+            const int z0 = L - j * kKeys;       // first stale key of the tile
+            const int nz = (kKeys - z0) * 16;   // 16-byte chunks over both halves
+            for (int c = r; c < nz; c += 128) {
+              const int key = z0 + c / 16, ch = c % 16;
+              const int h = ch >> 3, cc = ch & 7, kr = key & 7;
+              st_shared_v4(vst + (key >> 3) * 2048 + h * 1024 + kr * 128 + ((cc ^ kr) << 4), 0, 0, 0, 0);
+            }
+          } else {
+            fail();
+          }
+          fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+        }
+        tc_fence_before();  // the tcgen05.st of P -> the MMA thread
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kPFull + qt]);
+      }
+      // ---- epilogue: O / l -> out ----
+      const uint32_t lastp = (uint32_t)((ntiles - 1) & 1);
+      bool fin = ok && !flags[0] && ntiles > 0 && mbar_wait(&bars[kPvDone + qt], lastp);
+      fin = __all_sync(0xffffffffu, fin);
+      if (!fin && ntiles > 0) fail();
+      tc_fence_after();
+      const bool write = tok < ntok;
+      const float inv = (fin && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
+      T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * kD;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(to + 32 * c, o);
+        tmem_wait_ld();
+        if (write) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = TT::pack(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+            v.y = TT::pack(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            v.z = TT::pack(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            v.w = TT::pack(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *reinterpret_cast<uint4 *>(dst + 32 * c + i) = v;
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+template <typename T, int BS>
+cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
+  auto fn = encode_fn_tc();
+  if (!fn) return cudaErrorNotSupported;
+  const int G = a.group;
+  const int TPT = kRows / G;
+  CUtensorMap tmq, tmk, tmv;
+  {  // q viewed as [tokens][Hk][G][D]; box = TPT tokens x G heads x 64 columns
+    cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)G, (cuuint64_t)a.num_kv_heads,
+                          (cuuint64_t)a.num_q_tokens};
+    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)G * kD * 2, (cuuint64_t)a.num_heads * kD * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)TPT};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (fn(&tmq, TcType<T>::kTma, 4, const_cast<void *>(a.q), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  for (int i = 0; i < 2; ++i) {
+    // a cache viewed as [block x kv head][row group][half][8 rows][64 columns]
+    // (innermost first below): one box = one (block, kv head) tile, landing
+    // as [row group][half][8 rows][128 B]
+    cuuint64_t dims[5] = {64, 8, 2, (cuuint64_t)(BS / 8), (cuuint64_t)a.num_blocks * a.num_kv_heads};
+    cuuint64_t strides[4] = {(cuuint64_t)kD * 2, 128, (cuuint64_t)8 * kD * 2, (cuuint64_t)BS * kD * 2};
+    cuuint32_t box[5] = {64, 8, 2, (cuuint32_t)(BS / 8), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (fn(i ? &tmv : &tmk, TcType<T>::kTma, 5, const_cast<void *>(i ? a.v_cache : a.k_cache), dims,
+           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto kern = chunk_pp_kernel<T, BS>;
+  {
+    cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  // (sequence, KV head, pair of Q tiles)
+  const int tiles = (a.max_query_len + kQTiles * TPT - 1) / (kQTiles * TPT);
+  const int64_t grid = (int64_t)a.num_seqs * a.num_kv_heads * tiles;
+  if (grid == 0) return cudaSuccess;
+  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+  kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, tmq, tmk, tmv, tiles);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_pp_supported(const AttnArgs &a, int dtype) {
+  return (dtype == PA_BF16 || dtype == PA_F16) && a.head_dim == kD && a.group >= 1 &&
+         a.group <= kRows && kRows % a.group == 0 && (a.block_size == 16 || a.block_size == 32) &&
+         encode_fn_tc() != nullptr;
+}
+
+cudaError_t launch_chunk_pp(const AttnArgs &a, int dtype, cudaStream_t stream) {
+  if (dtype == PA_BF16)
+    return a.block_size == 16 ? launch_pp_t<__nv_bfloat16, 16>(a, stream)
+                              : launch_pp_t<__nv_bfloat16, 32>(a, stream);
+  return a.block_size == 16 ? launch_pp_t<__half, 16>(a, stream) : launch_pp_t<__half, 32>(a, stream);
+}
+
+}  // namespace pa

@@ -228,6 +228,11 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
         }
       }
     }
+    // the copies this warp started land before the CTA may exit
+    if (lane == 0 && !(drain_ring(full, C::STAGES, it) & drain_ring(qfull, 2, k))) {
+      if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
     return;
   }
 

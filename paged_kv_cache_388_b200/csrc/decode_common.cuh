@@ -63,18 +63,6 @@ struct BatchSmem {
   }
 };
 
-// Units a (sequence, KV head) pair weighs in the balanced partition beyond
-// its KV blocks: the fixed cost of an item (q load, cross-warp merge, output
-// store, next-item set-up) measured on B200 at 1.3-2.4 us against ~0.9 us per
-// block, so a CTA that holds many short items is given fewer blocks.
-// Measured (pa_decode, CUDA graphs): 1 / 2 / 3 / 4 units -> Llama-3-8B-shaped
-// batch 0.1700 / 0.1680 / 0.1677 / 0.1691 ms, Llama-2-7B-shaped MHA batch
-// 0.1719 / 0.1700 / 0.1681 / 0.1681 ms, parallel-sampling shared-prefix call
-// 0.1345 / 0.1266 / 0.1211 / 0.1170 ms.
-#ifndef PA_ITEM_UNITS
-#define PA_ITEM_UNITS 3
-#endif
-constexpr int kItemUnits = PA_ITEM_UNITS;
 
 // Partition units of a decode sequence (one query row, valid length) per KV
 // head: its KV blocks after the `pre` shared-prefix blocks plus kItemUnits,
@@ -82,7 +70,7 @@ constexpr int kItemUnits = PA_ITEM_UNITS;
 __device__ __forceinline__ int unit_blocks(const AttnArgs &a, int L, int qlen, int pre) {
   if (qlen != 1 || L <= 0 || L > a.max_context_len) return 0;
   const int tail = L - pre * a.block_size;
-  return tail > 0 ? ceil_div(tail, a.block_size) + kItemUnits : 0;
+  return tail > 0 ? ceil_div(tail, a.block_size) + a.item_units : 0;
 }
 
 // Shared-prefix groups -> b.pre[s], the leading KV blocks of sequence s that
@@ -212,7 +200,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs &a, const BatchSmem &
 // ---------------------------------------------------------------------------
 // Balanced partition.  The work of the launch is the concatenation, over
 // decode sequences s and then KV heads, of each (s, kvh) pair's units:
-// kItemUnits leading units that stand for the pair's fixed cost, then one
+// item_units leading units that stand for the pair's fixed cost, then one
 // unit per KV block; W = sum_s units(s) * Hk.  CTA i of G takes the flat
 // range [i*W/G, (i+1)*W/G), so every CTA carries the same cost (+-1 unit)
 // whatever the length mix; a CTA whose piece of a pair holds leading units
@@ -288,14 +276,14 @@ struct SegIter {
       }
       s = lo;
       const int nu = b.prefix[lo + 1] - b.prefix[lo];  // units per KV head (> 0 here)
-      const int nb = nu - kItemUnits;                  // KV blocks per KV head
+      const int nb = nu - a.item_units;                // KV blocks per KV head
       const int off = (int)(pos - (int64_t)b.prefix[lo] * Hk);  // < nu * Hk
       const int kvh = off / nu;
       const int u0 = off - kvh * nu;
       const int64_t left = end - pos;
       const int u1 = left < nu - u0 ? u0 + (int)left : nu;
       pos += u1 - u0;
-      const int b0 = max(0, u0 - kItemUnits), b1 = max(0, u1 - kItemUnits);
+      const int b0 = max(0, u0 - a.item_units), b1 = max(0, u1 - a.item_units);
       if (b1 == b0) continue;  // leading units only
       Item &it = seg->it;
       it.seq = a.seq_begin + lo;

@@ -343,6 +343,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
               const int row = (pb * a.num_kv_heads + item.kvh) * BS;
               const uint32_t dst = ring + slot * L::kStage;
               mbar_arrive_expect_tx(&full[slot], L::kStage);
+#ifdef PA_TEST_LOST_COPY
+              // Test build only (libpa_waittest.so): ring use PA_TEST_LOST_COPY
+              // of CTA 0 is announced on its barrier but never copied, so the
+              // consumers' wait for it expires and the CTA unwinds.
+              if (blockIdx.x == 0 && it - 1 == (uint32_t)PA_TEST_LOST_COPY) {
+              } else
+#endif
               if constexpr (F8) {  // each E4M3 tile is one contiguous run of BS * D bytes
                 const int64_t off = (int64_t)row * D;
                 bulk_load(smem + lay.ring + slot * L::kStage,
@@ -395,6 +402,11 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
       seg = nxt;
       have = have_nxt;
       if (have) have_nxt = iter.next(a, bsm, n, &nxt);
+    }
+    // the copies this warp started land before the CTA may exit
+    if (lane == 0 && !(drain_ring(full, L::kStages, it) & drain_ring(qfull, 2, k))) {
+      if (!*abort_flag) raise_error(a.err, PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
     }
     return;
   }
@@ -730,7 +742,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
       // This CTA holds the first piece of a pair cut at its range end: leave
       // the merge kernel a descriptor {record slot, kv head, last covering
       // CTA, query row}.
-      const int nu = ceil_div(item.L, a.block_size) + kItemUnits;  // the pair's units
+      const int nu = ceil_div(item.L, a.block_size) + a.item_units;  // the pair's units
       const int64_t W = (int64_t)bsm.prefix[n] * a.num_kv_heads;
       const int64_t ps = (int64_t)bsm.prefix[item.seq - a.seq_begin] * a.num_kv_heads +
                          (int64_t)item.kvh * nu;

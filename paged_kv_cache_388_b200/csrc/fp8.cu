@@ -254,6 +254,7 @@ int pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_c
   a.scale_log2 = scale * k_scale * 1.4426950408889634f;
   a.v_inv = 1.f / v_scale;
   a.balanced = 1;
+  a.item_units = kItemUnitsFp8;
   a.grid = decode_mma_grid_fp8(a, q_dtype, dev.sm_count);
   if (a.grid <= 0) return PA_ERR_CUDA;
   const size_t rec = balanced_record_bytes(a.grid, group, head_dim);

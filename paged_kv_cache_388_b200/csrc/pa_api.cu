@@ -251,6 +251,7 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
   const bool use_mma = !want_simt && !a.rows_mode && decode_mma_supported(a, dtype);
   // Balanced partition unless the caller fixed the split size.
   a.balanced = (use_mma && kv_split_tokens == 0) ? 1 : 0;
+  a.item_units = kItemUnits16;
   const int step = decode_max_seqs_per_launch();
   if (a.balanced) {
     AttnArgs probe = a;
@@ -403,6 +404,7 @@ int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const
   a.num_q_tokens = num_seqs;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.balanced = 1;
+  a.item_units = kItemUnits16;
   if (!decode_mma_supported(a, dtype) || !prefix_supported(a, dtype)) return PA_ERR_UNSUPPORTED;
   a.grid = decode_mma_grid(a, dtype, dev.sm_count);
   if (a.grid <= 0) return PA_ERR_CUDA;

@@ -14,8 +14,12 @@
 namespace pa {
 
 // Longest time any wait inside a kernel may spin before it gives up, sets
-// PA_DEVERR_TIMEOUT and unwinds (nanoseconds of %globaltimer).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// PA_DEVERR_TIMEOUT and unwinds (nanoseconds of %globaltimer).  The test
+// build of the decode kernel (libpa_waittest.so) sets a short one.
+#ifndef PA_WAIT_LIMIT_NS
+#define PA_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = PA_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -72,6 +76,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
   return true;
+}
+
+// Wait (each wait bounded) until the copies into the last `issued` uses of a
+// ring of `stages` full barriers have landed: use i of the ring is stage
+// i % stages in phase (i / stages) & 1.  A use that was only arrived on
+// (aborted or skipped) completes at once.  The issuing thread calls this
+// before its CTA may exit, so that a CTA unwinding early never leaves a bulk
+// copy in flight into shared memory that the SM may hand to the next CTA.
+// Returns false if a wait expired.
+__device__ __forceinline__ bool drain_ring(uint64_t *full, uint32_t stages, uint32_t issued) {
+  bool ok = true;
+  const uint32_t first = issued > stages ? issued - stages : 0u;
+  for (uint32_t i = first; i < issued; ++i) ok = mbar_wait(&full[i % stages], (i / stages) & 1u) && ok;
+  return ok;
 }
 
 // ---- bulk async copy global -> shared (completes on an mbarrier) ------------

@@ -38,6 +38,7 @@ struct AttnArgs {
   int rows_mode;      // 1: the decode kernel also takes rows of Q>1 sequences (one item per row)
   int balanced;       // 1: balanced flat partition (records in part_o), 0: fixed splits
   int grid;           // CTAs of the balanced launch (records are per CTA)
+  int item_units;     // balanced: units a (sequence, KV head) pair weighs beyond its blocks
   int *bal_prefix;    // balanced: [num_seqs + 1] block prefix written by CTA 0
   int *bal_desc;      // balanced: [grid][4] cut-pair descriptors written by the decode kernel
   float scale_log2;   // scale * log2(e)
@@ -55,6 +56,26 @@ struct AttnArgs {
   // scale_log2), value elements codes * v_scale; v_inv = 1 / v_scale.
   float v_inv;
 };
+
+// Units a (sequence, KV head) pair weighs in the balanced partition beyond
+// its KV blocks (AttnArgs::item_units): the fixed cost of an item (q load,
+// cross-warp merge, output store, next-item set-up) measured on B200 at
+// 1.3-2.4 us against ~0.9 us per 16-bit block, so a CTA that holds many short
+// items is given fewer blocks.  Measured (pa_decode, CUDA graphs): 1 / 2 / 3 /
+// 4 units -> Llama-3-8B-shaped batch 0.1700 / 0.1680 / 0.1677 / 0.1691 ms,
+// Llama-2-7B-shaped MHA batch 0.1719 / 0.1700 / 0.1681 / 0.1681 ms,
+// parallel-sampling shared-prefix call 0.1345 / 0.1266 / 0.1211 / 0.1170 ms.
+// An FP8 block moves half the bytes, so the same fixed cost weighs more
+// blocks: 3 -> 5 units took pa_decode_fp8 on the Llama-3-8B-shaped batch from
+// 0.1209 to 0.1163 ms.
+#ifndef PA_ITEM_UNITS
+#define PA_ITEM_UNITS 3
+#endif
+#ifndef PA_ITEM_UNITS_FP8
+#define PA_ITEM_UNITS_FP8 5
+#endif
+constexpr int kItemUnits16 = PA_ITEM_UNITS;
+constexpr int kItemUnitsFp8 = PA_ITEM_UNITS_FP8;
 
 struct DevInfo {
   int sm_count;
@@ -110,6 +131,11 @@ bool chunk_tc_supported(const AttnArgs &a, int dtype);
 cudaError_t launch_chunk_tc(const AttnArgs &a, int dtype, cudaStream_t stream);
 // The same kernel as the shared-prefix pass (group rows, records out)
 cudaError_t launch_prefix_tc(const AttnArgs &a, int dtype, cudaStream_t stream);
+
+// Implemented in chunk_pp.cu (tcgen05 chunked-query kernel, two Q tiles in
+// ping-pong over 128-key tiles; head_dim 128, 16-bit caches)
+bool chunk_pp_supported(const AttnArgs &a, int dtype);
+cudaError_t launch_chunk_pp(const AttnArgs &a, int dtype, cudaStream_t stream);
 
 // Implemented in chunk.cu
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int num_q_tokens, cudaStream_t stream);

@@ -148,6 +148,95 @@ class PagedKVCache:
                                 scale, max_context_len=max_context_len)
         return g.replay
 
+    def capture_pipelined_steps_from_host(self, steps, block_tables, scale, max_context_len=0,
+                                          warmup=2):
+        """Capture a run of decode steps fed from page-locked host memory into
+        one CUDA graph whose copies overlap the neighbouring steps' kernels.
+
+        ``steps`` is a list of dicts of pinned host tensors, one per step:
+        ``q``, ``key``, ``value``, ``slot_mapping``, ``context_lens``,
+        ``bt_index`` / ``bt_ids`` (int64 flat indices into ``block_tables``
+        and the int32 block ids to store there: the entries appended to the
+        tables since the previous step) and ``out`` (receives the attention
+        output).  ``block_tables`` is the device-resident table, updated in
+        place by every step.
+
+        Step i copies its inputs in on a host-to-device stream while step i-1
+        computes, runs reshape_and_cache + decode on the current stream, and
+        copies its output back on a device-to-host stream while step i+1
+        computes; two device staging sets alternate between the steps.
+        Returns a callable that replays the whole run."""
+        if not steps:
+            raise ValueError("no steps")
+        dev = self.device
+        names = ("q", "key", "value", "slot_mapping", "context_lens", "bt_index", "bt_ids")
+        stage = [{n: torch.empty(steps[0][n].shape, dtype=steps[0][n].dtype, device=dev)
+                  for n in names} for _ in range(2)]
+        outs = [torch.empty(steps[0]["out"].shape, dtype=steps[0]["out"].dtype, device=dev)
+                for _ in range(2)]
+        flat_bt = block_tables.view(-1)
+        mcl = max_context_len or block_tables.shape[1] * self.block_size
+        h2d = torch.cuda.Stream(device=dev)
+        d2h = torch.cuda.Stream(device=dev)
+
+        def run():
+            main = torch.cuda.current_stream(dev)
+            ev_k, ev_out = [], []
+            h2d.wait_stream(main)
+            d2h.wait_stream(main)
+            for i, st in enumerate(steps):
+                sb, ob = stage[i % 2], outs[i % 2]
+                if i >= 2:  # the staging set's previous user has finished its kernels
+                    h2d.wait_event(ev_k[i - 2])
+                with torch.cuda.stream(h2d):
+                    for n in names:
+                        sb[n].copy_(st[n], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(h2d)
+                main.wait_event(ev_in)
+                if i >= 2:  # its output buffer has been copied out
+                    main.wait_event(ev_out[i - 2])
+                flat_bt.index_copy_(0, sb["bt_index"], sb["bt_ids"])
+                self.write(sb["key"], sb["value"], sb["slot_mapping"])
+                self.attend(sb["q"], block_tables, sb["context_lens"], scale, out=ob,
+                            max_context_len=mcl)
+                ev = torch.cuda.Event()
+                ev.record(main)
+                ev_k.append(ev)
+                d2h.wait_event(ev)
+                with torch.cuda.stream(d2h):
+                    st["out"].copy_(ob, non_blocking=True)
+                eo = torch.cuda.Event()
+                eo.record(d2h)
+                ev_out.append(eo)
+            main.wait_stream(h2d)
+            main.wait_stream(d2h)
+
+        for _ in range(warmup):  # one-time library set-up happens outside capture
+            run()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        return g.replay
+
+    @staticmethod
+    def appended_table_entries(block_tables, context_lens, block_size, new_tokens=1):
+        """Flat indices into ``block_tables`` and the ids stored there for the
+        blocks that this step's last ``new_tokens`` tokens of each sequence
+        opened (a token at offset 0 of a block): what a decode step has to send
+        to a device-resident table."""
+        import numpy as np
+        idx, ids = [], []
+        width = block_tables.shape[1]
+        for i, L in enumerate(np.asarray(context_lens).tolist()):
+            for pos in range(max(0, L - new_tokens), L):
+                if pos % block_size == 0:
+                    b = pos // block_size
+                    idx.append(i * width + b)
+                    ids.append(int(block_tables[i, b]))
+        return (torch.tensor(idx, dtype=torch.int64), torch.tensor(ids, dtype=torch.int32))
+
     @staticmethod
     def host_bytes(*tensors) -> int:
         return int(sum(t.numel() * t.element_size() for t in tensors))

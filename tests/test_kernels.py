@@ -47,14 +47,15 @@ def decode_kernel(request, monkeypatch):
     return request.param
 
 
-@pytest.fixture(params=["auto", "mma"])
+@pytest.fixture(params=["auto", "tc64", "mma"])
 def chunk_kernel(request, monkeypatch):
-    """Chunked-query rows through the default kernel (tcgen05 at head_dim 128)
-    and through the mma.sync kernel forced."""
-    if request.param == "mma":
-        monkeypatch.setenv("PA_CHUNK_KERNEL", "mma")
-    else:
+    """Chunked-query rows through the default kernel (tcgen05 ping-pong over
+    128-key tiles at head_dim 128), through the tcgen05 kernel over 64-key
+    tiles and through the mma.sync kernel."""
+    if request.param == "auto":
         monkeypatch.delenv("PA_CHUNK_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("PA_CHUNK_KERNEL", request.param)
     return request.param
 
 

@@ -50,7 +50,7 @@ def _noalloc(lib, wl, b, d, split):
 
 
 @pytest.mark.parametrize("cfg,split,stale_cfg,stale_split",
-                         [("3s", 0, "4s", 64), ("3s32", 0, "3s", 16), ("4s", 64, "3s32", 0),
+                         [("3s", 0, "4s", 64), ("3s32", 0, "3s", 64), ("4s", 64, "3s32", 0),
                           ("g16", 0, "3s", 0)])
 def test_noalloc_matches_oracle_and_pa_decode_twice(cfg, split, stale_cfg, stale_split):
     from paged_kv_cache_388_b200 import _lib
