@@ -30,6 +30,16 @@
 //
 // Warps: 8 softmax (4 per Q tile; thread = row = TMEM lane), 1 TMA producer,
 // 1 MMA issuer (one elected thread) that also owns the TMEM allocation.
+//
+// PREFIX: the shared-prefix pass of pa_decode_shared_prefix.  The CTA is
+// (group, up to 256 member rows, KV head): its rows are the decode rows of
+// the group's members (one query row per sequence, 128/GROUP members per Q
+// tile), its keys the group's shared blocks read through the group's first
+// table, with no causal mask; the softmax warps check every member's table
+// over the shared range while the first tile loads, and the epilogue writes
+// one record (o unnormalised, reference max in base 2, sum; NaN sum for a
+// member whose table differs) per (member, head) for the decode kernel to
+// fold in.
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "tc_common.cuh"
@@ -56,7 +66,8 @@ constexpr int kOffQ = 0;
 constexpr int kHalfStage = kKeys * kD * 2;        // K (or V) of one tile: 32 KB
 constexpr int kStageBytes = 2 * kHalfStage;
 constexpr int kOffKV = kOffQ + kQTiles * kQBytes;
-constexpr int kOffBar = kOffKV + kStages * kStageBytes;
+constexpr int kOffMemBad = kOffKV + kStages * kStageBytes;  // prefix mode: [256] member flags
+constexpr int kOffBar = kOffMemBad + 256;
 enum {
   kQFull = 0,
   kKFull = 1,                      // [kStages] the K half of a stage landed
@@ -75,7 +86,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 __device__ __forceinline__ uint32_t tmem_s_col(int t) { return (uint32_t)t * 256u; }
 __device__ __forceinline__ uint32_t tmem_o_col(int t) { return (uint32_t)t * 256u + 128u; }
 
-template <typename T, int BS>
+template <typename T, int BS, bool PREFIX>
 __global__ void __maxnreg__(200)
     chunk_pp_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -92,35 +103,53 @@ __global__ void __maxnreg__(200)
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- the CTA's rows: tokens t0 .. t0 + ntok - 1 of the sequence's chunk --
+  // (prefix mode: members q0 .. q0 + ntok - 1 of the group, one row each)
   const int G = a.group;
-  const int TPT = kRows / G;  // tokens per Q tile
+  const int TPT = kRows / G;  // tokens (members) per Q tile
   const int tile = blockIdx.x % tiles_per_seq;
   const int rest = blockIdx.x / tiles_per_seq;
   const int kvh = rest % a.num_kv_heads;
-  const int seq = a.seq_begin + rest / a.num_kv_heads;
-  const int q0 = a.query_start_loc[seq];
-  const int Q = a.query_start_loc[seq + 1] - q0;
-  if (Q <= 1 || q0 < 0 || q0 + Q > a.num_q_tokens) return;  // CTA-uniform exits, before any barrier
-  if (Q > a.max_query_len) {
-    if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
-    return;
-  }
-  const int t0 = tile * kQTiles * TPT;
-  if (t0 >= Q) return;
-  const int ntok = min(kQTiles * TPT, Q - t0);
-  const int nq = ntok > TPT ? 2 : 1;  // Q tiles holding rows of this chunk
-  const int L = a.context_lens[seq];
-  if (L < Q || L > a.max_context_len) {
-    if (tid == 0 && tile == 0 && kvh == 0)
-      raise_error(a.err, (L < 0 || L > a.max_context_len) ? PA_DEVERR_CONTEXT_LEN : PA_DEVERR_QUERY_LEN);
-    for (int idx = tid; idx < ntok * G * kD; idx += blockDim.x) {
-      const int r = idx / kD, dd = idx - r * kD;
-      static_cast<T *>(a.out)[((int64_t)(q0 + t0 + r / G) * a.num_heads + kvh * G + r % G) * kD + dd] =
-          Elem<T>::from_f(0.f);
+  int seq, q0, Q, t0, ntok, L;
+  if constexpr (PREFIX) {
+    const int jg = rest / a.num_kv_heads;
+    const int s0 = a.grp_start[jg], s1 = a.grp_start[jg + 1], P = a.grp_blocks[jg];
+    const int m0 = s0 + tile * kQTiles * TPT;
+    // CTA-uniform exits, before any barrier (malformed groups are reported by the decode kernel)
+    if (!(0 <= s0 && s0 <= s1 && s1 <= a.num_seqs && 0 < P && P <= a.max_blocks_per_seq && m0 < s1))
+      return;
+    seq = s0;  // the group's first sequence: its table holds the shared blocks
+    q0 = m0;   // one decode row per member: q row = sequence index
+    Q = 1;     // with t0 = 0 every row sees keys 0 .. L-1 (no causal mask)
+    t0 = 0;
+    ntok = min(kQTiles * TPT, s1 - m0);
+    L = P * BS;
+  } else {
+    seq = a.seq_begin + rest / a.num_kv_heads;
+    q0 = a.query_start_loc[seq];
+    Q = a.query_start_loc[seq + 1] - q0;
+    if (Q <= 1 || q0 < 0 || q0 + Q > a.num_q_tokens) return;  // CTA-uniform exits, before any barrier
+    if (Q > a.max_query_len) {
+      if (tid == 0 && tile == 0) raise_error(a.err, PA_DEVERR_QUERY_LEN);
+      return;
     }
-    return;
+    t0 = tile * kQTiles * TPT;
+    if (t0 >= Q) return;
+    ntok = min(kQTiles * TPT, Q - t0);
+    L = a.context_lens[seq];
+    if (L < Q || L > a.max_context_len) {
+      if (tid == 0 && tile == 0 && kvh == 0)
+        raise_error(a.err, (L < 0 || L > a.max_context_len) ? PA_DEVERR_CONTEXT_LEN : PA_DEVERR_QUERY_LEN);
+      for (int idx = tid; idx < ntok * G * kD; idx += blockDim.x) {
+        const int r = idx / kD, dd = idx - r * kD;
+        static_cast<T *>(a.out)[((int64_t)(q0 + t0 + r / G) * a.num_heads + kvh * G + r % G) * kD + dd] =
+            Elem<T>::from_f(0.f);
+      }
+      return;
+    }
   }
+  const int nq = ntok > TPT ? 2 : 1;   // Q tiles holding rows of this CTA
   const int kend = L - Q + t0 + ntok;  // keys [0, kend) are visible to some row
+  volatile unsigned char *bad_member = smem + kOffMemBad;
   const int ntiles = (kend + kKeys - 1) / kKeys;
   const int nblk = (L + BS - 1) / BS;
 
@@ -140,6 +169,8 @@ __global__ void __maxnreg__(200)
     mbar_init(&bars[kDone], 1);
     flags[0] = 0;
     flags[1] = 0;
+    if constexpr (PREFIX)
+      for (int i = 0; i < kQTiles * kRows; ++i) bad_member[i] = 0;
     mbar_init_fence();
   }
   if (warp == kMmaWarp) {
@@ -323,6 +354,33 @@ __global__ void __maxnreg__(200)
       const int limit = min(L - Q + t0 + tok, L - 1);       // last key this row may see
       const int limit_lo = L - Q + t0 + qt * TPT;           // the tile's smallest limit
       const float sl2 = a.scale_log2;
+      if constexpr (PREFIX) {
+        // Every member's table must hold the group's ids over the shared
+        // range.  All of the checks' loads are issued together here, while the
+        // first tile is in flight, instead of one dependent round trip per tile.
+        const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
+        const int sid = qt * kRows + r;  // 0 .. nq*128 - 1
+        const int nth = nq * kRows;
+        for (int x0 = sid; x0 < ntok * nblk; x0 += nth * 8) {
+          int mine[8], ref[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int x = x0 + u * nth;
+            const int i = x / nblk, b = x - i * nblk;
+            mine[u] = x < ntok * nblk ? a.block_tables[(int64_t)(q0 + i) * a.max_blocks_per_seq + b] : 0;
+            ref[u] = x < ntok * nblk ? table[b] : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int x = x0 + u * nth;
+            if (x < ntok * nblk && mine[u] != ref[u]) {
+              const int i = x / nblk;
+              if (!bad_member[i]) raise_error(a.err, PA_DEVERR_PREFIX);
+              bad_member[i] = 1;
+            }
+          }
+        }
+      }
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < ntiles; ++j) {
@@ -437,6 +495,32 @@ __global__ void __maxnreg__(200)
       if (!fin && ntiles > 0) fail();
       tc_fence_after();
       const bool write = tok < ntok;
+      if constexpr (PREFIX) {
+        // the member flags of every active softmax warp (named barrier 1)
+        named_sync(1, nq * kRows);
+        // record of (member q0 + tok, head): o unnormalised, the reference max
+        // (base 2) o and l are relative to, l; NaN l marks a poisoned record
+        const bool poison = !fin || flags[1] || (write && bad_member[tok]);
+        float *rec = a.pre_rec + ((int64_t)(q0 + tok) * a.num_heads + kvh * G + r % G) * (kD + 4);
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(to + 32 * c, o);
+          tmem_wait_ld();
+          if (write) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4 *>(rec + 32 * c + i) =
+                  make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]), __uint_as_float(o[i + 2]),
+                              __uint_as_float(o[i + 3]));
+          }
+        }
+        if (write) {
+          rec[kD] = m_used;
+          rec[kD + 1] = poison ? __int_as_float(0x7fc00000) : l;
+        }
+        tc_fence_before();
+      } else {
       const float inv = (fin && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
       T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * kD;
 #pragma unroll 1
@@ -457,6 +541,7 @@ __global__ void __maxnreg__(200)
         }
       }
       tc_fence_before();
+      }
     }
   }
   __syncthreads();
@@ -467,7 +552,7 @@ __global__ void __maxnreg__(200)
   }
 }
 
-template <typename T, int BS>
+template <typename T, int BS, bool PREFIX>
 cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
   auto fn = encode_fn_tc();
   if (!fn) return cudaErrorNotSupported;
@@ -498,14 +583,16 @@ cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = chunk_pp_kernel<T, BS>;
+  auto kern = chunk_pp_kernel<T, BS, PREFIX>;
   {
     cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmemBytes);
     if (e != cudaSuccess) return e;
   }
-  // (sequence, KV head, pair of Q tiles)
-  const int tiles = (a.max_query_len + kQTiles * TPT - 1) / (kQTiles * TPT);
-  const int64_t grid = (int64_t)a.num_seqs * a.num_kv_heads * tiles;
+  // chunk rows: (sequence, KV head, pair of Q tiles); prefix: (group, KV
+  // head, pair of member tiles)
+  const int rows = PREFIX ? a.max_group : a.max_query_len;
+  const int tiles = (rows + kQTiles * TPT - 1) / (kQTiles * TPT);
+  const int64_t grid = (int64_t)(PREFIX ? a.num_groups : a.num_seqs) * a.num_kv_heads * tiles;
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
   kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, tmq, tmk, tmv, tiles);
@@ -522,9 +609,18 @@ bool chunk_pp_supported(const AttnArgs &a, int dtype) {
 
 cudaError_t launch_chunk_pp(const AttnArgs &a, int dtype, cudaStream_t stream) {
   if (dtype == PA_BF16)
-    return a.block_size == 16 ? launch_pp_t<__nv_bfloat16, 16>(a, stream)
-                              : launch_pp_t<__nv_bfloat16, 32>(a, stream);
-  return a.block_size == 16 ? launch_pp_t<__half, 16>(a, stream) : launch_pp_t<__half, 32>(a, stream);
+    return a.block_size == 16 ? launch_pp_t<__nv_bfloat16, 16, false>(a, stream)
+                              : launch_pp_t<__nv_bfloat16, 32, false>(a, stream);
+  return a.block_size == 16 ? launch_pp_t<__half, 16, false>(a, stream)
+                            : launch_pp_t<__half, 32, false>(a, stream);
+}
+
+cudaError_t launch_prefix_pp(const AttnArgs &a, int dtype, cudaStream_t stream) {
+  if (dtype == PA_BF16)
+    return a.block_size == 16 ? launch_pp_t<__nv_bfloat16, 16, true>(a, stream)
+                              : launch_pp_t<__nv_bfloat16, 32, true>(a, stream);
+  return a.block_size == 16 ? launch_pp_t<__half, 16, true>(a, stream)
+                            : launch_pp_t<__half, 32, true>(a, stream);
 }
 
 }  // namespace pa

@@ -427,11 +427,15 @@ int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const
   cudaError_t e = cudaSuccess;
   if (num_groups > 0) {
     // the shared blocks on the 5th-generation tensor cores (head_dim 128,
-    // group dividing 128) unless PA_PREFIX_KERNEL=mma asks for the mma.sync
-    // cluster kernel, which serves every other shape
+    // group dividing 128): the ping-pong kernel over 128-key tiles, or with
+    // PA_PREFIX_KERNEL=tc64 the earlier one over 64-key tiles; PA_PREFIX_KERNEL=mma
+    // asks for the mma.sync cluster kernel, which serves every other shape
     const char *sel = getenv("PA_PREFIX_KERNEL");
     const bool want_mma = sel && strcmp(sel, "mma") == 0;
-    if (!want_mma && chunk_tc_supported(a, dtype)) {
+    const bool want_tc64 = sel && strcmp(sel, "tc64") == 0;
+    if (!want_mma && !want_tc64 && chunk_pp_supported(a, dtype)) {
+      e = launch_prefix_pp(a, dtype, s);
+    } else if (!want_mma && chunk_tc_supported(a, dtype)) {
       e = launch_prefix_tc(a, dtype, s);
     } else {
       const int64_t units = (int64_t)num_groups * a.grp_chunks * num_kv_heads;

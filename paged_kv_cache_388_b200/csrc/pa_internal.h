@@ -136,6 +136,9 @@ cudaError_t launch_prefix_tc(const AttnArgs &a, int dtype, cudaStream_t stream);
 // ping-pong over 128-key tiles; head_dim 128, 16-bit caches)
 bool chunk_pp_supported(const AttnArgs &a, int dtype);
 cudaError_t launch_chunk_pp(const AttnArgs &a, int dtype, cudaStream_t stream);
+// The same kernel as the shared-prefix pass (member rows of a group over the
+// group's shared blocks, records out; uses a.max_group and a.num_groups)
+cudaError_t launch_prefix_pp(const AttnArgs &a, int dtype, cudaStream_t stream);
 
 // Implemented in chunk.cu
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int num_q_tokens, cudaStream_t stream);

@@ -67,6 +67,18 @@ def _plain(lib, wl, batch, d):
     return out
 
 
+@pytest.fixture(params=["auto", "tc64", "mma"])
+def prefix_kernel(request, monkeypatch):
+    """The shared-prefix pass through the default kernel (tcgen05 ping-pong over
+    128-key tiles at head_dim 128), the tcgen05 kernel over 64-key tiles and
+    the mma.sync cluster kernel."""
+    if request.param == "auto":
+        monkeypatch.delenv("PA_PREFIX_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("PA_PREFIX_KERNEL", request.param)
+    return request.param
+
+
 def _run(lib, wl, rows=None):
     vals = workloads.values(wl)
     batch = build_batch(wl)
@@ -83,7 +95,7 @@ def _run(lib, wl, rows=None):
 
 
 @pytest.mark.parametrize("cfg", ["4s", "4cows"])
-def test_small_configs(lib, cfg):
+def test_small_configs(lib, prefix_kernel, cfg):
     _run(lib, workloads.make(cfg))
 
 
@@ -109,7 +121,7 @@ def test_agrees_with_plain_decode(lib):
     (64, 8, 128, 32, "bf16", 11),   # 11 samples of group 8 -> chunks of 8 and 3
     (24, 8, 128, 16, "f16", 7),     # group 3: 21 members per tile, 63 rows
 ])
-def test_shapes(lib, H, Hk, D, bs, dtype, samples):
+def test_shapes(lib, prefix_kernel, H, Hk, D, bs, dtype, samples):
     wl = workloads.shared_prefix_workload(f"sp_{H}_{Hk}_{D}_{bs}_{dtype}_{samples}", 4100 + H + bs,
                                           3, samples, 5 * bs + 3, 3 * bs, H, Hk, D, bs, dtype)
     _run(lib, wl)
@@ -139,7 +151,7 @@ def _ref(wl, qn, kp, vp, bt, cl):
                          wl.scale, wl.dtype)
 
 
-def test_member_with_only_shared_keys(lib):
+def test_member_with_only_shared_keys(lib, prefix_kernel):
     wl, batch, d, kp, vp, qn = _setup(lib)
     gs, gb, mg = _groups(batch, wl.block_size)
     p = int(gb[0])
@@ -173,7 +185,7 @@ def test_no_groups_is_plain_decode(lib):
                  what="no groups")
 
 
-def test_member_table_mismatch(lib):
+def test_member_table_mismatch(lib, prefix_kernel):
     wl, batch, d, kp, vp, qn = _setup(lib)
     gs, gb, mg = _groups(batch, wl.block_size)
     bt = batch.block_tables.copy()
@@ -186,7 +198,7 @@ def test_member_table_mismatch(lib):
     assert_close(out, ref, wl.dtype, rows=keep, what="other members")
 
 
-def test_context_shorter_than_prefix(lib):
+def test_context_shorter_than_prefix(lib, prefix_kernel):
     wl, batch, d, kp, vp, qn = _setup(lib)
     gs, gb, mg = _groups(batch, wl.block_size)
     cl = batch.context_lens.copy()
@@ -199,7 +211,7 @@ def test_context_shorter_than_prefix(lib):
                  what="other members")
 
 
-def test_bad_block_id_in_shared_range(lib):
+def test_bad_block_id_in_shared_range(lib, prefix_kernel):
     wl, batch, d, kp, vp, qn = _setup(lib)
     gs, gb, mg = _groups(batch, wl.block_size)
     bt = batch.block_tables.copy()
