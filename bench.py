@@ -59,7 +59,7 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
-FLUSH_BYTES = 256 * 2 ** 20          # >= 2x L2: a memset of this evicts every cached line
+FLUSH_BYTES = 256 * 2 ** 20          # >= 2x L2: reading this evicts every cached line
 EXTRA_CONFIGS = ("2", "3fp8", "4", "4cow", "5", "5bs32", "1")
 
 
@@ -307,7 +307,9 @@ class Timer:
                for _ in range(iters)]
         torch.cuda.synchronize(self.dev)
         for e0, e1 in evs:
-            self._flush.zero_()  # ~40-80 us on the device: the replay below is enqueued meanwhile
+            # a read of FLUSH_BYTES evicts the L2 and leaves no dirty line to be
+            # written back inside the timed call (~40 us; the replay is enqueued meanwhile)
+            torch.amax(self._flush)
             e0.record(self.stream)
             g.replay()
             e1.record(self.stream)
@@ -488,6 +490,10 @@ def measure_config(db, timer, k):
                               "bf16 tensor peak)", "tensor_peak_TFLOPs": tc,
                               "tensor_peak_kind": tc_kind,
                               "frac": bound_ms / call["median_ms"]}
+    # one whole step last, so that db.out is the step's output on the step's
+    # cache (the lone copy_blocks / write timings above left other contents)
+    db.step()
+    torch.cuda.synchronize(db.dev)
     return res
 
 

@@ -40,6 +40,9 @@
 // one record (o unnormalised, reference max in base 2, sum; NaN sum for a
 // member whose table differs) per (member, head) for the decode kernel to
 // fold in.
+#include <stdlib.h>
+#include <string.h>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "tc_common.cuh"
@@ -87,10 +90,10 @@ __device__ __forceinline__ uint32_t tmem_s_col(int t) { return (uint32_t)t * 256
 __device__ __forceinline__ uint32_t tmem_o_col(int t) { return (uint32_t)t * 256u + 128u; }
 
 template <typename T, int BS, bool PREFIX>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     chunk_pp_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                    int tiles_per_seq) {
+                    int tiles_per_seq, int five_d) {
   using TT = TcType<T>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -100,6 +103,11 @@ __global__ void __maxnreg__(200)
   volatile int *flags = reinterpret_cast<volatile int *>(tmem_slot + 1);  // [0] abort, [1] bad block
   const uint32_t sbase = smem_addr(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // K/V stage layout: key k, 64-column half h at (k / 8) * GS + h * HS + (k % 8) * 128.
+  // 5-D boxes: [8-key group][half][8 rows] (GS 2 KB, HS 1 KB); 2-D boxes (one
+  // per block and half): [half][key] (GS 1 KB, HS 16 KB).
+  const uint32_t GS = five_d ? 2048u : 1024u;
+  const uint32_t HS = five_d ? 1024u : (uint32_t)(kKeys * 128);
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- the CTA's rows: tokens t0 .. t0 + ntok - 1 of the sequence's chunk --
@@ -244,16 +252,33 @@ __global__ void __maxnreg__(200)
             pbs[b] = 0;  // load a valid block; the CTA's rows are written as zeros
           }
         }
+        if (five_d) {
 #pragma unroll
-        for (int b = 0; b < kBpt; ++b)
-          if (b < nb)
-            tma_load_5d(kdst + b * BS * kD * 2, &tmk, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
-                        &bars[kKFull + st]);
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb)
+              tma_load_5d(kdst + b * BS * kD * 2, &tmk, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
+                          &bars[kKFull + st]);
 #pragma unroll
-        for (int b = 0; b < kBpt; ++b)
-          if (b < nb)
-            tma_load_5d(vdst + b * BS * kD * 2, &tmv, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
-                        &bars[kVFull + st]);
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb)
+              tma_load_5d(vdst + b * BS * kD * 2, &tmv, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
+                          &bars[kVFull + st]);
+        } else {
+#pragma unroll
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb) {
+              const int row = (pbs[b] * a.num_kv_heads + kvh) * BS;
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(kdst + h * HS + b * BS * 128, &tmk, h * 64, row, &bars[kKFull + st]);
+            }
+#pragma unroll
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb) {
+              const int row = (pbs[b] * a.num_kv_heads + kvh) * BS;
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(vdst + h * HS + b * BS * 128, &tmv, h * 64, row, &bars[kVFull + st]);
+            }
+        }
 #pragma unroll
         for (int s2 = 0; s2 < kStages; ++s2)
           if (s2 == st) last_issued[s2] = j;
@@ -277,7 +302,7 @@ __global__ void __maxnreg__(200)
       constexpr uint32_t idesc_s = umma_idesc(TT::kFmt, 0, 0, kRows, kKeys);
       constexpr uint32_t idesc_pv = umma_idesc(TT::kFmt, 0, 1, kRows, kD);
       // S_t(j) = Q_t K_j^T: both operands K-major; K rows of 8-key group g at
-      // 2 KB steps (SBO), the two 64-column halves 1 KB apart
+      // GS steps (SBO), the two 64-column halves HS apart
       auto issue_s = [&](int t, int j) {
         const uint32_t kst = sbase + kOffKV + (j % kStages) * kStageBytes;
         const uint32_t qst = sbase + kOffQ + t * kQBytes;
@@ -285,18 +310,18 @@ __global__ void __maxnreg__(200)
         for (int ks = 0; ks < kD / 16; ++ks) {
           const int h = ks >> 2, kk = ks & 3;
           const uint64_t da = umma_desc(qst + h * (kQBytes / 2) + kk * 32, 16, 1024);
-          const uint64_t db = umma_desc(kst + h * 1024 + kk * 32, 16, 2048);
+          const uint64_t db = umma_desc(kst + h * HS + kk * 32, 16, GS);
           umma(tmem + tmem_s_col(t), da, db, idesc_s, ks > 0 ? 1u : 0u);
         }
         umma_commit(&bars[kSFull + t]);
       };
       // O_t += P_t(j) V_j: A = P from tensor memory (16 keys in 8 columns per
-      // word kind), B = V MN-major (64-column atoms 1 KB apart, 8-key groups 2 KB)
+      // word kind), B = V MN-major (64-column atoms HS apart, 8-key groups GS)
       auto issue_pv = [&](int t, int j) {
         const uint32_t vst = sbase + kOffKV + (j % kStages) * kStageBytes + kHalfStage;
 #pragma unroll
         for (int ks = 0; ks < kKeys / 16; ++ks) {
-          const uint64_t db = umma_desc(vst + ks * 4096, 1024, 2048);
+          const uint64_t db = umma_desc(vst + ks * 2 * GS, HS, GS);
           if constexpr (TT::kSplitP) {
             umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + ks * 16, db, idesc_pv,
                     (j > 0 || ks > 0) ? 1u : 0u);
@@ -387,26 +412,29 @@ __global__ void __maxnreg__(200)
         ok = !flags[0] && mbar_wait(&bars[kSFull + qt], (uint32_t)(j & 1));
         if (!__all_sync(0xffffffffu, ok)) { ok = false; fail(); break; }  // tcgen05.ld is collective
         tc_fence_after();
-        uint32_t s[kKeys];
-#pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) {
-          uint32_t (&part)[32] = *reinterpret_cast<uint32_t (*)[32]>(&s[32 * c]);
-          tmem_ld32(ts + 32 * c, part);
-        }
-        tmem_wait_ld();
-        // causal mask (only tiles reaching past the tile's first limit), row max
-        float mx = -INFINITY;
+        // Pass 1: row max over the tile's S columns, 32 at a time (the next
+        // chunk's load is in flight while this one is reduced).  Keys past
+        // the row's causal limit are masked (only in tiles reaching past the
+        // Q tile's smallest limit).
         const int k0 = j * kKeys;
-        if (k0 + kKeys - 1 > limit_lo) {
+        const bool masked = k0 + kKeys - 1 > limit_lo;
+        float mx = -INFINITY;
+        {
+          uint32_t ca[32], cb[32];
+          tmem_ld32(ts, ca);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kKeys; ++c) {
-            const float v = (k0 + c <= limit) ? __uint_as_float(s[c]) : -INFINITY;
-            s[c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
+          for (int c = 0; c < kKeys / 32; ++c) {
+            uint32_t (&cur)[32] = (c & 1) ? cb : ca;
+            uint32_t (&nxt)[32] = (c & 1) ? ca : cb;
+            if (c + 1 < kKeys / 32) tmem_ld32(ts + 32 * (c + 1), nxt);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float v = (!masked || k0 + 32 * c + i <= limit) ? __uint_as_float(cur[i]) : -INFINITY;
+              mx = fmaxf(mx, v);
+            }
+            tmem_wait_ld();
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
         }
         mx *= sl2;
         // lazy rescale: move the reference max only when the tile max exceeds
@@ -430,35 +458,42 @@ __global__ void __maxnreg__(200)
             tmem_st32(to + 32 * c, o);
           }
         }
-        // P = 2^(s*scale*log2e - m) over this tile's S columns
+        // Pass 2: P = 2^(s*scale*log2e - m), chunk by chunk over the same
+        // columns; chunk c's P words go over S columns the pass has already
+        // read (bf16: [32c, 32c+32), fp16: [16c, 16c+16)).
         const float neg = -m_used;
         float psum = 0.f;
+        {
+#pragma unroll 1
+          for (int c = 0; c < kKeys / 32; ++c) {
+            uint32_t cur[32];
+            tmem_ld32(ts + 32 * c, cur);
+            tmem_wait_ld();
+            uint32_t w[16];
 #pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) {
-          uint32_t w[32];
+            for (int g2 = 0; g2 < 2; ++g2) {
 #pragma unroll
-          for (int g2 = 0; g2 < 2; ++g2) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int k = 32 * c + 16 * g2 + 2 * i;
-              const float p0 = fast_exp2(fmaf(__uint_as_float(s[k]), sl2, neg));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(s[k + 1]), sl2, neg));
-              psum += p0 + p1;
-              const uint32_t hi = TT::pack(p0, p1);
-              if constexpr (TT::kSplitP) {
-                // 16 keys: 8 hi words then 8 lo words (columns 16g .. 16g+15)
-                const float2 hv = TT::unpack(hi);
-                w[16 * g2 + i] = hi;
-                w[16 * g2 + 8 + i] = TT::pack(p0 - hv.x, p1 - hv.y);
-              } else {
-                w[8 * g2 + i] = hi;  // 16 keys: 8 words (columns 8g .. 8g+7)
+              for (int i = 0; i < 8; ++i) {
+                const int kk = 16 * g2 + 2 * i;  // key within the chunk
+                const int key = k0 + 32 * c + kk;
+                const float x0 = (!masked || key <= limit) ? __uint_as_float(cur[kk]) : -INFINITY;
+                const float x1 = (!masked || key + 1 <= limit) ? __uint_as_float(cur[kk + 1]) : -INFINITY;
+                const float p0 = fast_exp2(fmaf(x0, sl2, neg));
+                const float p1 = fast_exp2(fmaf(x1, sl2, neg));
+                psum += p0 + p1;
+                const uint32_t hi = TT::pack(p0, p1);
+                if constexpr (TT::kSplitP) {
+                  // 16 keys: 8 hi words then 8 lo words (columns 16g .. 16g+15)
+                  const float2 hv = TT::unpack(hi);
+                  w[i] = hi;
+                  w[8 + i] = TT::pack(p0 - hv.x, p1 - hv.y);
+                } else {
+                  w[8 * g2 + i] = hi;  // 16 keys: 8 words (columns 8g .. 8g+7)
+                }
               }
+              if constexpr (TT::kSplitP) tmem_st16(ts + 32 * c + 16 * g2, w);
             }
-          }
-          if constexpr (TT::kSplitP) {
-            tmem_st32(ts + 32 * c, w);
-          } else {
-            tmem_st16(ts + 16 * c, w);
+            if constexpr (!TT::kSplitP) tmem_st16(ts + 16 * c, w);
           }
         }
         tmem_wait_st();
@@ -477,7 +512,7 @@ __global__ void __maxnreg__(200)
             for (int c = r; c < nz; c += 128) {
               const int key = z0 + c / 16, ch = c % 16;
               const int h = ch >> 3, cc = ch & 7, kr = key & 7;
-              st_shared_v4(vst + (key >> 3) * 2048 + h * 1024 + kr * 128 + ((cc ^ kr) << 4), 0, 0, 0, 0);
+              st_shared_v4(vst + (key >> 3) * GS + h * HS + kr * 128 + ((cc ^ kr) << 4), 0, 0, 0, 0);
             }
           } else {
             fail();
@@ -565,12 +600,24 @@ cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)G * kD * 2, (cuuint64_t)a.num_heads * kD * 2};
     cuuint32_t box[4] = {64, (cuuint32_t)G, 1, (cuuint32_t)TPT};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (fn(&tmq, TcType<T>::kTma, 4, const_cast<void *>(a.q), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    const CUresult r = fn(&tmq, TcType<T>::kTma, 4, const_cast<void *>(a.q), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      debug_log("chunk_pp: Q tensor map refused (CUresult %d)", (int)r);
       return cudaErrorInvalidValue;
+    }
   }
-  for (int i = 0; i < 2; ++i) {
+  // K/V: one box per (block, KV head) through a 5-D view whose half-of-row
+  // dimension sits between the rows and the 8-row groups (when asked for and
+  // the driver accepts the view), else two 2-D boxes per block (one per
+  // 64-column half).
+  // Two 2-D boxes per block unless PA_CHUNK_PP_BOXES=5d: on the long mixed
+  // batch the whole call measured 1.382 ms with two boxes and 1.393 ms with
+  // one -- the box rate does not bound this kernel.
+  const char *boxes = getenv("PA_CHUNK_PP_BOXES");
+  int five_d = (boxes && strcmp(boxes, "5d") == 0) ? 1 : 0;
+  for (int i = 0; i < 2 && five_d; ++i) {
     // a cache viewed as [block x kv head][row group][half][8 rows][64 columns]
     // (innermost first below): one box = one (block, kv head) tile, landing
     // as [row group][half][8 rows][128 B]
@@ -578,15 +625,38 @@ cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
     cuuint64_t strides[4] = {(cuuint64_t)kD * 2, 128, (cuuint64_t)8 * kD * 2, (cuuint64_t)BS * kD * 2};
     cuuint32_t box[5] = {64, 8, 2, (cuuint32_t)(BS / 8), 1};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    if (fn(i ? &tmv : &tmk, TcType<T>::kTma, 5, const_cast<void *>(i ? a.v_cache : a.k_cache), dims,
-           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+    const CUresult r = fn(i ? &tmv : &tmk, TcType<T>::kTma, 5, const_cast<void *>(i ? a.v_cache : a.k_cache),
+                          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      debug_log("chunk_pp: 5-D K/V tensor map refused (CUresult %d); two 2-D boxes per block", (int)r);
+      five_d = 0;
+    }
+  }
+  if (!five_d) {
+    for (int i = 0; i < 2; ++i) {
+      cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)a.num_blocks * a.num_kv_heads * BS};
+      cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+      cuuint32_t box[2] = {64, (cuuint32_t)BS};
+      cuuint32_t estr[2] = {1, 1};
+      const CUresult r = fn(i ? &tmv : &tmk, TcType<T>::kTma, 2, const_cast<void *>(i ? a.v_cache : a.k_cache),
+                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) {
+        debug_log("chunk_pp: 2-D K/V tensor map refused (CUresult %d)", (int)r);
+        return cudaErrorInvalidValue;
+      }
+    }
   }
   auto kern = chunk_pp_kernel<T, BS, PREFIX>;
   {
     cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmemBytes);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      debug_log("chunk_pp: shared-memory limit %d refused: %s", kSmemBytes, cudaGetErrorString(e));
+      return e;
+    }
   }
   // chunk rows: (sequence, KV head, pair of Q tiles); prefix: (group, KV
   // head, pair of member tiles)
@@ -595,8 +665,10 @@ cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
   const int64_t grid = (int64_t)(PREFIX ? a.num_groups : a.num_seqs) * a.num_kv_heads * tiles;
   if (grid == 0) return cudaSuccess;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-  kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, tmq, tmk, tmv, tiles);
-  return cudaGetLastError();
+  kern<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, tmq, tmk, tmv, tiles, five_d);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) debug_log("chunk_pp: launch failed: %s", cudaGetErrorString(e));
+  return e;
 }
 
 }  // namespace

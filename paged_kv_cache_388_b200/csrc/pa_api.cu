@@ -3,6 +3,8 @@
 // Nothing here allocates device memory.  The only device state the library
 // owns is one error word per device (a file-scope __device__ variable), whose
 // address is looked up once per device.
+#include <stdarg.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -63,6 +65,17 @@ cudaError_t device_info(DevInfo *info) {
   }
   *info = g_dev[dev];
   return cudaSuccess;
+}
+
+void debug_log(const char *fmt, ...) {
+  static const bool on = getenv("PA_DEBUG") != nullptr;
+  if (!on) return;
+  va_list ap;
+  va_start(ap, fmt);
+  fputs("[libpa] ", stderr);
+  vfprintf(stderr, fmt, ap);
+  fputc('\n', stderr);
+  va_end(ap);
 }
 
 cudaError_t set_smem_limit_once(const void *func, int bytes) {
@@ -427,13 +440,16 @@ int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const
   cudaError_t e = cudaSuccess;
   if (num_groups > 0) {
     // the shared blocks on the 5th-generation tensor cores (head_dim 128,
-    // group dividing 128): the ping-pong kernel over 128-key tiles, or with
-    // PA_PREFIX_KERNEL=tc64 the earlier one over 64-key tiles; PA_PREFIX_KERNEL=mma
-    // asks for the mma.sync cluster kernel, which serves every other shape
+    // group dividing 128): the kernel over 64-key tiles with three S/P
+    // buffers; PA_PREFIX_KERNEL=pp selects the ping-pong kernel over 128-key
+    // tiles (slower here: a group's rows fill one Q tile at most, so it has no
+    // second tile to overlap with -- 0.145 vs 0.122 ms on the parallel-sampling
+    // batch), PA_PREFIX_KERNEL=mma the mma.sync cluster kernel, which serves
+    // every other shape
     const char *sel = getenv("PA_PREFIX_KERNEL");
     const bool want_mma = sel && strcmp(sel, "mma") == 0;
-    const bool want_tc64 = sel && strcmp(sel, "tc64") == 0;
-    if (!want_mma && !want_tc64 && chunk_pp_supported(a, dtype)) {
+    const bool want_pp = sel && strcmp(sel, "pp") == 0;
+    if (want_pp && chunk_pp_supported(a, dtype)) {
       e = launch_prefix_pp(a, dtype, s);
     } else if (!want_mma && chunk_tc_supported(a, dtype)) {
       e = launch_prefix_tc(a, dtype, s);

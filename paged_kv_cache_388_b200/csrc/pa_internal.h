@@ -85,6 +85,10 @@ struct DevInfo {
 // Implemented in pa_api.cu
 cudaError_t device_info(DevInfo *info);
 
+// printf-style line on stderr when the environment variable PA_DEBUG is set
+// (host-side failures that only surface as PA_ERR_CUDA otherwise).
+void debug_log(const char *fmt, ...);
+
 // Raise the dynamic shared-memory limit of kernel `func` to `bytes` on the
 // current device, once per (kernel, device); thread-safe.  Later calls for the
 // same pair return the first call's result without touching the runtime.

@@ -47,13 +47,18 @@ def decode_kernel(request, monkeypatch):
     return request.param
 
 
-@pytest.fixture(params=["auto", "tc64", "mma"])
+@pytest.fixture(params=["auto", "pp5d", "tc64", "mma"])
 def chunk_kernel(request, monkeypatch):
     """Chunked-query rows through the default kernel (tcgen05 ping-pong over
-    128-key tiles at head_dim 128), through the tcgen05 kernel over 64-key
-    tiles and through the mma.sync kernel."""
+    128-key tiles at head_dim 128), the same kernel with one 5-D K/V box per
+    block instead of two 2-D boxes, the tcgen05 kernel over 64-key tiles and
+    the mma.sync kernel."""
+    monkeypatch.delenv("PA_CHUNK_PP_BOXES", raising=False)
     if request.param == "auto":
         monkeypatch.delenv("PA_CHUNK_KERNEL", raising=False)
+    elif request.param == "pp5d":
+        monkeypatch.delenv("PA_CHUNK_KERNEL", raising=False)
+        monkeypatch.setenv("PA_CHUNK_PP_BOXES", "5d")
     else:
         monkeypatch.setenv("PA_CHUNK_KERNEL", request.param)
     return request.param

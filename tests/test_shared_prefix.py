@@ -67,11 +67,11 @@ def _plain(lib, wl, batch, d):
     return out
 
 
-@pytest.fixture(params=["auto", "tc64", "mma"])
+@pytest.fixture(params=["auto", "pp", "mma"])
 def prefix_kernel(request, monkeypatch):
-    """The shared-prefix pass through the default kernel (tcgen05 ping-pong over
-    128-key tiles at head_dim 128), the tcgen05 kernel over 64-key tiles and
-    the mma.sync cluster kernel."""
+    """The shared-prefix pass through the default kernel (tcgen05 over 64-key
+    tiles at head_dim 128), the tcgen05 ping-pong kernel over 128-key tiles
+    and the mma.sync cluster kernel."""
     if request.param == "auto":
         monkeypatch.delenv("PA_PREFIX_KERNEL", raising=False)
     else:
