@@ -500,6 +500,14 @@ def measure_config(db, timer, k):
 # --------------------------------------------------------------------------
 # CPU oracle legs (cpu_baseline and --impl reference)
 # --------------------------------------------------------------------------
+def host_cores():
+    """Host cores this process may run on (its CPU affinity set)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def oracle_runner(wl, vals, batch):
     """Returns run(n_seqs) -> (seconds, bytes, n_seqs): the oracle doing the
     step for the first n_seqs sequences (their new tokens' writes into a copy
@@ -518,13 +526,13 @@ def oracle_runner(wl, vals, batch):
         t0 = time.perf_counter()
         oracle.reshape_and_cache(kp, vp, key[:n], value[:n], batch.slot_mapping[:n], wl.dtype)
         oracle.decode(q, kp, vp, batch.block_tables, batch.context_lens, wl.scale, wl.dtype,
-                      rows=range(n))
+                      rows=range(n), threads=host_cores())
         dt = time.perf_counter() - t0
         dec, _, _ = seq_bytes(wl, batch, range(n))
         nbytes = dec + 2 * (2 * n * wl.num_kv_heads * wl.head_dim * e) + n * 8
         return dt, nbytes, n
 
-    return run, oracle.max_threads()
+    return run, host_cores()
 
 
 def size_sample(run, total, target_s):
@@ -563,6 +571,7 @@ def oracle_config_leg(db, gpu_out, target_s=1.5):
                                  wl.dtype)
     q = workloads.to_numpy_raw(vals["q"])
     qsl = batch.query_start_loc
+    cores = host_cores()  # every run names its thread count: OpenMP keeps the last one set
 
     def decode(rows, threads):
         t0 = time.perf_counter()
@@ -588,12 +597,12 @@ def oracle_config_leg(db, gpu_out, target_s=1.5):
         keys, row_seq = np.asarray(keys), np.asarray(row_seq)
     order = np.random.default_rng(7).permutation(keys.shape[0])
     probe = order[: max(1, min(8, keys.shape[0]))]
-    dt, _ = decode(probe.tolist(), 0)
+    dt, _ = decode(probe.tolist(), cores)
     per_key = dt / max(1, int(keys[probe].sum()))
     csum = np.cumsum(keys[order])
     n = int(np.searchsorted(csum, target_s / max(per_key, 1e-12))) + 1
     rows = np.sort(order[: max(1, min(n, keys.shape[0]))])
-    dt, ref = decode(rows.tolist(), 0)
+    dt, ref = decode(rows.tolist(), cores)
     e = elem_bytes(wl.dtype)
     ekv = 1 if db.kv_fp8 else e
     kv_bytes = int(keys[rows].sum()) * 2 * wl.num_kv_heads * wl.head_dim * ekv
@@ -605,7 +614,7 @@ def oracle_config_leg(db, gpu_out, target_s=1.5):
     leg = {"rows": int(rows.shape[0]), "of_rows": int(keys.shape[0]),
            "sample": "query rows drawn uniformly at random (seed 7), all heads; GB/s counts the "
                      "KV bytes each sampled row reads (no sharing between rows)",
-           "threads_all": {"cores": oracle.max_threads(), "s": dt, "GBps": nbytes / dt / 1e9},
+           "threads_all": {"cores": cores, "s": dt, "GBps": nbytes / dt / 1e9},
            "max_abs_err_vs_gpu": float(err.max()),
            "max_rel_err_vs_gpu_ref_gt_1e-3": float((err[big] / np.abs(r[big])).max()) if big.any() else 0.0}
     if db.cfg in ("1", "2", "3"):

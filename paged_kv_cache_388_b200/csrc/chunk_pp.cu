@@ -414,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // Pass 1: row max over the tile's S columns, 32 at a time (the next
         // chunk's load is in flight while this one is reduced).  Keys past
-        // the row's causal limit are masked (only in tiles reaching past the
-        // Q tile's smallest limit).
+        // the row's causal limit are masked, in the tiles that reach past the
+        // Q tile's smallest limit only (warp-uniform branch).
         const int k0 = j * kKeys;
         const bool masked = k0 + kKeys - 1 > limit_lo;
         float mx = -INFINITY;
@@ -428,11 +428,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t (&cur)[32] = (c & 1) ? cb : ca;
             uint32_t (&nxt)[32] = (c & 1) ? ca : cb;
             if (c + 1 < kKeys / 32) tmem_ld32(ts + 32 * (c + 1), nxt);
+            if (masked) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float v = (!masked || k0 + 32 * c + i <= limit) ? __uint_as_float(cur[i]) : -INFINITY;
-              mx = fmaxf(mx, v);
+              for (int i = 0; i < 32; ++i)
+                if (k0 + 32 * c + i > limit) cur[i] = __float_as_uint(-INFINITY);
             }
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(cur[i]), __uint_as_float(cur[i + 1]));
             tmem_wait_ld();
           }
         }
@@ -459,34 +461,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // Pass 2: P = 2^(s*scale*log2e - m), chunk by chunk over the same
-        // columns; chunk c's P words go over S columns the pass has already
-        // read (bf16: [32c, 32c+32), fp16: [16c, 16c+16)).
-        const float neg = -m_used;
-        float psum = 0.f;
-        {
+        // columns (next chunk prefetched); chunk c's P words go over S columns
+        // the pass has already read (bf16: [32c, 32c+32), fp16: [16c, 16c+16)).
+        // Key pairs are computed with packed f32x2 arithmetic.
+        const float2 sl2x2 = make_float2(sl2, sl2);
+        const float2 negx2 = make_float2(-m_used, -m_used);
+        float2 psum2 = make_float2(0.f, 0.f);
 #pragma unroll 1
-          for (int c = 0; c < kKeys / 32; ++c) {
-            uint32_t cur[32];
-            tmem_ld32(ts + 32 * c, cur);
-            tmem_wait_ld();
+        for (int cp = 0; cp < kKeys / 64; ++cp) {  // pairs of 32-column chunks
+          uint32_t ca[32], cb[32];
+          tmem_ld32(ts + 64 * cp, ca);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = 2 * cp + h;
+            uint32_t (&cur)[32] = h ? cb : ca;
+            if (h == 0) tmem_ld32(ts + 64 * cp + 32, cb);  // lands while chunk 2cp is computed
+            if (masked) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (k0 + 32 * c + i > limit) cur[i] = __float_as_uint(-INFINITY);
+            }
             uint32_t w[16];
 #pragma unroll
             for (int g2 = 0; g2 < 2; ++g2) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const int kk = 16 * g2 + 2 * i;  // key within the chunk
-                const int key = k0 + 32 * c + kk;
-                const float x0 = (!masked || key <= limit) ? __uint_as_float(cur[kk]) : -INFINITY;
-                const float x1 = (!masked || key + 1 <= limit) ? __uint_as_float(cur[kk + 1]) : -INFINITY;
-                const float p0 = fast_exp2(fmaf(x0, sl2, neg));
-                const float p1 = fast_exp2(fmaf(x1, sl2, neg));
-                psum += p0 + p1;
-                const uint32_t hi = TT::pack(p0, p1);
+                const float2 x = make_float2(__uint_as_float(cur[kk]), __uint_as_float(cur[kk + 1]));
+                const float2 t = __ffma2_rn(x, sl2x2, negx2);
+                const float2 pp = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+                psum2 = __fadd2_rn(psum2, pp);
+                const uint32_t hi = TT::pack(pp.x, pp.y);
                 if constexpr (TT::kSplitP) {
                   // 16 keys: 8 hi words then 8 lo words (columns 16g .. 16g+15)
                   const float2 hv = TT::unpack(hi);
+                  const float2 rv = __ffma2_rn(hv, make_float2(-1.f, -1.f), pp);  // p - hi
                   w[i] = hi;
-                  w[8 + i] = TT::pack(p0 - hv.x, p1 - hv.y);
+                  w[8 + i] = TT::pack(rv.x, rv.y);
                 } else {
                   w[8 * g2 + i] = hi;  // 16 keys: 8 words (columns 8g .. 8g+7)
                 }
@@ -494,8 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               if constexpr (TT::kSplitP) tmem_st16(ts + 32 * c + 16 * g2, w);
             }
             if constexpr (!TT::kSplitP) tmem_st16(ts + 16 * c, w);
+            tmem_wait_ld();
           }
         }
+        const float psum = psum2.x + psum2.y;
         tmem_wait_st();
         l += psum;
         // keys past the context end in the sequence's last tile: zero their V
