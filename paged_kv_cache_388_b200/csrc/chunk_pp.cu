@@ -58,29 +58,8 @@ constexpr int kQTiles = 2;
 #define PA_CHUNK_PP_STAGES 2
 #endif
 constexpr int kStages = PA_CHUNK_PP_STAGES;  // K/V tiles in flight
-// 1: the K half of a stage is released once the S products of its tile ran,
-// the V half once the P V products did (K of a tile then goes out about a
-// P V earlier); 0: both halves once the P V products ran.  Measured on one
-// B200 (long mixed batch, whole call back to back): 1.266 ms split vs 1.282 /
-// 1.285 ms unified with 2-D boxes, 1.281 vs 1.304 ms with 5-D boxes -- within
-// the 1-2 % the same build varies by between runs, and up to 6 % between
-// boxes; the simpler unified release is the default.
-#ifndef PA_CHUNK_PP_SPLIT_RELEASE
-#define PA_CHUNK_PP_SPLIT_RELEASE 0
-#endif
-constexpr bool kSplitRelease = PA_CHUNK_PP_SPLIT_RELEASE != 0;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: P stays <= 2^8 between rescales
-// Softmax warps per TMEM lane quadrant of a Q tile: with two, each takes 64 of
-// a tile's 128 keys and 64 of O's columns, and the pair exchanges row maxima
-// and sums through shared memory.
-#ifndef PA_CHUNK_PP_HALVES
-#define PA_CHUNK_PP_HALVES 2
-#endif
-constexpr int kHalves = PA_CHUNK_PP_HALVES;
-static_assert(kHalves == 1 || kHalves == 2, "one or two softmax warps per lane quadrant");
-constexpr int kKeysPerWarp = kKeys / kHalves;
-constexpr int kOColsPerWarp = kD / kHalves;
-constexpr int kSoftmaxWarps = 4 * kHalves * kQTiles;
+constexpr int kSoftmaxWarps = 4 * kQTiles;
 constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
 constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
 
@@ -91,38 +70,20 @@ constexpr int kHalfStage = kKeys * kD * 2;        // K (or V) of one tile: 32 KB
 constexpr int kStageBytes = 2 * kHalfStage;
 constexpr int kOffKV = kOffQ + kQTiles * kQBytes;
 constexpr int kOffMemBad = kOffKV + kStages * kStageBytes;  // prefix mode: [256] member flags
-// row-max exchange [Q tile][2 buffers][kHalves][128] and row-sum exchange [Q tile][kHalves][128]
-constexpr int kOffXMax = kOffMemBad + 256;
-constexpr int kOffXL = kOffXMax + kQTiles * 2 * kHalves * kRows * 4;
-constexpr int kOffBar = kOffXL + kQTiles * kHalves * kRows * 4;
+constexpr int kOffBar = kOffMemBad + 256;
 enum {
   kQFull = 0,
   kKFull = 1,                      // [kStages] the K half of a stage landed
   kVFull = kKFull + kStages,       // [kStages] the V half landed
-  kKEmpty = kVFull + kStages,      // [kStages] the stage's K read by every S product
-  kVEmpty = kKEmpty + kStages,     // [kStages] the stage's V read by every P V product
-  kSFull = kVEmpty + kStages,      // [Q tile] S in TMEM
+  kKvEmpty = kVFull + kStages,     // [kStages] both Q tiles' products of the stage done
+  kSFull = kKvEmpty + kStages,     // [Q tile] S in TMEM
   kPFull = kSFull + kQTiles,       // [Q tile] P written over S (4 softmax warps)
   kPvDone = kPFull + kQTiles,      // [Q tile] P V complete
   kDone = kPvDone + kQTiles,
-  kXFull = kDone + 1,              // [Q tile][quadrant][buffer] a row-max pair written
-  kLFull = kXFull + kQTiles * 8,   // [Q tile][quadrant] a row-sum pair written
-  kNumBars = kLFull + kQTiles * 4
+  kNumBars = kDone + 1
 };
 constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 64 + 1024;  // + TMEM slot, flags, alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
-
-// TMEM column, within a Q tile's S/P region, of the P words of keys 16g ..
-// 16g+15: bf16 hi + lo words sit over those keys' own S columns (16g .. +15);
-// one fp16 word per key pair takes 8 columns, packed at the front of the
-// region of the softmax warp that owns the keys, so that a warp never writes
-// S columns its partner has still to read.
-template <bool kSplit>
-__device__ __forceinline__ uint32_t p_col(int g) {
-  if constexpr (kSplit) return (uint32_t)g * 16u;
-  constexpr int kGroupsPerWarp = kKeysPerWarp / 16;
-  return (uint32_t)((g / kGroupsPerWarp) * kKeysPerWarp + (g % kGroupsPerWarp) * 8);
-}
 
 // TMEM columns: Q tile t's S/P at t*256, its O at t*256 + 128.
 __device__ __forceinline__ uint32_t tmem_s_col(int t) { return (uint32_t)t * 256u; }
@@ -206,17 +167,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars[kKFull + s], 1);
       mbar_init(&bars[kVFull + s], 1);
-      mbar_init(&bars[kKEmpty + s], 1);
-      mbar_init(&bars[kVEmpty + s], 1);
+      mbar_init(&bars[kKvEmpty + s], 1);
     }
     for (int t = 0; t < kQTiles; ++t) {
       mbar_init(&bars[kSFull + t], 1);
-      mbar_init(&bars[kPFull + t], 4 * kHalves);
+      mbar_init(&bars[kPFull + t], 4);
       mbar_init(&bars[kPvDone + t], 1);
     }
     mbar_init(&bars[kDone], 1);
-    for (int b = 0; b < kQTiles * 8; ++b) mbar_init(&bars[kXFull + b], 32 * kHalves);
-    for (int b = 0; b < kQTiles * 4; ++b) mbar_init(&bars[kLFull + b], 32 * kHalves);
     flags[0] = 0;
     flags[1] = 0;
     if constexpr (PREFIX)
@@ -257,9 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int grp = 0;
     int ids = lane < nblk ? table[lane] : 0;
     int ids_next = 32 + lane < nblk ? table[32 + lane] : 0;
-    int last_issued[kStages], v_issued[kStages];  // last tile whose K (V) went into each stage
+    int last_issued[kStages];
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) last_issued[s] = v_issued[s] = -1;
+    for (int s = 0; s < kStages; ++s) last_issued[s] = -1;
     bool aborted = false;
     for (int j = 0; j < ntiles && !aborted; ++j) {
       const int st = j % kStages;
@@ -273,11 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pbs[kBpt];
 #pragma unroll
       for (int b = 0; b < kBpt; ++b) pbs[b] = __shfl_sync(0xffffffffu, ids, (b0 - grp + b) & 31);
-      // The K half of a stage is free once both S products of its previous
-      // tile were issued and ran, the V half once both P V products did: K
-      // of tile j goes out about a P V ahead of its V.
-      const uint32_t epar = ((j / kStages) & 1) ^ 1;
-      bool ok = !flags[0] && mbar_wait(&bars[kKEmpty + st], epar);
+      bool ok = !flags[0] && mbar_wait(&bars[kKvEmpty + st], ((j / kStages) & 1) ^ 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) fail();
@@ -289,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vdst = kdst + kHalfStage;
         const uint32_t bytes = nb * BS * kD * 2;
         mbar_arrive_expect_tx(&bars[kKFull + st], bytes);
+        mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
 #pragma unroll
         for (int b = 0; b < kBpt; ++b) {
           if (b < nb && (pbs[b] < 0 || pbs[b] >= a.num_blocks)) {
@@ -297,39 +252,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             pbs[b] = 0;  // load a valid block; the CTA's rows are written as zeros
           }
         }
+        if (five_d) {
 #pragma unroll
-        for (int b = 0; b < kBpt; ++b)
-          if (b < nb) {
-            if (five_d) {
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb)
               tma_load_5d(kdst + b * BS * kD * 2, &tmk, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
                           &bars[kKFull + st]);
-            } else {
+#pragma unroll
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb)
+              tma_load_5d(vdst + b * BS * kD * 2, &tmv, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
+                          &bars[kVFull + st]);
+        } else {
+#pragma unroll
+          for (int b = 0; b < kBpt; ++b)
+            if (b < nb) {
               const int row = (pbs[b] * a.num_kv_heads + kvh) * BS;
               for (int h = 0; h < 2; ++h)
                 tma_load_2d(kdst + h * HS + b * BS * 128, &tmk, h * 64, row, &bars[kKFull + st]);
             }
-          }
-        // V of this tile: its half of the stage must have been read by the P V
-        // products of the stage's previous tile
-        if (kSplitRelease && !mbar_wait(&bars[kVEmpty + st], epar)) {
-          fail();  // V of this tile is never issued; its waiters' bounded waits end
-        } else {
-          mbar_arrive_expect_tx(&bars[kVFull + st], bytes);
 #pragma unroll
           for (int b = 0; b < kBpt; ++b)
             if (b < nb) {
-              if (five_d) {
-                tma_load_5d(vdst + b * BS * kD * 2, &tmv, 0, 0, 0, 0, pbs[b] * a.num_kv_heads + kvh,
-                            &bars[kVFull + st]);
-              } else {
-                const int row = (pbs[b] * a.num_kv_heads + kvh) * BS;
-                for (int h = 0; h < 2; ++h)
-                  tma_load_2d(vdst + h * HS + b * BS * 128, &tmv, h * 64, row, &bars[kVFull + st]);
-              }
+              const int row = (pbs[b] * a.num_kv_heads + kvh) * BS;
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(vdst + h * HS + b * BS * 128, &tmv, h * 64, row, &bars[kVFull + st]);
             }
-#pragma unroll
-          for (int s2 = 0; s2 < kStages; ++s2)
-            if (s2 == st) v_issued[s2] = j;
         }
 #pragma unroll
         for (int s2 = 0; s2 < kStages; ++s2)
@@ -343,8 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[kQFull], 0);
 #pragma unroll
       for (int s = 0; s < kStages; ++s) {
-        if (last_issued[s] >= 0 && !mbar_wait(&bars[kKFull + s], (last_issued[s] / kStages) & 1)) fail();
-        if (v_issued[s] >= 0 && !mbar_wait(&bars[kVFull + s], (v_issued[s] / kStages) & 1)) fail();
+        if (last_issued[s] < 0) continue;
+        const uint32_t par = (last_issued[s] / kStages) & 1;
+        if (!mbar_wait(&bars[kKFull + s], par) || !mbar_wait(&bars[kVFull + s], par)) fail();
       }
     }
   } else if (warp == kMmaWarp) {
@@ -378,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     (j > 0 || ks > 0) ? 1u : 0u);
             umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + ks * 16 + 8, db, idesc_pv, 1u);
           } else {
-            umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + p_col<false>(ks), db, idesc_pv,
+            umma_ts(tmem + tmem_o_col(t), tmem + tmem_s_col(t) + ks * 8, db, idesc_pv,
                     (j > 0 || ks > 0) ? 1u : 0u);
           }
         }
@@ -389,7 +338,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_s(0, 0);
         if (nq > 1) issue_s(1, 0);
-        if (kSplitRelease) umma_commit(&bars[kKEmpty]);  // K of tile 0 is free once these S products finish
       } else {
         fail();
       }
@@ -404,10 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           issue_pv(t, j);
-          if (t == nq - 1) {  // V (and without the split, K too) of tile j is free once these finish
-            umma_commit(&bars[kVEmpty + st]);
-            if (!kSplitRelease) umma_commit(&bars[kKEmpty + st]);
-          }
+          if (t == nq - 1) umma_commit(&bars[kKvEmpty + st]);  // the stage is free once these finish
           if (more) {
             // S(j+1) overwrites P(j) of this Q tile: its P V must be complete
             ok = mbar_wait(&bars[kPvDone + t], par) &&
@@ -415,7 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             issue_s(t, jn);
-            if (kSplitRelease && t == nq - 1) umma_commit(&bars[kKEmpty + (jn % kStages)]);  // K of tile j+1
           }
         }
         if (!ok) fail();
@@ -425,20 +369,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ======================= softmax warps =================================
-    // warp = (Q tile qt, key half hf, lane quadrant qd): rows 32 qd .. 32 qd + 31
-    // (TMEM lanes; a warp may only reach quadrant warp % 4), keys hf * kKeysPerWarp ..
-    // of every tile, O columns hf * kOColsPerWarp ..
-    const int qt = warp / (4 * kHalves), wl = warp % (4 * kHalves);
-    const int qd = wl & 3, hf = wl >> 2;
-    const int r = qd * 32 + lane;          // row of the Q tile = TMEM lane
-    const int sid = hf * kRows + r;        // 0 .. 128 * kHalves - 1 within the Q tile
-    float *xmax = reinterpret_cast<float *>(smem + kOffXMax);  // [qt][buf][hf][row]
-    float *xl = reinterpret_cast<float *>(smem + kOffXL);      // [qt][hf][row]
+    const int qt = warp >> 2, qd = warp & 3;
+    const int r = qd * 32 + lane;  // row of the Q tile = TMEM lane
     if (qt < nq) {
       const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-      const uint32_t ts = tmem + tmem_s_col(qt) + lane_off + hf * kKeysPerWarp;  // this warp's S columns
-      const uint32_t to = tmem + tmem_o_col(qt) + lane_off + hf * kOColsPerWarp; // and O columns
-      const uint32_t ts_p = tmem + tmem_s_col(qt) + lane_off;                    // P columns (p_col)
+      const uint32_t ts = tmem + tmem_s_col(qt) + lane_off;
+      const uint32_t to = tmem + tmem_o_col(qt) + lane_off;
       const int tok = qt * TPT + r / G;                     // token among the CTA's rows
       const int limit = min(L - Q + t0 + tok, L - 1);       // last key this row may see
       const int limit_lo = L - Q + t0 + qt * TPT;           // the tile's smallest limit
@@ -448,9 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // range.  All of the checks' loads are issued together here, while the
         // first tile is in flight, instead of one dependent round trip per tile.
         const int32_t *table = a.block_tables + (int64_t)seq * a.max_blocks_per_seq;
-        const int cid = qt * kHalves * kRows + sid;  // 0 .. nq * 128 * kHalves - 1
-        const int nth = nq * kHalves * kRows;
-        for (int x0 = cid; x0 < ntok * nblk; x0 += nth * 8) {
+        const int sid = qt * kRows + r;  // 0 .. nq*128 - 1
+        const int nth = nq * kRows;
+        for (int x0 = sid; x0 < ntok * nblk; x0 += nth * 8) {
           int mine[8], ref[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -480,41 +416,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         // chunk's load is in flight while this one is reduced).  Keys past
         // the row's causal limit are masked, in the tiles that reach past the
         // Q tile's smallest limit only (warp-uniform branch).
-        const int k0 = j * kKeys + hf * kKeysPerWarp;  // first key of this warp's columns
-        const bool masked = j * kKeys + kKeys - 1 > limit_lo;
+        const int k0 = j * kKeys;
+        const bool masked = k0 + kKeys - 1 > limit_lo;
         float mx = -INFINITY;
         {
-          // 16 columns per load, the next one in flight while this one is reduced
-          constexpr int kG = kKeysPerWarp / 16;
-          uint32_t ca[16], cb[16];
-          tmem_ld16(ts, ca);
+          uint32_t ca[32], cb[32];
+          tmem_ld32(ts, ca);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kG; ++c) {
-            uint32_t (&cur)[16] = (c & 1) ? cb : ca;
-            uint32_t (&nxt)[16] = (c & 1) ? ca : cb;
-            if (c + 1 < kG) tmem_ld16(ts + 16 * (c + 1), nxt);
+          for (int c = 0; c < kKeys / 32; ++c) {
+            uint32_t (&cur)[32] = (c & 1) ? cb : ca;
+            uint32_t (&nxt)[32] = (c & 1) ? ca : cb;
+            if (c + 1 < kKeys / 32) tmem_ld32(ts + 32 * (c + 1), nxt);
             if (masked) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (k0 + 16 * c + i > limit) cur[i] = __float_as_uint(-INFINITY);
+              for (int i = 0; i < 32; ++i)
+                if (k0 + 32 * c + i > limit) cur[i] = __float_as_uint(-INFINITY);
             }
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) mx = fmax3(mx, __uint_as_float(cur[i]), __uint_as_float(cur[i + 1]));
+            for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(cur[i]), __uint_as_float(cur[i + 1]));
             tmem_wait_ld();
           }
-        }
-        if constexpr (kHalves > 1) {
-          // the row's max over the whole tile: exchange with the partner warp
-          // (two buffers: the partner can be one tile ahead, never two)
-          const int xb = j & 1;
-          float *xm = xmax + (qt * 2 + xb) * kHalves * kRows;
-          xm[hf * kRows + r] = mx;
-          mbar_arrive(&bars[kXFull + qt * 8 + qd * 2 + xb]);
-          const bool got = mbar_wait(&bars[kXFull + qt * 8 + qd * 2 + xb], (uint32_t)((j >> 1) & 1));
-          if (!__all_sync(0xffffffffu, got)) { ok = false; fail(); break; }
-#pragma unroll
-          for (int h2 = 0; h2 < kHalves; ++h2) mx = fmaxf(mx, xm[h2 * kRows + r]);
         }
         mx *= sl2;
         // lazy rescale: move the reference max only when the tile max exceeds
@@ -529,64 +451,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-          for (int c = 0; c < kOColsPerWarp / 16; ++c) {
-            uint32_t o[16];
-            tmem_ld16(to + 16 * c, o);
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(to + 32 * c, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st16(to + 16 * c, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(to + 32 * c, o);
           }
         }
-        // Pass 2: P = 2^(s*scale*log2e - m) group by group; a group's P words
-        // go over S columns this warp has already read (p_col).  Key pairs are
-        // computed with packed f32x2 arithmetic.
+        // Pass 2: P = 2^(s*scale*log2e - m), chunk by chunk over the same
+        // columns (next chunk prefetched); chunk c's P words go over S columns
+        // the pass has already read (bf16: [32c, 32c+32), fp16: [16c, 16c+16)).
+        // Key pairs are computed with packed f32x2 arithmetic.
         const float2 sl2x2 = make_float2(sl2, sl2);
         const float2 negx2 = make_float2(-m_used, -m_used);
         float2 psum2 = make_float2(0.f, 0.f);
-        {
-          // one 16-key group per load (its P words written back before the
-          // next group's S columns are read), the next group in flight
-          constexpr int kG = kKeysPerWarp / 16;
-          const int g0 = (k0 - j * kKeys) / 16;  // this warp's first 16-key group of the tile
 #pragma unroll 1
-          for (int cp = 0; cp < kG; cp += 2) {  // pairs of groups: the second loads during the first
-          uint32_t ca[16], cb[16];
-          tmem_ld16(ts + 16 * cp, ca);
+        for (int cp = 0; cp < kKeys / 64; ++cp) {  // pairs of 32-column chunks
+          uint32_t ca[32], cb[32];
+          tmem_ld32(ts + 64 * cp, ca);
           tmem_wait_ld();
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int c = cp + h;
-            uint32_t (&cur)[16] = h ? cb : ca;
-            if (h == 0) tmem_ld16(ts + 16 * (c + 1), cb);
+            const int c = 2 * cp + h;
+            uint32_t (&cur)[32] = h ? cb : ca;
+            if (h == 0) tmem_ld32(ts + 64 * cp + 32, cb);  // lands while chunk 2cp is computed
             if (masked) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (k0 + 16 * c + i > limit) cur[i] = __float_as_uint(-INFINITY);
+              for (int i = 0; i < 32; ++i)
+                if (k0 + 32 * c + i > limit) cur[i] = __float_as_uint(-INFINITY);
             }
             uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 x = make_float2(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1]));
-              const float2 t = __ffma2_rn(x, sl2x2, negx2);
-              const float2 pp = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-              psum2 = __fadd2_rn(psum2, pp);
-              const uint32_t hi = TT::pack(pp.x, pp.y);
-              w[i] = hi;
-              if constexpr (TT::kSplitP) {
-                // 8 hi words then 8 lo words over the group's own 16 S columns
-                const float2 hv = TT::unpack(hi);
-                const float2 rv = __ffma2_rn(hv, make_float2(-1.f, -1.f), pp);  // p - hi
-                w[8 + i] = TT::pack(rv.x, rv.y);
+            for (int g2 = 0; g2 < 2; ++g2) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int kk = 16 * g2 + 2 * i;  // key within the chunk
+                const float2 x = make_float2(__uint_as_float(cur[kk]), __uint_as_float(cur[kk + 1]));
+                const float2 t = __ffma2_rn(x, sl2x2, negx2);
+                const float2 pp = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+                psum2 = __fadd2_rn(psum2, pp);
+                const uint32_t hi = TT::pack(pp.x, pp.y);
+                if constexpr (TT::kSplitP) {
+                  // 16 keys: 8 hi words then 8 lo words (columns 16g .. 16g+15)
+                  const float2 hv = TT::unpack(hi);
+                  const float2 rv = __ffma2_rn(hv, make_float2(-1.f, -1.f), pp);  // p - hi
+                  w[i] = hi;
+                  w[8 + i] = TT::pack(rv.x, rv.y);
+                } else {
+                  w[8 * g2 + i] = hi;  // 16 keys: 8 words (columns 8g .. 8g+7)
+                }
               }
+              if constexpr (TT::kSplitP) tmem_st16(ts + 32 * c + 16 * g2, w);
             }
-            if constexpr (TT::kSplitP) {
-              tmem_st16(ts_p + p_col<true>(g0 + c), w);
-            } else {
-              tmem_st8(ts_p + p_col<false>(g0 + c), w);
-            }
+            if constexpr (!TT::kSplitP) tmem_st16(ts + 16 * c, w);
             tmem_wait_ld();
-          }
           }
         }
         const float psum = psum2.x + psum2.y;
@@ -603,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t vst = sbase + kOffKV + st * kStageBytes + kHalfStage;
             const int z0 = L - j * kKeys;       // first stale key of the tile
             const int nz = (kKeys - z0) * 16;   // 16-byte chunks over both halves
-            for (int c = sid; c < nz; c += kHalves * kRows) {
+            for (int c = r; c < nz; c += 128) {
               const int key = z0 + c / 16, ch = c % 16;
               const int h = ch >> 3, cc = ch & 7, kr = key & 7;
               st_shared_v4(vst + (key >> 3) * GS + h * HS + kr * 128 + ((cc ^ kr) << 4), 0, 0, 0, 0);
@@ -622,65 +542,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool fin = ok && !flags[0] && ntiles > 0 && mbar_wait(&bars[kPvDone + qt], lastp);
       fin = __all_sync(0xffffffffu, fin);
       if (!fin && ntiles > 0) fail();
-      if constexpr (kHalves > 1) {  // the row's sum over both warps' keys
-        float *xs = xl + qt * kHalves * kRows;
-        xs[hf * kRows + r] = l;
-        mbar_arrive(&bars[kLFull + qt * 4 + qd]);
-        if (mbar_wait(&bars[kLFull + qt * 4 + qd], 0)) {
-          l = 0.f;
-#pragma unroll
-          for (int h2 = 0; h2 < kHalves; ++h2) l += xs[h2 * kRows + r];
-        } else {
-          fail();
-          fin = false;
-        }
-        fin = __all_sync(0xffffffffu, fin);
-      }
       tc_fence_after();
       const bool write = tok < ntok;
       if constexpr (PREFIX) {
         // the member flags of every active softmax warp (named barrier 1)
-        named_sync(1, nq * kHalves * kRows);
+        named_sync(1, nq * kRows);
         // record of (member q0 + tok, head): o unnormalised, the reference max
         // (base 2) o and l are relative to, l; NaN l marks a poisoned record
         const bool poison = !fin || flags[1] || (write && bad_member[tok]);
         float *rec = a.pre_rec + ((int64_t)(q0 + tok) * a.num_heads + kvh * G + r % G) * (kD + 4);
 #pragma unroll 1
-        for (int c = 0; c < kOColsPerWarp / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(to + 16 * c, o);
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(to + 32 * c, o);
           tmem_wait_ld();
           if (write) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<float4 *>(rec + hf * kOColsPerWarp + 16 * c + i) =
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4 *>(rec + 32 * c + i) =
                   make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]), __uint_as_float(o[i + 2]),
                               __uint_as_float(o[i + 3]));
           }
         }
-        if (write && hf == 0) {
+        if (write) {
           rec[kD] = m_used;
           rec[kD + 1] = poison ? __int_as_float(0x7fc00000) : l;
         }
         tc_fence_before();
       } else {
       const float inv = (fin && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
-      T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * kD +
-               hf * kOColsPerWarp;
+      T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * kD;
 #pragma unroll 1
-      for (int c = 0; c < kOColsPerWarp / 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(to + 16 * c, o);
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(to + 32 * c, o);
         tmem_wait_ld();
         if (write) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 8) {
+          for (int i = 0; i < 32; i += 8) {
             uint4 v;
             v.x = TT::pack(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
             v.y = TT::pack(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
             v.z = TT::pack(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
             v.w = TT::pack(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-            *reinterpret_cast<uint4 *>(dst + 16 * c + i) = v;
+            *reinterpret_cast<uint4 *>(dst + 32 * c + i) = v;
           }
         }
       }
