@@ -70,7 +70,11 @@ constexpr int kHalfStage = kKeys * kD * 2;        // K (or V) of one tile: 32 KB
 constexpr int kStageBytes = 2 * kHalfStage;
 constexpr int kOffKV = kOffQ + kQTiles * kQBytes;
 constexpr int kOffMemBad = kOffKV + kStages * kStageBytes;  // prefix mode: [256] member flags
-constexpr int kOffBar = kOffMemBad + 256;
+// Barriers follow the member flags, which only the prefix mode has: without
+// them a chunk-row CTA (~193 KB) leaves room on its SM for a decode CTA of a
+// mixed batch (~33 KB), both with 1 KB reserved, within the SM's 228 KB.
+template <bool PREFIX>
+constexpr int off_bar() { return kOffMemBad + (PREFIX ? 256 : 0); }
 enum {
   kQFull = 0,
   kKFull = 1,                      // [kStages] the K half of a stage landed
@@ -82,8 +86,9 @@ enum {
   kDone = kPvDone + kQTiles,
   kNumBars = kDone + 1
 };
-constexpr int kSmemBytes = kOffBar + 8 * kNumBars + 64 + 1024;  // + TMEM slot, flags, alignment
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+template <bool PREFIX>
+constexpr int smem_bytes() { return off_bar<PREFIX>() + 8 * kNumBars + 64 + 1024; }  // + TMEM slot, flags, alignment
+static_assert(smem_bytes<true>() <= 227 * 1024, "shared memory per CTA");
 
 // TMEM columns: Q tile t's S/P at t*256, its O at t*256 + 128.
 __device__ __forceinline__ uint32_t tmem_s_col(int t) { return (uint32_t)t * 256u; }
@@ -98,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int kOffBar = off_bar<PREFIX>();
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * kNumBars);
   volatile int *flags = reinterpret_cast<volatile int *>(tmem_slot + 1);  // [0] abort, [1] bad block
@@ -665,8 +671,9 @@ cudaError_t launch_pp_t(const AttnArgs &a, cudaStream_t stream) {
     }
   }
   auto kern = chunk_pp_kernel<T, BS, PREFIX>;
+  constexpr int kSmemBytes = smem_bytes<PREFIX>();
   {
-    cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmemBytes);
+    cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmemBytes, true);
     if (e != cudaSuccess) {
       debug_log("chunk_pp: shared-memory limit %d refused: %s", kSmemBytes, cudaGetErrorString(e));
       return e;

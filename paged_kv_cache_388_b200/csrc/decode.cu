@@ -150,7 +150,6 @@ __global__ void __launch_bounds__(32 * (MAXW + 1), MAXW == 4 ? PA_DECODE_MIN_CTA
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int nthreads = blockDim.x;
 
   // ---- prologue: barriers, per-sequence lengths and rows, item prefix sum --
   if (tid == 0) {

@@ -884,7 +884,7 @@ cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   const L lay(a.num_seqs, a.group);
   const L big(kMaxSeqsPerLaunch, 8 * NT);
-  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes);
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes, true);
   if (e != cudaSuccess) return e;
   int occ = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1), lay.bytes);
@@ -900,7 +900,9 @@ cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
   if (grid < 1) grid = 1;
   // programmatic dependent launch: the grid may be scheduled while the
   // previous kernel in the stream finishes; it waits (griddepcontrol.wait)
-  // before touching global memory.
+  // before touching global memory.  Not beside a mixed batch's chunk rows
+  // forked to another stream: there the decode CTAs, all resident at once,
+  // would take every SM before the chunk kernel placed its CTAs.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(32 * (NCW + 1));
@@ -910,7 +912,7 @@ cudaError_t launch_mma_t(const AttnArgs &a, int sm_count, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.no_pdl ? 0 : 1;
   return cudaLaunchKernelEx(&cfg, kern, a, tmk, tmv);
 }
 
@@ -920,7 +922,7 @@ int grid_mma_t(const AttnArgs &a, int sm_count) {
   using L = MmaLayout<D, BS, NT, NCW, F8>;
   auto kern = paged_decode_mma_kernel<T, D, BS, NT, NCW, F8>;
   const L big(kMaxSeqsPerLaunch, 8 * NT);
-  if (set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes) != cudaSuccess) return 0;
+  if (set_smem_limit_once(reinterpret_cast<const void *>(kern), big.bytes, true) != cudaSuccess) return 0;
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * (NCW + 1),
                                                     L(a.num_seqs, a.group).bytes) != cudaSuccess)
@@ -950,7 +952,7 @@ cudaError_t launch_bal_reduce_t(const AttnArgs &a, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.no_pdl ? 0 : 1;
   if (a.head_dim == 64) return cudaLaunchKernelEx(&cfg, balanced_merge_kernel<T, 64>, a);
   return cudaLaunchKernelEx(&cfg, balanced_merge_kernel<T, 128>, a);
 }

@@ -61,10 +61,14 @@ int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void 
   if (rc != PA_OK) return rc;
   // pa_decode checks the scratch it needs against the array's size and
   // returns PA_ERR_WORKSPACE, launching nothing, when the batch needs more.
-  return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                   query_start_loc, num_seqs, num_q_tokens, max_query_len, num_heads,
-                   num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
-                   kv_split_tokens, dtype, scratch, (size_t)PA_NOALLOC_SCRATCH_BYTES, stream);
+  // A mixed batch's chunk rows stay on the caller's stream: the side stream
+  // pa_decode forks them onto is created on first use, and this entry point
+  // creates nothing.
+  return pa::decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                         query_start_loc, num_seqs, num_q_tokens, max_query_len, num_heads,
+                         num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
+                         kv_split_tokens, dtype, scratch, (size_t)PA_NOALLOC_SCRATCH_BYTES, stream,
+                         false);
 }
 
 }  // extern "C"

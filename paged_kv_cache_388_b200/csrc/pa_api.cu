@@ -2,7 +2,9 @@
 //
 // Nothing here allocates device memory.  The only device state the library
 // owns is one error word per device (a file-scope __device__ variable), whose
-// address is looked up once per device.
+// address is looked up once per device, and, once a device has served a mixed
+// batch through pa_decode, a stream of the device's highest priority and two
+// events that let the batch's chunk rows run beside its decode rows.
 #include <stdarg.h>
 #include <stdio.h>
 #include <stdlib.h>
@@ -78,7 +80,7 @@ void debug_log(const char *fmt, ...) {
   va_end(ap);
 }
 
-cudaError_t set_smem_limit_once(const void *func, int bytes) {
+cudaError_t set_smem_limit_once(const void *func, int bytes, bool max_shared) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -89,6 +91,9 @@ cudaError_t set_smem_limit_once(const void *func, int bytes) {
   const auto it = done.find(key);
   if (it != done.end()) return it->second;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && max_shared)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done.emplace(key, e);  // failures are retried on the next call
   return e;
 }
@@ -116,6 +121,86 @@ void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_contex
   *split_blocks = sb;
   *max_splits = ceil_div(nblk_max, sb);
 }
+
+namespace {
+
+// A mixed batch's chunk rows (tensor-bound) and decode rows (HBM-bound) read
+// the same caches and write disjoint output rows, so they need no order between
+// them.  The chunk kernel goes to a second stream of the device's highest
+// priority, forked from the caller's stream and joined back into it with
+// events, and the decode kernel follows on the caller's stream without
+// programmatic dependent launch, so that the chunk grid is placed first.  The
+// block scheduler places a later grid's CTAs only once the earlier grid has
+// none left waiting for an SM, so the decode CTAs start when the chunk grid's
+// last wave is placed: on the SMs that wave leaves empty (40 of 148 on the long
+// mixed batch) and beside its CTAs (both kernels ask for the largest
+// shared-memory carve-out, and a decode CTA fits in what a chunk CTA leaves).
+// PA_MIXED_OVERLAP=0 keeps the two on the caller's stream, one after the other.
+struct SideStream {
+  std::mutex mu;  // held from the fork to the join: one fork-join per device at a time
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ready = false, failed = false;
+};
+SideStream g_side[kMaxDevices];
+
+bool overlap_wanted() {
+  static const bool on = [] {
+    const char *v = getenv("PA_MIXED_OVERLAP");
+    return !(v && strcmp(v, "0") == 0);
+  }();
+  return on;
+}
+
+// Forks the current device's side stream from `caller` and returns it locked,
+// or returns nullptr (nothing enqueued, nothing locked): the work then stays on
+// the caller's stream.  The stream and events are created on the first mixed
+// batch outside a stream capture.
+SideStream *side_fork(cudaStream_t caller) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  SideStream &sd = g_side[dev];
+  sd.mu.lock();
+  if (!sd.ready) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (sd.failed || cudaStreamIsCapturing(caller, &cap) != cudaSuccess ||
+        cap != cudaStreamCaptureStatusNone) {
+      cudaGetLastError();
+      sd.mu.unlock();
+      return nullptr;
+    }
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
+        cudaStreamCreateWithPriority(&sd.stream, cudaStreamNonBlocking, greatest) == cudaSuccess &&
+        cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) == cudaSuccess) {
+      sd.ready = true;
+    } else {
+      debug_log("side stream for mixed batches not created: %s", cudaGetErrorString(cudaGetLastError()));
+      sd.failed = true;
+      sd.mu.unlock();
+      return nullptr;
+    }
+  }
+  if (cudaEventRecord(sd.fork, caller) != cudaSuccess ||
+      cudaStreamWaitEvent(sd.stream, sd.fork, 0) != cudaSuccess) {
+    debug_log("mixed-batch fork failed: %s", cudaGetErrorString(cudaGetLastError()));
+    sd.mu.unlock();
+    return nullptr;
+  }
+  return &sd;
+}
+
+// Joins the side stream back into `caller` (also after a failed launch, so that
+// a capture in progress stays well formed) and unlocks it.
+cudaError_t side_join(SideStream *sd, cudaStream_t caller) {
+  cudaError_t e = cudaEventRecord(sd->join, sd->stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(caller, sd->join, 0);
+  sd->mu.unlock();
+  return e;
+}
+
+}  // namespace
 
 }  // namespace pa
 
@@ -194,12 +279,16 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
   return fixed > bal ? fixed : bal;
 }
 
-int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
-              const int32_t *query_start_loc, int num_seqs, int num_q_tokens, int max_query_len,
-              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
-              float scale, int max_context_len, int kv_split_tokens, int dtype, void *workspace,
-              size_t workspace_bytes, struct CUstream_st *stream) {
+}  // extern "C"
+
+namespace pa {
+
+int decode_call(void *out, const void *q, const void *k_cache, const void *v_cache,
+                const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                const int32_t *query_start_loc, int num_seqs, int num_q_tokens, int max_query_len,
+                int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                float scale, int max_context_len, int kv_split_tokens, int dtype, void *workspace,
+                size_t workspace_bytes, struct CUstream_st *stream, bool overlap) {
   if (num_seqs < 0 || num_q_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
       num_blocks <= 0 || max_blocks_per_seq <= 0 || !dtype_ok(dtype) || kv_split_tokens < 0)
     return PA_ERR_INVALID_ARG;
@@ -286,18 +375,42 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
   }
 
   cudaStream_t s = (cudaStream_t)stream;
-  for (int s0 = 0; s0 < num_seqs; s0 += step) {
+  const bool chunk_rows = max_query_len > 1 && !a.rows_mode;
+  SideStream *side = (overlap && chunk_rows && overlap_wanted()) ? side_fork(s) : nullptr;
+  a.no_pdl = side ? 1 : 0;
+  cudaError_t e = cudaSuccess;
+  for (int s0 = 0; s0 < num_seqs && e == cudaSuccess; s0 += step) {
     a.seq_begin = s0;
     a.num_seqs = num_seqs - s0 < step ? num_seqs - s0 : step;
-    cudaError_t e = use_mma ? launch_decode_mma(a, dtype, dev.sm_count, s)
-                            : launch_decode(a, dtype, dev.sm_count, s);
+    // forked: the chunk rows first, so that their CTAs are placed before the decode kernel's
+    if (side) e = launch_chunk(a, dtype, num_q_tokens, side->stream);
+    if (e == cudaSuccess)
+      e = use_mma ? launch_decode_mma(a, dtype, dev.sm_count, s) : launch_decode(a, dtype, dev.sm_count, s);
     if (e == cudaSuccess && a.balanced) e = launch_balanced_reduce(a, dtype, s);
     else if (e == cudaSuccess && max_splits > 1) e = launch_reduce(a, dtype, s);
-    if (e == cudaSuccess && max_query_len > 1 && !a.rows_mode)
-      e = launch_chunk(a, dtype, num_q_tokens, s);
-    if (e != cudaSuccess) return PA_ERR_CUDA;
+    if (e == cudaSuccess && chunk_rows && !side) e = launch_chunk(a, dtype, num_q_tokens, s);
   }
-  return PA_OK;
+  if (side) {
+    const cudaError_t j = side_join(side, s);
+    if (e == cudaSuccess) e = j;
+  }
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace pa
+
+extern "C" {
+
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+              const int32_t *query_start_loc, int num_seqs, int num_q_tokens, int max_query_len,
+              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+              float scale, int max_context_len, int kv_split_tokens, int dtype, void *workspace,
+              size_t workspace_bytes, struct CUstream_st *stream) {
+  return decode_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     query_start_loc, num_seqs, num_q_tokens, max_query_len, num_heads,
+                     num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
+                     kv_split_tokens, dtype, workspace, workspace_bytes, stream, true);
 }
 
 namespace {

@@ -39,6 +39,7 @@ struct AttnArgs {
   int balanced;       // 1: balanced flat partition (records in part_o), 0: fixed splits
   int grid;           // CTAs of the balanced launch (records are per CTA)
   int item_units;     // balanced: units a (sequence, KV head) pair weighs beyond its blocks
+  int no_pdl;         // host only: launch the decode and merge kernels without programmatic dependent launch
   int *bal_prefix;    // balanced: [num_seqs + 1] block prefix written by CTA 0
   int *bal_desc;      // balanced: [grid][4] cut-pair descriptors written by the decode kernel
   float scale_log2;   // scale * log2(e)
@@ -85,6 +86,16 @@ struct DevInfo {
 // Implemented in pa_api.cu
 cudaError_t device_info(DevInfo *info);
 
+// pa_decode with its arguments; overlap = false keeps a mixed batch's chunk
+// rows on the caller's stream after its decode rows (no side stream or events
+// are created), as pa_decode_noalloc needs.
+int decode_call(void *out, const void *q, const void *k_cache, const void *v_cache,
+                const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                const int32_t *query_start_loc, int num_seqs, int num_q_tokens, int max_query_len,
+                int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                float scale, int max_context_len, int kv_split_tokens, int dtype, void *workspace,
+                size_t workspace_bytes, struct CUstream_st *stream, bool overlap);
+
 // printf-style line on stderr when the environment variable PA_DEBUG is set
 // (host-side failures that only surface as PA_ERR_CUDA otherwise).
 void debug_log(const char *fmt, ...);
@@ -92,7 +103,10 @@ void debug_log(const char *fmt, ...);
 // Raise the dynamic shared-memory limit of kernel `func` to `bytes` on the
 // current device, once per (kernel, device); thread-safe.  Later calls for the
 // same pair return the first call's result without touching the runtime.
-cudaError_t set_smem_limit_once(const void *func, int bytes);
+// max_shared also asks for the largest shared-memory carve-out, so that the
+// kernel's CTAs and those of another kernel with the same preference can share
+// an SM's whole 228 KB (the chunk-row and decode kernels of a mixed batch).
+cudaError_t set_smem_limit_once(const void *func, int bytes, bool max_shared = false);
 
 // Split policy: KV blocks per split and the largest split count per sequence.
 void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_context_len,
