@@ -263,6 +263,15 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
  *                     (may be NULL when that size is 0); contents need no
  *                     initialisation and are not meaningful after the call.
  * Context length 0 gives zero output.
+ * A batch with both decode rows and chunk rows (max_query_len > 1) runs its
+ * chunk rows on a library stream of the device's highest priority, forked
+ * from `stream` and joined back into it with events: work enqueued on
+ * `stream` after the call is ordered after all of it, also inside a CUDA
+ * graph capture.  That stream and its two events are created on the first
+ * such call on a device made outside a stream capture (until then, and with
+ * the environment variable PA_MIXED_OVERLAP=0, both parts run on `stream`,
+ * one after the other).  One fork-join at a time per device: concurrent
+ * calls from several host threads serialise their enqueueing.
  */
 int pa_decode(void *out, const void *q, const void *k_cache,
               const void *v_cache, const int32_t *block_tables,
@@ -285,7 +294,8 @@ int pa_decode(void *out, const void *q, const void *k_cache,
  * instead from a static device array of PA_NOALLOC_SCRATCH_BYTES bytes built
  * into the library; every GPU that loads the library holds it until the
  * process exits.  This function allocates nothing and calls no allocating
- * routine.
+ * routine; a mixed batch's chunk rows run on `stream` after its decode rows
+ * (no side stream or event is created).
  *
  * Arguments and results are those of pa_decode (without workspace).
  * PA_ERR_WORKSPACE (nothing launched) if the batch needs more scratch than
