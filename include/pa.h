@@ -60,7 +60,8 @@
  *    PA_DEVERR_* bits that kernels OR in atomically.
  *  - Added entry points for the rows after the core path:
  *    pa_decode_shared_prefix (+ its workspace size), pa_reshape_and_cache_fp8,
- *    pa_decode_fp8, pa_swap_blocks, pa_decode_noalloc (+
+ *    pa_decode_fp8, pa_decode_fp8_rows (+ its workspace size),
+ *    pa_swap_blocks, pa_decode_noalloc (+
  *    pa_noalloc_scratch_bytes) and pa_abi_version.
  */
 #ifndef PA_H_
@@ -99,6 +100,8 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
                                       group's shared prefix, or a member whose block
                                       table differs from the group's first sequence
                                       over the shared range */
+#define PA_DEVERR_STAGING 0x40u    /* pa_decode_fp8_rows: the chunk-row sequences hold
+                                      more blocks than staged_blocks */
 
 /*
  * pa_reshape_and_cache -- write this step's new K/V into their cache slots.
@@ -216,6 +219,47 @@ int pa_decode_fp8(void *out, const void *q, const void *k_cache,
                   float v_scale, int max_context_len, int q_dtype,
                   void *workspace, size_t workspace_bytes,
                   struct CUstream_st *stream);
+
+/*
+ * pa_decode_fp8_rows -- pa_decode_fp8 for a batch that also holds chunked-
+ * prefill rows (query_start_loc, num_q_tokens and max_query_len as in
+ * pa_decode): decode rows as pa_decode_fp8; the rows of a sequence with Q > 1
+ * see keys 0 .. L-Q+t ("PagedAttention 实战", section Chunked Prefill) over the
+ * same FP8 codes (key = code * k_scale, value = code * v_scale).
+ *
+ * The chunk rows run on the 16-bit tensor-core chunk kernel: the blocks of
+ * every sequence with Q > 1 are first copied out of the cache into a staging
+ * pool inside the workspace as the 16-bit values of their codes (q's type;
+ * every E4M3 value is exact there), k_scale folded into the logit scale and
+ * v_scale applied to O / l.
+ *
+ *   staged_blocks  host-side bound of the staging pool in blocks: at least
+ *                  sum over the sequences with Q > 1 of
+ *                  ceil(context_len / block_size); > 0 when max_query_len > 1.
+ *                  A batch holding more blocks sets PA_DEVERR_STAGING, and the
+ *                  rows of the sequences whose blocks did not fit are written
+ *                  as zeros (with PA_DEVERR_BLOCK_ID).
+ *   workspace      >= pa_decode_fp8_rows_workspace_size(...) bytes.
+ * Other arguments as for pa_decode_fp8; the chunk rows need head_dim 128 and
+ * group <= 64 for the tensor-core kernels (else the mma.sync chunk kernel).
+ * Both parts run on `stream`, the chunk rows first.
+ */
+size_t pa_decode_fp8_rows_workspace_size(int num_seqs, int num_heads,
+                                         int num_kv_heads, int head_dim,
+                                         int block_size, int max_context_len,
+                                         int max_blocks_per_seq,
+                                         int staged_blocks);
+
+int pa_decode_fp8_rows(void *out, const void *q, const void *k_cache,
+                       const void *v_cache, const int32_t *block_tables,
+                       int max_blocks_per_seq, const int32_t *context_lens,
+                       const int32_t *query_start_loc, int num_seqs,
+                       int num_q_tokens, int max_query_len, int num_heads,
+                       int num_kv_heads, int head_dim, int block_size,
+                       int num_blocks, float scale, float k_scale,
+                       float v_scale, int max_context_len, int staged_blocks,
+                       int q_dtype, void *workspace, size_t workspace_bytes,
+                       struct CUstream_st *stream);
 
 /*
  * pa_decode_workspace_size -- bytes of device scratch pa_decode needs for

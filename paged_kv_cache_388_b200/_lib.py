@@ -36,6 +36,11 @@ _lib.pa_reshape_and_cache_fp8.restype = I
 _lib.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, P]
 _lib.pa_decode_fp8.restype = I
 _lib.pa_decode_fp8.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I, I, F, F, F, I, I, P, SZ, P]
+_lib.pa_decode_fp8_rows.restype = I
+_lib.pa_decode_fp8_rows.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, F, F, I, I, I,
+                                    P, SZ, P]
+_lib.pa_decode_fp8_rows_workspace_size.restype = SZ
+_lib.pa_decode_fp8_rows_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
 _lib.pa_swap_blocks.restype = I
 _lib.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P]
 _lib.pa_decode_workspace_size.restype = SZ
@@ -68,6 +73,7 @@ PA_DEVERR_CONTEXT_LEN = 0x4
 PA_DEVERR_QUERY_LEN = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 PA_DEVERR_PREFIX = 0x20
+PA_DEVERR_STAGING = 0x40
 
 
 class PAError(RuntimeError):
@@ -197,12 +203,26 @@ def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale
     _check(rc, "pa_reshape_and_cache_fp8")
 
 
+def pa_decode_fp8_rows_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, max_blocks_per_seq, staged_blocks) -> int:
+    return int(_lib.pa_decode_fp8_rows_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                      block_size, max_context_len,
+                                                      max_blocks_per_seq, staged_blocks))
+
+
 def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale,
-                  max_context_len=0, workspace=None, stream=None):
+                  max_context_len=0, workspace=None, query_start_loc=None, max_query_len=1,
+                  staged_blocks=0, stream=None):
     """out/q [S, H, D] fp16/bf16; caches uint8 E4M3 codes [NB, Hk, bs, D];
-    workspace: uint8 CUDA tensor of >= pa_decode_workspace_size(...) bytes."""
-    s, h, d, nb, hk, bs, _, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
-                                                  context_lens)
+    workspace: uint8 CUDA tensor of >= pa_decode_workspace_size(...) bytes.
+    With query_start_loc (chunked-prefill rows as in pa_decode) the call is
+    pa_decode_fp8_rows: staged_blocks bounds the blocks of the sequences with
+    more than one row (batch.staged_blocks_needed), and the workspace must hold
+    pa_decode_fp8_rows_workspace_size(...) bytes."""
+    tq, h, d, nb, hk, bs, s, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                   context_lens, query_start_loc)
+    if query_start_loc is not None:
+        _dev(query_start_loc, "query_start_loc", torch.int32)
     _dev(q, "q")
     _dev(out, "out", q.dtype)
     _dev(k_cache, "k_cache", torch.uint8)
@@ -212,11 +232,44 @@ def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k
     if workspace is not None:
         _dev(workspace, "workspace")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if query_start_loc is not None:
+        pa_decode_fp8_rows(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                           scale, k_scale, v_scale, max_query_len, staged_blocks,
+                           max_context_len=max_context_len, workspace=workspace, stream=stream)
+        return
     rc = _lib.pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                             mbps, _ptr(context_lens), s, h, hk, d, bs, nb, float(scale),
                             float(k_scale), float(v_scale), int(max_context_len), _DT[q.dtype],
                             _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "pa_decode_fp8")
+
+
+def pa_decode_fp8_rows(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                       scale, k_scale, v_scale, max_query_len, staged_blocks, max_context_len=0,
+                       workspace=None, stream=None):
+    """pa_decode_fp8 over a batch with chunked-prefill rows: q/out [Tq, H, D],
+    query_start_loc int32 [S + 1]; staged_blocks bounds the blocks of the
+    sequences with more than one row; workspace uint8 of
+    >= pa_decode_fp8_rows_workspace_size(...) bytes."""
+    tq, h, d, nb, hk, bs, s, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                   context_lens, query_start_loc)
+    _dev(q, "q")
+    _dev(out, "out", q.dtype)
+    _dev(k_cache, "k_cache", torch.uint8)
+    _dev(v_cache, "v_cache", torch.uint8)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    _dev(query_start_loc, "query_start_loc", torch.int32)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.pa_decode_fp8_rows(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(block_tables), mbps, _ptr(context_lens),
+                                 _ptr(query_start_loc), s, tq, int(max_query_len), h, hk, d, bs,
+                                 nb, float(scale), float(k_scale), float(v_scale),
+                                 int(max_context_len), int(staged_blocks), _DT[q.dtype],
+                                 _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "pa_decode_fp8_rows")
 
 
 def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None):

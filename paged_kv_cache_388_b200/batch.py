@@ -121,3 +121,12 @@ def shared_prefix_groups(block_tables: np.ndarray, context_lens: np.ndarray, blo
         starts.append(e)
         s = e
     return np.asarray(starts, dtype=np.int32), np.asarray(shared, dtype=np.int32)
+
+
+def staged_blocks_needed(query_start_loc, context_lens, block_size) -> int:
+    """Blocks pa_decode_fp8_rows stages for a batch over an FP8 cache: those of
+    the sequences with more than one query row (host arrays or CPU tensors)."""
+    qsl = np.asarray(query_start_loc, dtype=np.int64)
+    cl = np.asarray(context_lens, dtype=np.int64)
+    q = qsl[1:] - qsl[:-1]
+    return int(((cl + block_size - 1) // block_size)[(q > 1) & (cl > 0)].sum())

@@ -258,8 +258,8 @@ __global__ void __launch_bounds__(128) chunk_kernel(const AttnArgs a, int tiles_
   l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
   __syncthreads();
   const bool bad = s_bad != 0;  // a bad block id anywhere: the tile's rows are zeros
-  const float inv_a = (l_a > 0.f && !bad) ? 1.f / l_a : 0.f;
-  const float inv_b = (l_b > 0.f && !bad) ? 1.f / l_b : 0.f;
+  const float inv_a = (l_a > 0.f && !bad) ? (1.f / l_a) * a.o_scale : 0.f;
+  const float inv_b = (l_b > 0.f && !bad) ? (1.f / l_b) * a.o_scale : 0.f;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const int r = half ? row_b : row_a;

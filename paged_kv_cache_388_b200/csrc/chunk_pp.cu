@@ -576,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       } else {
-      const float inv = (fin && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
+      const float inv = (fin && l > 0.f && !flags[1]) ? (1.f / l) * a.o_scale : 0.f;
       T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * kD;
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {

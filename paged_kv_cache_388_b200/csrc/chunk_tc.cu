@@ -640,7 +640,7 @@ __global__ void __launch_bounds__(32 * (4 * kHalves * NQ + 2), PA_CHUNK_TC_MIN_C
         rec[D + 1] = poison ? __int_as_float(0x7fc00000) : l;
       }
     } else {
-      const float inv = (ok && l > 0.f && !flags[1]) ? 1.f / l : 0.f;
+      const float inv = (ok && l > 0.f && !flags[1]) ? (1.f / l) * a.o_scale : 0.f;
       T *dst = static_cast<T *>(a.out) + ((int64_t)(q0 + t0 + tok) * a.num_heads + kvh * G + r % G) * D;
 #pragma unroll 1
       for (int cblk = 0; cblk < kOColsPerHalf / 32; ++cblk) {

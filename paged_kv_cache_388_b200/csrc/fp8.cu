@@ -147,6 +147,179 @@ cudaError_t reshape_fp8_d(int head_dim, int block_size, const cudaLaunchConfig_t
                                 num_kv_heads, num_slots, ks, vs, err);
 }
 
+// ---- chunk rows over an FP8 cache -----------------------------------------
+// The tensor-core chunk kernels read 16-bit K/V tiles through TMA.  For a
+// mixed batch over an FP8 cache the blocks of the sequences with chunk rows
+// are first staged into a 16-bit pool of their codes' values (every E4M3
+// value is exact in fp16 and bf16), in the plain [block_size][head_dim] tile
+// layout, with per-sequence tables into that pool; k_scale goes into the
+// logit scale and v_scale onto O / l, as for the decode rows.
+
+// A sequence has staged blocks when it has more than one query row and a
+// context length the kernels accept.
+__device__ __forceinline__ int staged_blocks_of(const AttnArgs &a, int s) {
+  const int Q = a.query_start_loc[s + 1] - a.query_start_loc[s];
+  const int L = a.context_lens[s];
+  if (Q <= 1 || L <= 0 || L > a.max_context_len) return 0;
+  return (L + a.block_size - 1) / a.block_size;
+}
+
+// base[s] = first staged block of sequence s, base[num_seqs] = their total.
+// One CTA of 1024 threads; PA_DEVERR_STAGING if the total exceeds capacity.
+__global__ void __launch_bounds__(1024) fp8_stage_plan_kernel(const AttnArgs a, int *base,
+                                                             int capacity) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int s0 = 0; s0 < a.num_seqs; s0 += 1024) {
+    const int s = s0 + tid;
+    const int c = s < a.num_seqs ? staged_blocks_of(a, s) : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_tot[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int before = carry + (warp > 0 ? warp_tot[warp - 1] : 0);
+    if (s < a.num_seqs) base[s] = before + incl - c;
+    __syncthreads();
+    if (tid == 0) carry += warp_tot[31];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    base[a.num_seqs] = carry;
+    if (carry > capacity) raise_error(a.err, PA_DEVERR_STAGING);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2_t(float lo, float hi);
+template <>
+__device__ __forceinline__ uint32_t pack2_t<__nv_bfloat16>(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2_t<__half>(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ float e4m3_value(unsigned char code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw(code, __NV_E4M3)));
+}
+
+// Blocks of chunk-row sequences -> the 16-bit pool (sk, sv) and the tables
+// `tab` [num_seqs][max_blocks_per_seq] (-1 for a block not staged: an id
+// outside the cache, or past the pool's capacity).  Grid (x: blocks, y:
+// sequences); a CTA converts one (block, KV head) K tile and V tile at a time
+// through shared memory, each thread eight consecutive outputs of a row.
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(256) fp8_stage_kernel(const AttnArgs a, const int *base,
+                                                       int32_t *tab, T *sk, T *sv, int capacity) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ __align__(16) unsigned char kc[BS * D];
+  __shared__ __align__(16) unsigned char vc[BS * D];
+  const int s = blockIdx.y;
+  const int nblk = staged_blocks_of(a, s);
+  const unsigned char *kcache = static_cast<const unsigned char *>(a.k_cache);
+  const unsigned char *vcache = static_cast<const unsigned char *>(a.v_cache);
+  for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
+    const int id = base[s] + b;
+    const int src = a.block_tables[(int64_t)s * a.max_blocks_per_seq + b];
+    const bool src_ok = src >= 0 && src < a.num_blocks;
+    const bool ok = src_ok && id < capacity;
+    if (threadIdx.x == 0) {
+      tab[(int64_t)s * a.max_blocks_per_seq + b] = ok ? id : -1;
+      if (!src_ok) raise_error(a.err, PA_DEVERR_BLOCK_ID);
+    }
+    if (!ok) continue;  // uniform over the CTA
+    for (int h = 0; h < a.num_kv_heads; ++h) {
+      const int64_t tile = ((int64_t)src * a.num_kv_heads + h) * (BS * D);
+      __syncthreads();  // the previous tile's codes have been read
+      for (int i = threadIdx.x; i < BS * D / 16; i += blockDim.x) {
+        reinterpret_cast<uint4 *>(kc)[i] = reinterpret_cast<const uint4 *>(kcache + tile)[i];
+        reinterpret_cast<uint4 *>(vc)[i] = reinterpret_cast<const uint4 *>(vcache + tile)[i];
+      }
+      __syncthreads();
+      T *dk = sk + ((int64_t)id * a.num_kv_heads + h) * (BS * D);
+      T *dv = sv + ((int64_t)id * a.num_kv_heads + h) * (BS * D);
+      for (int o = threadIdx.x; o < BS * D / 8; o += blockDim.x) {
+        const int r = o / (D / 8), d0 = (o % (D / 8)) * 8;
+        // key r of the V tile: k-step kk, column cc of its 16 keys
+        const int kk = r >> 4, cc = r & 15;
+        const int vt = (cc & 7) >> 1, vi = (cc & 1) + 2 * (cc >> 3);
+        const int vpos = BS == 16 ? 4 * vt + vi : 8 * vt + 4 * kk + vi;
+        float fk[8], fv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int d = d0 + e;
+          const int j = d >> 6, k = (d >> 4) & 3, c = d & 15;
+          const int t = (c & 7) >> 1, i = (c & 1) + 2 * (c >> 3);
+          fk[e] = e4m3_value(kc[r * D + (((4 * j + t) ^ (r & (D / 16 - 1))) << 4) + 4 * k + i]);
+          fv[e] = e4m3_value(vc[d * BS + vpos]);
+        }
+        uint4 wk, wv;
+        wk.x = pack2_t<T>(fk[0], fk[1]); wk.y = pack2_t<T>(fk[2], fk[3]);
+        wk.z = pack2_t<T>(fk[4], fk[5]); wk.w = pack2_t<T>(fk[6], fk[7]);
+        wv.x = pack2_t<T>(fv[0], fv[1]); wv.y = pack2_t<T>(fv[2], fv[3]);
+        wv.z = pack2_t<T>(fv[4], fv[5]); wv.w = pack2_t<T>(fv[6], fv[7]);
+        *reinterpret_cast<uint4 *>(dk + r * D + d0) = wk;
+        *reinterpret_cast<uint4 *>(dv + r * D + d0) = wv;
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_stage_t(const AttnArgs &a, const int *base, int32_t *tab, void *sk, void *sv,
+                           int capacity, cudaStream_t s) {
+  const int gx = a.max_blocks_per_seq < 256 ? a.max_blocks_per_seq : 256;
+  const dim3 grid((unsigned)gx, (unsigned)a.num_seqs);
+  if (a.block_size == 16)
+    fp8_stage_kernel<T, D, 16><<<grid, 256, 0, s>>>(a, base, tab, static_cast<T *>(sk),
+                                                      static_cast<T *>(sv), capacity);
+  else
+    fp8_stage_kernel<T, D, 32><<<grid, 256, 0, s>>>(a, base, tab, static_cast<T *>(sk),
+                                                      static_cast<T *>(sv), capacity);
+  return cudaGetLastError();
+}
+
+// Workspace of pa_decode_fp8_rows: the decode rows' records (the bound of
+// pa_decode_workspace_size), base [num_seqs + 1], the staged tables
+// [num_seqs][max_blocks_per_seq] and the K and V pools of staged_blocks
+// 16-bit blocks, each part 1 KiB aligned.
+struct RowsWs {
+  size_t base, tab, k, v, total;
+};
+RowsWs rows_ws(size_t dec, int num_seqs, int num_kv_heads, int head_dim, int block_size,
+               int max_blocks_per_seq, int staged_blocks) {
+  auto up = [](size_t x) { return (x + 1023) / 1024 * 1024; };
+  RowsWs w;
+  w.base = up(dec);
+  w.tab = w.base + up((size_t)(num_seqs + 1) * sizeof(int));
+  w.k = w.tab + up((size_t)num_seqs * max_blocks_per_seq * sizeof(int32_t));
+  const size_t pool = up((size_t)staged_blocks * num_kv_heads * block_size * head_dim * 2);
+  w.v = w.k + pool;
+  w.total = w.v + pool;
+  return w;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool scale_ok(float s) { return s > 0.f && s < 3.0e38f; }
@@ -155,6 +328,127 @@ bool scale_ok(float s) { return s > 0.f && s < 3.0e38f; }
 }  // namespace pa
 
 using namespace pa;
+
+namespace pa {
+namespace {
+
+int decode_fp8_call(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *context_lens, const int32_t *query_start_loc, int num_seqs,
+                    int num_q_tokens, int max_query_len, int num_heads, int num_kv_heads,
+                    int head_dim, int block_size, int num_blocks, float scale, float k_scale,
+                    float v_scale, int max_context_len, int staged_blocks, int q_dtype,
+                    void *workspace, size_t workspace_bytes, struct CUstream_st *stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!scale_ok(k_scale) || !scale_ok(v_scale)) return PA_ERR_INVALID_ARG;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > decode_max_seqs_per_launch()) return PA_ERR_UNSUPPORTED;
+  if (!query_start_loc) {
+    if (num_q_tokens != num_seqs) return PA_ERR_INVALID_ARG;
+    max_query_len = 1;
+  } else if (max_query_len < 1 || num_q_tokens < num_seqs) {
+    return PA_ERR_INVALID_ARG;
+  }
+  const bool chunk_rows = max_query_len > 1;
+  if (staged_blocks < 0 || (chunk_rows && staged_blocks == 0)) return PA_ERR_INVALID_ARG;
+  if (chunk_rows && group > 64) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || num_q_tokens == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (out == q) return PA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30) return PA_ERR_UNSUPPORTED;
+  const int cap = max_blocks_per_seq * block_size;
+  if (max_context_len <= 0 || max_context_len > cap) max_context_len = cap;
+
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  AttnArgs a{};
+  a.o_scale = 1.f;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.err = dev.err;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.split_blocks = 1;
+  a.max_splits = 1;
+  a.query_start_loc = query_start_loc;
+  a.max_query_len = max_query_len;
+  a.max_context_len = max_context_len;
+  a.num_q_tokens = num_q_tokens;
+  a.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  a.v_inv = 1.f / v_scale;
+  a.balanced = 1;
+  a.item_units = kItemUnitsFp8;
+  a.grid = decode_mma_grid_fp8(a, q_dtype, dev.sm_count);
+  if (a.grid <= 0) return PA_ERR_CUDA;
+  const size_t rec = balanced_record_bytes(a.grid, group, head_dim);
+  const size_t desc = balanced_desc_bytes(a.grid);
+  const size_t need = rec + desc + (size_t)(num_seqs + 1) * sizeof(int);
+  RowsWs w{};
+  if (chunk_rows) {
+    w = rows_ws(pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                         max_context_len, 0),
+                num_seqs, num_kv_heads, head_dim, block_size, max_blocks_per_seq, staged_blocks);
+    if (need > w.base) return PA_ERR_WORKSPACE;
+  }
+  if (!workspace || workspace_bytes < (chunk_rows ? w.total : need) || !aligned16(workspace))
+    return PA_ERR_WORKSPACE;
+  char *ws = static_cast<char *>(workspace);
+  a.part_o = static_cast<float *>(workspace);
+  a.bal_desc = reinterpret_cast<int *>(ws + rec);
+  a.bal_prefix = reinterpret_cast<int *>(ws + rec + desc);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (chunk_rows) {
+    // the chunk rows: stage their sequences' blocks, then the 16-bit chunk kernel
+    int *base = reinterpret_cast<int *>(ws + w.base);
+    int32_t *tab = reinterpret_cast<int32_t *>(ws + w.tab);
+    fp8_stage_plan_kernel<<<1, 1024, 0, s>>>(a, base, staged_blocks);
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = q_dtype == PA_BF16
+              ? (head_dim == 64 ? launch_stage_t<__nv_bfloat16, 64>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s)
+                                : launch_stage_t<__nv_bfloat16, 128>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s))
+              : (head_dim == 64 ? launch_stage_t<__half, 64>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s)
+                                : launch_stage_t<__half, 128>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s));
+    if (e == cudaSuccess) {
+      AttnArgs c = a;
+      c.k_cache = ws + w.k;
+      c.v_cache = ws + w.v;
+      c.block_tables = tab;
+      c.num_blocks = staged_blocks;
+      c.o_scale = v_scale;
+      c.seq_begin = 0;
+      e = launch_chunk(c, q_dtype, num_q_tokens, s);
+    }
+  }
+  if (e == cudaSuccess) e = launch_decode_mma_fp8(a, q_dtype, dev.sm_count, s);
+  if (e == cudaSuccess) e = launch_balanced_reduce(a, q_dtype, s);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+
+}  // namespace
+}  // namespace pa
 
 extern "C" {
 
@@ -207,67 +501,38 @@ int pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_c
                   int head_dim, int block_size, int num_blocks, float scale, float k_scale,
                   float v_scale, int max_context_len, int q_dtype, void *workspace,
                   size_t workspace_bytes, struct CUstream_st *stream) {
-  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
-      max_blocks_per_seq <= 0)
-    return PA_ERR_INVALID_ARG;
-  if (!scale_ok(k_scale) || !scale_ok(v_scale)) return PA_ERR_INVALID_ARG;
-  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
-  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
-  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-  const int group = num_heads / num_kv_heads;
-  if (group > 16) return PA_ERR_UNSUPPORTED;
-  if (num_seqs > decode_max_seqs_per_launch()) return PA_ERR_UNSUPPORTED;
-  if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
-    return PA_ERR_INVALID_ARG;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return PA_ERR_INVALID_ARG;
-  if (out == q) return PA_ERR_INVALID_ARG;
-  if ((int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30) return PA_ERR_UNSUPPORTED;
+  return decode_fp8_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                         nullptr, num_seqs, num_seqs, 1, num_heads, num_kv_heads, head_dim,
+                         block_size, num_blocks, scale, k_scale, v_scale, max_context_len, 0,
+                         q_dtype, workspace, workspace_bytes, stream);
+}
+
+size_t pa_decode_fp8_rows_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int block_size, int max_context_len,
+                                         int max_blocks_per_seq, int staged_blocks) {
+  if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_blocks_per_seq <= 0 || staged_blocks < 0 ||
+      (int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30)
+    return 0;
   const int cap = max_blocks_per_seq * block_size;
   if (max_context_len <= 0 || max_context_len > cap) max_context_len = cap;
+  return rows_ws(pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                          max_context_len, 0),
+                 num_seqs, num_kv_heads, head_dim, block_size, max_blocks_per_seq, staged_blocks)
+      .total;
+}
 
-  DevInfo dev;
-  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  AttnArgs a{};
-  a.out = out;
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
-  a.err = dev.err;
-  a.num_seqs = num_seqs;
-  a.num_heads = num_heads;
-  a.num_kv_heads = num_kv_heads;
-  a.group = group;
-  a.head_dim = head_dim;
-  a.block_size = block_size;
-  a.num_blocks = num_blocks;
-  a.max_blocks_per_seq = max_blocks_per_seq;
-  a.split_blocks = 1;
-  a.max_splits = 1;
-  a.max_query_len = 1;
-  a.max_context_len = max_context_len;
-  a.num_q_tokens = num_seqs;
-  a.scale_log2 = scale * k_scale * 1.4426950408889634f;
-  a.v_inv = 1.f / v_scale;
-  a.balanced = 1;
-  a.item_units = kItemUnitsFp8;
-  a.grid = decode_mma_grid_fp8(a, q_dtype, dev.sm_count);
-  if (a.grid <= 0) return PA_ERR_CUDA;
-  const size_t rec = balanced_record_bytes(a.grid, group, head_dim);
-  const size_t desc = balanced_desc_bytes(a.grid);
-  const size_t need = rec + desc + (size_t)(num_seqs + 1) * sizeof(int);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
-  a.part_o = static_cast<float *>(workspace);
-  a.bal_desc = reinterpret_cast<int *>(static_cast<char *>(workspace) + rec);
-  a.bal_prefix = reinterpret_cast<int *>(static_cast<char *>(workspace) + rec + desc);
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_decode_mma_fp8(a, q_dtype, dev.sm_count, s);
-  if (e == cudaSuccess) e = launch_balanced_reduce(a, q_dtype, s);
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+int pa_decode_fp8_rows(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, int max_blocks_per_seq,
+                       const int32_t *context_lens, const int32_t *query_start_loc, int num_seqs,
+                       int num_q_tokens, int max_query_len, int num_heads, int num_kv_heads,
+                       int head_dim, int block_size, int num_blocks, float scale, float k_scale,
+                       float v_scale, int max_context_len, int staged_blocks, int q_dtype,
+                       void *workspace, size_t workspace_bytes, struct CUstream_st *stream) {
+  return decode_fp8_call(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                         query_start_loc, num_seqs, num_q_tokens, max_query_len, num_heads,
+                         num_kv_heads, head_dim, block_size, num_blocks, scale, k_scale, v_scale,
+                         max_context_len, staged_blocks, q_dtype, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

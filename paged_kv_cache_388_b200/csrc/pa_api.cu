@@ -321,6 +321,7 @@ int decode_call(void *out, const void *q, const void *k_cache, const void *v_cac
                &split_blocks, &max_splits);
 
   AttnArgs a{};
+  a.o_scale = 1.f;
   a.out = out;
   a.q = q;
   a.k_cache = k_cache;
@@ -506,6 +507,7 @@ int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const
   DevInfo dev;
   if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
   AttnArgs a{};
+  a.o_scale = 1.f;
   a.out = out;
   a.q = q;
   a.k_cache = k_cache;

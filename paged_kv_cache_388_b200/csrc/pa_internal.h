@@ -56,6 +56,7 @@ struct AttnArgs {
   // FP8 (E4M3) cache: key elements are codes * k_scale (folded into
   // scale_log2), value elements codes * v_scale; v_inv = 1 / v_scale.
   float v_inv;
+  float o_scale;      // chunk rows: factor on O / l (v_scale over an FP8 cache staged as its codes; else 1)
 };
 
 // Units a (sequence, KV head) pair weighs in the balanced partition beyond

@@ -71,17 +71,37 @@ class PagedKVCache:
         return self._ws if need else None
 
     def attend(self, q, block_tables, context_lens, scale, out=None, query_start_loc=None,
-               max_query_len=1, max_context_len=0, kv_split_tokens=0):
+               max_query_len=1, max_context_len=0, kv_split_tokens=0, staged_blocks=None):
+        """Over an FP8 cache, chunked-prefill rows (max_query_len > 1) stage
+        their sequences' blocks as 16-bit values: ``staged_blocks`` bounds
+        them (``batch.staged_blocks_needed``); when it is None it is counted
+        from query_start_loc and context_lens, which copies both to the host."""
         if out is None:
             out = torch.empty_like(q)
         mcl = max_context_len or block_tables.shape[1] * self.block_size
-        ws = self.workspace(block_tables.shape[0], q.shape[1], mcl, kv_split_tokens)
         if self.fp8:
-            if query_start_loc is not None or kv_split_tokens:
-                raise ValueError("an FP8 cache serves decode rows (one per sequence) only")
+            if kv_split_tokens:
+                raise ValueError("an FP8 cache takes the library's split policy (kv_split_tokens=0)")
+            if query_start_loc is not None and max_query_len > 1:
+                if staged_blocks is None:
+                    from .batch import staged_blocks_needed
+                    staged_blocks = staged_blocks_needed(query_start_loc.cpu(), context_lens.cpu(),
+                                                         self.block_size)
+                need = _lib.pa_decode_fp8_rows_workspace_size(
+                    block_tables.shape[0], q.shape[1], self.num_kv_heads, self.head_dim,
+                    self.block_size, mcl, block_tables.shape[1], max(1, staged_blocks))
+                if self._ws.numel() < need:
+                    self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+                _lib.pa_decode_fp8(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
+                                   scale, self.k_scale, self.v_scale, max_context_len=mcl,
+                                   workspace=self._ws, query_start_loc=query_start_loc,
+                                   max_query_len=max_query_len, staged_blocks=max(1, staged_blocks))
+                return out
+            ws = self.workspace(block_tables.shape[0], q.shape[1], mcl)
             _lib.pa_decode_fp8(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
                                self.k_scale, self.v_scale, max_context_len=mcl, workspace=ws)
             return out
+        ws = self.workspace(block_tables.shape[0], q.shape[1], mcl, kv_split_tokens)
         _lib.pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
                        query_start_loc=query_start_loc, max_query_len=max_query_len,
                        max_context_len=mcl, kv_split_tokens=kv_split_tokens, workspace=ws)

@@ -15,7 +15,7 @@ import torch
 import oracle
 import workloads
 from gpu_harness import assert_close
-from paged_kv_cache_388_b200.batch import build_batch
+from paged_kv_cache_388_b200.batch import build_batch, staged_blocks_needed
 
 pytestmark = pytest.mark.gpu
 
@@ -36,9 +36,14 @@ def _quant(t, s):
     return (t.float() / torch.tensor(s, dtype=torch.float32)).to(torch.float8_e4m3fn).view(torch.uint8)
 
 
-def _run(lib, wl, rows=None, q_mul=1.0):
+def _run(lib, wl, rows=None, q_mul=1.0, staged=None, expect_err=0):
+    """One step over an FP8 cache; mixed batches (chunk rows) go through
+    pa_decode_fp8_rows with `staged` blocks of staging (default: exactly what
+    the batch needs).  With expect_err the device error word must hold those
+    bits and every compared row is either the oracle's or zero."""
     vals = workloads.values(wl)
     batch = build_batch(wl)
+    mixed = batch.query_start_loc is not None and batch.max_query_len > 1
     ks = _scale(vals["k_pool"], vals["new_key"])
     vs = _scale(vals["v_pool"], vals["new_value"])
     kp, vp = _quant(vals["k_pool"], ks), _quant(vals["v_pool"], vs)
@@ -53,14 +58,27 @@ def _run(lib, wl, rows=None, q_mul=1.0):
     if cow.shape[0]:
         lib.pa_copy_blocks(k8, v8, cow)
     lib.pa_reshape_and_cache_fp8(key, value, k8, v8, slot, ks, vs)
-    out = torch.empty_like(q, device=dev)
-    size = lib.pa_decode_workspace_size(batch.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
-                                        wl.block_size, batch.max_context_len, 0)
-    ws = torch.empty(max(size, 16), dtype=torch.uint8, device=dev)
-    lib.pa_decode_fp8(out, q.to(dev), k8, v8, bt, cl, wl.scale, ks, vs,
-                      max_context_len=batch.max_context_len, workspace=ws)
+    out = torch.full_like(q, float("nan"), device=dev)
+    if mixed:
+        if staged is None:
+            staged = staged_blocks_needed(batch.query_start_loc, batch.context_lens, wl.block_size)
+        size = lib.pa_decode_fp8_rows_workspace_size(batch.num_seqs, wl.num_heads, wl.num_kv_heads,
+                                                     wl.head_dim, wl.block_size,
+                                                     batch.max_context_len,
+                                                     batch.block_tables.shape[1], staged)
+        ws = torch.empty(max(size, 16), dtype=torch.uint8, device=dev)
+        lib.pa_decode_fp8(out, q.to(dev), k8, v8, bt, cl, wl.scale, ks, vs,
+                          max_context_len=batch.max_context_len, workspace=ws,
+                          query_start_loc=torch.from_numpy(batch.query_start_loc).to(dev),
+                          max_query_len=batch.max_query_len, staged_blocks=staged)
+    else:
+        size = lib.pa_decode_workspace_size(batch.num_seqs, wl.num_heads, wl.num_kv_heads,
+                                            wl.head_dim, wl.block_size, batch.max_context_len, 0)
+        ws = torch.empty(max(size, 16), dtype=torch.uint8, device=dev)
+        lib.pa_decode_fp8(out, q.to(dev), k8, v8, bt, cl, wl.scale, ks, vs,
+                          max_context_len=batch.max_context_len, workspace=ws)
     torch.cuda.synchronize()
-    assert lib.pa_get_device_error() == 0
+    assert lib.pa_get_device_error() == expect_err
     # the oracle, from the same starting codes
     kpn, vpn = kp.numpy().copy(), vp.numpy().copy()
     if batch.cow_pairs.shape[0]:
@@ -71,7 +89,10 @@ def _run(lib, wl, rows=None, q_mul=1.0):
     assert np.array_equal(k8.cpu().numpy(), kpn), "K codes differ from the oracle"
     assert np.array_equal(v8.cpu().numpy(), vpn), "V codes differ from the oracle"
     ref = oracle.decode_fp8(workloads.to_numpy_raw(q), wl.dtype, kpn, vpn, ks, vs,
-                            batch.block_tables, batch.context_lens, wl.scale, rows=rows)
+                            batch.block_tables, batch.context_lens, wl.scale,
+                            query_start_loc=batch.query_start_loc if mixed else None, rows=rows)
+    if expect_err:
+        return out, ref
     assert_close(out, ref, "bf16", rows=rows, what=wl.name + " fp8")
     return out
 
@@ -157,3 +178,57 @@ def test_session_fp8_step(lib):
                        max_context_len=batch.max_context_len)
     ref = _run(lib, wl)
     assert torch.equal(out, ref)
+
+
+# ---- chunked-prefill rows over an FP8 cache (pa_decode_fp8_rows) ------------
+
+@pytest.mark.parametrize("cfg", ["5s", "5s32"])
+def test_chunk_rows_small(lib, cfg):
+    """Decode rows and 96-token chunks over 700-token prefixes, every row."""
+    _run(lib, workloads.make(cfg))
+
+
+@pytest.mark.parametrize("H,Hk,D,bs,dtype", [(16, 4, 128, 16, "f16"), (8, 2, 64, 32, "bf16"),
+                                             (16, 2, 64, 16, "f16")])
+def test_chunk_rows_shapes(lib, H, Hk, D, bs, dtype):
+    """Other groups, head_dim 64 (the mma.sync chunk kernel) and fp16 q."""
+    wl = workloads.mixed_workload(f"fp8_chunk_{H}_{Hk}_{D}_{bs}_{dtype}", 3400, 2, 100, 900, 3, 150,
+                                  37, H, Hk, D, bs, dtype)
+    _run(lib, wl)
+
+
+def _sample_rows(wl):
+    batch = build_batch(wl)
+    qsl = batch.query_start_loc
+    rows = []
+    for i in range(batch.num_seqs):
+        q0, q1 = int(qsl[i]), int(qsl[i + 1])
+        if q1 - q0 == 1:
+            rows.append(q0)
+        else:
+            rows += list(range(q0, q1, 8)) + [q1 - 1]
+    return sorted(set(rows))
+
+
+@pytest.mark.parametrize("cfg", ["5", "5bs32"])
+def test_chunk_rows_full(lib, cfg):
+    """The long mixed batch over an FP8 cache: every decode row, every 8th
+    chunk row and each chunk's last row."""
+    wl = workloads.make(cfg)
+    _run(lib, wl, rows=_sample_rows(wl))
+
+
+def test_staging_overflow(lib):
+    """A staging bound one block short: PA_DEVERR_STAGING (and BLOCK_ID for
+    the block left out), the rows whose keys reach that block are zeros and
+    every other row is the oracle's."""
+    wl = workloads.make("5s")
+    batch = build_batch(wl)
+    need = staged_blocks_needed(batch.query_start_loc, batch.context_lens, wl.block_size)
+    out, ref = _run(lib, wl, staged=need - 1,
+                    expect_err=lib.PA_DEVERR_STAGING | lib.PA_DEVERR_BLOCK_ID)
+    g = out.float().cpu().numpy().astype(np.float64)
+    zero = np.all(g == 0.0, axis=(1, 2))
+    ok = np.all(np.abs(g - ref) <= 2e-3 + 1e-2 * np.abs(ref), axis=(1, 2))
+    assert np.all(zero | ok)
+    assert zero.any() and ok.any()
