@@ -51,7 +51,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import workloads  # noqa: E402
-from paged_kv_cache_388_b200.batch import build_batch, shared_prefix_groups  # noqa: E402
+from paged_kv_cache_388_b200.batch import (build_batch, shared_prefix_groups,  # noqa: E402
+                                           staged_blocks_needed)
 
 METRIC = "paged decode attention: achieved HBM GB/s (% of peak) and decode tokens/s"
 UNIT = "GB/s"
@@ -60,7 +61,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
 FLUSH_BYTES = 256 * 2 ** 20          # >= 2x L2: reading this evicts every cached line
-EXTRA_CONFIGS = ("2", "3fp8", "4", "4cow", "5", "5bs32", "1")
+EXTRA_CONFIGS = ("2", "3fp8", "4", "4cow", "5", "5bs32", "5fp8", "1")
 
 
 def _peaks():
@@ -374,11 +375,17 @@ class DeviceBatch:
             self.gb_np = gb_np
             self.max_group = int(np.diff(gs_np).max())
         self.bytes = step_bytes(wl, batch, 1 if kv_fp8 else None)
+        # an FP8 cache stages the blocks of chunk-row sequences: the bound is
+        # counted here, on the host, not inside the timed (captured) calls
+        self.staged = None
+        if kv_fp8 and batch.query_start_loc is not None and batch.max_query_len > 1:
+            self.staged = staged_blocks_needed(batch.query_start_loc, batch.context_lens,
+                                               wl.block_size)
 
     def attend_plain(self):
         self.cache.attend(self.q, self.bt, self.cl, self.wl.scale, out=self.out,
                           query_start_loc=self.qsl, max_query_len=self.batch.max_query_len,
-                          max_context_len=self.mcl)
+                          max_context_len=self.mcl, staged_blocks=self.staged)
 
     def attend(self):
         if self.shared:
@@ -406,7 +413,8 @@ class DeviceBatch:
         splits = _lib.pa_decode_workspace_size(b.num_seqs, self.wl.num_heads, self.wl.num_kv_heads,
                                                self.wl.head_dim, self.wl.block_size, self.mcl, 0) > 0
         return 1 + 1 + (1 if splits else 0) + (1 if self.cow.shape[0] else 0) + \
-            (1 if b.max_query_len > 1 else 0) + (1 if self.shared else 0)
+            (1 if b.max_query_len > 1 else 0) + (1 if self.shared else 0) + \
+            (2 if self.staged else 0)  # FP8 chunk rows: staging plan + staging copy
 
     def rows_callable(self, ids):
         """A call attending only the query rows of sequences `ids` (the decode
@@ -421,9 +429,12 @@ class DeviceBatch:
         if t_qsl is not None and mql == 1:
             t_qsl = None
         mcl = int(scl.max())
+        staged = None
+        if self.kv_fp8 and t_qsl is not None:
+            staged = staged_blocks_needed(sqsl, scl, self.wl.block_size)
         return lambda: self.cache.attend(sq, t_bt, t_cl, self.wl.scale, out=sout,
                                          query_start_loc=t_qsl, max_query_len=mql,
-                                         max_context_len=mcl)
+                                         max_context_len=mcl, staged_blocks=staged)
 
 
 def _rate(nbytes, ms):
@@ -577,7 +588,8 @@ def oracle_config_leg(db, gpu_out, target_s=1.5):
         t0 = time.perf_counter()
         if db.kv_fp8:
             ref = oracle.decode_fp8(q, wl.dtype, kp, vp, db.ks, db.vs, batch.block_tables,
-                                    batch.context_lens, wl.scale, rows=rows, threads=threads)
+                                    batch.context_lens, wl.scale, query_start_loc=qsl, rows=rows,
+                                    threads=threads)
         else:
             ref = oracle.decode(q, kp, vp, batch.block_tables, batch.context_lens, wl.scale,
                                 wl.dtype, query_start_loc=qsl, rows=rows, threads=threads)

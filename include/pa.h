@@ -242,7 +242,10 @@ int pa_decode_fp8(void *out, const void *q, const void *k_cache,
  *   workspace      >= pa_decode_fp8_rows_workspace_size(...) bytes.
  * Other arguments as for pa_decode_fp8; the chunk rows need head_dim 128 and
  * group <= 64 for the tensor-core kernels (else the mma.sync chunk kernel).
- * Both parts run on `stream`, the chunk rows first.
+ * The chunk rows (staging and chunk kernel) run on the library's
+ * high-priority stream beside the decode rows, forked from `stream` and
+ * joined back into it as in pa_decode (PA_MIXED_OVERLAP=0: one after the
+ * other on `stream`).
  */
 size_t pa_decode_fp8_rows_workspace_size(int num_seqs, int num_heads,
                                          int num_kv_heads, int head_dim,

@@ -214,90 +214,150 @@ __device__ __forceinline__ uint32_t pack2_t<__nv_bfloat16>(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
 }
-template <>
-__device__ __forceinline__ uint32_t pack2_t<__half>(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&h);
-}
 
-__device__ __forceinline__ float e4m3_value(unsigned char code) {
-  return __half2float(__half(__nv_cvt_fp8_to_halfraw(code, __NV_E4M3)));
-}
 
 // Blocks of chunk-row sequences -> the 16-bit pool (sk, sv) and the tables
 // `tab` [num_seqs][max_blocks_per_seq] (-1 for a block not staged: an id
-// outside the cache, or past the pool's capacity).  Grid (x: blocks, y:
-// sequences); a CTA converts one (block, KV head) K tile and V tile at a time
-// through shared memory, each thread eight consecutive outputs of a row.
+// outside the cache, or past the pool's capacity).  Grid (x: (block, group of
+// up to kStageHeads KV heads), y: sequences).  The K (and V) tiles of
+// consecutive KV heads of a block are one contiguous run in the cache and in
+// the pool.  A thread loads 16-byte runs of codes (all in flight at once),
+// converts each pair of codes with one cvt and stores the values at their
+// places in a plain [head][row][column] tile in shared memory; the group then
+// goes out with 16-byte stores.
+//   K run at byte 16q of a tile: row r = q / (D/16), chunk p = q mod (D/16)
+//     holds k-steps 0..3 of fragment column group 4j + t = p ^ (r mod D/16):
+//     word k, bytes 0,1 -> columns 64j + 16k + 2t, +1; bytes 2,3 -> +8, +9.
+//   V run at byte 16q: column d = 16q / BS, bytes b0 .. b0+15 (b0 = 16q mod
+//     BS) of its transposed keys; byte b is key 16 kk + 2t + (i & 1) + 8 (i >> 1)
+//     with i = b mod 4, and t = b / 4 (BS 16) or t = b / 8, kk = (b / 4) mod 2
+//     (BS 32).
+constexpr int kStageHeads = 4;
+
+template <typename T>
+__device__ __forceinline__ uint32_t e4m3x2_to(uint16_t two);
+template <>
+__device__ __forceinline__ uint32_t e4m3x2_to<__half>(uint16_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);  // low code -> .x
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+template <>
+__device__ __forceinline__ uint32_t e4m3x2_to<__nv_bfloat16>(uint16_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+  return pack2_t<__nv_bfloat16>(f.x, f.y);
+}
+
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(256) fp8_stage_kernel(const AttnArgs a, const int *base,
                                                        int32_t *tab, T *sk, T *sv, int capacity) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ __align__(16) unsigned char kc[BS * D];
-  __shared__ __align__(16) unsigned char vc[BS * D];
+  extern __shared__ __align__(16) unsigned char stage_sm[];  // [K | V][kStageHeads][BS][D] of T
+  constexpr int kTile = BS * D;                               // elements (= code bytes) per tile
+  constexpr int kQ = kTile / 16;                              // 16-byte code runs per tile
+  constexpr int kPer = kStageHeads * kQ / 256;                // runs per thread for K and for V
+  constexpr int G16 = D / 16;
+  uint16_t *ok_sm = reinterpret_cast<uint16_t *>(stage_sm);
+  uint16_t *ov_sm = ok_sm + kStageHeads * kTile;
   const int s = blockIdx.y;
   const int nblk = staged_blocks_of(a, s);
+  const int ngrp = (a.num_kv_heads + kStageHeads - 1) / kStageHeads;
   const unsigned char *kcache = static_cast<const unsigned char *>(a.k_cache);
   const unsigned char *vcache = static_cast<const unsigned char *>(a.v_cache);
-  for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
+  for (int bg = blockIdx.x; bg < nblk * ngrp; bg += gridDim.x) {
+    const int b = bg / ngrp, h0 = (bg - b * ngrp) * kStageHeads;
+    const int nh = min(kStageHeads, a.num_kv_heads - h0);
     const int id = base[s] + b;
     const int src = a.block_tables[(int64_t)s * a.max_blocks_per_seq + b];
     const bool src_ok = src >= 0 && src < a.num_blocks;
     const bool ok = src_ok && id < capacity;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && h0 == 0) {
       tab[(int64_t)s * a.max_blocks_per_seq + b] = ok ? id : -1;
       if (!src_ok) raise_error(a.err, PA_DEVERR_BLOCK_ID);
     }
     if (!ok) continue;  // uniform over the CTA
-    for (int h = 0; h < a.num_kv_heads; ++h) {
-      const int64_t tile = ((int64_t)src * a.num_kv_heads + h) * (BS * D);
-      __syncthreads();  // the previous tile's codes have been read
-      for (int i = threadIdx.x; i < BS * D / 16; i += blockDim.x) {
-        reinterpret_cast<uint4 *>(kc)[i] = reinterpret_cast<const uint4 *>(kcache + tile)[i];
-        reinterpret_cast<uint4 *>(vc)[i] = reinterpret_cast<const uint4 *>(vcache + tile)[i];
-      }
-      __syncthreads();
-      T *dk = sk + ((int64_t)id * a.num_kv_heads + h) * (BS * D);
-      T *dv = sv + ((int64_t)id * a.num_kv_heads + h) * (BS * D);
-      for (int o = threadIdx.x; o < BS * D / 8; o += blockDim.x) {
-        const int r = o / (D / 8), d0 = (o % (D / 8)) * 8;
-        // key r of the V tile: k-step kk, column cc of its 16 keys
-        const int kk = r >> 4, cc = r & 15;
-        const int vt = (cc & 7) >> 1, vi = (cc & 1) + 2 * (cc >> 3);
-        const int vpos = BS == 16 ? 4 * vt + vi : 8 * vt + 4 * kk + vi;
-        float fk[8], fv[8];
+    const int64_t run = ((int64_t)src * a.num_kv_heads + h0) * kTile;
+    const int n16 = nh * kQ;
+    uint4 rk[kPer], rv[kPer];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int d = d0 + e;
-          const int j = d >> 6, k = (d >> 4) & 3, c = d & 15;
-          const int t = (c & 7) >> 1, i = (c & 1) + 2 * (c >> 3);
-          fk[e] = e4m3_value(kc[r * D + (((4 * j + t) ^ (r & (D / 16 - 1))) << 4) + 4 * k + i]);
-          fv[e] = e4m3_value(vc[d * BS + vpos]);
-        }
-        uint4 wk, wv;
-        wk.x = pack2_t<T>(fk[0], fk[1]); wk.y = pack2_t<T>(fk[2], fk[3]);
-        wk.z = pack2_t<T>(fk[4], fk[5]); wk.w = pack2_t<T>(fk[6], fk[7]);
-        wv.x = pack2_t<T>(fv[0], fv[1]); wv.y = pack2_t<T>(fv[2], fv[3]);
-        wv.z = pack2_t<T>(fv[4], fv[5]); wv.w = pack2_t<T>(fv[6], fv[7]);
-        *reinterpret_cast<uint4 *>(dk + r * D + d0) = wk;
-        *reinterpret_cast<uint4 *>(dv + r * D + d0) = wv;
+    for (int u = 0; u < kPer; ++u) {
+      const int i = threadIdx.x + u * 256;
+      if (i < n16) {
+        rk[u] = reinterpret_cast<const uint4 *>(kcache + run)[i];
+        rv[u] = reinterpret_cast<const uint4 *>(vcache + run)[i];
       }
     }
+    __syncthreads();  // the previous group's tile has been copied out
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = threadIdx.x + u * 256;
+      if (i < n16) {
+        const int hh = i / kQ, q = i - hh * kQ;
+        // K: four words, one per k-step, each two adjacent column pairs
+        {
+          const int r = q / G16, p = q - r * G16;
+          const int jt = p ^ (r & (G16 - 1));
+          const int col = 64 * (jt >> 2) + 2 * (jt & 3);
+          uint16_t *row = ok_sm + hh * kTile + r * D;
+          const uint32_t w[4] = {rk[u].x, rk[u].y, rk[u].z, rk[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            *reinterpret_cast<uint32_t *>(row + col + 16 * k) = e4m3x2_to<T>((uint16_t)(w[k] & 0xffffu));
+            *reinterpret_cast<uint32_t *>(row + col + 16 * k + 8) = e4m3x2_to<T>((uint16_t)(w[k] >> 16));
+          }
+        }
+        // V: sixteen keys of one column
+        {
+          const int d = (16 * q) / BS, b0 = (16 * q) % BS;
+          uint16_t *tile = ov_sm + hh * kTile;
+          const uint32_t w[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};
+#pragma unroll
+          for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t two = e4m3x2_to<T>((uint16_t)(half ? w[wi] >> 16 : w[wi] & 0xffffu));
+              const int bb = b0 + 4 * wi + 2 * half;  // byte of the first code of the pair
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int byte = bb + e, i4 = byte & 3;
+                const int t = BS == 16 ? (byte >> 2) : (byte >> 3);
+                const int kk = BS == 16 ? 0 : ((byte >> 2) & 1);
+                const int key = 16 * kk + 2 * t + (i4 & 1) + 8 * (i4 >> 1);
+                tile[key * D + d] = (uint16_t)(e ? two >> 16 : two & 0xffffu);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+    const int64_t dst = ((int64_t)id * a.num_kv_heads + h0) * kTile;
+    for (int i = threadIdx.x; i < nh * kTile / 8; i += blockDim.x) {
+      reinterpret_cast<uint4 *>(sk + dst)[i] = reinterpret_cast<const uint4 *>(ok_sm)[i];
+      reinterpret_cast<uint4 *>(sv + dst)[i] = reinterpret_cast<const uint4 *>(ov_sm)[i];
+    }
   }
+}
+
+template <typename T, int D, int BS>
+cudaError_t launch_stage_bs(const AttnArgs &a, const int *base, int32_t *tab, void *sk, void *sv,
+                            int capacity, cudaStream_t s) {
+  auto kern = fp8_stage_kernel<T, D, BS>;
+  constexpr int kSmem = 2 * kStageHeads * BS * D * 2;
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmem);
+  if (e != cudaSuccess) return e;
+  const int ngrp = (a.num_kv_heads + kStageHeads - 1) / kStageHeads;
+  const int64_t work = (int64_t)a.max_blocks_per_seq * ngrp;
+  const dim3 grid((unsigned)(work < 1024 ? work : 1024), (unsigned)a.num_seqs);
+  kern<<<grid, 256, kSmem, s>>>(a, base, tab, static_cast<T *>(sk), static_cast<T *>(sv), capacity);
+  return cudaGetLastError();
 }
 
 template <typename T, int D>
 cudaError_t launch_stage_t(const AttnArgs &a, const int *base, int32_t *tab, void *sk, void *sv,
                            int capacity, cudaStream_t s) {
-  const int gx = a.max_blocks_per_seq < 256 ? a.max_blocks_per_seq : 256;
-  const dim3 grid((unsigned)gx, (unsigned)a.num_seqs);
-  if (a.block_size == 16)
-    fp8_stage_kernel<T, D, 16><<<grid, 256, 0, s>>>(a, base, tab, static_cast<T *>(sk),
-                                                      static_cast<T *>(sv), capacity);
-  else
-    fp8_stage_kernel<T, D, 32><<<grid, 256, 0, s>>>(a, base, tab, static_cast<T *>(sk),
-                                                      static_cast<T *>(sv), capacity);
-  return cudaGetLastError();
+  return a.block_size == 16 ? launch_stage_bs<T, D, 16>(a, base, tab, sk, sv, capacity, s)
+                            : launch_stage_bs<T, D, 32>(a, base, tab, sk, sv, capacity, s);
 }
 
 // Workspace of pa_decode_fp8_rows: the decode rows' records (the bound of
@@ -418,18 +478,22 @@ int decode_fp8_call(void *out, const void *q, const void *k_cache, const void *v
   a.bal_prefix = reinterpret_cast<int *>(ws + rec + desc);
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
+  // the chunk rows (staging + 16-bit chunk kernel) fork onto the library's
+  // high-priority stream beside the decode rows, as in pa_decode
+  SideStream *side = (chunk_rows && mixed_overlap_wanted()) ? side_fork(s) : nullptr;
+  const cudaStream_t cs = side ? side->stream : s;
+  a.no_pdl = side ? 1 : 0;
   if (chunk_rows) {
-    // the chunk rows: stage their sequences' blocks, then the 16-bit chunk kernel
     int *base = reinterpret_cast<int *>(ws + w.base);
     int32_t *tab = reinterpret_cast<int32_t *>(ws + w.tab);
-    fp8_stage_plan_kernel<<<1, 1024, 0, s>>>(a, base, staged_blocks);
+    fp8_stage_plan_kernel<<<1, 1024, 0, cs>>>(a, base, staged_blocks);
     e = cudaGetLastError();
     if (e == cudaSuccess)
       e = q_dtype == PA_BF16
-              ? (head_dim == 64 ? launch_stage_t<__nv_bfloat16, 64>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s)
-                                : launch_stage_t<__nv_bfloat16, 128>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s))
-              : (head_dim == 64 ? launch_stage_t<__half, 64>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s)
-                                : launch_stage_t<__half, 128>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, s));
+              ? (head_dim == 64 ? launch_stage_t<__nv_bfloat16, 64>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, cs)
+                                : launch_stage_t<__nv_bfloat16, 128>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, cs))
+              : (head_dim == 64 ? launch_stage_t<__half, 64>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, cs)
+                                : launch_stage_t<__half, 128>(a, base, tab, ws + w.k, ws + w.v, staged_blocks, cs));
     if (e == cudaSuccess) {
       AttnArgs c = a;
       c.k_cache = ws + w.k;
@@ -438,11 +502,15 @@ int decode_fp8_call(void *out, const void *q, const void *k_cache, const void *v
       c.num_blocks = staged_blocks;
       c.o_scale = v_scale;
       c.seq_begin = 0;
-      e = launch_chunk(c, q_dtype, num_q_tokens, s);
+      e = launch_chunk(c, q_dtype, num_q_tokens, cs);
     }
   }
   if (e == cudaSuccess) e = launch_decode_mma_fp8(a, q_dtype, dev.sm_count, s);
   if (e == cudaSuccess) e = launch_balanced_reduce(a, q_dtype, s);
+  if (side) {
+    const cudaError_t j = side_join(side, s);  // also after a failed launch
+    if (e == cudaSuccess) e = j;
+  }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -122,7 +122,6 @@ void split_policy(int num_seqs, int num_kv_heads, int block_size, int max_contex
   *max_splits = ceil_div(nblk_max, sb);
 }
 
-namespace {
 
 // A mixed batch's chunk rows (tensor-bound) and decode rows (HBM-bound) read
 // the same caches and write disjoint output rows, so they need no order between
@@ -136,15 +135,11 @@ namespace {
 // mixed batch) and beside its CTAs (both kernels ask for the largest
 // shared-memory carve-out, and a decode CTA fits in what a chunk CTA leaves).
 // PA_MIXED_OVERLAP=0 keeps the two on the caller's stream, one after the other.
-struct SideStream {
-  std::mutex mu;  // held from the fork to the join: one fork-join per device at a time
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-  bool ready = false, failed = false;
-};
+namespace {
 SideStream g_side[kMaxDevices];
+}  // namespace
 
-bool overlap_wanted() {
+bool mixed_overlap_wanted() {
   static const bool on = [] {
     const char *v = getenv("PA_MIXED_OVERLAP");
     return !(v && strcmp(v, "0") == 0);
@@ -200,7 +195,6 @@ cudaError_t side_join(SideStream *sd, cudaStream_t caller) {
   return e;
 }
 
-}  // namespace
 
 }  // namespace pa
 
@@ -377,7 +371,7 @@ int decode_call(void *out, const void *q, const void *k_cache, const void *v_cac
 
   cudaStream_t s = (cudaStream_t)stream;
   const bool chunk_rows = max_query_len > 1 && !a.rows_mode;
-  SideStream *side = (overlap && chunk_rows && overlap_wanted()) ? side_fork(s) : nullptr;
+  SideStream *side = (overlap && chunk_rows && mixed_overlap_wanted()) ? side_fork(s) : nullptr;
   a.no_pdl = side ? 1 : 0;
   cudaError_t e = cudaSuccess;
   for (int s0 = 0; s0 < num_seqs && e == cudaSuccess; s0 += step) {

@@ -1,6 +1,8 @@
 // pa_internal.h -- host-side declarations shared by the libpa translation units.
 #pragma once
 
+#include <mutex>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -86,6 +88,21 @@ struct DevInfo {
 
 // Implemented in pa_api.cu
 cudaError_t device_info(DevInfo *info);
+
+// A second stream of the device's highest priority for a mixed batch's chunk
+// rows, forked from the caller's stream and joined back into it with events
+// (pa_api.cu).  side_fork returns it locked, or nullptr (nothing enqueued):
+// the work then stays on the caller's stream.  mixed_overlap_wanted() is false
+// under PA_MIXED_OVERLAP=0.
+struct SideStream {
+  std::mutex mu;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ready = false, failed = false;
+};
+bool mixed_overlap_wanted();
+SideStream *side_fork(cudaStream_t caller);
+cudaError_t side_join(SideStream *sd, cudaStream_t caller);
 
 // pa_decode with its arguments; overlap = false keeps a mixed batch's chunk
 // rows on the caller's stream after its decode rows (no side stream or events
