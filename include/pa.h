@@ -61,6 +61,7 @@
  *  - Added entry points for the rows after the core path:
  *    pa_decode_shared_prefix (+ its workspace size), pa_reshape_and_cache_fp8,
  *    pa_decode_fp8, pa_decode_fp8_rows (+ its workspace size),
+ *    pa_decode_shared_prefix_fp8 (+ its workspace size),
  *    pa_swap_blocks, pa_decode_noalloc (+
  *    pa_noalloc_scratch_bytes) and pa_abi_version.
  */
@@ -100,8 +101,8 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2, PA_FP8_E4M3 = 3 } pa_dtype;
                                       group's shared prefix, or a member whose block
                                       table differs from the group's first sequence
                                       over the shared range */
-#define PA_DEVERR_STAGING 0x40u    /* pa_decode_fp8_rows: the chunk-row sequences hold
-                                      more blocks than staged_blocks */
+#define PA_DEVERR_STAGING 0x40u    /* pa_decode_fp8_rows / pa_decode_shared_prefix_fp8:
+                                      the blocks to stage exceed staged_blocks */
 
 /*
  * pa_reshape_and_cache -- write this step's new K/V into their cache slots.
@@ -432,6 +433,50 @@ size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_heads,
                                               int num_kv_heads, int head_dim,
                                               int block_size,
                                               int max_context_len);
+
+/*
+ * pa_decode_shared_prefix_fp8 -- pa_decode_shared_prefix over FP8 (E4M3)
+ * caches written by pa_reshape_and_cache_fp8 (key = code * k_scale, value =
+ * code * v_scale), q/out of q_dtype (PA_F16 or PA_BF16).  The shared blocks of
+ * each group's first sequence are copied into a staging pool inside the
+ * workspace as the 16-bit values of their codes (exact) and the prefix pass
+ * of pa_decode_shared_prefix runs over that pool (k_scale in the logit scale,
+ * its partial sums kept in units of 1/v_scale); the private tails run on the
+ * FP8 decode kernel, which folds the prefix partials in.  A member whose
+ * table differs from its group's first sequence over the shared range is
+ * reported and zeroed as in pa_decode_shared_prefix.
+ *
+ *   staged_blocks  host-side bound of the staging pool in blocks: at least
+ *                  sum over groups of group_shared_blocks[j]; > 0 when
+ *                  num_groups > 0.  A batch holding more sets
+ *                  PA_DEVERR_STAGING (the groups past the bound read as bad
+ *                  blocks: their members' rows are zeros).
+ *   workspace      >= pa_decode_shared_prefix_fp8_workspace_size(...) bytes.
+ * Supported: group = num_heads / num_kv_heads <= 16, num_seqs <= 2048.
+ */
+int pa_decode_shared_prefix_fp8(void *out, const void *q, const void *k_cache,
+                                const void *v_cache, const int32_t *block_tables,
+                                int max_blocks_per_seq,
+                                const int32_t *context_lens, int num_seqs,
+                                const int32_t *group_start,
+                                const int32_t *group_shared_blocks,
+                                int num_groups, int max_group_size,
+                                int num_heads, int num_kv_heads, int head_dim,
+                                int block_size, int num_blocks, float scale,
+                                float k_scale, float v_scale,
+                                int max_context_len, int staged_blocks,
+                                int q_dtype, void *workspace,
+                                size_t workspace_bytes,
+                                struct CUstream_st *stream);
+
+/* Workspace bytes pa_decode_shared_prefix_fp8 needs (current device). */
+size_t pa_decode_shared_prefix_fp8_workspace_size(int num_seqs, int num_heads,
+                                                  int num_kv_heads,
+                                                  int head_dim, int block_size,
+                                                  int max_context_len,
+                                                  int max_blocks_per_seq,
+                                                  int num_groups,
+                                                  int staged_blocks);
 
 /*
  * pa_get_device_error -- synchronise `stream`, then read and clear the

@@ -54,6 +54,11 @@ _lib.pa_decode_shared_prefix.argtypes = [P, P, P, P, P, I, P, I, P, P, I, I, I, 
                                          P, SZ, P]
 _lib.pa_decode_shared_prefix_workspace_size.restype = SZ
 _lib.pa_decode_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I]
+_lib.pa_decode_shared_prefix_fp8.restype = I
+_lib.pa_decode_shared_prefix_fp8.argtypes = [P, P, P, P, P, I, P, I, P, P, I, I, I, I, I, I, I, F,
+                                             F, F, I, I, I, P, SZ, P]
+_lib.pa_decode_shared_prefix_fp8_workspace_size.restype = SZ
+_lib.pa_decode_shared_prefix_fp8_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I]
 _lib.pa_noalloc_scratch_bytes.restype = SZ
 _lib.pa_noalloc_scratch_bytes.argtypes = []
 _lib.pa_get_device_error.restype = I
@@ -393,6 +398,48 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
                                       int(max_context_len), _DT[q.dtype], _ptr(workspace),
                                       ws_bytes, _stream(stream))
     _check(rc, "pa_decode_shared_prefix")
+
+
+def pa_decode_shared_prefix_fp8_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                               block_size, max_context_len, max_blocks_per_seq,
+                                               num_groups, staged_blocks) -> int:
+    return int(_lib.pa_decode_shared_prefix_fp8_workspace_size(
+        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+        max_blocks_per_seq, num_groups, staged_blocks))
+
+
+def pa_decode_shared_prefix_fp8(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                                group_shared_blocks, scale, k_scale, v_scale, staged_blocks,
+                                max_group_size=0, max_context_len=0, workspace=None, stream=None):
+    """pa_decode_shared_prefix over FP8 (E4M3) caches (uint8 codes); out/q
+    fp16/bf16 [S, H, D]; staged_blocks bounds the groups' shared blocks
+    (their sum); workspace uint8 of
+    >= pa_decode_shared_prefix_fp8_workspace_size(...) bytes."""
+    s, h, d, nb, hk, bs, _, mbps = _decode_shapes(out, q, k_cache, v_cache, block_tables,
+                                                  context_lens)
+    _shape(group_start.dim() == 1 and group_shared_blocks.dim() == 1 and
+           group_start.shape[0] == group_shared_blocks.shape[0] + 1,
+           "group_start must have one more entry than group_shared_blocks")
+    _dev(q, "q")
+    _dev(out, "out", q.dtype)
+    _dev(k_cache, "k_cache", torch.uint8)
+    _dev(v_cache, "v_cache", torch.uint8)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    _dev(group_start, "group_start", torch.int32)
+    _dev(group_shared_blocks, "group_shared_blocks", torch.int32)
+    if workspace is not None:
+        _dev(workspace, "workspace")
+    g = group_shared_blocks.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.pa_decode_shared_prefix_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(block_tables), mbps, _ptr(context_lens), s,
+                                          _ptr(group_start), _ptr(group_shared_blocks), g,
+                                          int(max_group_size), h, hk, d, bs, nb, float(scale),
+                                          float(k_scale), float(v_scale), int(max_context_len),
+                                          int(staged_blocks), _DT[q.dtype], _ptr(workspace),
+                                          ws_bytes, _stream(stream))
+    _check(rc, "pa_decode_shared_prefix_fp8")
 
 
 def pa_noalloc_scratch_bytes() -> int:

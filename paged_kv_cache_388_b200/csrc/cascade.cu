@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (part == 0) {
         rec[D] = M;
-        rec[D + 1] = rbad ? __int_as_float(0x7fc00000) : l;
+        rec[D + 1] = rbad ? __int_as_float(0x7fc00000) : l / a.o_scale;
       }
     }
   }

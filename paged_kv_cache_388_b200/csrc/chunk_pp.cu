@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (write) {
           rec[kD] = m_used;
-          rec[kD + 1] = poison ? __int_as_float(0x7fc00000) : l;
+          rec[kD + 1] = poison ? __int_as_float(0x7fc00000) : l / a.o_scale;
         }
         tc_fence_before();
       } else {

@@ -637,7 +637,7 @@ __global__ void __launch_bounds__(32 * (4 * kHalves * NQ + 2), PA_CHUNK_TC_MIN_C
       }
       if (write && hf == 0) {
         rec[D] = m_used;
-        rec[D + 1] = poison ? __int_as_float(0x7fc00000) : l;
+        rec[D + 1] = poison ? __int_as_float(0x7fc00000) : l / a.o_scale;
       }
     } else {
       const float inv = (ok && l > 0.f && !flags[1]) ? (1.f / l) * a.o_scale : 0.f;

@@ -248,25 +248,91 @@ __device__ __forceinline__ uint32_t e4m3x2_to<__nv_bfloat16>(uint16_t two) {
   return pack2_t<__nv_bfloat16>(f.x, f.y);
 }
 
+// Converts the K and V tiles of KV heads h0 .. h0+nh-1 of cache block `src`
+// into pool block `id` (CTA-wide: every thread of the CTA calls it).
+template <typename T, int D, int BS>
+__device__ __forceinline__ void stage_group(const AttnArgs &a, int src, int id, int h0, int nh,
+                                            T *sk, T *sv, unsigned char *stage_sm) {
+  constexpr int kTile = BS * D;                 // elements (= code bytes) per tile
+  constexpr int kQ = kTile / 16;                // 16-byte code runs per tile
+  constexpr int kPer = kStageHeads * kQ / 256;  // runs per thread for K and for V
+  constexpr int G16 = D / 16;
+  uint16_t *ok_sm = reinterpret_cast<uint16_t *>(stage_sm);
+  uint16_t *ov_sm = ok_sm + kStageHeads * kTile;
+  const unsigned char *kcache = static_cast<const unsigned char *>(a.k_cache);
+  const unsigned char *vcache = static_cast<const unsigned char *>(a.v_cache);
+  const int64_t run = ((int64_t)src * a.num_kv_heads + h0) * kTile;
+  const int n16 = nh * kQ;
+  uint4 rk[kPer], rv[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + u * 256;
+    if (i < n16) {
+      rk[u] = reinterpret_cast<const uint4 *>(kcache + run)[i];
+      rv[u] = reinterpret_cast<const uint4 *>(vcache + run)[i];
+    }
+  }
+  __syncthreads();  // the previous group's tile has been copied out
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = threadIdx.x + u * 256;
+    if (i < n16) {
+      const int hh = i / kQ, q = i - hh * kQ;
+      // K: four words, one per k-step, each two adjacent column pairs
+      {
+        const int r = q / G16, p = q - r * G16;
+        const int jt = p ^ (r & (G16 - 1));
+        const int col = 64 * (jt >> 2) + 2 * (jt & 3);
+        uint16_t *row = ok_sm + hh * kTile + r * D;
+        const uint32_t w[4] = {rk[u].x, rk[u].y, rk[u].z, rk[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          *reinterpret_cast<uint32_t *>(row + col + 16 * k) = e4m3x2_to<T>((uint16_t)(w[k] & 0xffffu));
+          *reinterpret_cast<uint32_t *>(row + col + 16 * k + 8) = e4m3x2_to<T>((uint16_t)(w[k] >> 16));
+        }
+      }
+      // V: sixteen keys of one column
+      {
+        const int d = (16 * q) / BS, b0 = (16 * q) % BS;
+        uint16_t *tile = ov_sm + hh * kTile;
+        const uint32_t w[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t two = e4m3x2_to<T>((uint16_t)(half ? w[wi] >> 16 : w[wi] & 0xffffu));
+            const int bb = b0 + 4 * wi + 2 * half;  // byte of the first code of the pair
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int byte = bb + e, i4 = byte & 3;
+              const int t = BS == 16 ? (byte >> 2) : (byte >> 3);
+              const int kk = BS == 16 ? 0 : ((byte >> 2) & 1);
+              const int key = 16 * kk + 2 * t + (i4 & 1) + 8 * (i4 >> 1);
+              tile[key * D + d] = (uint16_t)(e ? two >> 16 : two & 0xffffu);
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int64_t dst = ((int64_t)id * a.num_kv_heads + h0) * kTile;
+  for (int i = threadIdx.x; i < nh * kTile / 8; i += blockDim.x) {
+    reinterpret_cast<uint4 *>(sk + dst)[i] = reinterpret_cast<const uint4 *>(ok_sm)[i];
+    reinterpret_cast<uint4 *>(sv + dst)[i] = reinterpret_cast<const uint4 *>(ov_sm)[i];
+  }
+}
+
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(256) fp8_stage_kernel(const AttnArgs a, const int *base,
                                                        int32_t *tab, T *sk, T *sv, int capacity) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) unsigned char stage_sm[];  // [K | V][kStageHeads][BS][D] of T
-  constexpr int kTile = BS * D;                               // elements (= code bytes) per tile
-  constexpr int kQ = kTile / 16;                              // 16-byte code runs per tile
-  constexpr int kPer = kStageHeads * kQ / 256;                // runs per thread for K and for V
-  constexpr int G16 = D / 16;
-  uint16_t *ok_sm = reinterpret_cast<uint16_t *>(stage_sm);
-  uint16_t *ov_sm = ok_sm + kStageHeads * kTile;
   const int s = blockIdx.y;
   const int nblk = staged_blocks_of(a, s);
   const int ngrp = (a.num_kv_heads + kStageHeads - 1) / kStageHeads;
-  const unsigned char *kcache = static_cast<const unsigned char *>(a.k_cache);
-  const unsigned char *vcache = static_cast<const unsigned char *>(a.v_cache);
   for (int bg = blockIdx.x; bg < nblk * ngrp; bg += gridDim.x) {
     const int b = bg / ngrp, h0 = (bg - b * ngrp) * kStageHeads;
-    const int nh = min(kStageHeads, a.num_kv_heads - h0);
     const int id = base[s] + b;
     const int src = a.block_tables[(int64_t)s * a.max_blocks_per_seq + b];
     const bool src_ok = src >= 0 && src < a.num_blocks;
@@ -276,67 +342,112 @@ __global__ void __launch_bounds__(256) fp8_stage_kernel(const AttnArgs a, const 
       if (!src_ok) raise_error(a.err, PA_DEVERR_BLOCK_ID);
     }
     if (!ok) continue;  // uniform over the CTA
-    const int64_t run = ((int64_t)src * a.num_kv_heads + h0) * kTile;
-    const int n16 = nh * kQ;
-    uint4 rk[kPer], rv[kPer];
+    stage_group<T, D, BS>(a, src, id, h0, min(kStageHeads, a.num_kv_heads - h0), sk, sv, stage_sm);
+  }
+}
+
+// Shared prefixes over an FP8 cache: group j (sequences grp_start[j] ..
+// grp_start[j+1]-1 sharing grp_blocks[j] leading blocks) stages those blocks
+// of its first sequence at pool blocks base[j] ..; gbase[num_groups] = total.
+__device__ __forceinline__ int group_blocks_of(const AttnArgs &a, int j) {
+  const int s0 = a.grp_start[j], s1 = a.grp_start[j + 1], P = a.grp_blocks[j];
+  const bool valid = 0 <= s0 && s0 < s1 && s1 <= a.num_seqs && 0 < P && P <= a.max_blocks_per_seq;
+  return valid ? P : 0;
+}
+
+__global__ void __launch_bounds__(1024) fp8_group_plan_kernel(const AttnArgs a, int *gbase,
+                                                             int capacity) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int j0 = 0; j0 < a.num_groups; j0 += 1024) {
+    const int j = j0 + tid;
+    const int c = j < a.num_groups ? group_blocks_of(a, j) : 0;
+    int incl = c;
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = threadIdx.x + u * 256;
-      if (i < n16) {
-        rk[u] = reinterpret_cast<const uint4 *>(kcache + run)[i];
-        rv[u] = reinterpret_cast<const uint4 *>(vcache + run)[i];
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    __syncthreads();  // the previous group's tile has been copied out
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_tot[lane];
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = threadIdx.x + u * 256;
-      if (i < n16) {
-        const int hh = i / kQ, q = i - hh * kQ;
-        // K: four words, one per k-step, each two adjacent column pairs
-        {
-          const int r = q / G16, p = q - r * G16;
-          const int jt = p ^ (r & (G16 - 1));
-          const int col = 64 * (jt >> 2) + 2 * (jt & 3);
-          uint16_t *row = ok_sm + hh * kTile + r * D;
-          const uint32_t w[4] = {rk[u].x, rk[u].y, rk[u].z, rk[u].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            *reinterpret_cast<uint32_t *>(row + col + 16 * k) = e4m3x2_to<T>((uint16_t)(w[k] & 0xffffu));
-            *reinterpret_cast<uint32_t *>(row + col + 16 * k + 8) = e4m3x2_to<T>((uint16_t)(w[k] >> 16));
-          }
-        }
-        // V: sixteen keys of one column
-        {
-          const int d = (16 * q) / BS, b0 = (16 * q) % BS;
-          uint16_t *tile = ov_sm + hh * kTile;
-          const uint32_t w[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};
-#pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const uint32_t two = e4m3x2_to<T>((uint16_t)(half ? w[wi] >> 16 : w[wi] & 0xffffu));
-              const int bb = b0 + 4 * wi + 2 * half;  // byte of the first code of the pair
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int byte = bb + e, i4 = byte & 3;
-                const int t = BS == 16 ? (byte >> 2) : (byte >> 3);
-                const int kk = BS == 16 ? 0 : ((byte >> 2) & 1);
-                const int key = 16 * kk + 2 * t + (i4 & 1) + 8 * (i4 >> 1);
-                tile[key * D + d] = (uint16_t)(e ? two >> 16 : two & 0xffffu);
-              }
-            }
-          }
-        }
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
       }
+      warp_tot[lane] = w;
     }
     __syncthreads();
-    const int64_t dst = ((int64_t)id * a.num_kv_heads + h0) * kTile;
-    for (int i = threadIdx.x; i < nh * kTile / 8; i += blockDim.x) {
-      reinterpret_cast<uint4 *>(sk + dst)[i] = reinterpret_cast<const uint4 *>(ok_sm)[i];
-      reinterpret_cast<uint4 *>(sv + dst)[i] = reinterpret_cast<const uint4 *>(ov_sm)[i];
-    }
+    const int before = carry + (warp > 0 ? warp_tot[warp - 1] : 0);
+    if (j < a.num_groups) gbase[j] = before + incl - c;
+    __syncthreads();
+    if (tid == 0) carry += warp_tot[31];
+    __syncthreads();
   }
+  if (tid == 0) {
+    gbase[a.num_groups] = carry;
+    if (carry > capacity) raise_error(a.err, PA_DEVERR_STAGING);
+  }
+}
+
+// Grid (x: (shared block, group of KV heads), y: groups).  Every member's
+// table row over the shared range gets the staged id where it holds the first
+// sequence's block and -1 where it does not, so that the prefix kernel's
+// member check still sees a member whose table differs.
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(256) fp8_group_stage_kernel(const AttnArgs a, const int *gbase,
+                                                             int32_t *tab, T *sk, T *sv,
+                                                             int capacity) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ __align__(16) unsigned char stage_sm[];
+  const int j = blockIdx.y;
+  const int P = group_blocks_of(a, j);
+  if (P == 0) return;
+  const int s0 = a.grp_start[j], s1 = a.grp_start[j + 1];
+  const int ngrp = (a.num_kv_heads + kStageHeads - 1) / kStageHeads;
+  for (int bg = blockIdx.x; bg < P * ngrp; bg += gridDim.x) {
+    const int b = bg / ngrp, h0 = (bg - b * ngrp) * kStageHeads;
+    const int id = gbase[j] + b;
+    const int src = a.block_tables[(int64_t)s0 * a.max_blocks_per_seq + b];
+    const bool src_ok = src >= 0 && src < a.num_blocks;
+    const bool ok = src_ok && id < capacity;
+    if (h0 == 0) {
+      for (int m = s0 + (int)threadIdx.x; m < s1; m += blockDim.x) {
+        const int mine = a.block_tables[(int64_t)m * a.max_blocks_per_seq + b];
+        tab[(int64_t)m * a.max_blocks_per_seq + b] = (ok && mine == src) ? id : -1;
+      }
+      if (threadIdx.x == 0 && !src_ok) raise_error(a.err, PA_DEVERR_BLOCK_ID);
+    }
+    if (!ok) continue;  // uniform over the CTA
+    stage_group<T, D, BS>(a, src, id, h0, min(kStageHeads, a.num_kv_heads - h0), sk, sv, stage_sm);
+  }
+}
+
+template <typename T, int D, int BS>
+cudaError_t launch_group_stage_bs(const AttnArgs &a, const int *gbase, int32_t *tab, void *sk,
+                                  void *sv, int capacity, cudaStream_t s) {
+  auto kern = fp8_group_stage_kernel<T, D, BS>;
+  constexpr int kSmem = 2 * kStageHeads * BS * D * 2;
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(kern), kSmem);
+  if (e != cudaSuccess) return e;
+  const int ngrp = (a.num_kv_heads + kStageHeads - 1) / kStageHeads;
+  const int64_t work = (int64_t)a.max_blocks_per_seq * ngrp;
+  const dim3 grid((unsigned)(work < 1024 ? work : 1024), (unsigned)a.num_groups);
+  kern<<<grid, 256, kSmem, s>>>(a, gbase, tab, static_cast<T *>(sk), static_cast<T *>(sv), capacity);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_group_stage_t(const AttnArgs &a, const int *gbase, int32_t *tab, void *sk,
+                                 void *sv, int capacity, cudaStream_t s) {
+  return a.block_size == 16 ? launch_group_stage_bs<T, D, 16>(a, gbase, tab, sk, sv, capacity, s)
+                            : launch_group_stage_bs<T, D, 32>(a, gbase, tab, sk, sv, capacity, s);
 }
 
 template <typename T, int D, int BS>
@@ -385,6 +496,24 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool scale_ok(float s) { return s > 0.f && s < 3.0e38f; }
 
 }  // namespace
+
+cudaError_t launch_fp8_group_stage(const AttnArgs &a, int q_dtype, int *gbase, int32_t *tab,
+                                   void *sk, void *sv, int capacity, cudaStream_t s) {
+  if (a.num_groups <= 0) return cudaSuccess;
+  fp8_group_plan_kernel<<<1, 1024, 0, s>>>(a, gbase, capacity);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (q_dtype == PA_BF16)
+    return a.head_dim == 64 ? launch_group_stage_t<__nv_bfloat16, 64>(a, gbase, tab, sk, sv, capacity, s)
+                            : launch_group_stage_t<__nv_bfloat16, 128>(a, gbase, tab, sk, sv, capacity, s);
+  return a.head_dim == 64 ? launch_group_stage_t<__half, 64>(a, gbase, tab, sk, sv, capacity, s)
+                          : launch_group_stage_t<__half, 128>(a, gbase, tab, sk, sv, capacity, s);
+}
+
+size_t fp8_pool_bytes(int staged_blocks, int num_kv_heads, int head_dim, int block_size) {
+  return ((size_t)staged_blocks * num_kv_heads * block_size * head_dim * 2 + 1023) / 1024 * 1024;
+}
+
 }  // namespace pa
 
 using namespace pa;

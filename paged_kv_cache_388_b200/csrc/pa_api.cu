@@ -572,6 +572,145 @@ int pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// Workspace of pa_decode_shared_prefix_fp8: that of pa_decode_shared_prefix,
+// then the staging plan (gbase), the staged tables and the two 16-bit pools.
+size_t pa_decode_shared_prefix_fp8_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                                  int head_dim, int block_size,
+                                                  int max_context_len, int max_blocks_per_seq,
+                                                  int num_groups, int staged_blocks) {
+  if (max_blocks_per_seq <= 0 || num_groups < 0 || staged_blocks < 0 || block_size <= 0) return 0;
+  const size_t base = pa_decode_shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads,
+                                                             head_dim, block_size, max_context_len);
+  if (base == 0) return 0;
+  auto up = [](size_t x) { return (x + 1023) / 1024 * 1024; };
+  return up(base) + up((size_t)(num_groups + 1) * sizeof(int)) +
+         up((size_t)num_seqs * max_blocks_per_seq * sizeof(int32_t)) +
+         2 * fp8_pool_bytes(staged_blocks, num_kv_heads, head_dim, block_size);
+}
+
+int pa_decode_shared_prefix_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *context_lens, int num_seqs,
+                                const int32_t *group_start, const int32_t *group_shared_blocks,
+                                int num_groups, int max_group_size, int num_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                float scale, float k_scale, float v_scale, int max_context_len,
+                                int staged_blocks, int q_dtype, void *workspace,
+                                size_t workspace_bytes, struct CUstream_st *stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || num_groups < 0 || staged_blocks < 0)
+    return PA_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f && k_scale < 3.0e38f) || !(v_scale > 0.f && v_scale < 3.0e38f))
+    return PA_ERR_INVALID_ARG;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_heads / num_kv_heads;
+  if (!group_supported(group) || group > 16) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > decode_max_seqs_per_launch()) return PA_ERR_UNSUPPORTED;
+  if (num_groups > 0 && staged_blocks == 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (num_groups > 0 && (!group_start || !group_shared_blocks)) return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (out == q) return PA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * block_size > (int64_t)1 << 30) return PA_ERR_UNSUPPORTED;
+  const int cap = max_blocks_per_seq * block_size;
+  if (max_context_len <= 0 || max_context_len > cap) max_context_len = cap;
+  if (max_group_size <= 0 || max_group_size > num_seqs) max_group_size = num_seqs;
+
+  DevInfo dev;
+  if (device_info(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  AttnArgs a{};
+  a.o_scale = 1.f;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start_loc = nullptr;
+  a.err = dev.err;
+  a.num_seqs = num_seqs;
+  a.seq_begin = 0;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.split_blocks = 1;
+  a.max_splits = 1;
+  a.max_query_len = 1;
+  a.max_context_len = max_context_len;
+  a.num_q_tokens = num_seqs;
+  a.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  a.v_inv = 1.f / v_scale;
+  a.balanced = 1;
+  a.item_units = kItemUnitsFp8;
+  if (!prefix_supported(a, q_dtype)) return PA_ERR_UNSUPPORTED;
+  a.grid = decode_mma_grid_fp8(a, q_dtype, dev.sm_count);
+  if (a.grid <= 0) return PA_ERR_CUDA;
+  const SharedPrefixWs w = shared_prefix_ws(num_seqs, num_heads, head_dim, group, a.grid);
+  auto up = [](size_t x) { return (x + 1023) / 1024 * 1024; };
+  const size_t off_g = up(shared_prefix_ws(num_seqs, num_heads, head_dim, group, dev.sm_count * 8).total);
+  const size_t off_t = off_g + up((size_t)(num_groups + 1) * sizeof(int));
+  const size_t off_k = off_t + up((size_t)num_seqs * max_blocks_per_seq * sizeof(int32_t));
+  const size_t pool = fp8_pool_bytes(staged_blocks, num_kv_heads, head_dim, block_size);
+  const size_t total = off_k + 2 * pool;
+  if (w.total > off_g || !workspace || workspace_bytes < total || !aligned16(workspace))
+    return PA_ERR_WORKSPACE;
+  char *ws = static_cast<char *>(workspace);
+  a.part_o = reinterpret_cast<float *>(ws);
+  a.bal_desc = reinterpret_cast<int *>(ws + w.desc);
+  a.bal_prefix = reinterpret_cast<int *>(ws + w.prefix);
+  a.seq_pre = reinterpret_cast<int *>(ws + w.seq_pre);
+  a.pre_rec = reinterpret_cast<float *>(ws + w.pre_rec);
+  a.grp_start = group_start;
+  a.grp_blocks = group_shared_blocks;
+  a.num_groups = num_groups;
+  const int mpc = kPrefixRows / group;
+  a.grp_chunks = (max_group_size + mpc - 1) / mpc;
+  a.max_group = max_group_size;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (num_groups > 0) {
+    // the shared blocks: staged as 16-bit values of their codes, then the
+    // prefix pass of pa_decode_shared_prefix over that pool (k_scale in the
+    // logit scale; its records hold l / v_scale, the decode kernel's units)
+    int *gbase = reinterpret_cast<int *>(ws + off_g);
+    int32_t *tab = reinterpret_cast<int32_t *>(ws + off_t);
+    e = launch_fp8_group_stage(a, q_dtype, gbase, tab, ws + off_k, ws + off_k + pool, staged_blocks, s);
+    AttnArgs p = a;
+    p.k_cache = ws + off_k;
+    p.v_cache = ws + off_k + pool;
+    p.block_tables = tab;
+    p.num_blocks = staged_blocks;
+    p.o_scale = v_scale;
+    const char *sel = getenv("PA_PREFIX_KERNEL");
+    const bool want_mma = sel && strcmp(sel, "mma") == 0;
+    const bool want_pp = sel && strcmp(sel, "pp") == 0;
+    if (e == cudaSuccess) {
+      if (want_pp && chunk_pp_supported(p, q_dtype)) {
+        e = launch_prefix_pp(p, q_dtype, s);
+      } else if (!want_mma && chunk_tc_supported(p, q_dtype)) {
+        e = launch_prefix_tc(p, q_dtype, s);
+      } else {
+        const int64_t units = (int64_t)num_groups * a.grp_chunks * num_kv_heads;
+        e = launch_prefix(p, q_dtype, prefix_cluster(units, dev.sm_count), s);
+      }
+    }
+  }
+  if (e == cudaSuccess) e = launch_decode_mma_fp8(a, q_dtype, dev.sm_count, s);
+  if (e == cudaSuccess) e = launch_balanced_reduce(a, q_dtype, s);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int pa_get_device_error(unsigned int *code_out, struct CUstream_st *stream) {
   if (!code_out) return PA_ERR_INVALID_ARG;
   DevInfo dev;

@@ -58,7 +58,8 @@ struct AttnArgs {
   // FP8 (E4M3) cache: key elements are codes * k_scale (folded into
   // scale_log2), value elements codes * v_scale; v_inv = 1 / v_scale.
   float v_inv;
-  float o_scale;      // chunk rows: factor on O / l (v_scale over an FP8 cache staged as its codes; else 1)
+  float o_scale;      // factor on O / l: v_scale over an FP8 cache staged as its codes, else 1
+                      // (chunk rows scale their output by it, prefix records store l / o_scale)
 };
 
 // Units a (sequence, KV head) pair weighs in the balanced partition beyond
@@ -178,6 +179,16 @@ cudaError_t launch_prefix_pp(const AttnArgs &a, int dtype, cudaStream_t stream);
 
 // Implemented in chunk.cu
 cudaError_t launch_chunk(const AttnArgs &a, int dtype, int num_q_tokens, cudaStream_t stream);
+
+// FP8 shared prefixes (fp8.cu): stage the shared blocks of every group of `a`
+// (an FP8 cache, grp_* set) into 16-bit pools sk/sv of `capacity` blocks with
+// tables `tab` (same row stride as a.block_tables; -1 where a member's block
+// differs from its group's first sequence), gbase [num_groups + 1] scratch;
+// PA_DEVERR_STAGING when the groups hold more than capacity blocks.
+cudaError_t launch_fp8_group_stage(const AttnArgs &a, int q_dtype, int *gbase, int32_t *tab,
+                                   void *sk, void *sv, int capacity, cudaStream_t s);
+// Bytes of one staging pool (K or V) of `staged_blocks` 16-bit blocks, 1 KiB aligned.
+size_t fp8_pool_bytes(int staged_blocks, int num_kv_heads, int head_dim, int block_size);
 
 // Implemented in cache_ops.cu
 cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache,

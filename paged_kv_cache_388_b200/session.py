@@ -108,15 +108,35 @@ class PagedKVCache:
         return out
 
     def attend_shared_prefix(self, q, block_tables, context_lens, group_start, group_shared_blocks,
-                             scale, max_group_size=0, out=None, max_context_len=0):
+                             scale, max_group_size=0, out=None, max_context_len=0,
+                             staged_blocks=None):
         """Decode (one query row per sequence) where groups of consecutive
         sequences share the leading blocks of their tables: group j is
         sequences group_start[j] .. group_start[j+1]-1 sharing
         group_shared_blocks[j] blocks (see ``batch.shared_prefix_groups``).
-        Same result as ``attend``; the shared blocks are read once per group."""
+        Same result as ``attend``; the shared blocks are read once per group.
+        Over an FP8 cache the shared blocks are staged as 16-bit values:
+        ``staged_blocks`` bounds their total (when None it is summed from
+        group_shared_blocks, which copies it to the host)."""
         if out is None:
             out = torch.empty_like(q)
         mcl = max_context_len or block_tables.shape[1] * self.block_size
+        if self.fp8:
+            if staged_blocks is None:
+                staged_blocks = int(group_shared_blocks.cpu().clamp(min=0).sum())
+            staged_blocks = max(1, int(staged_blocks))
+            need = _lib.pa_decode_shared_prefix_fp8_workspace_size(
+                block_tables.shape[0], q.shape[1], self.num_kv_heads, self.head_dim,
+                self.block_size, mcl, block_tables.shape[1], group_shared_blocks.shape[0],
+                staged_blocks)
+            if self._ws.numel() < need:
+                self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            _lib.pa_decode_shared_prefix_fp8(out, q, self.k_cache, self.v_cache, block_tables,
+                                             context_lens, group_start, group_shared_blocks, scale,
+                                             self.k_scale, self.v_scale, staged_blocks,
+                                             max_group_size=max_group_size, max_context_len=mcl,
+                                             workspace=self._ws)
+            return out
         need = _lib.pa_decode_shared_prefix_workspace_size(block_tables.shape[0], q.shape[1],
                                                            self.num_kv_heads, self.head_dim,
                                                            self.block_size, mcl)

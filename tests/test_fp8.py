@@ -15,7 +15,7 @@ import torch
 import oracle
 import workloads
 from gpu_harness import assert_close
-from paged_kv_cache_388_b200.batch import build_batch, staged_blocks_needed
+from paged_kv_cache_388_b200.batch import build_batch, shared_prefix_groups, staged_blocks_needed
 
 pytestmark = pytest.mark.gpu
 
@@ -227,6 +227,104 @@ def test_staging_overflow(lib):
     need = staged_blocks_needed(batch.query_start_loc, batch.context_lens, wl.block_size)
     out, ref = _run(lib, wl, staged=need - 1,
                     expect_err=lib.PA_DEVERR_STAGING | lib.PA_DEVERR_BLOCK_ID)
+    g = out.float().cpu().numpy().astype(np.float64)
+    zero = np.all(g == 0.0, axis=(1, 2))
+    ok = np.all(np.abs(g - ref) <= 2e-3 + 1e-2 * np.abs(ref), axis=(1, 2))
+    assert np.all(zero | ok)
+    assert zero.any() and ok.any()
+
+
+# ---- shared prefixes over an FP8 cache (pa_decode_shared_prefix_fp8) --------
+
+def _run_shared(lib, wl, staged=None, expect_err=0, mutate=None):
+    """One step over an FP8 cache through pa_decode_shared_prefix_fp8 with the
+    batch's shared-prefix groups, against the oracle's plain FP8 decode (the
+    same attention).  `mutate(block_tables) -> block_tables` alters the tables
+    the call and the oracle see; returns (out, ref)."""
+    vals = workloads.values(wl)
+    batch = build_batch(wl)
+    ks = _scale(vals["k_pool"], vals["new_key"])
+    vs = _scale(vals["v_pool"], vals["new_value"])
+    kp, vp = _quant(vals["k_pool"], ks), _quant(vals["v_pool"], vs)
+    dev = "cuda"
+    k8, v8 = kp.to(dev), vp.to(dev)
+    cow = torch.from_numpy(np.ascontiguousarray(batch.cow_pairs)).to(dev)
+    if cow.shape[0]:
+        lib.pa_copy_blocks(k8, v8, cow)
+    lib.pa_reshape_and_cache_fp8(vals["new_key"].to(dev), vals["new_value"].to(dev), k8, v8,
+                                 torch.from_numpy(batch.slot_mapping).to(dev), ks, vs)
+    gs, gb = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)
+    assert int(gb.max()) > 0, "the workload must share blocks"
+    bt_np = batch.block_tables if mutate is None else mutate(batch.block_tables.copy())
+    if staged is None:
+        staged = int(gb.sum())
+    size = lib.pa_decode_shared_prefix_fp8_workspace_size(
+        batch.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+        batch.max_context_len, batch.block_tables.shape[1], gb.shape[0], staged)
+    ws = torch.empty(size, dtype=torch.uint8, device=dev)
+    q = vals["q"].to(dev)
+    out = torch.full_like(q, float("nan"))
+    lib.pa_decode_shared_prefix_fp8(out, q, k8, v8, torch.from_numpy(bt_np).to(dev),
+                                    torch.from_numpy(batch.context_lens).to(dev),
+                                    torch.from_numpy(gs).to(dev), torch.from_numpy(gb).to(dev),
+                                    wl.scale, ks, vs, staged, max_group_size=int(np.diff(gs).max()),
+                                    max_context_len=batch.max_context_len, workspace=ws)
+    torch.cuda.synchronize()
+    assert lib.pa_get_device_error() == expect_err
+    kpn, vpn = kp.numpy().copy(), vp.numpy().copy()
+    if batch.cow_pairs.shape[0]:
+        oracle.copy_blocks(kpn, vpn, batch.cow_pairs, "fp8")
+    oracle.reshape_and_cache_fp8(kpn, vpn, workloads.to_numpy_raw(vals["new_key"]),
+                                 workloads.to_numpy_raw(vals["new_value"]), wl.dtype,
+                                 batch.slot_mapping, ks, vs)
+    ref = oracle.decode_fp8(workloads.to_numpy_raw(vals["q"]), wl.dtype, kpn, vpn, ks, vs, bt_np,
+                            batch.context_lens, wl.scale)
+    return out, ref
+
+
+@pytest.mark.parametrize("prefix_kernel", ["auto", "pp", "mma"])
+@pytest.mark.parametrize("cfg", ["4s", "4cows"])
+def test_shared_prefix_small(lib, monkeypatch, cfg, prefix_kernel):
+    """Every prefix kernel over the staged shared blocks, every row."""
+    if prefix_kernel == "auto":
+        monkeypatch.delenv("PA_PREFIX_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("PA_PREFIX_KERNEL", prefix_kernel)
+    wl = workloads.make(cfg)
+    out, ref = _run_shared(lib, wl)
+    assert_close(out, ref, "bf16", what=wl.name + " fp8 shared-prefix")
+
+
+@pytest.mark.parametrize("cfg", ["4", "4cow"])
+def test_shared_prefix_full(lib, cfg):
+    """Full-size parallel-sampling batches over an FP8 cache, every row."""
+    wl = workloads.make(cfg)
+    out, ref = _run_shared(lib, wl)
+    assert_close(out, ref, "bf16", what=wl.name + " fp8 shared-prefix")
+
+
+def test_shared_prefix_member_mismatch(lib):
+    """A member whose table leaves its group's block: PA_DEVERR_PREFIX and a
+    zero row for it, every other row the oracle's."""
+    wl = workloads.make("4s")
+
+    def mutate(bt):
+        bt[2, 1] = bt[9, 1]  # sequence 2 no longer holds its group's block 1
+        return bt
+    out, ref = _run_shared(lib, wl, expect_err=lib.PA_DEVERR_PREFIX, mutate=mutate)
+    assert torch.count_nonzero(out[2]) == 0
+    keep = [i for i in range(out.shape[0]) if i != 2]
+    assert_close(out, ref, "bf16", rows=keep, what="fp8 shared-prefix other members")
+
+
+def test_shared_prefix_staging_overflow(lib):
+    """A staging bound one block short: PA_DEVERR_STAGING (and BLOCK_ID for the
+    block left out); each row is the oracle's or zeros, some of each."""
+    wl = workloads.make("4s")
+    batch = build_batch(wl)
+    gb = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)[1]
+    out, ref = _run_shared(lib, wl, staged=int(gb.sum()) - 1,
+                           expect_err=lib.PA_DEVERR_STAGING | lib.PA_DEVERR_BLOCK_ID)
     g = out.float().cpu().numpy().astype(np.float64)
     zero = np.all(g == 0.0, axis=(1, 2))
     ok = np.all(np.abs(g - ref) <= 2e-3 + 1e-2 * np.abs(ref), axis=(1, 2))
