@@ -61,7 +61,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
 FLUSH_BYTES = 256 * 2 ** 20          # >= 2x L2: reading this evicts every cached line
-EXTRA_CONFIGS = ("2", "3fp8", "4", "4cow", "5", "5bs32", "5fp8", "1")
+EXTRA_CONFIGS = ("2", "3fp8", "4", "4cow", "4fp8", "5", "5bs32", "5fp8", "1")
 
 
 def _peaks():
@@ -367,7 +367,7 @@ class DeviceBatch:
         self.out = torch.empty_like(self.q)
         self.mcl = batch.max_context_len
         self.cache.workspace(batch.num_seqs, wl.num_heads, self.mcl)
-        self.shared = wl.kind == "shared_prefix" and not plain_decode and not kv_fp8
+        self.shared = wl.kind == "shared_prefix" and not plain_decode
         if self.shared:
             gs_np, gb_np = shared_prefix_groups(batch.block_tables, batch.context_lens, wl.block_size)
             self.gs = torch.from_numpy(gs_np).to(dev)
@@ -391,7 +391,9 @@ class DeviceBatch:
         if self.shared:
             self.cache.attend_shared_prefix(self.q, self.bt, self.cl, self.gs, self.gb,
                                             self.wl.scale, max_group_size=self.max_group,
-                                            out=self.out, max_context_len=self.mcl)
+                                            out=self.out, max_context_len=self.mcl,
+                                            staged_blocks=int(self.gb_np.sum()) if self.kv_fp8
+                                            else None)
         else:
             self.attend_plain()
 
@@ -414,7 +416,7 @@ class DeviceBatch:
                                                self.wl.head_dim, self.wl.block_size, self.mcl, 0) > 0
         return 1 + 1 + (1 if splits else 0) + (1 if self.cow.shape[0] else 0) + \
             (1 if b.max_query_len > 1 else 0) + (1 if self.shared else 0) + \
-            (2 if self.staged else 0)  # FP8 chunk rows: staging plan + staging copy
+            (2 if self.staged or (self.kv_fp8 and self.shared) else 0)  # FP8: staging plan + copy
 
     def rows_callable(self, ids):
         """A call attending only the query rows of sequences `ids` (the decode
@@ -452,7 +454,7 @@ def measure_config(db, timer, k):
     res = {"workload": wl.name, "dtype": ("fp8_e4m3 KV, " + wl.dtype + " q/out") if db.kv_fp8
            else wl.dtype, "seqs": batch.num_seqs, "q_rows": db.bytes["q_rows"],
            "kv_tokens": db.bytes["kv_tokens"], "decode_bytes": db.bytes["decode"]}
-    name = "pa_decode_shared_prefix" if db.shared else ("pa_decode_fp8" if db.kv_fp8 else "pa_decode")
+    name = ("pa_decode_shared_prefix" if db.shared else "pa_decode") + ("_fp8" if db.kv_fp8 else "")
     call = timer.flushed(db.attend)
     call["avg_ms_back_to_back"] = timer.back_to_back(db.attend, k)
     call["GBps"] = _rate(db.bytes["decode"], call["median_ms"])
@@ -822,8 +824,8 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = hbm_peak()
     achieved = nbytes["decode"] / (dec_avg * 1e-3) / 1e9
     value = job_bytes / (ms * 1e-3) / 1e9
-    call_name = ("pa_decode_shared_prefix" if args.config.startswith("4") and not args.plain_decode
-                 else ("pa_decode_fp8" if args.kv_fp8 else "pa_decode"))
+    call_name = (("pa_decode_shared_prefix" if args.config.startswith("4") and not args.plain_decode
+                  else "pa_decode") + ("_fp8" if args.kv_fp8 else ""))
     res = {
         "metric": METRIC,
         "value": value,

@@ -59,7 +59,7 @@ __device__ __forceinline__ uint32_t quant2(float a, float b, float scale) {
   return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
 }
 
-// One thread per (token, kv head, group of 16 columns).  The cache tile of a
+// K: one thread per (token, kv head, group of 16 columns); V: see below.  The cache tile of a
 // (block, kv head) is laid out for the decode kernel's fragment loads:
 //   K [BS][D]: column d = 64j + 16k + c of row r goes to byte
 //     ((4j + t) ^ (r mod D/16)) * 16 + 4k + i of the row, t = (c mod 8) / 2,
@@ -106,14 +106,34 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
       const int chunk = (4 * j + t) ^ (r & (G16 - 1));
       *reinterpret_cast<uint32_t *>(krow + chunk * 16 + 4 * k) = w;
     }
-    load8<T>(value + src, *reinterpret_cast<float(*)[8]>(x));
-    load8<T>(value + src + 8, *reinterpret_cast<float(*)[8]>(x + 8));
+  }
+  // V: a thread takes 8 columns of one token; the 16 lanes of a half-warp take
+  // 16 consecutive tokens, so that when they fill consecutive slots of a
+  // block their bytes of a column form whole 16-byte runs of the transposed
+  // tile (one store transaction instead of sixteen)
+  const int64_t vtotal = (int64_t)((num_tokens + 15) / 16) * num_kv_heads * G16 * 32;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < vtotal;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int lo = (int)(i & 15), half = (int)((i >> 4) & 1);
+    int64_t rest = i >> 5;
+    const int g16 = (int)(rest % G16);
+    rest /= G16;
+    const int h = (int)(rest % num_kv_heads);
+    const int64_t tok = (rest / num_kv_heads) * 16 + lo;
+    if (tok >= num_tokens) continue;
+    const int64_t slot = slot_mapping[tok];
+    if (slot < 0 || slot >= num_slots) continue;  // reported by the K loop
+    const int64_t blk = slot / BS;
+    const int r = (int)(slot - blk * BS);
+    const int64_t tile = (blk * num_kv_heads + h) * (int64_t)(BS * D);
+    float x[8];
+    load8<T>(value + (tok * num_kv_heads + h) * D + g16 * 16 + half * 8, x);
     const int kk = r >> 4, c = r & 15;
     const int vpos = BS == 16 ? 4 * ((c & 7) >> 1) + (c & 1) + 2 * (c >> 3)
                               : 8 * ((c & 7) >> 1) + 4 * kk + (c & 1) + 2 * (c >> 3);
-    unsigned char *vcol = v_cache + tile + (int64_t)(g16 * 16) * BS + vpos;
+    unsigned char *vcol = v_cache + tile + (int64_t)(g16 * 16 + half * 8) * BS + vpos;
 #pragma unroll
-    for (int e = 0; e < 16; e += 2) {
+    for (int e = 0; e < 8; e += 2) {
       const uint32_t two = quant2(x[e], x[e + 1], v_scale);
       vcol[(int64_t)e * BS] = (unsigned char)(two & 0xffu);
       vcol[(int64_t)(e + 1) * BS] = (unsigned char)(two >> 8);
