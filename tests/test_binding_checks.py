@@ -111,3 +111,42 @@ def test_tensor_on_another_device_is_refused(monkeypatch):
         _lib._dev(_FakeCudaTensor(), "q")
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
     assert isinstance(_lib._dev(_FakeCudaTensor(), "q"), _FakeCudaTensor)
+
+
+def _fp8_args(S=2, tq=None):
+    a = _decode_args(S=S, tq=tq)
+    a["k_cache"] = torch.zeros(8, 2, 16, 128, dtype=torch.uint8)
+    a["v_cache"] = torch.zeros(8, 2, 16, 128, dtype=torch.uint8)
+    return a
+
+
+def test_fp8_rows_and_shared_prefix_fp8_shape_disagreements():
+    a = _fp8_args(tq=5)
+    with pytest.raises(ValueError, match="num_seqs \\+ 1"):
+        _lib.pa_decode_fp8_rows(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                                a["context_lens"], torch.tensor([0, 5], dtype=torch.int32), 0.1,
+                                1.0, 1.0, 4, 1)
+    a = _fp8_args()
+    a["context_lens"] = torch.zeros(3, dtype=torch.int32)
+    with pytest.raises(ValueError, match="number of sequences"):
+        _lib.pa_decode_shared_prefix_fp8(a["out"], a["q"], a["k_cache"], a["v_cache"],
+                                         a["block_tables"], a["context_lens"],
+                                         torch.tensor([0, 2], dtype=torch.int32),
+                                         torch.tensor([1], dtype=torch.int32), 0.1, 1.0, 1.0, 1)
+    a = _fp8_args()
+    with pytest.raises(ValueError, match="one more entry"):
+        _lib.pa_decode_shared_prefix_fp8(a["out"], a["q"], a["k_cache"], a["v_cache"],
+                                         a["block_tables"], a["context_lens"],
+                                         torch.tensor([0, 2], dtype=torch.int32),
+                                         torch.tensor([1, 1], dtype=torch.int32), 0.1, 1.0, 1.0, 2)
+
+
+def test_staged_blocks_needed():
+    """The staging bound counts the blocks of the sequences with more than one
+    query row (ceil(L / block_size)), nothing for decode rows or empty ones."""
+    from paged_kv_cache_388_b200.batch import staged_blocks_needed
+    qsl = [0, 1, 97, 98, 98, 610]          # rows 1, 96, 1, 0, 512
+    lens = [5000, 796, 17, 0, 16896]
+    assert staged_blocks_needed(qsl, lens, 16) == 50 + 1056
+    assert staged_blocks_needed(qsl, lens, 32) == 25 + 528
+    assert staged_blocks_needed([0, 1, 2], [10, 20], 16) == 0

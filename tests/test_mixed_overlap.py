@@ -104,3 +104,43 @@ def test_forked_mixed_8k_long_chunks():
     rows += list(range(int(qsl[-1]) - 64, int(qsl[-1])))  # the last chunk's final rows
     _, _, ref = oracle_step(wl, vals, rows=np.asarray(rows))
     assert_close(out, ref, wl.dtype, rows=rows, what="overlap_mixed_8k")
+
+
+def test_concurrent_callers():
+    """Two host threads, each with its own stream and workspace, call
+    pa_decode on mixed batches at once: the library's side stream is shared,
+    so each fork-join holds it; every result equals the serial order's."""
+    import threading
+    lib, wl, vals, batch, d, _ = _setup("5s")
+    serial = torch.empty_like(d["q"])
+    lib.pa_decode_noalloc(serial, d["q"], d["k_cache"], d["v_cache"], d["block_tables"],
+                          d["context_lens"], wl.scale, query_start_loc=d["qsl"],
+                          max_query_len=batch.max_query_len, max_context_len=batch.max_context_len)
+    torch.cuda.synchronize()
+    size = lib.pa_decode_workspace_size(batch.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                                        wl.block_size, batch.max_context_len, 0)
+    outs, errors = [], []
+
+    def worker():
+        try:
+            st = torch.cuda.Stream()
+            ws = torch.empty(max(16, size), dtype=torch.uint8, device="cuda")
+            res = [torch.empty_like(d["q"]) for _ in range(6)]
+            with torch.cuda.stream(st):
+                for o in res:
+                    _forked(lib, wl, batch, d, ws, o)
+            st.synchronize()
+            outs.extend(res)
+        except Exception as e:  # noqa: BLE001 -- surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker) for _ in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    assert lib.pa_get_device_error() == 0
+    assert len(outs) == 12
+    for o in outs:
+        assert torch.equal(o, serial)
