@@ -485,7 +485,7 @@ def measure_config(db, timer, k):
         dec_ids = [i for i in range(batch.num_seqs) if qsl[i + 1] - qsl[i] == 1]
         chk_ids = [i for i in range(batch.num_seqs) if qsl[i + 1] - qsl[i] > 1]
         flops = chunk_flops(batch) * wl.num_heads * wl.head_dim * 4
-        dbytes, _, _ = seq_bytes(wl, batch, dec_ids)
+        dbytes, _, _ = seq_bytes(wl, batch, dec_ids, kv_elem=1 if db.kv_fp8 else None)
         if dec_ids:
             d = timer.flushed(db.rows_callable(dec_ids))
             d["GBps"] = _rate(dbytes, d["median_ms"])
