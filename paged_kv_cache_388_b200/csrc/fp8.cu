@@ -53,13 +53,37 @@ __device__ __forceinline__ void load8<__half>(const __half *p, float (&x)[8]) {
   }
 }
 
+// Two consecutive elements as floats.
+template <typename T>
+__device__ __forceinline__ void load2(const T *p, float &a, float &b);
+template <>
+__device__ __forceinline__ void load2<float>(const float *p, float &a, float &b) {
+  const float2 v = __ldcs(reinterpret_cast<const float2 *>(p));
+  a = v.x;
+  b = v.y;
+}
+template <>
+__device__ __forceinline__ void load2<__nv_bfloat16>(const __nv_bfloat16 *p, float &a, float &b) {
+  const uint32_t u = __ldcs(reinterpret_cast<const unsigned int *>(p));
+  a = __uint_as_float(u << 16);
+  b = __uint_as_float(u & 0xffff0000u);
+}
+template <>
+__device__ __forceinline__ void load2<__half>(const __half *p, float &a, float &b) {
+  const uint32_t u = __ldcs(reinterpret_cast<const unsigned int *>(p));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&u));
+  a = f.x;
+  b = f.y;
+}
+
 // Two elements -> two E4M3 codes of x / scale (the first in the low byte).
 __device__ __forceinline__ uint32_t quant2(float a, float b, float scale) {
   const float2 q = make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale));
   return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
 }
 
-// K: one thread per (token, kv head, group of 16 columns); V: see below.  The cache tile of a
+// K: one thread per (token, kv head, 16-byte chunk of the row), so that the
+// lanes of a warp write whole rows; V: see below.  The cache tile of a
 // (block, kv head) is laid out for the decode kernel's fragment loads:
 //   K [BS][D]: column d = 64j + 16k + c of row r goes to byte
 //     ((4j + t) ^ (r mod D/16)) * 16 + 4k + i of the row, t = (c mod 8) / 2,
@@ -88,24 +112,25 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(
       if (rest == 0) raise_error(err, PA_DEVERR_SLOT);
       continue;
     }
+    // the row's 16-byte chunk of fragment column group jt = 4j + t: word k
+    // holds columns 64j + 16k + 2t, +1 (low half) and +8, +9 (high half)
     const int h = (int)(rest / G16);
-    const int g16 = (int)(rest - (int64_t)h * G16);
-    const int j = g16 >> 2, k = g16 & 3;
+    const int jt = (int)(rest - (int64_t)h * G16);
+    const int j = jt >> 2, t = jt & 3;
     const int64_t blk = slot / BS;
     const int r = (int)(slot - blk * BS);
     const int64_t tile = (blk * num_kv_heads + h) * (int64_t)(BS * D);
-    const int64_t src = (tok * num_kv_heads + h) * D + g16 * 16;
-    float x[16];
-    load8<T>(key + src, *reinterpret_cast<float(*)[8]>(x));
-    load8<T>(key + src + 8, *reinterpret_cast<float(*)[8]>(x + 8));
-    unsigned char *krow = k_cache + tile + (int64_t)r * D;
+    const T *kp = key + (tok * num_kv_heads + h) * D + 64 * j + 2 * t;
+    uint32_t w[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const uint32_t w = quant2(x[2 * t], x[2 * t + 1], k_scale) |
-                         (quant2(x[2 * t + 8], x[2 * t + 9], k_scale) << 16);
-      const int chunk = (4 * j + t) ^ (r & (G16 - 1));
-      *reinterpret_cast<uint32_t *>(krow + chunk * 16 + 4 * k) = w;
+    for (int k = 0; k < 4; ++k) {
+      float a0, a1, b0, b1;
+      load2<T>(kp + 16 * k, a0, a1);
+      load2<T>(kp + 16 * k + 8, b0, b1);
+      w[k] = quant2(a0, a1, k_scale) | (quant2(b0, b1, k_scale) << 16);
     }
+    unsigned char *krow = k_cache + tile + (int64_t)r * D;
+    *reinterpret_cast<uint4 *>(krow + ((jt ^ (r & (G16 - 1))) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   // V: a thread takes 8 columns of one token; the 16 lanes of a half-warp take
   // 16 consecutive tokens, so that when they fill consecutive slots of a
