@@ -124,6 +124,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// Transpose of an 8x8 16-bit matrix held as the warp's m8n8 fragment (lane
+// 4r + c holds row r, columns 2c and 2c + 1; lower column in the low half).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -166,8 +174,7 @@ struct MmaLayout {
   static constexpr int kTile = BS * D * kElem;    // bytes of one (block, kv-head) K or V tile
   static constexpr int kStage = 2 * kTile;
   static constexpr int kStages = (PA_MMA_RING_KB * 1024) / kStage < 2 ? 2 : (PA_MMA_RING_KB * 1024) / kStage;
-  static constexpr int kPbuf = NT * 2 * 8 * 16 * 2;  // per warp: P^T hi+lo [nt][8 heads][16 keys]
-  int ring, qbuf, full, empty, qfull, qempty, bad, misc, batch, pbuf, merge, bytes, qbytes;
+  int ring, qbuf, full, empty, qfull, qempty, bad, misc, batch, merge, bytes, qbytes;
   // merge area: [warp][group heads][D + 4] floats
   __host__ __device__ MmaLayout(int n, int group) {
     qbytes = group * D * 2;
@@ -180,8 +187,7 @@ struct MmaLayout {
     bad = qempty + 16;
     misc = align_up(bad + 4 * kStages, 16);
     batch = misc + 16;
-    pbuf = align_up(batch + BatchSmem::bytes(n), 128);
-    merge = align_up(pbuf + NCW * kPbuf, 128);
+    merge = align_up(batch + BatchSmem::bytes(n), 128);
     bytes = merge + NCW * group * (D + 4) * 4 + 1024;  // + alignment slack
   }
 };
@@ -413,7 +419,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
 
   // ======================= consumer warps ==================================
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
-  unsigned char *pbuf = smem + lay.pbuf + warp * L::kPbuf;  // [nt][hi|lo][8 heads][16 keys] 16-bit
   float *merge = reinterpret_cast<float *>(smem + lay.merge);
   const int mstride = a.group * (D + 4);
   const float sl2 = a.scale_log2;
@@ -582,7 +587,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
             uint32_t pb_hi[NT][2], pb_lo[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              float p[4];
+              float p[4], alpha[2];
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
                 const float x0 = v0 ? s[nt][hh] * qf[nt][hh] : -INFINITY;
@@ -592,35 +597,42 @@ __global__ void __launch_bounds__(32 * (NCW + 1), NT == 1 ? PA_MMA_MIN_CTAS : 2)
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 const float mn = fmaxf(m[nt][hh], mx);
-                const float alpha = fast_exp2(m[nt][hh] - mn);
+                alpha[hh] = fast_exp2(m[nt][hh] - mn);
                 m[nt][hh] = mn;
                 p[hh] = fast_exp2(x0 - mn);
                 p[2 + hh] = fast_exp2(x1 - mn);
-                l[nt][hh] = l[nt][hh] * alpha + p[hh] + p[2 + hh];
+                l[nt][hh] = l[nt][hh] * alpha[hh] + p[hh] + p[2 + hh];
+              }
+              // O^T columns of heads whose max moved; skipped when every
+              // factor of the warp is exactly 1 (the product would be o)
+              if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                  o[nt][mt][hh] *= alpha;
-                  o[nt][mt][2 + hh] *= alpha;
+                  o[nt][mt][0] *= alpha[0];
+                  o[nt][mt][1] *= alpha[1];
+                  o[nt][mt][2] *= alpha[0];
+                  o[nt][mt][3] *= alpha[1];
                 }
               }
-              // P^T via shared memory: P[head][key] 16-bit, rows of 16 keys
-              uint16_t *ph = reinterpret_cast<uint16_t *>(pbuf) + nt * 2 * 128;
-              uint16_t *pl = ph + 128;
+              // P^T as the B operand: the S^T accumulator holds, per 8-key
+              // half, rows = keys g and columns = heads 2t, 2t+1, i.e. the
+              // m8n8 16-bit fragment of P^T transposed; movmatrix turns it
+              // into rows = head g, columns = keys 2t, 2t+1
+              uint32_t hw[2], lw[2];
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int head = 2 * t + (c & 1), key = g + (c >> 1) * 8;
-                const uint16_t hi = MmaT<Tc>::bits(p[c]);
-                ph[head * 16 + key] = hi;
-                if constexpr (MmaT<Tc>::kSplitP) pl[head * 16 + key] = MmaT<Tc>::bits(p[c] - MmaT<Tc>::back(hi));
+              for (int half = 0; half < 2; ++half) {
+                const uint16_t h0 = MmaT<Tc>::bits(p[2 * half]), h1 = MmaT<Tc>::bits(p[2 * half + 1]);
+                hw[half] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                if constexpr (MmaT<Tc>::kSplitP)
+                  lw[half] = (uint32_t)MmaT<Tc>::bits(p[2 * half] - MmaT<Tc>::back(h0)) |
+                             ((uint32_t)MmaT<Tc>::bits(p[2 * half + 1] - MmaT<Tc>::back(h1)) << 16);
               }
-              __syncwarp();
-              pb_hi[nt][0] = *reinterpret_cast<const uint32_t *>(ph + g * 16 + 2 * t);
-              pb_hi[nt][1] = *reinterpret_cast<const uint32_t *>(ph + g * 16 + 8 + 2 * t);
+              pb_hi[nt][0] = movmatrix_t(hw[0]);
+              pb_hi[nt][1] = movmatrix_t(hw[1]);
               if constexpr (MmaT<Tc>::kSplitP) {
-                pb_lo[nt][0] = *reinterpret_cast<const uint32_t *>(pl + g * 16 + 2 * t);
-                pb_lo[nt][1] = *reinterpret_cast<const uint32_t *>(pl + g * 16 + 8 + 2 * t);
+                pb_lo[nt][0] = movmatrix_t(lw[0]);
+                pb_lo[nt][1] = movmatrix_t(lw[1]);
               }
-              __syncwarp();
             }
             // ---- rows past the context end may hold anything (even NaN):
             //      zero them in the staged V tile, as P is 0 there ----
