@@ -757,23 +757,28 @@ def run_ours(args, rank, world, local_rank):
 
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # The clock record spans the timed steps and the per-call timings that
+    # the roofline figures come from (the K steps alone last a few ms, less
+    # than the sampling period).
     with ClockSampler(local_rank) as clocks:
         barrier()
         t_start.record(stream)
         g_steps.replay()
         t_end.record(stream)
         barrier()
-    ms_local = t_start.elapsed_time(t_end)
-    job_bytes, ms = aggregate(nbytes["step"] * K, ms_local, dev)
-    assert _lib.pa_get_device_error() == 0
-    clk = clocks.summary()
-    del g_steps, g_warm
+        ms_local = t_start.elapsed_time(t_end)
+        job_bytes, ms = aggregate(nbytes["step"] * K, ms_local, dev)
+        assert _lib.pa_get_device_error() == 0
+        del g_steps, g_warm
 
-    # per-call device time of the step's calls: K back-to-back calls in one
-    # graph (inputs larger than L2) and 50 single calls after an L2 flush
-    dec_avg = timer.back_to_back(db.attend, K)
-    res_avg = timer.back_to_back(db.write, K)
-    dec_flushed = timer.flushed(db.attend)
+        # per-call device time of the step's calls: K back-to-back calls in one
+        # graph (inputs larger than L2) and 50 single calls after an L2 flush
+        dec_avg = timer.back_to_back(db.attend, K)
+        res_avg = timer.back_to_back(db.write, K)
+        dec_flushed = timer.flushed(db.attend)
+        torch.cuda.synchronize(dev)
+    clk = clocks.summary()
+    clk["window"] = "timed steps and the per-call timings of the step's calls"
 
     # ---- end to end through the public API, host (pinned) buffers ----------
     e2e = None
