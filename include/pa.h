@@ -354,7 +354,8 @@ int pa_decode(void *out, const void *q, const void *k_cache,
  * bytes plus a few KiB, so on a 148-SM B200 every group <= 8 at head_dim
  * 128 and every group <= 16 at head_dim 64 fits whatever the occupancy;
  * group 16 at head_dim 128 fits at the occupancy the decode kernel reaches
- * (5 CTAs per SM, about 12.5 MiB) but not at the bound.  Fixed splits
+ * for groups above 8 (2 CTAs per SM at its 232 registers per thread, about
+ * 5 MiB) but not at the bound.  Fixed splits
  * (kv_split_tokens > 0) need num_seqs * num_heads * splits * (head_dim + 2)
  * * 4 bytes.
  * The first call on a device looks up the array's device address
